@@ -1,0 +1,298 @@
+/*
+ * mmh3.h -- C ABI of the B200 (sm_100a) packed multimodal DiT block library.
+ *
+ * The hot path is the forward pass of a MiniMax-H3-shaped packed-token DiT
+ * block: one sequence [text | audio | video] with no batching and no
+ * cross-attention, modulated per token through a segment table over a
+ * rank-24 adaLN timestep curve.  Operations follow the page
+ * "cortiq_engine/mmh3.rs" (docs.rs, cortiq-engine 0.5.72); the encoder-layer
+ * entry points follow "ffai-argus 0.7.0 src/siglip.rs".
+ *
+ * Conventions (every entry point):
+ *  - Matrices are row-major; projection weights are [out, in].
+ *  - "device" pointers are CUDA device memory owned by the caller; "host"
+ *    pointers are ordinary host memory.  The library never allocates or
+ *    frees device memory and never synchronises the stream, except where an
+ *    entry point says so (mmh3_device_status).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *  - Argument errors are reported before anything is launched; the return
+ *    value is an mmh3_status and mmh3_last_error() gives a message (thread
+ *    local, valid until the next call on the same thread).
+ *  - Activation / GEMM-operand dtype: MMH3_BF16 (bf16 storage, fp32
+ *    accumulate on tcgen05 kind::f16) or MMH3_F32 (fp32 storage, tcgen05
+ *    kind::tf32).  The residual stream x is always fp32.  Norm gains, adaLN
+ *    basis / bias / table and output-head biases are always fp32.
+ *  - Kernel waits are bounded (default 2 s, MMH3_WAIT_LIMIT_MS or
+ *    mmh3_set_wait_limit_ns); a kernel that gives up records a device status
+ *    that mmh3_device_status() returns as MMH3_ERR_TIMEOUT.
+ */
+#ifndef MMH3_H_
+#define MMH3_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MMH3_OK = 0,
+  MMH3_ERR_ARG = 1,          /* null pointer, bad enum, inconsistent argument */
+  MMH3_ERR_SHAPE = 2,        /* unsupported or inconsistent sizes */
+  MMH3_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned */
+  MMH3_ERR_WORKSPACE = 4,    /* workspace missing or too small */
+  MMH3_ERR_UNSUPPORTED = 5,  /* more than two distinct timesteps, etc. */
+  MMH3_ERR_CUDA = 6,         /* a CUDA runtime / driver call failed */
+  MMH3_ERR_TIMEOUT = 7       /* a kernel gave up waiting (device status) */
+} mmh3_status;
+
+typedef enum { MMH3_F32 = 0, MMH3_BF16 = 1 } mmh3_dtype;
+
+/* Block hyper-parameters.  rope_k = rotary frequencies per position axis
+ * (3*rope_k pairs rotate, dims >= 6*rope_k do not); 16 for head_dim 128. */
+typedef struct {
+  int hidden;        /* H, multiple of 128 */
+  int heads;         /* nh */
+  int head_dim;      /* hd: 64 or 128; inner = heads*head_dim == hidden */
+  int ffn;           /* F (SwiGLU inner), multiple of 128 */
+  int rank;          /* adaLN curve rank R (24), <= 32 */
+  int grid;          /* timestep-curve table rows G (1025) */
+  int rope_k;        /* hd/8 */
+  float eps;         /* RMSNorm eps for norm1 / norm2 / final norm (1e-5) */
+  float qk_eps;      /* q/k RMSNorm eps (1e-5) */
+  float rope_theta;  /* rotary base (10000) */
+  int act_dtype;     /* mmh3_dtype of activations and projection weights */
+} mmh3_dims;
+
+/* One contiguous run of tokens sharing a modality tag and a flow clock.
+ * tag: 0 video, 1 text, 2 audio (adaLN row order).  clock: 0 = the video
+ * clock (t_v = 1 - max(sigma_v, 1e-6)), 1 = the audio clock
+ * (t_a = 1 - sigma_a).  Text uses the video clock.  Segments must be sorted,
+ * contiguous and cover [0, n) exactly; at most 8. */
+typedef struct {
+  uint32_t start, stop;
+  uint8_t tag, clock;
+  uint8_t pad[2];
+} mmh3_segment;
+
+/* One block's weights (device pointers).
+ *  norm1, norm2 [H] fp32; q_norm, k_norm [hd] fp32;
+ *  wqkv [3*inner, H] act dtype, rows [q | k | v], heads contiguous;
+ *  wout [H, inner]; wfc2 [H, F];
+ *  wfc1 [2F, H] act dtype in the INTERLEAVED order written by
+ *       mmh3_prepare_fc1 (not the checkpoint's [gate | up] order);
+ *  adaln_w [2*3*6*H, R], adaln_b [2*3*6*H], adaln_table [G, R] fp32. */
+typedef struct {
+  const float* norm1;
+  const float* norm2;
+  const void* wqkv;
+  const void* wout;
+  const float* q_norm;
+  const float* k_norm;
+  const void* wfc1;
+  const void* wfc2;
+  const float* adaln_w;
+  const float* adaln_b;
+  const float* adaln_table;
+} mmh3_block_weights;
+
+/* Final layer (output heads).  final_norm [H] fp32; adaln_w [2*2*H, R],
+ * adaln_b [2*2*H], adaln_table [G, R] fp32 (one modality, chunks shift,
+ * scale); w_video [out_video, H] / w_audio [out_audio, H] act dtype;
+ * b_video / b_audio fp32.  out_* must be multiples of 32. */
+typedef struct {
+  const float* final_norm;
+  const float* adaln_w;
+  const float* adaln_b;
+  const float* adaln_table;
+  const void* w_video;
+  const float* b_video;
+  const void* w_audio;
+  const float* b_audio;
+  int out_video;
+  int out_audio;
+} mmh3_head_weights;
+
+/* ------------------------------------------------------------ host helpers */
+
+/* sigma on the to_shift schedule at the same base-grid point:
+ * b = s / (f + s (1 - f)),  s' = t b / (1 + (t - 1) b)
+ * ("cortiq_engine/mmh3.rs", time_shift_sigma).  Host only, never fails. */
+double mmh3_time_shift_sigma(double sigma, double from_shift, double to_shift);
+
+/* The t2va layout [text | audio | video] ("cortiq_engine/mmh3.rs",
+ * Layout::t2va / build_full): text rows (i, 0, 0); stereo audio rows
+ * channel-major from t = text_len with w at the frame grid's extremes; video
+ * frames advancing t by (5/3)*[1,4,4,4,4][k%5] over the 2x2-patch h/w grid
+ * of axis_from_sqrt_area.  Positions are computed in fp64 and rounded to
+ * fp32.  Host buffers: segs [>= 3], pos [pos_capacity * 3] (t, h, w).
+ * *n_out = text_len + 2*audio_t + latent_t*(lat_h/2)*(lat_w/2); returns
+ * MMH3_ERR_SHAPE if pos_capacity is smaller (pos may be NULL to query n). */
+mmh3_status mmh3_layout_t2va(int text_len, int latent_t, int lat_h, int lat_w, int audio_t,
+                             mmh3_segment* segs, int* n_seg, float* pos, int pos_capacity,
+                             int* n_out);
+
+/* Image mode [text | reference image | target image]: the reference image is
+ * placed like a reference still of "cortiq_engine/mmh3.rs" build_full (rows
+ * at the cursor t with their own h/w grid, cursor + 1), the target at the
+ * next t; image rows are tag video on clock 0.  Same buffers as above. */
+mmh3_status mmh3_layout_image(int text_len, int ref_lat_h, int ref_lat_w, int lat_h, int lat_w,
+                              mmh3_segment* segs, int* n_seg, float* pos, int pos_capacity,
+                              int* n_out);
+
+/* Distinct timesteps (ascending, de-duplicated) of the clocks the segments
+ * use, and each segment's block adaLN row slot(clock)*3 + tag
+ * ("cortiq_engine/mmh3.rs", forward).  Host buffers: ts [2], seg_rows
+ * [n_seg].  MMH3_ERR_UNSUPPORTED if the clocks give > 2 timesteps. */
+mmh3_status mmh3_plan_timesteps(const mmh3_segment* segs, int n_seg, int n, double sigma_v,
+                                double sigma_a, double* ts, int* n_ts, int* seg_rows);
+
+/* ------------------------------------------------------------ device steps */
+
+/* Writes the per-token adaLN row (int32 [n], device) that the fused
+ * norm/modulate gather uses: rows[i] = slot(clock)*3 + tag of i's segment. */
+mmh3_status mmh3_resolve_rows(const mmh3_segment* segs, int n_seg, int n, double sigma_v,
+                              double sigma_a, int32_t* rows_dev, void* stream);
+
+/* adaLN as a curve ("cortiq_engine/mmh3.rs", Adaln::eval): for each distinct
+ * timestep slot s (ts from the segments, sigma_v, sigma_a):
+ *   p = clamp(t,0,1)*(G-1), i0 = min(floor p, G-2), f = p - i0,
+ *   c = (1-f) table[i0] + f table[i0+1],
+ *   out[s*rows_per_slot + r] = w[s*rows_per_slot + r] . c + b[...]
+ * rows_per_slot = 18*H for a block (3 tags x 6 chunks), 2*H for the final
+ * layer.  out: device fp32 [n_ts * rows_per_slot].  *n_ts receives T_s. */
+mmh3_status mmh3_adaln_modulation(const mmh3_dims* dims, const float* w, const float* b,
+                                  const float* table, int rows_per_slot, const mmh3_segment* segs,
+                                  int n_seg, int n, double sigma_v, double sigma_a, float* out,
+                                  int* n_ts, void* stream);
+
+/* Rewrites fc1 [2F, H] from the checkpoint order [gate | up] into the tile
+ * order the fused fc1+SwiGLU kernel reads: blocks of 256 rows, 128 gate rows
+ * then the 128 matching up rows.  Device in/out, act dtype, distinct. */
+mmh3_status mmh3_prepare_fc1(const mmh3_dims* dims, const void* fc1_gate_up, void* fc1_tiled,
+                             void* stream);
+
+/* Bytes of device workspace mmh3_block_forward / mmh3_stack_forward need for
+ * n tokens.  Layout (each region 256-byte aligned, in this order): mods fp32
+ * [2*3, 6H]; rope (cos, sin) fp32x2 [n, 3*rope_k]; xn1 [n, H]; qkv [n, 3*inner]
+ * (q and k after qk-norm + rotation); attn [n, inner]; xn2 [n, H]; act [n, F];
+ * head scratch [n, H] and final mods fp32 [2, 2H] -- all act dtype unless
+ * stated.  After a block call the regions hold that block's intermediates. */
+mmh3_status mmh3_workspace_size(const mmh3_dims* dims, int n, size_t* bytes);
+
+/* Full bidirectional attention over packed sequences (one 128-row query
+ * tile per CTA, tcgen05): for each sequence b < n_seq of `seq` tokens
+ * starting at row b*seq of the qkv panel [n_seq*seq, 3*heads*head_dim]
+ * (rows [q | k | v], heads contiguous, act dtype, device), per head:
+ * out = softmax(q k^T * scale) v, written to out [n_seq*seq, heads*head_dim]
+ * ("cortiq_engine/mmh3.rs", attention; softmax_inplace).  scale is applied
+ * to the scores (pass 1/sqrt(hd); 1 when it is folded into q). */
+mmh3_status mmh3_attention(const void* qkv, int n_seq, int seq, int heads, int head_dim,
+                           int act_dtype, float scale, void* out, void* stream);
+
+/* One modulated block, in place on x [n, H] fp32 (device)
+ * ("cortiq_engine/mmh3.rs", block_forward + ffn_tail):
+ *   mods = adaLN(ts); xn1 = RMSNorm(x; norm1)(1+scale_msa)+shift_msa;
+ *   qkv = xn1 Wqkv^T; q,k = RMSNorm per head (q_norm/k_norm) + partial
+ *   split-half 3-axis rotation by pos; attn = softmax(q k^T/sqrt(hd)) v;
+ *   x += gate_msa * (attn Wout^T); xn2 = RMSNorm(x; norm2)(1+scale_mlp)
+ *   +shift_mlp; act = silu(xn2 Wg^T) * (xn2 Wu^T); x += gate_mlp * (act W2^T).
+ * The modulation row of token i is given by its segment (mmh3_segment).
+ * pos_dev: device fp32 [n, 3] (t, h, w), or NULL for no rotation.
+ * modulated = 0 runs the unmodulated form (plain residuals, no adaLN; the
+ * weights' adaln pointers may be NULL).  workspace: mmh3_workspace_size. */
+mmh3_status mmh3_block_forward(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
+                               const mmh3_segment* segs, int n_seg, const float* pos_dev,
+                               double sigma_v, double sigma_a, int modulated, void* workspace,
+                               size_t ws_bytes, void* stream);
+
+/* n_blocks blocks (blocks: host array of n_blocks weight structs) then,
+ * if heads != NULL, the two output heads ("cortiq_engine/mmh3.rs", forward
+ * "blocks" and "heads"): per stream (the video segment rows -> out_video
+ * [rows, out_video], the audio segment rows -> out_audio [rows, out_audio],
+ * fp32 device), RMSNorm(final_norm) -> (1+scale)+shift from the final adaLN
+ * row of the stream's timestep -> W^T + b -> negated.  The rotation table is
+ * computed once for all blocks. */
+mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* blocks,
+                               int n_blocks, const mmh3_head_weights* heads, float* x, int n,
+                               const mmh3_segment* segs, int n_seg, const float* pos_dev,
+                               double sigma_v, double sigma_a, float* out_video, float* out_audio,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------ SigLIP encoder layer */
+
+typedef struct {
+  int hidden;     /* H, multiple of 128 */
+  int heads;
+  int head_dim;   /* 64 */
+  int mlp;        /* multiple of 128 */
+  float ln_eps;
+} mmh3_vit_dims;
+
+/* ln1_g/ln1_b/ln2_g/ln2_b [H] fp32; wqkv [3H, H] bf16 with the attention
+ * scale folded into its q rows and bqkv [3H] fp32 likewise (see
+ * mmh3_vit_fold_qkv); wo [H, H], w1 [mlp, H], w2 [H, mlp] bf16; bo, b1, b2
+ * fp32. */
+typedef struct {
+  const float* ln1_g;
+  const float* ln1_b;
+  const void* wqkv;
+  const float* bqkv;
+  const void* wo;
+  const float* bo;
+  const float* ln2_g;
+  const float* ln2_b;
+  const void* w1;
+  const float* b1;
+  const void* w2;
+  const float* b2;
+} mmh3_vit_weights;
+
+/* Fuse q/k/v into one [3H, H] bf16 matrix and [3H] fp32 bias with the
+ * attention scale head_dim^-1/2 multiplied into the q rows and q bias
+ * ("ffai-argus 0.7.0 src/siglip.rs", Layer::load).  Device pointers. */
+mmh3_status mmh3_vit_fold_qkv(const mmh3_vit_dims* dims, const void* wq, const void* wk,
+                              const void* wv, const float* bq, const float* bk, const float* bv,
+                              void* wqkv, float* bqkv, void* stream);
+
+/* Workspace: h [B*S, H] bf16, qkv [B*S, 3H] bf16, attn [B*S, H] bf16,
+ * act [B*S, mlp] bf16 (256-byte aligned regions, in this order). */
+mmh3_status mmh3_vit_workspace_size(const mmh3_vit_dims* dims, int batch, int seq, size_t* bytes);
+
+/* One pre-norm encoder layer, in place on x [batch*seq, H] fp32
+ * ("ffai-argus 0.7.0 src/siglip.rs", Layer::forward + finish_attention):
+ *   y = x + (attn(LN1 x) Wo^T + bo),  z = y + (gelu_tanh(LN2 y W1^T + b1) W2^T + b2)
+ * with attention inside each image of `seq` tokens and LayerNorm's variance
+ * computed two-pass. */
+mmh3_status mmh3_vit_layer_forward(const mmh3_vit_dims* dims, const mmh3_vit_weights* w, float* x,
+                                   int batch, int seq, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* ------------------------------------------------------------ diagnostics */
+
+/* Synchronises `stream`, then reads and clears the device status word that
+ * bounded waits write.  *code receives the first device error (0 = none);
+ * returns MMH3_ERR_TIMEOUT if one was recorded. */
+mmh3_status mmh3_device_status(void* stream, int* code, int* site);
+
+/* Bound on every in-kernel wait, in nanoseconds (0 restores the default). */
+void mmh3_set_wait_limit_ns(uint64_t ns);
+
+/* Launches one warp that waits on an mbarrier nothing arrives at, with a
+ * wait limit of limit_ns, and synchronises the stream: exercises the
+ * bounded-wait error path without hanging anything.  Returns the status
+ * mmh3_device_status would (MMH3_ERR_TIMEOUT when the wait ran out). */
+mmh3_status mmh3_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* mmh3_last_error(void);
+
+/* Library version string. */
+const char* mmh3_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMH3_H_ */

@@ -1,0 +1,117 @@
+"""ctypes declarations of the C ABI in include/mmh3.h (argument marshalling
+only).  Loading fails loudly when libmmh3.so is missing: there is no CPU or
+Python fallback for any step of the path."""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmmh3.so")
+
+MMH3_F32, MMH3_BF16 = 0, 1
+
+STATUS_NAMES = {0: "MMH3_OK", 1: "MMH3_ERR_ARG", 2: "MMH3_ERR_SHAPE", 3: "MMH3_ERR_ALIGN",
+                4: "MMH3_ERR_WORKSPACE", 5: "MMH3_ERR_UNSUPPORTED", 6: "MMH3_ERR_CUDA",
+                7: "MMH3_ERR_TIMEOUT"}
+
+
+class Mmh3Error(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Dims(C.Structure):
+    _fields_ = [("hidden", C.c_int), ("heads", C.c_int), ("head_dim", C.c_int), ("ffn", C.c_int),
+                ("rank", C.c_int), ("grid", C.c_int), ("rope_k", C.c_int), ("eps", C.c_float),
+                ("qk_eps", C.c_float), ("rope_theta", C.c_float), ("act_dtype", C.c_int)]
+
+
+class Segment(C.Structure):
+    _fields_ = [("start", C.c_uint32), ("stop", C.c_uint32), ("tag", C.c_uint8),
+                ("clock", C.c_uint8), ("pad", C.c_uint8 * 2)]
+
+
+class BlockWeights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("norm1", "norm2", "wqkv", "wout", "q_norm", "k_norm",
+                                          "wfc1", "wfc2", "adaln_w", "adaln_b", "adaln_table")]
+
+
+class HeadWeights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("final_norm", "adaln_w", "adaln_b", "adaln_table",
+                                          "w_video", "b_video", "w_audio", "b_audio")] + \
+               [("out_video", C.c_int), ("out_audio", C.c_int)]
+
+
+class VitDims(C.Structure):
+    _fields_ = [("hidden", C.c_int), ("heads", C.c_int), ("head_dim", C.c_int), ("mlp", C.c_int),
+                ("ln_eps", C.c_float)]
+
+
+class VitWeights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("ln1_g", "ln1_b", "wqkv", "bqkv", "wo", "bo", "ln2_g",
+                                          "ln2_b", "w1", "b1", "w2", "b2")]
+
+
+_P = C.c_void_p
+_I = C.c_int
+_D = C.c_double
+_SEGP = C.POINTER(Segment)
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "mmh3_time_shift_sigma": (C.c_double, [_D, _D, _D]),
+    "mmh3_layout_t2va": (_I, [_I, _I, _I, _I, _I, _SEGP, C.POINTER(_I), C.POINTER(C.c_float), _I,
+                              C.POINTER(_I)]),
+    "mmh3_layout_image": (_I, [_I, _I, _I, _I, _I, _SEGP, C.POINTER(_I), C.POINTER(C.c_float), _I,
+                               C.POINTER(_I)]),
+    "mmh3_plan_timesteps": (_I, [_SEGP, _I, _I, _D, _D, C.POINTER(_D), C.POINTER(_I),
+                                 C.POINTER(_I)]),
+    "mmh3_resolve_rows": (_I, [_SEGP, _I, _I, _D, _D, _P, _P]),
+    "mmh3_adaln_modulation": (_I, [C.POINTER(Dims), _P, _P, _P, _I, _SEGP, _I, _I, _D, _D, _P,
+                                   C.POINTER(_I), _P]),
+    "mmh3_prepare_fc1": (_I, [C.POINTER(Dims), _P, _P, _P]),
+    "mmh3_workspace_size": (_I, [C.POINTER(Dims), _I, C.POINTER(C.c_size_t)]),
+    "mmh3_attention": (_I, [_P, _I, _I, _I, _I, _I, C.c_float, _P, _P]),
+    "mmh3_block_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _P,
+                                _D, _D, _I, _P, C.c_size_t, _P]),
+    "mmh3_stack_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _I,
+                                C.POINTER(HeadWeights), _P, _I, _SEGP, _I, _P, _D, _D, _P, _P, _P,
+                                C.c_size_t, _P]),
+    "mmh3_vit_fold_qkv": (_I, [C.POINTER(VitDims), _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "mmh3_vit_workspace_size": (_I, [C.POINTER(VitDims), _I, _I, C.POINTER(C.c_size_t)]),
+    "mmh3_vit_layer_forward": (_I, [C.POINTER(VitDims), C.POINTER(VitWeights), _P, _I, _I, _P,
+                                    C.c_size_t, _P]),
+    "mmh3_device_status": (_I, [_P, C.POINTER(_I), C.POINTER(_I)]),
+    "mmh3_set_wait_limit_ns": (None, [C.c_uint64]),
+    "mmh3_selftest_wait_timeout": (_I, [C.c_uint64, _P]),
+    "mmh3_last_error": (C.c_char_p, []),
+    "mmh3_version": (C.c_char_p, []),
+}
+
+_lib = None
+
+
+def load() -> C.CDLL:
+    """Load libmmh3.so (built by ``build.py``); raise if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m packed_multimodal_diffusion_b200.build` (no fallback exists)")
+    lib = C.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def check(code: int) -> None:
+    if code != 0:
+        msg = load().mmh3_last_error().decode(errors="replace")
+        raise Mmh3Error(code, msg)

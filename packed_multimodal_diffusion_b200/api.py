@@ -1,0 +1,267 @@
+"""Python binding of the C ABI for torch tensors (marshalling only: every step
+of the path runs in libmmh3.so's kernels on the caller's current CUDA
+stream).  Device tensors must be contiguous CUDA tensors; PyTorch provides
+device memory and streams, nothing else."""
+
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import (MMH3_BF16, MMH3_F32, BlockWeights, Dims, HeadWeights, Segment, VitDims,
+                   VitWeights, check, load)
+
+__all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_image",
+           "plan_timesteps", "time_shift_sigma", "resolve_rows", "adaln_modulation",
+           "prepare_fc1", "workspace_size", "attention", "BlockParams", "HeadParams",
+           "block_forward", "stack_forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
+           "vit_layer_forward", "device_status", "selftest_wait_timeout", "set_wait_limit_ns",
+           "MMH3_BF16", "MMH3_F32"]
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return t.data_ptr()
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return MMH3_BF16
+    if dt == torch.float32:
+        return MMH3_F32
+    raise ValueError(f"unsupported activation dtype {dt}")
+
+
+def make_dims(hidden, heads, head_dim, ffn, act_dtype=torch.bfloat16, rank=24, grid=1025,
+              eps=1e-5, qk_eps=1e-5, rope_theta=10000.0) -> Dims:
+    return Dims(hidden, heads, head_dim, ffn, rank, grid, head_dim // 8, eps, qk_eps, rope_theta,
+                _dtype_code(act_dtype))
+
+
+def segments(segs) -> C.Array:
+    """(start, stop, tag, clock) tuples -> a ctypes array of mmh3_segment."""
+    arr = (Segment * len(segs))()
+    for i, (a, b, tag, clock) in enumerate(segs):
+        arr[i].start, arr[i].stop, arr[i].tag, arr[i].clock = a, b, tag, clock
+    return arr
+
+
+def _seg_tuples(arr, n) -> list[tuple]:
+    return [(arr[i].start, arr[i].stop, arr[i].tag, arr[i].clock) for i in range(n)]
+
+
+def time_shift_sigma(sigma: float, from_shift: float, to_shift: float) -> float:
+    return load().mmh3_time_shift_sigma(sigma, from_shift, to_shift)
+
+
+def _layout(fn, *args):
+    segs = (Segment * 8)()
+    nseg, n = C.c_int(), C.c_int()
+    check(fn(*args, segs, C.byref(nseg), None, 0, C.byref(n)))
+    pos = np.zeros((n.value, 3), dtype=np.float32)
+    check(fn(*args, segs, C.byref(nseg), pos.ctypes.data_as(C.POINTER(C.c_float)), n.value,
+             C.byref(n)))
+    return _seg_tuples(segs, nseg.value), pos
+
+
+def layout_t2va(text_len, latent_t, lat_h, lat_w, audio_t):
+    """-> (segments [(start, stop, tag, clock)], pos float32 [n, 3])."""
+    return _layout(load().mmh3_layout_t2va, text_len, latent_t, lat_h, lat_w, audio_t)
+
+
+def layout_image(text_len, ref_lat_h, ref_lat_w, lat_h, lat_w):
+    return _layout(load().mmh3_layout_image, text_len, ref_lat_h, ref_lat_w, lat_h, lat_w)
+
+
+def plan_timesteps(segs, n, sigma_v, sigma_a):
+    arr = segments(segs)
+    ts = (C.c_double * 2)()
+    nts = C.c_int()
+    rows = (C.c_int * len(segs))()
+    check(load().mmh3_plan_timesteps(arr, len(segs), n, sigma_v, sigma_a, ts, C.byref(nts), rows))
+    return list(ts)[: nts.value], list(rows)
+
+
+def resolve_rows(segs, n, sigma_v, sigma_a, rows_out: torch.Tensor) -> None:
+    check(load().mmh3_resolve_rows(segments(segs), len(segs), n, sigma_v, sigma_a,
+                                   _ptr(rows_out), _stream()))
+
+
+def adaln_modulation(dims: Dims, w, b, table, rows_per_slot, segs, n, sigma_v, sigma_a,
+                     out: torch.Tensor) -> int:
+    nts = C.c_int()
+    check(load().mmh3_adaln_modulation(C.byref(dims), _ptr(w), _ptr(b), _ptr(table), rows_per_slot,
+                                       segments(segs), len(segs), n, sigma_v, sigma_a, _ptr(out),
+                                       C.byref(nts), _stream()))
+    return nts.value
+
+
+def prepare_fc1(dims: Dims, fc1_gate_up: torch.Tensor, out: torch.Tensor) -> None:
+    check(load().mmh3_prepare_fc1(C.byref(dims), _ptr(fc1_gate_up), _ptr(out), _stream()))
+
+
+def workspace_size(dims: Dims, n: int) -> int:
+    v = C.c_size_t()
+    check(load().mmh3_workspace_size(C.byref(dims), n, C.byref(v)))
+    return v.value
+
+
+def attention(qkv: torch.Tensor, n_seq: int, seq: int, heads: int, head_dim: int, scale: float,
+              out: torch.Tensor) -> None:
+    check(load().mmh3_attention(_ptr(qkv), n_seq, seq, heads, head_dim, _dtype_code(qkv.dtype),
+                                scale, _ptr(out), _stream()))
+
+
+@dataclass
+class BlockParams:
+    """Device tensors of one block (fc1 already in the fused kernel's tile
+    order, see prepare_fc1) and the matching C struct."""
+    tensors: dict
+
+    def struct(self) -> BlockWeights:
+        t = self.tensors
+        return BlockWeights(*[_ptr(t.get(k)) for k in ("norm1", "norm2", "wqkv", "wout", "q_norm",
+                                                        "k_norm", "wfc1_tiled", "wfc2", "adaln_w",
+                                                        "adaln_b", "adaln_table")])
+
+    @staticmethod
+    def from_host(dims: Dims, w: dict, device="cuda") -> "BlockParams":
+        """Copy a host weight dict (natural layouts) to the device and tile
+        fc1 for the fused SwiGLU kernel."""
+        t = {k: v.to(device).contiguous() for k, v in w.items() if k != "wfc1"}
+        fc1 = w["wfc1"].to(device).contiguous()
+        t["wfc1_tiled"] = torch.empty_like(fc1)
+        prepare_fc1(dims, fc1, t["wfc1_tiled"])
+        return BlockParams(t)
+
+
+@dataclass
+class HeadParams:
+    tensors: dict
+
+    def struct(self) -> HeadWeights:
+        t = self.tensors
+        return HeadWeights(*[_ptr(t.get(k)) for k in ("final_norm", "adaln_w", "adaln_b",
+                                                       "adaln_table", "w_video", "b_video",
+                                                       "w_audio", "b_audio")],
+                           t["w_video"].shape[0], t["w_audio"].shape[0])
+
+    @staticmethod
+    def from_host(w: dict, device="cuda") -> "HeadParams":
+        return HeadParams({k: v.to(device).contiguous() for k, v in w.items()})
+
+
+def block_forward(dims: Dims, params: BlockParams, x: torch.Tensor, segs, pos: torch.Tensor | None,
+                  sigma_v: float, sigma_a: float, workspace: torch.Tensor,
+                  modulated: bool = True) -> None:
+    """In place on x [n, H] fp32."""
+    st = params.struct()
+    check(load().mmh3_block_forward(C.byref(dims), C.byref(st), _ptr(x), x.shape[0],
+                                    segments(segs), len(segs), _ptr(pos), sigma_v, sigma_a,
+                                    1 if modulated else 0, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream()))
+
+
+def stack_forward(dims: Dims, blocks: list, heads: HeadParams | None, x: torch.Tensor, segs,
+                  pos, sigma_v, sigma_a, out_video, out_audio, workspace) -> None:
+    arr = (BlockWeights * max(1, len(blocks)))(*[b.struct() for b in blocks])
+    hs = heads.struct() if heads is not None else None
+    check(load().mmh3_stack_forward(C.byref(dims), arr, len(blocks),
+                                    C.byref(hs) if hs is not None else None, _ptr(x), x.shape[0],
+                                    segments(segs), len(segs), _ptr(pos), sigma_v, sigma_a,
+                                    _ptr(out_video), _ptr(out_audio), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream()))
+
+
+# -------------------------------------------------------------- encoder layer
+def vit_dims(hidden, heads, head_dim, mlp, ln_eps=1e-6) -> VitDims:
+    return VitDims(hidden, heads, head_dim, mlp, ln_eps)
+
+
+@dataclass
+class VitParams:
+    tensors: dict
+
+    def struct(self) -> VitWeights:
+        t = self.tensors
+        return VitWeights(*[_ptr(t[k]) for k in ("ln1_g", "ln1_b", "wqkv", "bqkv", "wo", "bo",
+                                                  "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")])
+
+    @staticmethod
+    def from_host(dims: VitDims, w: dict, device="cuda") -> "VitParams":
+        t = {k: v.to(device).contiguous() for k, v in w.items()}
+        H = dims.hidden
+        t["wqkv"] = torch.empty((3 * H, H), dtype=torch.bfloat16, device=device)
+        t["bqkv"] = torch.empty((3 * H,), dtype=torch.float32, device=device)
+        vit_fold_qkv(dims, t["wq"], t["wk"], t["wv"], t["bq"], t["bk"], t["bv"], t["wqkv"],
+                     t["bqkv"])
+        return VitParams(t)
+
+
+def vit_fold_qkv(dims: VitDims, wq, wk, wv, bq, bk, bv, wqkv, bqkv) -> None:
+    check(load().mmh3_vit_fold_qkv(C.byref(dims), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(bq), _ptr(bk),
+                                   _ptr(bv), _ptr(wqkv), _ptr(bqkv), _stream()))
+
+
+def vit_workspace_size(dims: VitDims, batch: int, seq: int) -> int:
+    v = C.c_size_t()
+    check(load().mmh3_vit_workspace_size(C.byref(dims), batch, seq, C.byref(v)))
+    return v.value
+
+
+def vit_layer_forward(dims: VitDims, params: VitParams, x: torch.Tensor, batch: int, seq: int,
+                      workspace: torch.Tensor) -> None:
+    st = params.struct()
+    check(load().mmh3_vit_layer_forward(C.byref(dims), C.byref(st), _ptr(x), batch, seq,
+                                        _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream()))
+
+
+# ---------------------------------------------------------------- diagnostics
+def device_status() -> tuple[int, int]:
+    """Synchronise the current stream; return (code, site) of a recorded
+    bounded-wait timeout, raising Mmh3Error(MMH3_ERR_TIMEOUT) if one was."""
+    code, site = C.c_int(), C.c_int()
+    check(load().mmh3_device_status(_stream(), C.byref(code), C.byref(site)))
+    return code.value, site.value
+
+
+def selftest_wait_timeout(limit_ns: int) -> int:
+    """Run the bounded-wait self test; returns the status code (7 expected)."""
+    return load().mmh3_selftest_wait_timeout(limit_ns, _stream())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    load().mmh3_set_wait_limit_ns(ns)
+
+
+def workspace_regions(dims: Dims, n: int, ws: torch.Tensor) -> dict:
+    """Views of the workspace regions (layout of mmh3_workspace_size) for
+    inspecting a block's intermediates."""
+    H, I, F = dims.hidden, dims.heads * dims.head_dim, dims.ffn
+    act = torch.bfloat16 if dims.act_dtype == MMH3_BF16 else torch.float32
+    es = 2 if dims.act_dtype == MMH3_BF16 else 4
+    a256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    sizes = [("mods", 2 * 3 * 6 * H * 4, torch.float32, (6, 6 * H)),
+             ("cs", n * 3 * dims.rope_k * 8, torch.float32, (n, 3 * dims.rope_k, 2)),
+             ("xn1", n * H * es, act, (n, H)), ("qkv", n * 3 * I * es, act, (n, 3 * I)),
+             ("attn", n * I * es, act, (n, I)), ("xn2", n * H * es, act, (n, H)),
+             ("act", n * F * es, act, (n, F)), ("head", n * H * es, act, (n, H)),
+             ("fmods", 2 * 2 * H * 4, torch.float32, (2, 2 * H))]
+    out, off = {}, 0
+    raw = ws.view(torch.uint8)
+    for name, nbytes, dt, shape in sizes:
+        out[name] = raw[off:off + nbytes].view(dt).view(shape)
+        off += a256(nbytes)
+    return out

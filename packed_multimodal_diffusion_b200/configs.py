@@ -128,28 +128,31 @@ _X_INDEX = 990
 _VIT_BASE = 800
 
 
-def block_weights(cfg: DitConfig, b: int, device="cpu", wdtype=None) -> dict:
+def block_weights(cfg: DitConfig, b: int, device="cpu", wdtype=None, keys=None) -> dict:
     """Synthetic weights of block ``b`` (natural layouts: qkv rows [q|k|v],
     fc1 rows [gate|up]).  Projections in ``wdtype`` (default: the config's
-    activation dtype), everything else fp32."""
+    activation dtype), everything else fp32.  ``keys`` limits the output to
+    those tensors (each has its own stream, so a subset is identical to the
+    same entries of the full set)."""
     wdtype = cfg.act_dtype if wdtype is None else wdtype
     H, I, F, R = cfg.hidden, cfg.inner, cfg.ffn, cfg.rank
     base = b * _BLOCK_STRIDE
     s = lambda j: synth.tensor_seed(cfg.cfg_seed, base + j)  # noqa: E731
     n = synth.normal
-    return {
-        "norm1": n((H,), s(0), 0.02, 1.0, device=device),
-        "norm2": n((H,), s(1), 0.02, 1.0, device=device),
-        "wqkv": n((3 * I, H), s(2), 0.02, dtype=wdtype, device=device),
-        "wout": n((H, I), s(3), 0.02, dtype=wdtype, device=device),
-        "q_norm": n((cfg.head_dim,), s(4), 0.02, 1.0, device=device),
-        "k_norm": n((cfg.head_dim,), s(5), 0.02, 1.0, device=device),
-        "wfc1": n((2 * F, H), s(6), 0.02, dtype=wdtype, device=device),
-        "wfc2": n((H, F), s(7), 0.02, dtype=wdtype, device=device),
-        "adaln_w": n((cfg.n_slots * 3 * 6 * H, R), s(8), 0.02, device=device),
-        "adaln_b": n((cfg.n_slots * 3 * 6 * H,), s(9), 0.02, device=device),
-        "adaln_table": n((cfg.grid, R), s(10), 1.0, device=device),
+    make = {
+        "norm1": lambda: n((H,), s(0), 0.02, 1.0, device=device),
+        "norm2": lambda: n((H,), s(1), 0.02, 1.0, device=device),
+        "wqkv": lambda: n((3 * I, H), s(2), 0.02, dtype=wdtype, device=device),
+        "wout": lambda: n((H, I), s(3), 0.02, dtype=wdtype, device=device),
+        "q_norm": lambda: n((cfg.head_dim,), s(4), 0.02, 1.0, device=device),
+        "k_norm": lambda: n((cfg.head_dim,), s(5), 0.02, 1.0, device=device),
+        "wfc1": lambda: n((2 * F, H), s(6), 0.02, dtype=wdtype, device=device),
+        "wfc2": lambda: n((H, F), s(7), 0.02, dtype=wdtype, device=device),
+        "adaln_w": lambda: n((cfg.n_slots * 3 * 6 * H, R), s(8), 0.02, device=device),
+        "adaln_b": lambda: n((cfg.n_slots * 3 * 6 * H,), s(9), 0.02, device=device),
+        "adaln_table": lambda: n((cfg.grid, R), s(10), 1.0, device=device),
     }
+    return {k: f() for k, f in make.items() if keys is None or k in keys}
 
 
 def head_weights(cfg: DitConfig, device="cpu", wdtype=None) -> dict:

@@ -1,0 +1,376 @@
+// The C ABI entry points that run the hot path: adaLN modulation, the
+// modulated block, the 50-block stack with its output heads, and the SigLIP
+// encoder layer.  Each entry point validates everything before the first
+// launch and then enqueues a fixed sequence of kernels on the caller's
+// stream (no host synchronisation, no allocation).
+//
+// Step order follows "cortiq_engine/mmh3.rs" (cortiq-engine 0.5.72):
+// MiniMaxH3::forward ("blocks", "heads"), block_forward and ffn_tail;
+// the encoder layer follows "ffai-argus 0.7.0 src/siglip.rs",
+// Layer::forward and finish_attention.
+#include <cmath>
+#include <cstring>
+
+#include "mmh3_internal.h"
+
+using namespace mmh3;
+
+namespace {
+
+struct Workspace {
+  float* mods;
+  float2* cs;
+  void* xn1;
+  void* qkv;
+  void* attn;
+  void* xn2;
+  void* act;
+  void* head;
+  float* fmods;
+  size_t bytes;
+};
+
+Workspace carve(const mmh3_dims& d, int n, void* base) {
+  const size_t es = (size_t)esize_of(d.act_dtype);
+  const size_t H = (size_t)d.hidden, I = (size_t)d.heads * d.head_dim, F = (size_t)d.ffn;
+  const size_t N = (size_t)n;
+  Workspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = static_cast<uint8_t*>(base) + off;
+    off += align256(bytes);
+    return base ? static_cast<void*>(p) : nullptr;
+  };
+  w.mods = static_cast<float*>(take(2 * 3 * 6 * H * 4));
+  w.cs = static_cast<float2*>(take(N * 3 * (size_t)d.rope_k * 8));
+  w.xn1 = take(N * H * es);
+  w.qkv = take(N * 3 * I * es);
+  w.attn = take(N * I * es);
+  w.xn2 = take(N * H * es);
+  w.act = take(N * F * es);
+  w.head = take(N * H * es);
+  w.fmods = static_cast<float*>(take(2 * 2 * H * 4));
+  w.bytes = off;
+  return w;
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; }
+
+mmh3_status check_dims(const mmh3_dims* d) {
+  if (d == nullptr) return fail(MMH3_ERR_ARG, "dims is null");
+  if (d->act_dtype != MMH3_BF16 && d->act_dtype != MMH3_F32) return fail(MMH3_ERR_ARG, "act_dtype %d", d->act_dtype);
+  if (d->hidden <= 0 || d->hidden % 128 != 0 || d->hidden > 4096)
+    return fail(MMH3_ERR_SHAPE, "hidden %d must be a positive multiple of 128 (<= 4096)", d->hidden);
+  if (d->head_dim != 64 && d->head_dim != 128) return fail(MMH3_ERR_SHAPE, "head_dim %d not in {64, 128}", d->head_dim);
+  if (d->act_dtype == MMH3_F32 && d->head_dim != 64)
+    return fail(MMH3_ERR_UNSUPPORTED, "fp32 activations support head_dim 64 only");
+  if (d->heads <= 0 || d->heads > 256)
+    return fail(MMH3_ERR_SHAPE, "heads = %d not in [1, 256]", d->heads);
+  if (d->ffn <= 0 || d->ffn % 128 != 0) return fail(MMH3_ERR_SHAPE, "ffn %d must be a multiple of 128", d->ffn);
+  if (d->rank < 1 || d->rank > 32) return fail(MMH3_ERR_SHAPE, "rank %d not in [1, 32]", d->rank);
+  if (d->grid < 2) return fail(MMH3_ERR_SHAPE, "grid %d < 2", d->grid);
+  if (d->rope_k != d->head_dim / 8) return fail(MMH3_ERR_SHAPE, "rope_k %d != head_dim/8", d->rope_k);
+  if (!(d->eps > 0) || !(d->qk_eps > 0)) return fail(MMH3_ERR_ARG, "eps must be positive");
+  return MMH3_OK;
+}
+
+mmh3_status check_block(const mmh3_dims& d, const mmh3_block_weights* w, bool modulated) {
+  if (w == nullptr) return fail(MMH3_ERR_ARG, "block weights are null");
+  const void* req[] = {w->norm1, w->norm2, w->wqkv, w->wout, w->q_norm, w->k_norm, w->wfc1, w->wfc2};
+  for (const void* p : req) {
+    if (p == nullptr) return fail(MMH3_ERR_ARG, "a block weight pointer is null");
+    if (misaligned(p)) return fail(MMH3_ERR_ALIGN, "a block weight pointer is not 16-byte aligned");
+  }
+  if (modulated) {
+    const void* ad[] = {w->adaln_w, w->adaln_b, w->adaln_table};
+    for (const void* p : ad) {
+      if (p == nullptr) return fail(MMH3_ERR_ARG, "adaLN pointer is null in a modulated block");
+      if (misaligned(p)) return fail(MMH3_ERR_ALIGN, "adaLN pointer is not 16-byte aligned");
+    }
+  }
+  (void)d;
+  return MMH3_OK;
+}
+
+// norm1-modulate -> qkv+qknorm+rope -> attention -> out+gated residual ->
+// norm2-modulate -> fc1+SwiGLU -> fc2+gated residual
+mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x, int n,
+                       const Plan& plan, const float* mods, const float2* cs, const Workspace& ws,
+                       cudaStream_t s) {
+  const int H = d.hidden, I = d.heads * d.head_dim, F = d.ffn;
+  const int dt = d.act_dtype;
+  const int stride = 6 * H;
+  cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm1, d.eps, mods, stride, 0 * H, 1 * H, plan.block_rows, 0,
+                                  ws.xn1, s);
+  if (e != cudaSuccess) return cuda_fail(e, "norm1/modulate launch");
+  mmh3_status st = gemm_qkv(dt, ws.xn1, w.wqkv, n, 3 * I, H, d.head_dim, I, w.q_norm, w.k_norm, cs, d.qk_eps,
+                            ws.qkv, s);
+  if (st != MMH3_OK) return st;
+  st = attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, 1.0f / std::sqrt((float)d.head_dim), ws.attn, s);
+  if (st != MMH3_OK) return st;
+  st = gemm_gated_residual(dt, ws.attn, w.wout, n, H, I, x, mods, stride, 2 * H, plan.block_rows, s);
+  if (st != MMH3_OK) return st;
+  e = launch_norm_mod(dt, x, n, H, w.norm2, d.eps, mods, stride, 3 * H, 4 * H, plan.block_rows, 0, ws.xn2, s);
+  if (e != cudaSuccess) return cuda_fail(e, "norm2/modulate launch");
+  st = gemm_swiglu(dt, ws.xn2, w.wfc1, n, F, H, ws.act, s);
+  if (st != MMH3_OK) return st;
+  return gemm_gated_residual(dt, ws.act, w.wfc2, n, H, F, x, mods, stride, 5 * H, plan.block_rows, s);
+}
+
+mmh3_status common_checks(const mmh3_dims* dims, float* x, int n, const float* pos, void* ws,
+                          size_t ws_bytes, Workspace* out_ws) {
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (x == nullptr) return fail(MMH3_ERR_ARG, "x is null");
+  if (misaligned(x) || (pos && misaligned(pos)) || misaligned(ws))
+    return fail(MMH3_ERR_ALIGN, "x / pos / workspace must be 16-byte aligned");
+  if (n < 1) return fail(MMH3_ERR_SHAPE, "n = %d < 1", n);
+  if (fault_injected("workspace")) return fail(MMH3_ERR_WORKSPACE, "injected fault at workspace");
+  const Workspace need = carve(*dims, n, nullptr);
+  if (ws == nullptr || ws_bytes < need.bytes)
+    return fail(MMH3_ERR_WORKSPACE, "workspace %zu bytes < %zu required", ws_bytes, need.bytes);
+  *out_ws = carve(*dims, n, ws);
+  return MMH3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mmh3_status mmh3_workspace_size(const mmh3_dims* dims, int n, size_t* bytes) {
+  clear_error();
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (bytes == nullptr) return fail(MMH3_ERR_ARG, "bytes is null");
+  if (n < 0) return fail(MMH3_ERR_SHAPE, "n < 0");
+  *bytes = carve(*dims, n, nullptr).bytes;
+  return MMH3_OK;
+}
+
+mmh3_status mmh3_resolve_rows(const mmh3_segment* segs, int n_seg, int n, double sigma_v, double sigma_a,
+                              int32_t* rows_dev, void* stream) {
+  clear_error();
+  if (rows_dev == nullptr) return fail(MMH3_ERR_ARG, "rows is null");
+  Plan plan;
+  mmh3_status st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+  if (st != MMH3_OK) return st;
+  cudaError_t e = launch_rows(plan.block_rows, n, rows_dev, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "rows launch");
+}
+
+mmh3_status mmh3_adaln_modulation(const mmh3_dims* dims, const float* w, const float* b, const float* table,
+                                  int rows_per_slot, const mmh3_segment* segs, int n_seg, int n,
+                                  double sigma_v, double sigma_a, float* out, int* n_ts, void* stream) {
+  clear_error();
+  if (dims == nullptr || w == nullptr || b == nullptr || table == nullptr || out == nullptr)
+    return fail(MMH3_ERR_ARG, "adaln: null pointer");
+  if (dims->rank < 1 || dims->rank > 32 || dims->grid < 2) return fail(MMH3_ERR_SHAPE, "adaln: rank/grid");
+  if (rows_per_slot < 1) return fail(MMH3_ERR_SHAPE, "adaln: rows_per_slot %d", rows_per_slot);
+  if (misaligned(w)) return fail(MMH3_ERR_ALIGN, "adaln: basis not 16-byte aligned");
+  Plan plan;
+  mmh3_status st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+  if (st != MMH3_OK) return st;
+  if (n_ts) *n_ts = plan.n_ts;
+  cudaError_t e = launch_adaln(w, b, table, dims->rank, dims->grid, rows_per_slot, plan, out,
+                               static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "adaln launch");
+}
+
+mmh3_status mmh3_prepare_fc1(const mmh3_dims* dims, const void* fc1_gate_up, void* fc1_tiled, void* stream) {
+  clear_error();
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (fc1_gate_up == nullptr || fc1_tiled == nullptr || fc1_gate_up == fc1_tiled)
+    return fail(MMH3_ERR_ARG, "prepare_fc1: null or aliased pointers");
+  if (misaligned(fc1_gate_up) || misaligned(fc1_tiled)) return fail(MMH3_ERR_ALIGN, "prepare_fc1: alignment");
+  cudaError_t e = launch_fc1_tile(esize_of(dims->act_dtype), fc1_gate_up, fc1_tiled, dims->ffn, dims->hidden,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "prepare_fc1 launch");
+}
+
+mmh3_status mmh3_block_forward(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
+                               const mmh3_segment* segs, int n_seg, const float* pos_dev, double sigma_v,
+                               double sigma_a, int modulated, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  clear_error();
+  Workspace ws;
+  mmh3_status st = common_checks(dims, x, n, pos_dev, workspace, ws_bytes, &ws);
+  if (st != MMH3_OK) return st;
+  st = check_block(*dims, w, modulated != 0);
+  if (st != MMH3_OK) return st;
+  Plan plan;
+  if (modulated) {
+    st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+    if (st != MMH3_OK) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = dims->hidden;
+  if (modulated) {
+    cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * H, plan,
+                                 ws.mods, s);
+    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
+  }
+  if (pos_dev) {
+    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  }
+  return block_core(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s);
+}
+
+mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* blocks, int n_blocks,
+                               const mmh3_head_weights* heads, float* x, int n, const mmh3_segment* segs,
+                               int n_seg, const float* pos_dev, double sigma_v, double sigma_a,
+                               float* out_video, float* out_audio, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  clear_error();
+  Workspace ws;
+  mmh3_status st = common_checks(dims, x, n, pos_dev, workspace, ws_bytes, &ws);
+  if (st != MMH3_OK) return st;
+  if (n_blocks < 0 || (n_blocks > 0 && blocks == nullptr)) return fail(MMH3_ERR_ARG, "blocks");
+  for (int i = 0; i < n_blocks; ++i) {
+    st = check_block(*dims, blocks + i, true);
+    if (st != MMH3_OK) return st;
+  }
+  Plan plan;
+  st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+  if (st != MMH3_OK) return st;
+  const int H = dims->hidden;
+  // output streams: the last video-tag segment and the last audio-tag segment
+  int vseg = -1, aseg = -1;
+  for (int k = 0; k < n_seg; ++k) {
+    if (segs[k].tag == 0) vseg = k;
+    if (segs[k].tag == 2) aseg = k;
+  }
+  if (heads) {
+    if (heads->final_norm == nullptr || heads->adaln_w == nullptr || heads->adaln_b == nullptr ||
+        heads->adaln_table == nullptr)
+      return fail(MMH3_ERR_ARG, "head weights: null pointer");
+    if (vseg >= 0 && (heads->w_video == nullptr || heads->b_video == nullptr || out_video == nullptr ||
+                      heads->out_video <= 0 || heads->out_video % 32 != 0))
+      return fail(MMH3_ERR_ARG, "video head: missing pointer or out_video %d not a positive multiple of 32",
+                  heads->out_video);
+    if (aseg >= 0 && (heads->w_audio == nullptr || heads->b_audio == nullptr || out_audio == nullptr ||
+                      heads->out_audio <= 0 || heads->out_audio % 32 != 0))
+      return fail(MMH3_ERR_ARG, "audio head: missing pointer or out_audio %d not a positive multiple of 32",
+                  heads->out_audio);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pos_dev) {
+    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  }
+  for (int i = 0; i < n_blocks; ++i) {
+    const mmh3_block_weights& w = blocks[i];
+    cudaError_t e = launch_adaln(w.adaln_w, w.adaln_b, w.adaln_table, dims->rank, dims->grid, 18 * H, plan,
+                                 ws.mods, s);
+    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
+    st = block_core(*dims, w, x, n, plan, ws.mods, pos_dev ? ws.cs : nullptr, ws, s);
+    if (st != MMH3_OK) return st;
+  }
+  if (heads == nullptr) return MMH3_OK;
+  cudaError_t e = launch_adaln(heads->adaln_w, heads->adaln_b, heads->adaln_table, dims->rank, dims->grid, 2 * H,
+                               plan, ws.fmods, s);
+  if (e != cudaSuccess) return cuda_fail(e, "final adaln launch");
+  const int sidx[2] = {vseg, aseg};
+  for (int k = 0; k < 2; ++k) {
+    if (sidx[k] < 0) continue;
+    const mmh3_segment& sg = segs[sidx[k]];
+    const int rows = (int)(sg.stop - sg.start);
+    e = launch_norm_mod(dims->act_dtype, x + (size_t)sg.start * H, rows, H, heads->final_norm, dims->eps,
+                        ws.fmods, 2 * H, 0, H, plan.final_rows, (int)sg.start, ws.head, s);
+    if (e != cudaSuccess) return cuda_fail(e, "final norm launch");
+    st = gemm_bias_act(dims->act_dtype, ws.head, k == 0 ? heads->w_video : heads->w_audio, rows,
+                       k == 0 ? heads->out_video : heads->out_audio, H, k == 0 ? heads->b_video : heads->b_audio, 2,
+                       k == 0 ? (void*)out_video : (void*)out_audio, s);
+    if (st != MMH3_OK) return st;
+  }
+  return MMH3_OK;
+}
+
+// ----------------------------------------------------------- encoder layer
+static mmh3_status check_vit(const mmh3_vit_dims* d) {
+  if (d == nullptr) return fail(MMH3_ERR_ARG, "vit dims null");
+  if (d->hidden <= 0 || d->hidden % 256 != 0 || d->hidden > 4096)
+    return fail(MMH3_ERR_SHAPE, "vit hidden %d must be a multiple of 256", d->hidden);
+  if (d->head_dim != 64 && d->head_dim != 128) return fail(MMH3_ERR_SHAPE, "vit head_dim %d", d->head_dim);
+  if (d->heads * d->head_dim != d->hidden) return fail(MMH3_ERR_SHAPE, "vit heads*head_dim != hidden");
+  if (d->mlp <= 0 || d->mlp % 256 != 0) return fail(MMH3_ERR_SHAPE, "vit mlp %d must be a multiple of 256", d->mlp);
+  if (!(d->ln_eps > 0)) return fail(MMH3_ERR_ARG, "vit ln_eps");
+  return MMH3_OK;
+}
+
+static size_t vit_carve(const mmh3_vit_dims& d, size_t rows, void* base, void** h, void** qkv, void** attn,
+                        void** act) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    void* p = base ? static_cast<void*>(static_cast<uint8_t*>(base) + off) : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  *h = take(rows * d.hidden * 2);
+  *qkv = take(rows * 3 * d.hidden * 2);
+  *attn = take(rows * d.hidden * 2);
+  *act = take(rows * d.mlp * 2);
+  return off;
+}
+
+mmh3_status mmh3_vit_workspace_size(const mmh3_vit_dims* dims, int batch, int seq, size_t* bytes) {
+  clear_error();
+  mmh3_status st = check_vit(dims);
+  if (st != MMH3_OK) return st;
+  if (bytes == nullptr || batch < 0 || seq < 0) return fail(MMH3_ERR_ARG, "vit workspace args");
+  void *a, *b, *c, *e;
+  *bytes = vit_carve(*dims, (size_t)batch * seq, nullptr, &a, &b, &c, &e);
+  return MMH3_OK;
+}
+
+mmh3_status mmh3_vit_fold_qkv(const mmh3_vit_dims* dims, const void* wq, const void* wk, const void* wv,
+                              const float* bq, const float* bk, const float* bv, void* wqkv, float* bqkv,
+                              void* stream) {
+  clear_error();
+  mmh3_status st = check_vit(dims);
+  if (st != MMH3_OK) return st;
+  if (!wq || !wk || !wv || !bq || !bk || !bv || !wqkv || !bqkv) return fail(MMH3_ERR_ARG, "vit fold: null");
+  const float scale = 1.0f / std::sqrt((float)dims->head_dim);
+  cudaError_t e = launch_vit_fold(wq, wk, wv, bq, bk, bv, scale, dims->hidden, wqkv, bqkv,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "vit fold launch");
+}
+
+mmh3_status mmh3_vit_layer_forward(const mmh3_vit_dims* dims, const mmh3_vit_weights* w, float* x, int batch,
+                                   int seq, void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  mmh3_status st = check_vit(dims);
+  if (st != MMH3_OK) return st;
+  if (w == nullptr || x == nullptr) return fail(MMH3_ERR_ARG, "vit: null pointer");
+  const void* req[] = {w->ln1_g, w->ln1_b, w->wqkv, w->bqkv, w->wo, w->bo, w->ln2_g, w->ln2_b, w->w1, w->b1, w->w2, w->b2};
+  for (const void* p : req) {
+    if (p == nullptr) return fail(MMH3_ERR_ARG, "vit: null weight pointer");
+    if (misaligned(p)) return fail(MMH3_ERR_ALIGN, "vit: weight pointer not 16-byte aligned");
+  }
+  if (batch < 1 || seq < 1) return fail(MMH3_ERR_SHAPE, "vit: batch %d seq %d", batch, seq);
+  if (misaligned(x) || misaligned(workspace)) return fail(MMH3_ERR_ALIGN, "vit: x / workspace alignment");
+  void *h, *qkv, *attn, *act;
+  const size_t rows = (size_t)batch * seq;
+  const size_t need = vit_carve(*dims, rows, nullptr, &h, &qkv, &attn, &act);
+  if (workspace == nullptr || ws_bytes < need)
+    return fail(MMH3_ERR_WORKSPACE, "vit workspace %zu < %zu", ws_bytes, need);
+  vit_carve(*dims, rows, workspace, &h, &qkv, &attn, &act);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = dims->hidden, M = (int)rows;
+  cudaError_t e = launch_layernorm(x, M, H, w->ln1_g, w->ln1_b, dims->ln_eps, static_cast<__nv_bfloat16*>(h), s);
+  if (e != cudaSuccess) return cuda_fail(e, "ln1 launch");
+  st = gemm_bias_act(MMH3_BF16, h, w->wqkv, M, 3 * H, H, w->bqkv, 0, qkv, s);
+  if (st != MMH3_OK) return st;
+  st = attention(MMH3_BF16, qkv, batch, seq, dims->heads, dims->head_dim, 1.0f, attn, s);
+  if (st != MMH3_OK) return st;
+  st = gemm_bias_residual(MMH3_BF16, attn, w->wo, M, H, H, w->bo, x, s);
+  if (st != MMH3_OK) return st;
+  e = launch_layernorm(x, M, H, w->ln2_g, w->ln2_b, dims->ln_eps, static_cast<__nv_bfloat16*>(h), s);
+  if (e != cudaSuccess) return cuda_fail(e, "ln2 launch");
+  st = gemm_bias_act(MMH3_BF16, h, w->w1, M, dims->mlp, H, w->b1, 1, act, s);
+  if (st != MMH3_OK) return st;
+  return gemm_bias_residual(MMH3_BF16, act, w->w2, M, H, dims->mlp, w->b2, x, s);
+}
+
+}  // extern "C"

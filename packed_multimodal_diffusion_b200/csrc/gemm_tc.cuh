@@ -1,0 +1,455 @@
+// Persistent, warp-specialised tcgen05 GEMM  C[M, N] = A[M, K] * B[N, K]^T
+// with the block's epilogues fused in.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A and B tiles into a STAGES-deep smem ring
+//   warp 1      MMA issuer: tcgen05.mma into one of two TMEM accumulators
+//   warps 2..5  epilogue: tcgen05.ld the accumulator rows, apply the fused
+//               epilogue, store; the second TMEM buffer lets the next tile's
+//               MMAs run under this tile's epilogue.
+// Tiles are 128 x BN x (128 bytes of K); operands are bf16 (kind::f16) or
+// fp32 read as tf32 (kind::tf32).  Every wait is bounded (mbar_wait) and a
+// timeout leaves the loops, drains in-flight copies and frees TMEM.
+#pragma once
+
+#include "mmh3_device.cuh"
+
+namespace mmh3 {
+
+template <typename T>
+struct ElemTraits;
+template <>
+struct ElemTraits<__nv_bfloat16> {
+  static constexpr bool kTf32 = false;
+  static constexpr int kBytes = 2;
+};
+template <>
+struct ElemTraits<float> {
+  static constexpr bool kTf32 = true;
+  static constexpr int kBytes = 4;
+};
+
+// ---------------------------------------------------------- store helpers
+// Store 32 fp32 values to 32 consecutive elements of type T (16-byte aligned).
+__device__ __forceinline__ void store32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = u;
+  }
+}
+__device__ __forceinline__ void store32(float* dst, const float (&v)[32]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__device__ __forceinline__ void ld_acc32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  return 0.5f * x * (1.0f + tanhf(k0 * (x + 0.044715f * x * x * x)));
+}
+
+// ------------------------------------------------------------- epilogues
+// Each epilogue gets: the TMEM address of this thread's accumulator row
+// (column 0 of the tile), the output row index, the tile's first column,
+// and whether the row is inside the matrix.  It must issue every tcgen05.ld
+// even for rows outside the matrix (the loads are warp-collective).
+
+// qkv projection: per 128-column head of the q and k planes, RMSNorm with
+// the q_norm / k_norm weight, then the partial split-half 3-axis rotation
+// from a per-row (cos, sin) table; the v plane is stored as is.
+template <typename T, int HD, int BN>
+struct EpiQkvNormRope {
+  T* out;            // [M, N] with N = 3 * inner
+  int N;
+  int inner;         // heads * HD
+  const float* q_norm;
+  const float* k_norm;
+  const float2* cs;  // [M, kPairs] (cos, sin), or null: no rotation
+  float eps;
+  static constexpr int kPairs = 3 * (HD / 8);
+
+  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+#pragma unroll 1
+    for (int g = 0; g < BN / HD; ++g) {
+      const int col0 = n0 + g * HD;
+      if (col0 >= N) break;  // uniform across the warp
+      float v[HD];
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        float t[32];
+        ld_acc32(tacc + g * HD + c * 32, t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[c * 32 + i] = t[i];
+      }
+      const int which = col0 / inner;  // 0 q, 1 k, 2 v
+      if (which < 2) {
+        const float* w = which == 0 ? q_norm : k_norm;
+        float ss = 0.f;
+#pragma unroll
+        for (int d = 0; d < HD; ++d) ss = fmaf(v[d], v[d], ss);
+        const float inv = rsqrtf(ss * (1.0f / HD) + eps);
+#pragma unroll
+        for (int d = 0; d < HD; ++d) v[d] = v[d] * inv * __ldg(w + d);
+        if (cs != nullptr && row_ok) {
+          const float2* c2 = cs + (size_t)row * kPairs;
+#pragma unroll
+          for (int j = 0; j < kPairs; ++j) {
+            const float2 a = __ldg(c2 + j);
+            const float lo = v[j], hi = v[j + kPairs];
+            v[j] = lo * a.x - hi * a.y;
+            v[j + kPairs] = lo * a.y + hi * a.x;
+          }
+        }
+      }
+      if (row_ok) {
+        T* dst = out + (size_t)row * N + col0;
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          float t[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) t[i] = v[c * 32 + i];
+          store32(dst + c * 32, t);
+        }
+      }
+    }
+  }
+};
+
+// x[row, :] += gate[row] * acc : the gated residual.  gate is chunk `chunk`
+// of the token's modulation row (row id from the segment table).  With
+// mods == null the residual is plain (x += acc).
+template <int BN>
+struct EpiGatedResidual {
+  float* x;          // [M, N] fp32, in place
+  int N;
+  const float* mods; // [rows, mods_stride] or null
+  int mods_stride;
+  int chunk_off;     // chunk * hidden
+  SegRows seg;
+
+  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+    const float* gate = nullptr;
+    if (mods != nullptr) gate = mods + (size_t)seg_row(seg, row) * mods_stride + chunk_off;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col = n0 + c * 32;
+      if (col >= N) break;
+      float v[32];
+      ld_acc32(tacc + c * 32, v);
+      if (row_ok) {
+        float4* xp = reinterpret_cast<float4*>(x + (size_t)row * N + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 xv = xp[q];
+          float4 gv = gate ? __ldg(reinterpret_cast<const float4*>(gate + col) + q)
+                           : make_float4(1.f, 1.f, 1.f, 1.f);
+          xv.x = fmaf(gv.x, v[4 * q + 0], xv.x);
+          xv.y = fmaf(gv.y, v[4 * q + 1], xv.y);
+          xv.z = fmaf(gv.z, v[4 * q + 2], xv.z);
+          xv.w = fmaf(gv.w, v[4 * q + 3], xv.w);
+          xp[q] = xv;
+        }
+      }
+    }
+  }
+};
+
+// fc1 + SwiGLU: the weight rows are interleaved so that tile columns
+// [0, BN/2) are gate rows and [BN/2, BN) the matching up rows; the output
+// column block is n0 / 2.
+template <typename T, int BN>
+struct EpiSwiGLU {
+  T* out;  // [M, F]
+  int F;
+
+  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+    const int f0 = n0 / 2;
+#pragma unroll 1
+    for (int c = 0; c < BN / 64; ++c) {
+      const int f = f0 + c * 32;
+      if (f >= F) break;
+      float g[32], u[32];
+      ld_acc32(tacc + c * 32, g);
+      ld_acc32(tacc + BN / 2 + c * 32, u);
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+        store32(out + (size_t)row * F + f, g);
+      }
+    }
+  }
+};
+
+// out = act(acc + bias) for the unmodulated encoder layer and the output
+// heads.  MODE 0: identity, 1: tanh-GELU, 2: negate (velocity sign).
+template <typename T, int BN, int MODE>
+struct EpiBiasAct {
+  T* out;
+  int N;
+  const float* bias;
+
+  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col = n0 + c * 32;
+      if (col >= N) break;
+      float v[32];
+      ld_acc32(tacc + c * 32, v);
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float t = v[i] + __ldg(bias + col + i);
+          if (MODE == 1) t = gelu_tanh_f(t);
+          if (MODE == 2) t = -t;
+          v[i] = t;
+        }
+        store32(out + (size_t)row * N + col, v);
+      }
+    }
+  }
+};
+
+// x += acc + bias : residual with the projection's bias folded in.
+template <int BN>
+struct EpiBiasResidual {
+  float* x;
+  int N;
+  const float* bias;
+
+  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col = n0 + c * 32;
+      if (col >= N) break;
+      float v[32];
+      ld_acc32(tacc + c * 32, v);
+      if (row_ok) {
+        float4* xp = reinterpret_cast<float4*>(x + (size_t)row * N + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 xv = xp[q];
+          const float4 bv = __ldg(reinterpret_cast<const float4*>(bias + col) + q);
+          xv.x += v[4 * q + 0] + bv.x;
+          xv.y += v[4 * q + 1] + bv.y;
+          xv.z += v[4 * q + 2] + bv.z;
+          xv.w += v[4 * q + 3] + bv.w;
+          xp[q] = xv;
+        }
+      }
+    }
+  }
+};
+
+// ------------------------------------------------------------------ kernel
+template <int BN>
+struct GemmShape {
+  static constexpr int BM = 128;
+  static constexpr int kABytes = BM * 128;  // 128 rows of 128 bytes
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+};
+
+template <int BN, int STAGES>
+constexpr int gemm_smem_bytes() {
+  return STAGES * GemmShape<BN>::kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+}
+
+template <typename T, int BN, int STAGES, class Epi>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   int M, int N, int K, Epi epi, DevStatus* status, uint64_t limit_ns) {
+  using Sh = GemmShape<BN>;
+  constexpr bool kTf32 = ElemTraits<T>::kTf32;
+  constexpr int kBK = 128 / ElemTraits<T>::kBytes;  // K elements per stage
+  constexpr uint32_t kIdesc = make_idesc(kTf32, 128, BN, false, false);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Sh::kStageBytes);
+  // bars: full[STAGES] empty[STAGES] tfull[2] tempty[2] drain; then the
+  // TMEM address slot and the CTA's abort flag
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Sh::kTmemCols);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_tiles = (M + Sh::BM - 1) / Sh::BM;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int k_blocks = (K + kBK - 1) / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;  // stages whose copies may still be in flight
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mt = tile % m_tiles, nt = tile / m_tiles;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (*abort_flag || !mbar_wait(empty_bar(stage), phase ^ 1u, limit_ns)) {
+            if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + stage * Sh::kStageBytes;
+          mbar_expect_tx(full_bar(stage), Sh::kStageBytes);
+          tma_load_2d(sa, &tmA, full_bar(stage), kb * kBK, mt * Sh::BM);
+          tma_load_2d(sa + Sh::kABytes, &tmB, full_bar(stage), kb * kBK, nt * BN);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Drain: every issued stage's copy must land before the CTA exits.
+        // The most recent min(issued, STAGES) stages may be outstanding.
+        int s = stage;
+        uint32_t ph = phase;
+        const int outstanding = issued < STAGES ? issued : STAGES;
+        for (int i = 0; i < outstanding; ++i) {
+          if (--s < 0) {
+            s = STAGES - 1;
+            ph ^= 1u;
+          }
+          mbar_wait(full_bar(s), ph, limit_ns);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (*abort_flag || !mbar_wait(tempty_bar(acc), acc_phase ^ 1u, limit_ns)) {
+          if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, 1000 + tile);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (*abort_flag || !mbar_wait(full_bar(stage), phase, limit_ns)) {
+            if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * Sh::kStageBytes;
+          const uint32_t sb = sa + Sh::kABytes;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = sdesc_sw128(sa + ks * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sb + ks * 32, 16, 1024);
+            umma_ss<kTf32>(d_tmem, ad, bd, kIdesc, (kb | ks) != 0 ? 1u : 0u);
+          }
+          umma_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // Drain: wait until every MMA this thread issued has completed before
+      // TMEM is released (a commit tracks all prior MMAs of the thread).
+      if (!ok) {
+        umma_commit(drain_bar);
+        mbar_wait(drain_bar, 0, limit_ns);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 (TMEM lane groups 2,3,0,1)
+    const int lgrp = warp & 3;
+    const uint32_t lane_off = (uint32_t)(lgrp * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      // warp-uniform decision: the epilogue's TMEM loads are warp-collective
+      const bool fail = *abort_flag || !mbar_wait(tfull_bar(acc), acc_phase, limit_ns);
+      if (__any_sync(0xffffffffu, fail)) {
+        if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_EPILOGUE, tile);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row = mt * Sh::BM + lgrp * 32 + lane;
+      epi(tmem_base + acc * BN + lane_off, row, nt * BN, row < M);
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Sh::kTmemCols);
+  }
+}
+
+}  // namespace mmh3

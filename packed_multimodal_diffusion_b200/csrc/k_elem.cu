@@ -1,0 +1,395 @@
+// Memory-bound kernels of the block: the adaLN curve evaluation, the fused
+// segment-gather RMSNorm + modulate, the rotary (cos, sin) table, the
+// encoder layer's LayerNorm and the weight-preparation copies; plus the
+// device status word written by bounded waits.
+//
+// Sources: "cortiq_engine/mmh3.rs" (cortiq-engine 0.5.72) -- Adaln::eval,
+// rms_norm_into, norm_rows, modulate, rope_angles; "inferencelayer 0.2.1
+// src/encoder_cpu.rs" -- layer_norm_rows (two-pass variance).
+#include <cmath>
+#include <cstdio>
+
+#include "mmh3_device.cuh"
+#include "mmh3_internal.h"
+
+namespace mmh3 {
+
+// ------------------------------------------------------------ status word
+__device__ DevStatus g_dev_status;
+
+DevStatus* device_status_ptr() {
+  static DevStatus* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<DevStatus*>(p);
+  }
+  return ptrs[dev];
+}
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = v > 0 ? v : 148;
+  }
+  return cached[dev];
+}
+
+// -------------------------------------------------------------- K1 adaLN
+// out[s*rows_per_slot + r] = w[row] . c_s + b[row], c_s the interpolated
+// curve coordinates of timestep slot s (rank <= 32).
+struct CurveArgs {
+  int i0[2];
+  float f[2];
+};
+
+__global__ void __launch_bounds__(256) adaln_kernel(const float* __restrict__ w,
+                                                    const float* __restrict__ b,
+                                                    const float* __restrict__ table, int rank,
+                                                    int rows_per_slot, int n_ts, CurveArgs ca,
+                                                    float* __restrict__ out) {
+  __shared__ float c[2][32];
+  if (threadIdx.x < n_ts * rank) {
+    const int s = threadIdx.x / rank, k = threadIdx.x % rank;
+    const float a = table[ca.i0[s] * rank + k];
+    const float bb = table[(ca.i0[s] + 1) * rank + k];
+    const float f = ca.f[s];
+    c[s][k] = (1.0f - f) * a + f * bb;
+  }
+  __syncthreads();
+  const int total = n_ts * rows_per_slot;
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < total; r += gridDim.x * blockDim.x) {
+    const int s = r / rows_per_slot;
+    const float* wr = w + (size_t)r * rank;
+    float acc = 0.f;
+    if (rank == 24) {
+      const float4* w4 = reinterpret_cast<const float4*>(wr);
+#pragma unroll
+      for (int q = 0; q < 6; ++q) {
+        const float4 v = __ldg(w4 + q);
+        acc = fmaf(v.x, c[s][4 * q + 0], acc);
+        acc = fmaf(v.y, c[s][4 * q + 1], acc);
+        acc = fmaf(v.z, c[s][4 * q + 2], acc);
+        acc = fmaf(v.w, c[s][4 * q + 3], acc);
+      }
+    } else {
+      for (int k = 0; k < rank; ++k) acc = fmaf(__ldg(wr + k), c[s][k], acc);
+    }
+    out[r] = acc + __ldg(b + r);
+  }
+}
+
+cudaError_t launch_adaln(const float* w, const float* b, const float* table, int rank, int grid,
+                         int rows_per_slot, const Plan& plan, float* out, cudaStream_t s) {
+  CurveArgs ca{};
+  for (int i = 0; i < plan.n_ts; ++i) curve_coords(plan.ts[i], grid, &ca.i0[i], &ca.f[i]);
+  const int total = plan.n_ts * rows_per_slot;
+  int blocks = (total + 255) / 256;
+  const int cap = num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  adaln_kernel<<<blocks, 256, 0, s>>>(w, b, table, rank, rows_per_slot, plan.n_ts, ca, out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------- rotary (cos, sin)
+// cs[i, j] = (cos a, sin a), a = pos[i, j / k] * inv_freq[j % k], the
+// product taken in fp64 and rounded to fp32 as rope_angles does.
+struct InvFreq {
+  float v[32];
+};
+
+__global__ void rope_table_kernel(const float* __restrict__ pos, int n, int k, InvFreq inv,
+                                  float2* __restrict__ cs) {
+  const int np = 3 * k;
+  const long total = (long)n * np;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(e / np), j = (int)(e % np);
+    const float a = (float)((double)pos[i * 3 + j / k] * (double)inv.v[j % k]);
+    float sv, cv;
+    sincosf(a, &sv, &cv);
+    cs[e] = make_float2(cv, sv);
+  }
+}
+
+cudaError_t launch_rope_table(const float* pos, int n, int k, float theta, float2* cs,
+                              cudaStream_t s) {
+  InvFreq inv{};
+  for (int i = 0; i < k && i < 32; ++i) inv.v[i] = (float)std::pow((double)theta, -(double)i / (double)k);
+  const long total = (long)n * 3 * k;
+  long blocks = (total + 255) / 256;
+  if (blocks > num_sms() * 16) blocks = num_sms() * 16;
+  rope_table_kernel<<<(int)blocks, 256, 0, s>>>(pos, n, k, inv, cs);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------- K2 RMSNorm + modulate gather
+// One warp per token row; VPL float4 per lane (H = 128 * VPL).  Row i reads
+// modulation row seg_row(i + row_base): y = (x * rsqrt(mean x^2 + eps) * g)
+// * (1 + scale) + shift, stored as the GEMM operand dtype.
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+  uint2 u;
+  u.x = pack_bf16x2(v.x, v.y);
+  u.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+
+template <typename TO, int VPL>
+__global__ void __launch_bounds__(256) norm_mod_kernel(const float* __restrict__ x, int n, int H,
+                                                       const float* __restrict__ g, float eps,
+                                                       const float* __restrict__ mods,
+                                                       int mods_stride, int shift_off,
+                                                       int scale_off, SegRows seg, int row_base,
+                                                       TO* __restrict__ out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= n) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * H);
+  float4 v[VPL];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    v[i] = __ldcs(xr + i * 32 + lane);
+    ss = fmaf(v[i].x, v[i].x, ss);
+    ss = fmaf(v[i].y, v[i].y, ss);
+    ss = fmaf(v[i].z, v[i].z, ss);
+    ss = fmaf(v[i].w, v[i].w, ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = rsqrtf(ss / (float)H + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  const float* m = mods ? mods + (size_t)seg_row(seg, row + row_base) * mods_stride : nullptr;
+  TO* o = out + (size_t)row * H;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int c4 = i * 32 + lane;
+    const float4 gg = __ldg(g4 + c4);
+    float4 y = make_float4(v[i].x * inv * gg.x, v[i].y * inv * gg.y, v[i].z * inv * gg.z,
+                           v[i].w * inv * gg.w);
+    if (m) {
+      const float4 sh = __ldg(reinterpret_cast<const float4*>(m + shift_off) + c4);
+      const float4 sc = __ldg(reinterpret_cast<const float4*>(m + scale_off) + c4);
+      y.x = fmaf(y.x, 1.0f + sc.x, sh.x);
+      y.y = fmaf(y.y, 1.0f + sc.y, sh.y);
+      y.z = fmaf(y.z, 1.0f + sc.z, sh.z);
+      y.w = fmaf(y.w, 1.0f + sc.w, sh.w);
+    }
+    store4(o + 4 * c4, y);
+  }
+}
+
+template <typename TO>
+static cudaError_t norm_mod_dispatch(const float* x, int n, int H, const float* g, float eps,
+                                     const float* mods, int ms, int so, int co, const SegRows& seg,
+                                     int rb, TO* out, cudaStream_t s) {
+  const int blocks = (n + 7) / 8;
+  switch (H / 128) {
+#define MMH3_NM(V) \
+  case V:          \
+    norm_mod_kernel<TO, V><<<blocks, 256, 0, s>>>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out); break;
+    MMH3_NM(1) MMH3_NM(2) MMH3_NM(4) MMH3_NM(6) MMH3_NM(8) MMH3_NM(16) MMH3_NM(21) MMH3_NM(24)
+    MMH3_NM(32)
+#undef MMH3_NM
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_norm_mod(int dtype, const float* x, int n, int H, const float* g, float eps,
+                            const float* mods, int mods_stride, int shift_off, int scale_off,
+                            const SegRows& seg, int row_base, void* out, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  if (dtype == MMH3_BF16)
+    return norm_mod_dispatch(x, n, H, g, eps, mods, mods_stride, shift_off, scale_off, seg, row_base,
+                             static_cast<__nv_bfloat16*>(out), s);
+  return norm_mod_dispatch(x, n, H, g, eps, mods, mods_stride, shift_off, scale_off, seg, row_base,
+                           static_cast<float*>(out), s);
+}
+
+// ------------------------------------------------------------ LayerNorm
+// One warp per row, two-pass variance over registers.
+template <int VPL>
+__global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int n, int H,
+                                                        const float* __restrict__ g,
+                                                        const float* __restrict__ b, float eps,
+                                                        __nv_bfloat16* __restrict__ out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= n) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * H);
+  float4 v[VPL];
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    v[i] = __ldcs(xr + i * 32 + lane);
+    sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mu = sum / (float)H;
+  float sq = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    v[i].x -= mu; v[i].y -= mu; v[i].z -= mu; v[i].w -= mu;
+    sq = fmaf(v[i].x, v[i].x, sq);
+    sq = fmaf(v[i].y, v[i].y, sq);
+    sq = fmaf(v[i].z, v[i].z, sq);
+    sq = fmaf(v[i].w, v[i].w, sq);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  const float inv = rsqrtf(sq / (float)H + eps);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int c4 = i * 32 + lane;
+    const float4 gg = __ldg(reinterpret_cast<const float4*>(g) + c4);
+    const float4 bb = __ldg(reinterpret_cast<const float4*>(b) + c4);
+    const float4 y = make_float4(fmaf(v[i].x * inv, gg.x, bb.x), fmaf(v[i].y * inv, gg.y, bb.y),
+                                 fmaf(v[i].z * inv, gg.z, bb.z), fmaf(v[i].w * inv, gg.w, bb.w));
+    store4(out + (size_t)row * H + 4 * c4, y);
+  }
+}
+
+cudaError_t launch_layernorm(const float* x, int n, int H, const float* g, const float* b,
+                             float eps, __nv_bfloat16* out, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int blocks = (n + 7) / 8;
+  switch (H / 128) {
+#define MMH3_LN(V) \
+  case V: layernorm_kernel<V><<<blocks, 256, 0, s>>>(x, n, H, g, b, eps, out); break;
+    MMH3_LN(2) MMH3_LN(4) MMH3_LN(6) MMH3_LN(8) MMH3_LN(16) MMH3_LN(21)
+#undef MMH3_LN
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ row table
+__global__ void rows_kernel(SegRows seg, int n, int32_t* __restrict__ rows) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    rows[i] = seg_row(seg, i);
+}
+
+cudaError_t launch_rows(const SegRows& seg, int n, int32_t* rows, cudaStream_t s) {
+  int blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  rows_kernel<<<blocks, 256, 0, s>>>(seg, n, rows);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------- fc1 tile interleave
+// out row (t*256 + j) = gate row (t*128 + j) for j < 128, else up row
+// (F + t*128 + j - 128); rows of `row_bytes` bytes copied as 16-byte words.
+__global__ void fc1_tile_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int F,
+                                int words_per_row) {
+  const long total = 2L * F * words_per_row;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+    const int orow = (int)(e / words_per_row), w = (int)(e % words_per_row);
+    const int t = orow / 256, j = orow % 256;
+    const int irow = j < 128 ? t * 128 + j : F + t * 128 + (j - 128);
+    out[e] = in[(long)irow * words_per_row + w];
+  }
+}
+
+cudaError_t launch_fc1_tile(int esize, const void* in, void* out, int F, int H, cudaStream_t s) {
+  const int words = H * esize / 16;
+  long total = 2L * F * words;
+  long blocks = (total + 255) / 256;
+  if (blocks > num_sms() * 32) blocks = num_sms() * 32;
+  fc1_tile_kernel<<<(int)blocks, 256, 0, s>>>(static_cast<const uint4*>(in), static_cast<uint4*>(out), F,
+                                              words);
+  return cudaGetLastError();
+}
+
+// -------------------------------------------------- encoder qkv folding
+__global__ void vit_fold_kernel(const __nv_bfloat16* __restrict__ wq, const __nv_bfloat16* __restrict__ wk,
+                                const __nv_bfloat16* __restrict__ wv, const float* __restrict__ bq,
+                                const float* __restrict__ bk, const float* __restrict__ bv, float scale,
+                                int H, __nv_bfloat16* __restrict__ wqkv, float* __restrict__ bqkv) {
+  const long hh = (long)H * H;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < 3 * hh; e += (long)gridDim.x * blockDim.x) {
+    const int part = (int)(e / hh);
+    const long off = e % hh;
+    float v = __bfloat162float(part == 0 ? wq[off] : part == 1 ? wk[off] : wv[off]);
+    if (part == 0) v *= scale;
+    wqkv[e] = __float2bfloat16_rn(v);
+    if (off < H) {
+      const float bb = part == 0 ? bq[off] * scale : part == 1 ? bk[off] : bv[off];
+      bqkv[part * H + off] = bb;
+    }
+  }
+}
+
+cudaError_t launch_vit_fold(const void* wq, const void* wk, const void* wv, const float* bq,
+                            const float* bk, const float* bv, float scale, int H, void* wqkv,
+                            float* bqkv, cudaStream_t s) {
+  long total = 3L * H * H;
+  long blocks = (total + 255) / 256;
+  if (blocks > num_sms() * 32) blocks = num_sms() * 32;
+  vit_fold_kernel<<<(int)blocks, 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(wq), static_cast<const __nv_bfloat16*>(wk),
+      static_cast<const __nv_bfloat16*>(wv), bq, bk, bv, scale, H, static_cast<__nv_bfloat16*>(wqkv), bqkv);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------ bounded-wait self test
+// One thread initialises an mbarrier that expects one arrival which never
+// comes, waits with the given limit and records the timeout.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, DevStatus* st) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    if (!mbar_wait(b, 0, limit_ns)) record_error(st, DEV_TIMEOUT_SELFTEST, 0);
+  }
+}
+
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns, device_status_ptr());
+  return cudaGetLastError();
+}
+
+}  // namespace mmh3
+
+using namespace mmh3;
+
+extern "C" mmh3_status mmh3_device_status(void* stream, int* code, int* site) {
+  clear_error();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "device_status: stream synchronize");
+  DevStatus* p = device_status_ptr();
+  if (p == nullptr) return fail(MMH3_ERR_CUDA, "device_status: no status symbol");
+  DevStatus h{};
+  e = cudaMemcpy(&h, p, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "device_status: read");
+  const DevStatus zero{};
+  e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "device_status: clear");
+  if (code) *code = h.code;
+  if (site) *site = h.site;
+  if (h.code != 0)
+    return fail(MMH3_ERR_TIMEOUT, "a kernel gave up waiting (code %d, site %d, %d CTAs)", h.code, h.site,
+                h.count);
+  return MMH3_OK;
+}
+
+extern "C" mmh3_status mmh3_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  clear_error();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_selftest_wait(limit_ns, s);
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  int code = 0, site = 0;
+  return mmh3_device_status(stream, &code, &site);
+}

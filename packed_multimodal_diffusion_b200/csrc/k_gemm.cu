@@ -1,0 +1,163 @@
+// Host launchers of the tcgen05 GEMM instantiations and the TMA tensor-map
+// encoder.  The block's four projections ("cortiq_engine/mmh3.rs",
+// block_forward / ffn_tail: qkv, out, fc1, fc2, and the output heads of
+// forward) and the encoder layer's four biased projections ("ffai-argus
+// 0.7.0 src/siglip.rs", Layer::forward / finish_attention) all go through
+// gemm_tc_kernel with the matching fused epilogue.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm_tc.cuh"
+#include "mmh3_internal.h"
+
+namespace mmh3 {
+
+// ----------------------------------------------------------- tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, uint64_t rows,
+                  uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / esize), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launch
+template <int BN>
+constexpr int stages_for() {
+  return BN >= 256 ? 4 : (BN >= 224 ? 5 : 6);
+}
+
+template <typename T, int BN, class Epi>
+static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, const Epi& epi,
+                            cudaStream_t s) {
+  constexpr int STAGES = stages_for<BN>();
+  constexpr int smem = gemm_smem_bytes<BN, STAGES>();
+  static_assert(smem <= 232448, "GEMM shared memory above the per-CTA limit");
+  if (M <= 0) return MMH3_OK;
+  if (fault_injected("tensormap")) return fail(MMH3_ERR_CUDA, "injected fault at tensormap");
+  const int es = (int)sizeof(T);
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15)
+    return fail(MMH3_ERR_ALIGN, "GEMM operand not 16-byte aligned");
+  if (((size_t)K * es) % 16 != 0) return fail(MMH3_ERR_SHAPE, "GEMM K=%d row pitch not a multiple of 16 bytes", K);
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, A, es, (uint64_t)K, (uint64_t)M, 128) ||
+      !make_tmap_2d(&tb, B, es, (uint64_t)K, (uint64_t)N, BN))
+    return fail(MMH3_ERR_CUDA, "cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
+  auto kern = gemm_tc_kernel<T, BN, STAGES, Epi>;
+  {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM smem attribute");
+  }
+  const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
+  kern<<<grid, 192, smem, s>>>(ta, tb, M, N, K, epi, device_status_ptr(), wait_limit_ns());
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+  return MMH3_OK;
+}
+
+// qkv + per-head RMSNorm + rotation
+mmh3_status gemm_qkv(int dtype, const void* A, const void* B, int M, int N, int K, int head_dim,
+                     int inner, const float* q_norm, const float* k_norm, const float2* cs,
+                     float eps, void* out, cudaStream_t s) {
+  if (dtype == MMH3_BF16 && head_dim == 128) {
+    EpiQkvNormRope<__nv_bfloat16, 128, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, eps};
+    return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
+  }
+  if (dtype == MMH3_BF16 && head_dim == 64) {
+    EpiQkvNormRope<__nv_bfloat16, 64, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, eps};
+    return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
+  }
+  if (dtype == MMH3_F32 && head_dim == 64) {
+    EpiQkvNormRope<float, 64, 256> e{static_cast<float*>(out), N, inner, q_norm, k_norm, cs, eps};
+    return run_gemm<float, 256>(A, B, M, N, K, e, s);
+  }
+  if (dtype == MMH3_F32 && head_dim == 128) {
+    EpiQkvNormRope<float, 128, 256> e{static_cast<float*>(out), N, inner, q_norm, k_norm, cs, eps};
+    return run_gemm<float, 256>(A, B, M, N, K, e, s);
+  }
+  return fail(MMH3_ERR_SHAPE, "qkv: head_dim %d unsupported", head_dim);
+}
+
+mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, int N, int K,
+                                float* x, const float* mods, int mods_stride, int chunk_off,
+                                const SegRows& seg, cudaStream_t s) {
+  if (dtype == MMH3_BF16) {
+    if (N % 256 == 0) {
+      EpiGatedResidual<256> e{x, N, mods, mods_stride, chunk_off, seg};
+      return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
+    }
+    if (N % 224 == 0) {
+      EpiGatedResidual<224> e{x, N, mods, mods_stride, chunk_off, seg};
+      return run_gemm<__nv_bfloat16, 224>(A, B, M, N, K, e, s);
+    }
+    EpiGatedResidual<128> e{x, N, mods, mods_stride, chunk_off, seg};
+    return run_gemm<__nv_bfloat16, 128>(A, B, M, N, K, e, s);
+  }
+  if (N % 256 == 0) {
+    EpiGatedResidual<256> e{x, N, mods, mods_stride, chunk_off, seg};
+    return run_gemm<float, 256>(A, B, M, N, K, e, s);
+  }
+  EpiGatedResidual<128> e{x, N, mods, mods_stride, chunk_off, seg};
+  return run_gemm<float, 128>(A, B, M, N, K, e, s);
+}
+
+mmh3_status gemm_swiglu(int dtype, const void* A, const void* B, int M, int F, int K, void* out,
+                        cudaStream_t s) {
+  if (dtype == MMH3_BF16) {
+    EpiSwiGLU<__nv_bfloat16, 256> e{static_cast<__nv_bfloat16*>(out), F};
+    return run_gemm<__nv_bfloat16, 256>(A, B, M, 2 * F, K, e, s);
+  }
+  EpiSwiGLU<float, 256> e{static_cast<float*>(out), F};
+  return run_gemm<float, 256>(A, B, M, 2 * F, K, e, s);
+}
+
+mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N, int K,
+                          const float* bias, int mode, void* out, cudaStream_t s) {
+  if (mode == 2) {  // output heads: fp32, negated, N = 128-wide tiles
+    if (dtype == MMH3_BF16) {
+      EpiBiasAct<float, 128, 2> e{static_cast<float*>(out), N, bias};
+      return run_gemm<__nv_bfloat16, 128>(A, B, M, N, K, e, s);
+    }
+    EpiBiasAct<float, 128, 2> e{static_cast<float*>(out), N, bias};
+    return run_gemm<float, 128>(A, B, M, N, K, e, s);
+  }
+  if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias/gelu epilogue: bf16 only");
+  if (mode == 1) {
+    EpiBiasAct<__nv_bfloat16, 256, 1> e{static_cast<__nv_bfloat16*>(out), N, bias};
+    return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
+  }
+  EpiBiasAct<__nv_bfloat16, 256, 0> e{static_cast<__nv_bfloat16*>(out), N, bias};
+  return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
+}
+
+mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,
+                               const float* bias, float* x, cudaStream_t s) {
+  if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias residual epilogue: bf16 only");
+  EpiBiasResidual<256> e{x, N, bias};
+  return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
+}
+
+}  // namespace mmh3

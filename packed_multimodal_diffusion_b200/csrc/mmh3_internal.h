@@ -1,0 +1,85 @@
+// Internal host-side interfaces shared by the library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mmh3.h"
+#include "mmh3_types.h"
+
+struct CUtensorMap_st;
+typedef struct CUtensorMap_st CUtensorMap;
+
+namespace mmh3 {
+
+// ---------------------------------------------------------------- errors
+mmh3_status fail(mmh3_status code, const char* fmt, ...);
+void clear_error();
+// MMH3_FAULT=<site>: the host planner fails at the named site (host-side
+// fault injection for tests; nothing is launched).
+bool fault_injected(const char* site);
+mmh3_status cuda_fail(cudaError_t e, const char* what);
+uint64_t wait_limit_ns();
+// Address of the device status word on the current device.
+DevStatus* device_status_ptr();
+int num_sms();
+
+// ------------------------------------------------------------------ plan
+struct Plan {
+  int n_ts = 0;
+  double ts[2] = {0, 0};
+  int slot[2] = {-1, -1};   // slot of clock 0 / 1 (-1: unused)
+  SegRows block_rows{};      // per segment: slot*3 + tag
+  SegRows final_rows{};      // per segment: slot
+  int seg_tag[kMaxSeg]{};
+};
+mmh3_status make_plan(const mmh3_segment* segs, int n_seg, int n, double sigma_v, double sigma_a,
+                      Plan* p);
+// Interpolation coordinates of timestep t on a table of `grid` rows.
+void curve_coords(double t, int grid, int* i0, float* f);
+
+// -------------------------------------------------------------- launches
+cudaError_t launch_adaln(const float* w, const float* b, const float* table, int rank, int grid,
+                         int rows_per_slot, const Plan& plan, float* out, cudaStream_t s);
+cudaError_t launch_rope_table(const float* pos, int n, int k, float theta, float2* cs,
+                              cudaStream_t s);
+cudaError_t launch_norm_mod(int dtype, const float* x, int n, int H, const float* g, float eps,
+                            const float* mods, int mods_stride, int shift_off, int scale_off,
+                            const SegRows& seg, int row_base, void* out, cudaStream_t s);
+cudaError_t launch_layernorm(const float* x, int n, int H, const float* g, const float* b,
+                             float eps, __nv_bfloat16* out, cudaStream_t s);
+cudaError_t launch_rows(const SegRows& seg, int n, int32_t* rows, cudaStream_t s);
+cudaError_t launch_fc1_tile(int esize, const void* in, void* out, int F, int H, cudaStream_t s);
+cudaError_t launch_vit_fold(const void* wq, const void* wk, const void* wv, const float* bq,
+                            const float* bk, const float* bv, float scale, int H, void* wqkv,
+                            float* bqkv, cudaStream_t s);
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s);
+
+// ------------------------------------------------------------------ GEMMs
+// C = A[M,K] B[N,K]^T with a fused epilogue; dtype = mmh3_dtype of A and B.
+mmh3_status gemm_qkv(int dtype, const void* A, const void* B, int M, int N, int K, int head_dim,
+                     int inner, const float* q_norm, const float* k_norm, const float2* cs,
+                     float eps, void* out, cudaStream_t s);
+mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, int N, int K,
+                                float* x, const float* mods, int mods_stride, int chunk_off,
+                                const SegRows& seg, cudaStream_t s);
+mmh3_status gemm_swiglu(int dtype, const void* A, const void* B, int M, int F, int K, void* out,
+                        cudaStream_t s);
+// mode 0: out(act dtype) = acc + bias; 1: gelu_tanh(acc + bias);
+// 2: out(fp32) = -(acc + bias)
+mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N, int K,
+                          const float* bias, int mode, void* out, cudaStream_t s);
+mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,
+                               const float* bias, float* x, cudaStream_t s);
+mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads, int head_dim,
+                      float scale, void* out, cudaStream_t s);
+
+// 2-D row-major tensor map, 128-byte swizzle, box {128 bytes, box_rows}.
+bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, uint64_t rows,
+                  uint32_t box_rows);
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline int esize_of(int dtype) { return dtype == MMH3_BF16 ? 2 : 4; }
+
+}  // namespace mmh3

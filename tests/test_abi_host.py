@@ -1,0 +1,109 @@
+"""CPU-side checks of the C ABI library: it loads, exports every entry point
+that include/mmh3.h declares, and its host helpers (layouts, the flow-clock
+remap, the timestep plan) agree exactly with the oracle.  No GPU compute."""
+
+import ctypes as C
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import mmh3_oracle as O
+from packed_multimodal_diffusion_b200 import _lib, api, configs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:mmh3_status|double|void|const char\s*\*)\s*(mmh3_\w+)\s*\(",
+                             text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_symbols()
+    assert len(names) >= 19
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(_lib.SIGNATURES) == names
+    assert lib.mmh3_version().startswith(b"mmh3-b200")
+
+
+def test_time_shift_matches_oracle():
+    for s in (1e-3, 0.1, 0.3, 0.5, 0.972973, 1.0):
+        for (f, t) in ((12.0, 3.0), (3.0, 12.0)):
+            assert api.time_shift_sigma(s, f, t) == O.time_shift_sigma(s, f, t)
+
+
+@pytest.mark.parametrize("name", ["tiny", "block", "stack", "image"])
+def test_layouts_bit_exact_against_oracle(name):
+    c = configs.CONFIGS[name]
+    if c.image_mode:
+        segs, pos = api.layout_image(c.text_len, c.ref_lat_h, c.ref_lat_w, c.lat_h, c.lat_w)
+        L = O.layout_image(c.text_len, c.ref_lat_h, c.ref_lat_w, c.lat_h, c.lat_w)
+    else:
+        segs, pos = api.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+        L = O.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+    assert [tuple(s) for s in segs] == [tuple(s) for s in L["segments"]]
+    np.testing.assert_array_equal(pos, L["pos"].astype(np.float32))
+
+
+def test_printed_t2va_layout_through_the_abi():
+    segs, pos = api.layout_t2va(8, 3, 8, 12, 5)
+    assert pos.shape == (90, 3)
+    assert [s[2] for s in segs] == [1, 2, 0]
+
+
+@pytest.mark.parametrize("sigma_v", [1e-9, 0.05, 0.3, 0.5, 0.9, 1.0])
+@pytest.mark.parametrize("name", ["tiny", "image"])
+def test_plan_timesteps_matches_oracle(name, sigma_v):
+    c = configs.CONFIGS[name]
+    if c.image_mode:
+        L = O.layout_image(c.text_len, c.ref_lat_h, c.ref_lat_w, c.lat_h, c.lat_w)
+    else:
+        L = O.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+    sa = O.time_shift_sigma(max(sigma_v, 1e-6), 12, 3)
+    ts_o, slot = O.plan_timesteps(sigma_v, sa, L["segments"])
+    ts, rows = api.plan_timesteps(L["segments"], L["seq_len"], sigma_v, sa)
+    assert ts == ts_o
+    rows_o = O.token_rows(L["segments"], slot, L["seq_len"])
+    for (a, b, _, _), r in zip(L["segments"], rows):
+        assert (rows_o[a:b] == r).all()
+
+
+def test_argument_errors_are_reported_before_launch():
+    lib = _lib.load()
+    d = api.make_dims(2688, 21, 128, 10752)
+    bad = api.make_dims(2688, 21, 96, 10752)
+    v = C.c_size_t()
+    assert lib.mmh3_workspace_size(C.byref(bad), 100, C.byref(v)) == 2
+    assert b"head_dim" in lib.mmh3_last_error()
+    assert lib.mmh3_workspace_size(C.byref(d), 100, C.byref(v)) == 0 and v.value > 0
+    # a block call with a null weight struct fails with MMH3_ERR_ARG, no CUDA involved
+    segs = api.segments([(0, 10, 1, 0)])
+    ws = C.c_void_p(256)  # never dereferenced: validation fails first
+    rc = lib.mmh3_block_forward(C.byref(d), None, C.c_void_p(256), 10, segs, 1, None, 0.5, 0.2, 1,
+                                ws, v.value, None)
+    assert rc in (1, 4)
+    # segments with a gap
+    with pytest.raises(_lib.Mmh3Error) as e:
+        api.plan_timesteps([(0, 4, 1, 0), (5, 9, 0, 0)], 9, 0.5, 0.2)
+    assert e.value.code == 2
+
+
+def test_host_fault_injection(monkeypatch):
+    monkeypatch.setenv("MMH3_FAULT", "plan")
+    with pytest.raises(_lib.Mmh3Error) as e:
+        api.plan_timesteps([(0, 4, 1, 0)], 4, 0.5, 0.2)
+    assert "injected fault at plan" in str(e.value)
+    monkeypatch.delenv("MMH3_FAULT")
+    ts, rows = api.plan_timesteps([(0, 4, 1, 0)], 4, 0.5, 0.2)
+    assert ts == [0.5] and rows == [1]

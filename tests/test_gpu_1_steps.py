@@ -1,0 +1,117 @@
+"""GPU parity of the individual steps against the oracle, through the C ABI:
+segment rows (exact), adaLN modulation (1e-4 relative), attention (bf16 bar)
+on ragged, single-token, multi-sequence and large-score inputs, and the
+bounded-wait error path."""
+
+import pytest
+
+from gpu_common import (BF16_COS, BF16_MAXABS, TF32_COS, TF32_MAXABS, O, api, assert_close,
+                        configs, f64, math, np, sigma_pair, synth, torch)
+
+pytestmark = pytest.mark.gpu
+
+
+def _layout(name):
+    c = configs.CONFIGS[name]
+    if c.image_mode:
+        return O.layout_image(c.text_len, c.ref_lat_h, c.ref_lat_w, c.lat_h, c.lat_w)
+    return O.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+
+
+@pytest.mark.parametrize("name", ["tiny", "block", "stack", "image"])
+@pytest.mark.parametrize("sigma_v", [0.3, 0.5, 1.0])
+def test_rows_exact(cuda_ok, name, sigma_v):
+    L = _layout(name)
+    sv, sa = sigma_pair(sigma_v)
+    ts, slot = O.plan_timesteps(sv, sa, L["segments"])
+    ref = O.token_rows(L["segments"], slot, L["seq_len"])
+    rows = torch.full((L["seq_len"],), -7, dtype=torch.int32, device="cuda")
+    api.resolve_rows(L["segments"], L["seq_len"], sv, sa, rows)
+    np.testing.assert_array_equal(rows.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("name", ["tiny", "block", "image"])
+@pytest.mark.parametrize("sigma_v", [0.0, 0.3, 0.5, 0.97, 1.0])
+def test_adaln_modulation(cuda_ok, name, sigma_v):
+    c = configs.CONFIGS[name]
+    L = _layout(name)
+    w = configs.block_weights(c, 0, keys=("adaln_w", "adaln_b", "adaln_table"))
+    sv, sa = sigma_pair(sigma_v)
+    ts, _ = O.plan_timesteps(sv, sa, L["segments"])
+    H = c.hidden
+    ref = O.block_mods(f64(w["adaln_w"]), f64(w["adaln_b"]), f64(w["adaln_table"]), ts, H)
+    out = torch.full((2 * 18 * H,), float("nan"), device="cuda")
+    dims = api.make_dims(H, c.heads, c.head_dim, c.ffn)
+    nts = api.adaln_modulation(dims, w["adaln_w"].cuda(), w["adaln_b"].cuda(),
+                               w["adaln_table"].cuda(), 18 * H, L["segments"], L["seq_len"], sv, sa, out)
+    assert nts == len(ts)
+    got = f64(out[: nts * 18 * H]).reshape(nts * 3, 6 * H)
+    np.testing.assert_allclose(got, ref, rtol=1e-4, atol=1e-6)
+
+
+def _qkv(n, heads, hd, seed, dtype=torch.bfloat16, qscale=1.0):
+    I = heads * hd
+    q = synth.normal((n, I), seed, qscale, dtype=dtype)
+    k = synth.normal((n, I), seed + 1, 1.0, dtype=dtype)
+    v = synth.normal((n, I), seed + 2, 1.0, dtype=dtype)
+    return torch.cat([q, k, v], dim=1).contiguous()
+
+
+@pytest.mark.parametrize("n,heads,hd", [(1, 2, 128), (127, 1, 128), (128, 2, 128), (129, 1, 128),
+                                        (300, 3, 128), (1000, 2, 128), (300, 4, 64)])
+def test_attention_bf16(cuda_ok, n, heads, hd):
+    qkv = _qkv(n, heads, hd, 100 + n)
+    out = torch.full((n, heads * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    api.attention(qkv.cuda(), 1, n, heads, hd, 1 / math.sqrt(hd), out)
+    api.device_status()
+    q, k, v = (f64(t).reshape(n, heads, hd) for t in qkv.split(heads * hd, dim=1))
+    ref = O.attention(q, k, v, 1 / math.sqrt(hd)).reshape(n, -1)
+    assert_close(out, ref, what=f"attention n={n}")
+
+
+def test_attention_large_scores_exercise_rescale(cuda_ok):
+    # scores with std ~6 make the running maximum grow by more than 2^8
+    # between key tiles, so the O rescale path runs.
+    n, heads, hd = 700, 2, 128
+    qkv = _qkv(n, heads, hd, 7, qscale=6.0)
+    out = torch.empty((n, heads * hd), dtype=torch.bfloat16, device="cuda")
+    api.attention(qkv.cuda(), 1, n, heads, hd, 1 / math.sqrt(hd), out)
+    api.device_status()
+    q, k, v = (f64(t).reshape(n, heads, hd) for t in qkv.split(heads * hd, dim=1))
+    ref = O.attention(q, k, v, 1 / math.sqrt(hd)).reshape(n, -1)
+    assert_close(out, ref, what="attention large scores")
+
+
+def test_attention_multi_sequence(cuda_ok):
+    n_seq, seq, heads, hd = 3, 200, 2, 64
+    qkv = _qkv(n_seq * seq, heads, hd, 11)
+    out = torch.empty((n_seq * seq, heads * hd), dtype=torch.bfloat16, device="cuda")
+    api.attention(qkv.cuda(), n_seq, seq, heads, hd, 0.125, out)
+    api.device_status()
+    for b in range(n_seq):
+        part = qkv[b * seq:(b + 1) * seq]
+        q, k, v = (f64(t).reshape(seq, heads, hd) for t in part.split(heads * hd, dim=1))
+        ref = O.attention(q, k, v, 0.125).reshape(seq, -1)
+        assert_close(out[b * seq:(b + 1) * seq], ref, what=f"sequence {b}")
+
+
+def test_attention_fp32_tf32(cuda_ok):
+    n, heads, hd = 200, 2, 64
+    qkv = _qkv(n, heads, hd, 21, dtype=torch.float32)
+    out = torch.empty((n, heads * hd), dtype=torch.float32, device="cuda")
+    api.attention(qkv.cuda(), 1, n, heads, hd, 1 / 8, out)
+    api.device_status()
+    q, k, v = (f64(t).reshape(n, heads, hd) for t in qkv.split(heads * hd, dim=1))
+    ref = O.attention(q, k, v, 1 / 8).reshape(n, -1)
+    assert_close(out, ref, TF32_MAXABS, TF32_COS, what="attention tf32")
+
+
+def test_bounded_wait_returns_timeout_and_context_survives(cuda_ok):
+    assert api.selftest_wait_timeout(1_000_000) == 7      # MMH3_ERR_TIMEOUT after ~1 ms
+    assert api.device_status() == (0, 0)                  # status was cleared
+    n, heads, hd = 130, 1, 128
+    qkv = _qkv(n, heads, hd, 5)
+    out = torch.empty((n, heads * hd), dtype=torch.bfloat16, device="cuda")
+    api.attention(qkv.cuda(), 1, n, heads, hd, 1 / math.sqrt(hd), out)
+    api.device_status()
+    assert torch.isfinite(out.float()).all()

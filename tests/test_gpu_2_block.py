@@ -1,0 +1,123 @@
+"""GPU parity of the whole modulated block (and its stack / heads) against
+the oracle, through mmh3_block_forward / mmh3_stack_forward: the output, the
+block delta (x_out - x_in) and every intermediate the workspace holds
+(xn1, post-rotation q and k, v, attn, xn2, act)."""
+
+import pytest
+
+from gpu_common import (BF16_COS, BF16_MAXABS, TF32_COS, TF32_MAXABS, O, api, assert_close,
+                        configs, f64, heads_split, np, oracle_block, run_block, sigma_pair,
+                        small_block_weights, small_dims, t2va, torch)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_block(dims_o, dims_c, w, x, segs, pos, sv, sa, bars, modulated=True):
+    keep = {}
+    ref, mods, rows = oracle_block(w, x, segs, pos, sv, sa, dims_o, keep=keep, modulated=modulated)
+    xg, reg = run_block(dims_c, w, x, segs, pos, sv, sa, modulated=modulated)
+    maxabs, cos = bars
+    assert_close(xg, ref, maxabs, cos, "x_out")
+    assert_close(xg.cpu().double() - x.double(), ref - f64(x), maxabs, cos, "block delta")
+    H, nh, hd = dims_o["hidden"], dims_o["heads"], dims_o["head_dim"]
+    n = x.shape[0]
+    assert_close(reg["xn1"], keep["xn1"], maxabs, cos, "xn1")
+    q, k, v = heads_split(reg["qkv"], nh, hd)
+    assert_close(q, keep["q"], maxabs, cos, "q after qk-norm + rotation")
+    assert_close(k, keep["k"], maxabs, cos, "k after qk-norm + rotation")
+    assert_close(v, keep["v"], maxabs, cos, "v")
+    assert_close(reg["attn"], keep["attn"], maxabs, cos, "attn")
+    assert_close(reg["xn2"], keep["xn2"], maxabs, cos, "xn2")
+    assert_close(reg["act"], keep["act"], maxabs, cos, "SwiGLU act")
+    return xg
+
+
+@pytest.mark.parametrize("layout,sigma_v", [((20, 3, 16, 20, 20), 0.5), ((5, 1, 4, 4, 3), 0.3),
+                                            ((130, 2, 16, 16, 64), 1.0)])
+def test_block_small_bf16(cuda_ok, layout, sigma_v):
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(*layout)
+    n = int(pos.shape[0])
+    w = small_block_weights(31, 256, 2, 128, 512)
+    x = configs.synth.normal((n, 256), 77, 1.0)
+    sv, sa = sigma_pair(sigma_v)
+    _check_block(dims_o, dims_c, w, x, segs, pos, sv, sa, (BF16_MAXABS, BF16_COS))
+
+
+def test_block_zero_gates_is_exact_identity(cuda_ok):
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    n = int(pos.shape[0])
+    w = small_block_weights(32, 256, 2, 128, 512)
+    H = 256
+    for e in (2, 5):
+        for r in range(6):
+            lo = r * 6 * H + e * H
+            w["adaln_w"][lo:lo + H] = 0
+            w["adaln_b"][lo:lo + H] = 0
+    x = configs.synth.normal((n, H), 78, 1.0)
+    xg, _ = run_block(dims_c, w, x, segs, pos, *sigma_pair(0.5))
+    assert torch.equal(xg.cpu(), x)
+
+
+def test_block_unmodulated_refiner_form(cuda_ok):
+    dims_o, dims_c = small_dims()
+    n = 150
+    w = small_block_weights(33, 256, 2, 128, 512)
+    x = configs.synth.normal((n, 256), 79, 1.0)
+    segs = [(0, n, 1, 0)]
+    _check_block(dims_o, dims_c, w, x, segs, None, 0.5, 0.2, (BF16_MAXABS, BF16_COS), modulated=False)
+
+
+def test_block_deterministic(cuda_ok):
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    w = small_block_weights(34, 256, 2, 128, 512)
+    x = configs.synth.normal((int(pos.shape[0]), 256), 80, 1.0)
+    a, _ = run_block(dims_c, w, x, segs, pos, *sigma_pair(0.5))
+    b, _ = run_block(dims_c, w, x, segs, pos, *sigma_pair(0.5))
+    assert torch.equal(a, b)
+
+
+def test_tiny_workload_fp32(cuda_ok):
+    c = configs.TINY
+    segs, pos = t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+    assert pos.shape[0] == 64
+    w = configs.block_weights(c, 0)
+    x = configs.hidden_states(c)
+    dims_c = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn, act_dtype=torch.float32)
+    _check_block(c.dims(), dims_c, w, x, segs, pos, *sigma_pair(c.sigma_v), (TF32_MAXABS, TF32_COS))
+
+
+def test_tiny_workload_bf16(cuda_ok):
+    c = configs.TINY
+    segs, pos = t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+    w = configs.block_weights(c, 0, wdtype=torch.bfloat16)
+    x = configs.hidden_states(c)
+    dims_c = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn, act_dtype=torch.bfloat16)
+    _check_block(c.dims(), dims_c, w, x, segs, pos, *sigma_pair(c.sigma_v), (BF16_MAXABS, BF16_COS))
+
+
+def test_block_workload_full_size_sampled_rows(cuda_ok):
+    """The 13 248-token MiniMax-H3 block in the launch configuration the bench
+    times; the oracle computes k and v for every token and the rest for a
+    sample of rows spanning text, audio, video and the ragged last tile."""
+    c = configs.BLOCK
+    segs, pos = t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+    n = int(pos.shape[0])
+    assert n == 13248
+    w = configs.block_weights(c, 0)
+    x = configs.hidden_states(c)
+    sv, sa = sigma_pair(c.sigma_v)
+    dims_c = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn)
+    xg, reg = run_block(dims_c, w, x, segs, pos, sv, sa)
+    sample = [0, 1, 255, 256, 511, 767, 768, 4000, 9000, 13119, 13120, 13200, 13247]
+    keep = {}
+    ref, _, _ = oracle_block(w, x, segs, pos, sv, sa, c.dims(), sample_rows=sample, keep=keep)
+    assert_close(xg[sample], ref, what="x_out rows")
+    assert_close(xg[sample].cpu().double() - x[sample].double(), ref - f64(x[sample]), what="delta rows")
+    q, k, v = heads_split(reg["qkv"][sample], c.heads, c.head_dim)
+    assert_close(q, keep["q"], what="q rows")
+    assert_close(k, keep["k"], what="k rows")
+    assert_close(reg["attn"][sample], keep["attn"], what="attn rows")
+    assert_close(reg["act"][sample], keep["act"], what="act rows")
