@@ -285,6 +285,20 @@ void mmh3_set_wait_limit_ns(uint64_t ns);
  * mmh3_device_status would (MMH3_ERR_TIMEOUT when the wait ran out). */
 mmh3_status mmh3_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
+/* Per-phase device-time profile of the block, in the nine phase slots of
+ * "cortiq_engine/mmh3.rs" (MMH3_PROF): 0 norm+modulate (with the adaLN curve
+ * and the rotation table), 1 qkv GEMM (qk-norm and rotation fused in; slot 2
+ * stays 0), 3 attention, 4 out GEMM + gated residual, 5 fc1 GEMM + SwiGLU
+ * (slot 6 stays 0), 7 fc2 GEMM + gated residual (slot 8 stays 0).
+ * mmh3_prof_enable(1) makes the block entry points record CUDA events on
+ * their stream between launches; mmh3_prof_collect waits for the recorded
+ * events and adds their times into ms[0..min(n_slots,9)) (cumulative since
+ * the last reset), with *n_blocks the number of blocks profiled.  Not thread
+ * safe; the events are created lazily and reused. */
+void mmh3_prof_enable(int on);
+mmh3_status mmh3_prof_collect(double* ms, int n_slots, long* n_blocks);
+void mmh3_prof_reset(void);
+
 /* Message of the last failing call on this thread ("" if none). */
 const char* mmh3_last_error(void);
 

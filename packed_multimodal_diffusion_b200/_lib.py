@@ -87,6 +87,9 @@ SIGNATURES = {
     "mmh3_device_status": (_I, [_P, C.POINTER(_I), C.POINTER(_I)]),
     "mmh3_set_wait_limit_ns": (None, [C.c_uint64]),
     "mmh3_selftest_wait_timeout": (_I, [C.c_uint64, _P]),
+    "mmh3_prof_enable": (None, [_I]),
+    "mmh3_prof_collect": (_I, [C.POINTER(C.c_double), _I, C.POINTER(C.c_long)]),
+    "mmh3_prof_reset": (None, []),
     "mmh3_last_error": (C.c_char_p, []),
     "mmh3_version": (C.c_char_p, []),
 }

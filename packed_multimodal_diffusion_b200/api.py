@@ -242,6 +242,26 @@ def selftest_wait_timeout(limit_ns: int) -> int:
     return load().mmh3_selftest_wait_timeout(limit_ns, _stream())
 
 
+PROF_SLOTS = ("norm+mod", "qkv gemm", "qknorm+rope", "attention", "out gemm", "fc1 gemm",
+              "swiglu", "fc2 gemm", "residual")
+
+
+def prof_enable(on: bool = True) -> None:
+    load().mmh3_prof_enable(1 if on else 0)
+
+
+def prof_reset() -> None:
+    load().mmh3_prof_reset()
+
+
+def prof_collect() -> tuple[dict, int]:
+    """Cumulative per-phase device milliseconds and the number of blocks."""
+    ms = (C.c_double * 9)()
+    nb = C.c_long()
+    check(load().mmh3_prof_collect(ms, 9, C.byref(nb)))
+    return dict(zip(PROF_SLOTS, list(ms))), nb.value
+
+
 def set_wait_limit_ns(ns: int) -> None:
     load().mmh3_set_wait_limit_ns(ns)
 

@@ -10,10 +10,64 @@
 // Layer::forward and finish_attention.
 #include <cmath>
 #include <cstring>
+#include <vector>
 
 #include "mmh3_internal.h"
 
 using namespace mmh3;
+
+
+// --------------------------------------------------------------- profiler
+// Per-phase device time of the block, in the nine slots of the reference's
+// phase profile ("cortiq_engine/mmh3.rs", MMH3_PROF): 0 norm+modulate (with
+// the adaLN curve and the rotation table), 1 qkv GEMM (qk-norm and rotation
+// are fused into it, so slot 2 stays 0), 3 attention, 4 out GEMM with the
+// gated residual, 5 fc1 GEMM with SwiGLU (slot 6 stays 0), 7 fc2 GEMM with
+// the gated residual (slot 8 stays 0).  Enabled by mmh3_prof_enable(1);
+// events are recorded on the caller's stream between the launches, so the
+// phases never overlap and are never counted twice.
+struct ProfRec {
+  int slot;
+  cudaEvent_t a, b;
+};
+static bool g_prof_on = false;
+static std::vector<ProfRec> g_prof_recs;
+static std::vector<cudaEvent_t> g_prof_free;
+static double g_prof_ms[9] = {0};
+static long g_prof_blocks = 0;
+
+static cudaEvent_t prof_event() {
+  cudaEvent_t e = nullptr;
+  if (!g_prof_free.empty()) {
+    e = g_prof_free.back();
+    g_prof_free.pop_back();
+  } else if (cudaEventCreate(&e) != cudaSuccess) {
+    e = nullptr;
+  }
+  return e;
+}
+
+struct PhaseMark {
+  cudaEvent_t last = nullptr;
+  cudaStream_t s;
+  explicit PhaseMark(cudaStream_t st) : s(st) {
+    if (g_prof_on && (last = prof_event()) != nullptr) cudaEventRecord(last, s);
+  }
+  // closes the running phase as `slot` and opens the next one
+  void mark(int slot) {
+    if (!g_prof_on || last == nullptr) return;
+    cudaEvent_t e = prof_event();
+    if (e == nullptr) return;
+    cudaEventRecord(e, s);
+    g_prof_recs.push_back({slot, last, e});
+    cudaEvent_t next = prof_event();
+    if (next) cudaEventRecord(next, s);
+    last = next;
+  }
+  ~PhaseMark() {
+    if (last) g_prof_free.push_back(last);
+  }
+};
 
 namespace {
 
@@ -96,25 +150,35 @@ mmh3_status check_block(const mmh3_dims& d, const mmh3_block_weights* w, bool mo
 // norm2-modulate -> fc1+SwiGLU -> fc2+gated residual
 mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x, int n,
                        const Plan& plan, const float* mods, const float2* cs, const Workspace& ws,
-                       cudaStream_t s) {
+                       cudaStream_t s, PhaseMark& pm) {
   const int H = d.hidden, I = d.heads * d.head_dim, F = d.ffn;
   const int dt = d.act_dtype;
   const int stride = 6 * H;
   cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm1, d.eps, mods, stride, 0 * H, 1 * H, plan.block_rows, 0,
                                   ws.xn1, s);
   if (e != cudaSuccess) return cuda_fail(e, "norm1/modulate launch");
+  pm.mark(0);
   mmh3_status st = gemm_qkv(dt, ws.xn1, w.wqkv, n, 3 * I, H, d.head_dim, I, w.q_norm, w.k_norm, cs, d.qk_eps,
                             ws.qkv, s);
   if (st != MMH3_OK) return st;
+  pm.mark(1);
   st = attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, 1.0f / std::sqrt((float)d.head_dim), ws.attn, s);
   if (st != MMH3_OK) return st;
+  pm.mark(3);
   st = gemm_gated_residual(dt, ws.attn, w.wout, n, H, I, x, mods, stride, 2 * H, plan.block_rows, s);
   if (st != MMH3_OK) return st;
+  pm.mark(4);
   e = launch_norm_mod(dt, x, n, H, w.norm2, d.eps, mods, stride, 3 * H, 4 * H, plan.block_rows, 0, ws.xn2, s);
   if (e != cudaSuccess) return cuda_fail(e, "norm2/modulate launch");
+  pm.mark(0);
   st = gemm_swiglu(dt, ws.xn2, w.wfc1, n, F, H, ws.act, s);
   if (st != MMH3_OK) return st;
-  return gemm_gated_residual(dt, ws.act, w.wfc2, n, H, F, x, mods, stride, 5 * H, plan.block_rows, s);
+  pm.mark(5);
+  st = gemm_gated_residual(dt, ws.act, w.wfc2, n, H, F, x, mods, stride, 5 * H, plan.block_rows, s);
+  if (st != MMH3_OK) return st;
+  pm.mark(7);
+  if (g_prof_on) ++g_prof_blocks;
+  return MMH3_OK;
 }
 
 mmh3_status common_checks(const mmh3_dims* dims, float* x, int n, const float* pos, void* ws,
@@ -205,6 +269,7 @@ mmh3_status mmh3_block_forward(const mmh3_dims* dims, const mmh3_block_weights* 
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden;
+  PhaseMark pm(s);
   if (modulated) {
     cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * H, plan,
                                  ws.mods, s);
@@ -214,7 +279,8 @@ mmh3_status mmh3_block_forward(const mmh3_dims* dims, const mmh3_block_weights* 
     cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
   }
-  return block_core(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s);
+  pm.mark(0);
+  return block_core(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s, pm);
 }
 
 mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* blocks, int n_blocks,
@@ -255,6 +321,7 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                   heads->out_audio);
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PhaseMark pm(s);
   if (pos_dev) {
     cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
@@ -264,7 +331,8 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
     cudaError_t e = launch_adaln(w.adaln_w, w.adaln_b, w.adaln_table, dims->rank, dims->grid, 18 * H, plan,
                                  ws.mods, s);
     if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
-    st = block_core(*dims, w, x, n, plan, ws.mods, pos_dev ? ws.cs : nullptr, ws, s);
+    pm.mark(0);
+    st = block_core(*dims, w, x, n, plan, ws.mods, pos_dev ? ws.cs : nullptr, ws, s, pm);
     if (st != MMH3_OK) return st;
   }
   if (heads == nullptr) return MMH3_OK;
@@ -371,6 +439,31 @@ mmh3_status mmh3_vit_layer_forward(const mmh3_vit_dims* dims, const mmh3_vit_wei
   st = gemm_bias_act(MMH3_BF16, h, w->w1, M, dims->mlp, H, w->b1, 1, act, s);
   if (st != MMH3_OK) return st;
   return gemm_bias_residual(MMH3_BF16, act, w->w2, M, H, dims->mlp, w->b2, x, s);
+}
+
+// ---------------------------------------------------------------- profiler
+void mmh3_prof_enable(int on) { g_prof_on = on != 0; }
+
+mmh3_status mmh3_prof_collect(double* ms, int n_slots, long* n_blocks) {
+  clear_error();
+  for (ProfRec& r : g_prof_recs) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "prof: event");
+    g_prof_ms[r.slot] += t;
+    g_prof_free.push_back(r.a);
+    g_prof_free.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  for (int i = 0; i < n_slots && i < 9; ++i) ms[i] = g_prof_ms[i];
+  if (n_blocks) *n_blocks = g_prof_blocks;
+  return MMH3_OK;
+}
+
+void mmh3_prof_reset(void) {
+  for (double& v : g_prof_ms) v = 0.0;
+  g_prof_blocks = 0;
 }
 
 }  // extern "C"

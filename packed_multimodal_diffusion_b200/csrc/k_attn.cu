@@ -8,6 +8,68 @@
 
 namespace mmh3 {
 
+// Exact-fp32 attention on CUDA cores for the fp32-storage path: one thread
+// per query row, 64-key tiles of K and V staged in shared memory, running
+// maximum and sum (online softmax), final division by the sum.
+template <int HD>
+__global__ void __launch_bounds__(64) attn_f32_simt_kernel(const float* __restrict__ qkv, float* __restrict__ out,
+                                                           int seq, int inner, float scale) {
+  __shared__ float ks[64][HD];
+  __shared__ float vs[64][HD];
+  const int head = blockIdx.y;
+  const int row0 = blockIdx.z * seq;
+  const int qi = blockIdx.x * 64 + threadIdx.x;
+  const int ld = 3 * inner;
+  const bool q_ok = qi < seq;
+  float q[HD], o[HD];
+#pragma unroll
+  for (int d = 0; d < HD; ++d) {
+    q[d] = q_ok ? qkv[(size_t)(row0 + qi) * ld + head * HD + d] * scale : 0.f;
+    o[d] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int k0 = 0; k0 < seq; k0 += 64) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * HD; e += 64) {
+      const int r = e / HD, d = e % HD;
+      const bool ok = k0 + r < seq;
+      const size_t base = (size_t)(row0 + k0 + r) * ld + head * HD + d;
+      ks[r][d] = ok ? qkv[base + inner] : 0.f;
+      vs[r][d] = ok ? qkv[base + 2 * inner] : 0.f;
+    }
+    __syncthreads();
+    const int nk = seq - k0 < 64 ? seq - k0 : 64;
+    for (int j = 0; j < nk; ++j) {
+      float sv = 0.f;
+#pragma unroll
+      for (int d = 0; d < HD; ++d) sv = fmaf(q[d], ks[j][d], sv);
+      const float m_new = fmaxf(m, sv);
+      const float alpha = expf(m - m_new);
+      const float p = expf(sv - m_new);
+      l = l * alpha + p;
+#pragma unroll
+      for (int d = 0; d < HD; ++d) o[d] = fmaf(o[d], alpha, p * vs[j][d]);
+      m = m_new;
+    }
+  }
+  if (q_ok) {
+    const float inv = l > 0.f ? 1.0f / l : 0.f;
+    float* dst = out + (size_t)(row0 + qi) * inner + head * HD;
+#pragma unroll
+    for (int d = 0; d < HD; ++d) dst[d] = o[d] * inv;
+  }
+}
+
+template <int HD>
+static mmh3_status run_attn_f32(const void* qkv, int n_seq, int seq, int heads, float scale, void* out,
+                                cudaStream_t s) {
+  dim3 grid((seq + 63) / 64, heads, n_seq);
+  attn_f32_simt_kernel<HD><<<grid, 64, 0, s>>>(static_cast<const float*>(qkv), static_cast<float*>(out), seq,
+                                                heads * HD, scale);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "fp32 attention launch");
+}
+
 template <typename T, int HD, int KV, int PB>
 static mmh3_status run_attn(const void* qkv, int n_seq, int seq, int heads, float scale, void* out,
                             cudaStream_t s) {
@@ -39,8 +101,7 @@ mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads,
     return run_attn<__nv_bfloat16, 128, 2, 2>(qkv, n_seq, seq, heads, scale, out, s);
   if (dtype == MMH3_BF16 && head_dim == 64)
     return run_attn<__nv_bfloat16, 64, 2, 2>(qkv, n_seq, seq, heads, scale, out, s);
-  if (dtype == MMH3_F32 && head_dim == 64)
-    return run_attn<float, 64, 2, 1>(qkv, n_seq, seq, heads, scale, out, s);
+  if (dtype == MMH3_F32 && head_dim == 64) return run_attn_f32<64>(qkv, n_seq, seq, heads, scale, out, s);
   return fail(MMH3_ERR_SHAPE, "attention: dtype %d head_dim %d unsupported", dtype, head_dim);
 }
 

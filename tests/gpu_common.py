@@ -2,13 +2,17 @@
 the comparison bars.
 
 Bars (floating point):
-  * bf16 path (block outputs, block deltas and every bf16 intermediate):
-    max-abs <= 2e-2 and cosine >= 0.9995.
+  * bf16 path, block outputs and block deltas (x_out - x_in): max-abs <= 2e-2
+    and cosine >= 0.9995.
+  * bf16-stored intermediates (xn1, q, k, v after qk-norm + rotation, attn,
+    xn2, act): cosine >= 0.9995 and, element-wise,
+    |gpu - ref| <= 2e-2 + 2^-7 |ref| -- rounding a value to bf16 alone moves
+    it by up to 2^-8 |ref|, which exceeds 2e-2 for |ref| > 5.
   * fp32 modulation vectors: |gpu - oracle| <= 1e-4 |oracle| + 1e-6.
-  * fp32-storage path (tcgen05 kind::tf32, 10-bit mantissa operands):
-    max-abs <= 5e-3 and cosine >= 0.99995 -- tf32 rounding (2^-11 relative
-    per operand) is 16x finer than bf16's 2^-7, so the bf16 bar tightened by
-    about that factor.
+  * fp32-storage path (tcgen05 kind::tf32 GEMMs, exact-fp32 attention):
+    max-abs <= 5e-3 and cosine >= 0.99995, intermediates + 2^-10 |ref| --
+    tf32 rounding (2^-11 relative per operand) is 16x finer than bf16's 2^-7,
+    so the bf16 bar tightened by about that factor.
 Integer work (rows, positions): exact.
 """
 
@@ -40,14 +44,28 @@ def cosine(a, b) -> float:
     return float(a @ b / (na * nb))
 
 
-def assert_close(gpu, ref, maxabs=BF16_MAXABS, cos=BF16_COS, what=""):
+def assert_close(gpu, ref, maxabs=BF16_MAXABS, cos=BF16_COS, what="", rel=0.0):
+    """max |gpu - ref| <= maxabs (+ rel * |ref| element-wise) and cosine >= cos.
+
+    rel > 0 is used for intermediates the GPU stores in a low-precision type:
+    rounding a value v to bf16 alone moves it by up to |v| * 2^-8, so such a
+    tensor gets the element-wise bound maxabs + 2^-7 |ref| (storage rounding
+    plus the same again for the rounding of its bf16 inputs)."""
     g, r = f64(gpu), f64(ref)
     assert g.shape == r.shape, (what, g.shape, r.shape)
     assert np.isfinite(g).all(), f"{what}: non-finite GPU values"
-    err = float(np.max(np.abs(g - r))) if g.size else 0.0
+    excess = np.abs(g - r) - rel * np.abs(r)
+    err = float(np.max(excess)) if g.size else 0.0
     c = cosine(g, r)
-    assert err <= maxabs and c >= cos, f"{what}: max-abs {err:.3e} (bar {maxabs}), cosine {c:.6f} (bar {cos})"
+    assert err <= maxabs and c >= cos, \
+        f"{what}: max-abs {err:.3e} beyond {rel:g}|ref| (bar {maxabs}), cosine {c:.6f} (bar {cos})"
     return err, c
+
+
+#: element-wise relative allowance for bf16-stored intermediates
+BF16_STORE_REL = 2.0 ** -7
+#: the same for tf32-rounded GEMM inputs with fp32 storage
+TF32_STORE_REL = 2.0 ** -10
 
 
 def small_dims(hidden=256, heads=2, head_dim=128, ffn=512, act=torch.bfloat16):
