@@ -201,13 +201,20 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       float s[128];
       {
-        uint32_t u[32];
+        // four loads in flight, one wait
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        const uint32_t ts = tmem + sb * 128 + lane_off;
+        tmem_ld32(ts + 0, u0);
+        tmem_ld32(ts + 32, u1);
+        tmem_ld32(ts + 64, u2);
+        tmem_ld32(ts + 96, u3);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tmem + sb * 128 + lane_off + c * 32, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(u[i]);
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(u0[i]);
+          s[32 + i] = __uint_as_float(u1[i]);
+          s[64 + i] = __uint_as_float(u2[i]);
+          s[96 + i] = __uint_as_float(u3[i]);
         }
       }
       tc_fence_before();
@@ -218,9 +225,14 @@ __global__ void __launch_bounds__(192, 1)
         for (int k = 0; k < 128; ++k)
           if (k >= valid) s[k] = -INFINITY;
       }
-      float mx = s[0];
+      // row maximum with eight independent partial maxima (short chains)
+      float pm[8];
 #pragma unroll
-      for (int k = 1; k < 128; ++k) mx = fmaxf(mx, s[k]);
+      for (int i = 0; i < 8; ++i) pm[i] = s[i];
+#pragma unroll
+      for (int k = 8; k < 128; ++k) pm[k & 7] = fmaxf(pm[k & 7], s[k]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       const float m_tile = mx * scale_log2;
       if (j == 0) {
         m_ref = m_tile;
@@ -259,7 +271,7 @@ __global__ void __launch_bounds__(192, 1)
       // p = 2^(s * scale * log2e - m_ref); write the row into the swizzled
       // K-major A tile: box = key / kEPB, 16-byte chunk index XOR (row % 8).
       uint8_t* prow = smem + Sh::kPOff + pb * Sh::kPBytes + r * 128;
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (kTf32) {
 #pragma unroll
         for (int k8 = 0; k8 < 128 / 4; ++k8) {
@@ -268,7 +280,7 @@ __global__ void __launch_bounds__(192, 1)
           q.y = ex2_approx(fmaf(s[4 * k8 + 1], scale_log2, -m_ref));
           q.z = ex2_approx(fmaf(s[4 * k8 + 2], scale_log2, -m_ref));
           q.w = ex2_approx(fmaf(s[4 * k8 + 3], scale_log2, -m_ref));
-          psum += (q.x + q.y) + (q.z + q.w);
+          ps[k8 & 3] += (q.x + q.y) + (q.z + q.w);
           const int box = k8 / 8, chunk = k8 % 8;
           *reinterpret_cast<float4*>(prow + box * Sh::kBoxBytes + ((chunk ^ (r & 7)) * 16)) = q;
         }
@@ -278,7 +290,7 @@ __global__ void __launch_bounds__(192, 1)
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) p[e] = ex2_approx(fmaf(s[8 * k8 + e], scale_log2, -m_ref));
-          psum += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+          ps[k8 & 3] += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
           uint4 q;
           q.x = pack_bf16x2(p[0], p[1]);
           q.y = pack_bf16x2(p[2], p[3]);
@@ -288,7 +300,7 @@ __global__ void __launch_bounds__(192, 1)
           *reinterpret_cast<uint4*>(prow + box * Sh::kBoxBytes + ((chunk ^ (r & 7)) * 16)) = q;
         }
       }
-      l_sum += psum;
+      l_sum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(B_PF + pb));

@@ -257,6 +257,21 @@ struct EpiBiasResidual {
 };
 
 // ------------------------------------------------------------------ kernel
+// Tile order: groups of kGroupM row tiles, all column tiles of a group
+// before the next group, so the A rows of a group and all of B stay in L2
+// while the group is processed (A is read from DRAM about once).
+constexpr int kGroupM = 16;
+
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mt, int& nt) {
+  const int per_group = kGroupM * n_tiles;
+  const int g = tile / per_group;
+  const int first_m = g * kGroupM;
+  const int gm = (m_tiles - first_m) < kGroupM ? (m_tiles - first_m) : kGroupM;
+  const int t = tile - g * per_group;
+  mt = first_m + t % gm;
+  nt = t / gm;
+}
+
 template <int BN>
 struct GemmShape {
   static constexpr int BM = 128;
@@ -332,7 +347,8 @@ __global__ void __launch_bounds__(192, 1)
       int issued = 0;  // stages whose copies may still be in flight
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile % m_tiles, nt = tile / m_tiles;
+        int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, mt, nt);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (*abort_flag || !mbar_wait(empty_bar(stage), phase ^ 1u, limit_ns)) {
             if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, tile);
@@ -426,7 +442,8 @@ __global__ void __launch_bounds__(192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, mt, nt);
       // warp-uniform decision: the epilogue's TMEM loads are warp-collective
       const bool fail = *abort_flag || !mbar_wait(tfull_bar(acc), acc_phase, limit_ns);
       if (__any_sync(0xffffffffu, fail)) {
