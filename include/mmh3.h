@@ -220,6 +220,35 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                                double sigma_v, double sigma_a, float* out_video, float* out_audio,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch that mmh3_block_forward_noalloc uses:
+ * 32 MiB, reserved on every GPU where the library's device code is loaded,
+ * until the process exits. */
+#define MMH3_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* mmh3_block_forward for callers that cannot allocate device memory (no
+ * counterpart in the pages; this is a library-usage addition).  Some hosts
+ * own every device allocation through their own pool and give plugins no
+ * allocator, and some runtimes must not call cudaMalloc on their hot path
+ * because it synchronises the device; such callers cannot provide the
+ * workspace mmh3_block_forward needs.  This entry point runs the same
+ * kernels with the block's intermediates in one fixed library-owned device
+ * array of MMH3_NOALLOC_SCRATCH_BYTES, and allocates nothing itself: the
+ * caller still passes x, the weights and the positions.
+ *  - Sizes whose intermediates (mmh3_workspace_size) exceed the array are
+ *    rejected with MMH3_ERR_WORKSPACE and a message giving the largest token
+ *    count that fits (556 tokens at hidden 2688, 21 x 128 heads, ffn 10752).
+ *  - The first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls share the array, which keeps the last call's contents; calls
+ *    whose kernels overlap on the GPU race on it.  Nothing in it needs to
+ *    start at zero.  The phase profile is not recorded by this entry point.
+ * Arguments and results are those of mmh3_block_forward without the
+ * workspace. */
+mmh3_status mmh3_block_forward_noalloc(const mmh3_dims* dims, const mmh3_block_weights* w, float* x,
+                                       int n, const mmh3_segment* segs, int n_seg,
+                                       const float* pos_dev, double sigma_v, double sigma_a,
+                                       int modulated, void* stream);
+
 /* ------------------------------------------------------ SigLIP encoder layer */
 
 typedef struct {

@@ -77,6 +77,8 @@ SIGNATURES = {
     "mmh3_attention": (_I, [_P, _I, _I, _I, _I, _I, C.c_float, _P, _P]),
     "mmh3_block_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _P,
                                 _D, _D, _I, _P, C.c_size_t, _P]),
+    "mmh3_block_forward_noalloc": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I,
+                                        _P, _D, _D, _I, _P]),
     "mmh3_stack_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _I,
                                 C.POINTER(HeadWeights), _P, _I, _SEGP, _I, _P, _D, _D, _P, _P, _P,
                                 C.c_size_t, _P]),

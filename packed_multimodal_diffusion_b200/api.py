@@ -173,6 +173,17 @@ def block_forward(dims: Dims, params: BlockParams, x: torch.Tensor, segs, pos: t
                                     workspace.numel() * workspace.element_size(), _stream()))
 
 
+def block_forward_noalloc(dims: Dims, params: BlockParams, x: torch.Tensor, segs,
+                          pos: torch.Tensor | None, sigma_v: float, sigma_a: float,
+                          modulated: bool = True) -> None:
+    """mmh3_block_forward on the library's fixed device scratch (no
+    workspace argument, nothing allocated by the call); in place on x."""
+    st = params.struct()
+    check(load().mmh3_block_forward_noalloc(C.byref(dims), C.byref(st), _ptr(x), x.shape[0],
+                                            segments(segs), len(segs), _ptr(pos), sigma_v, sigma_a,
+                                            1 if modulated else 0, _stream()))
+
+
 def stack_forward(dims: Dims, blocks: list, heads: HeadParams | None, x: torch.Tensor, segs,
                   pos, sigma_v, sigma_a, out_video, out_audio, workspace) -> None:
     arr = (BlockWeights * max(1, len(blocks)))(*[b.struct() for b in blocks])

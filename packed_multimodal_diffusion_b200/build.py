@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmmh3.so")
-SOURCES = ["host_planner.cpp", "k_elem.cu", "k_gemm.cu", "k_attn.cu", "api.cu"]
+SOURCES = ["host_planner.cpp", "k_elem.cu", "k_gemm.cu", "k_attn.cu", "api.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]

@@ -50,12 +50,13 @@ static cudaEvent_t prof_event() {
 struct PhaseMark {
   cudaEvent_t last = nullptr;
   cudaStream_t s;
-  explicit PhaseMark(cudaStream_t st) : s(st) {
-    if (g_prof_on && (last = prof_event()) != nullptr) cudaEventRecord(last, s);
+  bool on;
+  PhaseMark(cudaStream_t st, bool enabled) : s(st), on(enabled && g_prof_on) {
+    if (on && (last = prof_event()) != nullptr) cudaEventRecord(last, s);
   }
   // closes the running phase as `slot` and opens the next one
   void mark(int slot) {
-    if (!g_prof_on || last == nullptr) return;
+    if (!on || last == nullptr) return;
     cudaEvent_t e = prof_event();
     if (e == nullptr) return;
     cudaEventRecord(e, s);
@@ -177,7 +178,7 @@ mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x
   st = gemm_gated_residual(dt, ws.act, w.wfc2, n, H, F, x, mods, stride, 5 * H, plan.block_rows, s);
   if (st != MMH3_OK) return st;
   pm.mark(7);
-  if (g_prof_on) ++g_prof_blocks;
+  if (pm.on) ++g_prof_blocks;
   return MMH3_OK;
 }
 
@@ -199,7 +200,42 @@ mmh3_status common_checks(const mmh3_dims* dims, float* x, int n, const float* p
 
 }  // namespace
 
+// The whole modulated (or unmodulated) block on a caller-provided scratch
+// region; shared by the entry points that take a workspace and by the one
+// that uses the library's own static scratch.  `profile` = false records no
+// phase events.
+mmh3_status mmh3::block_forward_impl(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
+                                     const mmh3_segment* segs, int n_seg, const float* pos_dev, double sigma_v,
+                                     double sigma_a, int modulated, void* workspace, size_t ws_bytes,
+                                     void* stream, bool profile) {
+  Workspace ws;
+  mmh3_status st = common_checks(dims, x, n, pos_dev, workspace, ws_bytes, &ws);
+  if (st != MMH3_OK) return st;
+  st = check_block(*dims, w, modulated != 0);
+  if (st != MMH3_OK) return st;
+  Plan plan;
+  if (modulated) {
+    st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+    if (st != MMH3_OK) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = dims->hidden;
+  PhaseMark pm(s, profile);
+  if (modulated) {
+    cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * H, plan,
+                                 ws.mods, s);
+    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
+  }
+  if (pos_dev) {
+    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  }
+  pm.mark(0);
+  return block_core(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s, pm);
+}
+
 extern "C" {
+
 
 mmh3_status mmh3_workspace_size(const mmh3_dims* dims, int n, size_t* bytes) {
   clear_error();
@@ -257,30 +293,8 @@ mmh3_status mmh3_block_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                                double sigma_a, int modulated, void* workspace, size_t ws_bytes,
                                void* stream) {
   clear_error();
-  Workspace ws;
-  mmh3_status st = common_checks(dims, x, n, pos_dev, workspace, ws_bytes, &ws);
-  if (st != MMH3_OK) return st;
-  st = check_block(*dims, w, modulated != 0);
-  if (st != MMH3_OK) return st;
-  Plan plan;
-  if (modulated) {
-    st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
-    if (st != MMH3_OK) return st;
-  }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int H = dims->hidden;
-  PhaseMark pm(s);
-  if (modulated) {
-    cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * H, plan,
-                                 ws.mods, s);
-    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
-  }
-  if (pos_dev) {
-    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
-  }
-  pm.mark(0);
-  return block_core(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s, pm);
+  return block_forward_impl(dims, w, x, n, segs, n_seg, pos_dev, sigma_v, sigma_a, modulated, workspace,
+                            ws_bytes, stream, /*profile=*/true);
 }
 
 mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* blocks, int n_blocks,
@@ -321,7 +335,7 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                   heads->out_audio);
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  PhaseMark pm(s);
+  PhaseMark pm(s, true);
   if (pos_dev) {
     cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");

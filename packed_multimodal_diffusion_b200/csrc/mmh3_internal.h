@@ -75,6 +75,13 @@ mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, i
 mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads, int head_dim,
                       float scale, void* out, cudaStream_t s);
 
+// The block on a caller-provided scratch region (see mmh3_workspace_size);
+// profile = false records no phase-profile events.
+mmh3_status block_forward_impl(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
+                               const mmh3_segment* segs, int n_seg, const float* pos_dev, double sigma_v,
+                               double sigma_a, int modulated, void* workspace, size_t ws_bytes, void* stream,
+                               bool profile);
+
 // 2-D row-major tensor map, 128-byte swizzle, box {128 bytes, box_rows}.
 bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, uint64_t rows,
                   uint32_t box_rows);
