@@ -65,14 +65,81 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
 }
 
 // ------------------------------------------------------------- epilogues
-// Each epilogue gets: the TMEM address of this thread's accumulator row
-// (column 0 of the tile), the output row index, the tile's first column,
-// and whether the row is inside the matrix.  It must issue every tcgen05.ld
-// even for rows outside the matrix (the loads are warp-collective).
+constexpr int kEpiParts = 1;         // epilogue warp sets (4 warps each)
 
-// qkv projection: per 128-column head of the q and k planes, RMSNorm with
-// the q_norm / k_norm weight, then the partial split-half 3-axis rotation
-// from a per-row (cos, sin) table; the v plane is stored as is.
+template <int BN>
+__device__ __forceinline__ void part_chunks(int part, int& c0, int& c1) {
+  constexpr int nc = BN / 32;
+  constexpr int h = (nc + kEpiParts - 1) / kEpiParts;
+  c0 = part * h;
+  c1 = (part + 1) * h < nc ? (part + 1) * h : nc;
+}
+
+// Epilogue warps: kEpiParts sets of four warps; the warps of one set cover
+// the four TMEM lane quarters (rows), the sets split the tile's columns
+// (`part`).  Contract:
+//   bool operator()(tacc, row, n0, row_ok, part, wait, smem)
+// tacc is the TMEM address of this thread's accumulator row (column 0),
+// `wait()` blocks until the accumulator is complete (false on timeout,
+// warp-uniform); loads that do not depend on the accumulator are issued
+// before it.  Every tcgen05.ld is issued by all 32 lanes, also for rows
+// outside the matrix.  setup() stages small parameters in shared memory.
+
+template <int N>
+__device__ __forceinline__ void ld_acc(uint32_t taddr, float (&v)[N]) {
+  if constexpr (N == 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  } else if constexpr (N == 16) {
+    uint32_t r[16];
+    tmem_ld16(taddr, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  } else {
+    static_assert(N == 8, "8, 16 or 32 columns");
+    uint32_t r[8];
+    tmem_ld8(taddr, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+
+// N consecutive values (N multiple of 8) to dst (16-byte aligned).
+template <int N>
+__device__ __forceinline__ void store_n(__nv_bfloat16* dst, const float (&v)[N]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < N / 8; ++q) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = u;
+  }
+}
+template <int N>
+__device__ __forceinline__ void store_n(float* dst, const float (&v)[N]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+struct NoSetup {
+  static constexpr int kSmemFloats = 0;
+  __device__ __forceinline__ void setup(float*, int, int) const {}
+};
+
+// qkv projection: per head of the q and k planes, RMSNorm with the q_norm /
+// k_norm weight, then the partial split-half 3-axis rotation from a per-row
+// (cos, sin) table; v is stored as is.  Two passes over TMEM: the sum of
+// squares, then the rotation in three groups of G = HD/8 pairs (one position
+// axis each) and the unrotated tail -- small register footprint.
 template <typename T, int HD, int BN>
 struct EpiQkvNormRope {
   T* out;            // [M, N] with N = 3 * inner
@@ -83,134 +150,224 @@ struct EpiQkvNormRope {
   const float2* cs;  // [M, kPairs] (cos, sin), or null: no rotation
   float eps;
   static constexpr int kPairs = 3 * (HD / 8);
+  static constexpr int kG = HD / 8;
+  static constexpr int kSmemFloats = 2 * HD;
 
-  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+  __device__ __forceinline__ void setup(float* sm, int tid, int nthreads) const {
+    for (int i = tid; i < 2 * HD; i += nthreads) sm[i] = i < HD ? q_norm[i] : k_norm[i - HD];
+  }
+
+  template <class Wait>
+  __device__ __forceinline__ bool operator()(uint32_t tacc, int row, int n0, bool row_ok, int part,
+                                             Wait&& wait, const float* sm) const {
+    constexpr int kHeadsPerPart = BN / HD / kEpiParts;
+    if (!wait()) return false;
 #pragma unroll 1
-    for (int g = 0; g < BN / HD; ++g) {
+    for (int hh = 0; hh < kHeadsPerPart; ++hh) {
+      const int g = part * kHeadsPerPart + hh;
       const int col0 = n0 + g * HD;
       if (col0 >= N) break;  // uniform across the warp
-      float v[HD];
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        float t[32];
-        ld_acc32(tacc + g * HD + c * 32, t);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[c * 32 + i] = t[i];
-      }
+      const uint32_t th = tacc + g * HD;
+      T* dst = out + (size_t)row * N + col0;
       const int which = col0 / inner;  // 0 q, 1 k, 2 v
-      if (which < 2) {
-        const float* w = which == 0 ? q_norm : k_norm;
-        float ss = 0.f;
+      if (which == 2) {
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          float v[32];
+          ld_acc<32>(th + c * 32, v);
+          if (row_ok) store_n<32>(dst + c * 32, v);
+        }
+        continue;
+      }
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float v[32];
+        ld_acc<32>(th + c * 32, v);
 #pragma unroll
-        for (int d = 0; d < HD; ++d) ss = fmaf(v[d], v[d], ss);
-        const float inv = rsqrtf(ss * (1.0f / HD) + eps);
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+      }
+      const float inv = rsqrtf(ss * (1.0f / HD) + eps);
+      const float* w = sm + which * HD;
+      if (cs != nullptr) {
+#pragma unroll 1
+        for (int a = 0; a < 3; ++a) {
+          const int j0 = a * kG;
+          float lo[kG], hi[kG];
+          ld_acc<kG>(th + j0, lo);
+          ld_acc<kG>(th + j0 + kPairs, hi);
+          if (row_ok) {
+            const float2* c2 = cs + (size_t)row * kPairs + j0;
 #pragma unroll
-        for (int d = 0; d < HD; ++d) v[d] = v[d] * inv * __ldg(w + d);
-        if (cs != nullptr && row_ok) {
-          const float2* c2 = cs + (size_t)row * kPairs;
+            for (int i = 0; i < kG; ++i) {
+              const float2 e = __ldg(c2 + i);
+              const float yl = lo[i] * inv * w[j0 + i];
+              const float yh = hi[i] * inv * w[j0 + kPairs + i];
+              lo[i] = yl * e.x - yh * e.y;
+              hi[i] = yl * e.y + yh * e.x;
+            }
+            store_n<kG>(dst + j0, lo);
+            store_n<kG>(dst + j0 + kPairs, hi);
+          }
+        }
+        constexpr int kTail = HD - 2 * kPairs;  // 32 of 128, 16 of 64
+        float t[kTail];
+        ld_acc<kTail>(th + 2 * kPairs, t);
+        if (row_ok) {
 #pragma unroll
-          for (int j = 0; j < kPairs; ++j) {
-            const float2 a = __ldg(c2 + j);
-            const float lo = v[j], hi = v[j + kPairs];
-            v[j] = lo * a.x - hi * a.y;
-            v[j + kPairs] = lo * a.y + hi * a.x;
+          for (int i = 0; i < kTail; ++i) t[i] = t[i] * inv * w[2 * kPairs + i];
+          store_n<kTail>(dst + 2 * kPairs, t);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          float v[32];
+          ld_acc<32>(th + c * 32, v);
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = v[i] * inv * w[c * 32 + i];
+            store_n<32>(dst + c * 32, v);
           }
         }
       }
-      if (row_ok) {
-        T* dst = out + (size_t)row * N + col0;
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          float t[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) t[i] = v[c * 32 + i];
-          store32(dst + c * 32, t);
-        }
-      }
     }
+    return true;
   }
 };
 
-// x[row, :] += gate[row] * acc : the gated residual.  gate is chunk `chunk`
-// of the token's modulation row (row id from the segment table).  With
-// mods == null the residual is plain (x += acc).
-template <int BN>
-struct EpiGatedResidual {
+
+
+// x[row, :] += gate[row] * acc (the gated residual; gate = chunk of the
+// token's modulation row, found through the segment table), or x += acc when
+// mods is null, or x += acc + bias (the encoder layer's biased residual).
+// The x and gate/bias values of a chunk are loaded before the accumulator
+// chunk is read, and the next chunk's before the current one is stored.
+template <int BN, bool BIAS>
+struct EpiResidual : NoSetup {
   float* x;          // [M, N] fp32, in place
   int N;
-  const float* mods; // [rows, mods_stride] or null
+  const float* mods; // [rows, mods_stride] or null (gated form)
   int mods_stride;
   int chunk_off;     // chunk * hidden
   SegRows seg;
+  const float* bias; // [N] (biased form)
 
-  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
-    const float* gate = nullptr;
-    if (mods != nullptr) gate = mods + (size_t)seg_row(seg, row) * mods_stride + chunk_off;
+  __device__ __forceinline__ void load_x(int row, int col, bool row_ok, float4 (&xv)[8]) const {
+    if (row_ok) {
+      const float4* xp = reinterpret_cast<const float4*>(x + (size_t)row * N + col);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) xv[q] = xp[q];
+    }
+  }
+
+  template <class Wait>
+  __device__ __forceinline__ bool operator()(uint32_t tacc, int row, int n0, bool row_ok, int part,
+                                             Wait&& wait, const float*) const {
+    const float* g = nullptr;
+    if (BIAS) g = bias;
+    else if (mods != nullptr) g = mods + (size_t)seg_row(seg, row) * mods_stride + chunk_off;
+    int c0, c1;
+    part_chunks<BN>(part, c0, c1);
+    float4 xa[8];
+    if (c0 < c1 && n0 + c0 * 32 < N) load_x(row, n0 + c0 * 32, row_ok, xa);
+    if (!wait()) return false;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c0; c < c1; ++c) {
       const int col = n0 + c * 32;
       if (col >= N) break;
+      float4 gv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        gv[q] = g ? __ldg(reinterpret_cast<const float4*>(g + col) + q) : make_float4(1.f, 1.f, 1.f, 1.f);
       float v[32];
-      ld_acc32(tacc + c * 32, v);
+      ld_acc<32>(tacc + c * 32, v);
+      float4 xb[8];
+      const bool next = c + 1 < c1 && col + 32 < N;
+      if (next) load_x(row, col + 32, row_ok, xb);
       if (row_ok) {
         float4* xp = reinterpret_cast<float4*>(x + (size_t)row * N + col);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          float4 xv = xp[q];
-          float4 gv = gate ? __ldg(reinterpret_cast<const float4*>(gate + col) + q)
-                           : make_float4(1.f, 1.f, 1.f, 1.f);
-          xv.x = fmaf(gv.x, v[4 * q + 0], xv.x);
-          xv.y = fmaf(gv.y, v[4 * q + 1], xv.y);
-          xv.z = fmaf(gv.z, v[4 * q + 2], xv.z);
-          xv.w = fmaf(gv.w, v[4 * q + 3], xv.w);
-          xp[q] = xv;
+          float4 o = xa[q];
+          if (BIAS) {
+            o.x += v[4 * q + 0] + gv[q].x;
+            o.y += v[4 * q + 1] + gv[q].y;
+            o.z += v[4 * q + 2] + gv[q].z;
+            o.w += v[4 * q + 3] + gv[q].w;
+          } else {
+            o.x = fmaf(gv[q].x, v[4 * q + 0], o.x);
+            o.y = fmaf(gv[q].y, v[4 * q + 1], o.y);
+            o.z = fmaf(gv[q].z, v[4 * q + 2], o.z);
+            o.w = fmaf(gv[q].w, v[4 * q + 3], o.w);
+          }
+          xp[q] = o;
         }
       }
+      if (next) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) xa[q] = xb[q];
+      }
     }
+    return true;
   }
 };
+
+template <int BN>
+using EpiGatedResidual = EpiResidual<BN, false>;
+template <int BN>
+using EpiBiasResidual = EpiResidual<BN, true>;
 
 // fc1 + SwiGLU: the weight rows are interleaved so that tile columns
 // [0, BN/2) are gate rows and [BN/2, BN) the matching up rows; the output
 // column block is n0 / 2.
 template <typename T, int BN>
-struct EpiSwiGLU {
+struct EpiSwiGLU : NoSetup {
   T* out;  // [M, F]
   int F;
 
-  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+  template <class Wait>
+  __device__ __forceinline__ bool operator()(uint32_t tacc, int row, int n0, bool row_ok, int part,
+                                             Wait&& wait, const float*) const {
+    if (!wait()) return false;
+    constexpr int np = BN / 64;  // chunk pairs
     const int f0 = n0 / 2;
 #pragma unroll 1
-    for (int c = 0; c < BN / 64; ++c) {
+    for (int c = part * (np / kEpiParts); c < (part + 1) * (np / kEpiParts); ++c) {
       const int f = f0 + c * 32;
       if (f >= F) break;
-      float g[32], u[32];
-      ld_acc32(tacc + c * 32, g);
-      ld_acc32(tacc + BN / 2 + c * 32, u);
+      float gt[32], u[32];
+      ld_acc<32>(tacc + c * 32, gt);
+      ld_acc<32>(tacc + BN / 2 + c * 32, u);
       if (row_ok) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
-        store32(out + (size_t)row * F + f, g);
+        for (int i = 0; i < 32; ++i) gt[i] = silu_f(gt[i]) * u[i];
+        store_n<32>(out + (size_t)row * F + f, gt);
       }
     }
+    return true;
   }
 };
 
 // out = act(acc + bias) for the unmodulated encoder layer and the output
 // heads.  MODE 0: identity, 1: tanh-GELU, 2: negate (velocity sign).
 template <typename T, int BN, int MODE>
-struct EpiBiasAct {
+struct EpiBiasAct : NoSetup {
   T* out;
   int N;
   const float* bias;
 
-  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
+  template <class Wait>
+  __device__ __forceinline__ bool operator()(uint32_t tacc, int row, int n0, bool row_ok, int part,
+                                             Wait&& wait, const float*) const {
+    if (!wait()) return false;
+    int c0, c1;
+    part_chunks<BN>(part, c0, c1);
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c0; c < c1; ++c) {
       const int col = n0 + c * 32;
       if (col >= N) break;
       float v[32];
-      ld_acc32(tacc + c * 32, v);
+      ld_acc<32>(tacc + c * 32, v);
       if (row_ok) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -219,40 +376,10 @@ struct EpiBiasAct {
           if (MODE == 2) t = -t;
           v[i] = t;
         }
-        store32(out + (size_t)row * N + col, v);
+        store_n<32>(out + (size_t)row * N + col, v);
       }
     }
-  }
-};
-
-// x += acc + bias : residual with the projection's bias folded in.
-template <int BN>
-struct EpiBiasResidual {
-  float* x;
-  int N;
-  const float* bias;
-
-  __device__ __forceinline__ void operator()(uint32_t tacc, int row, int n0, bool row_ok) const {
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      const int col = n0 + c * 32;
-      if (col >= N) break;
-      float v[32];
-      ld_acc32(tacc + c * 32, v);
-      if (row_ok) {
-        float4* xp = reinterpret_cast<float4*>(x + (size_t)row * N + col);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float4 xv = xp[q];
-          const float4 bv = __ldg(reinterpret_cast<const float4*>(bias + col) + q);
-          xv.x += v[4 * q + 0] + bv.x;
-          xv.y += v[4 * q + 1] + bv.y;
-          xv.z += v[4 * q + 2] + bv.z;
-          xv.w += v[4 * q + 3] + bv.w;
-          xp[q] = xv;
-        }
-      }
-    }
+    return true;
   }
 };
 
@@ -282,13 +409,16 @@ struct GemmShape {
                                    : (2 * BN <= 256) ? 256 : 512;
 };
 
+constexpr int kEpiSmemBytes = 2048;  // staged epilogue parameters
+constexpr int kGemmThreads = 64 + 128 * kEpiParts;  // producer, MMA, epilogue
+
 template <int BN, int STAGES>
 constexpr int gemm_smem_bytes() {
-  return STAGES * GemmShape<BN>::kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  return STAGES * GemmShape<BN>::kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiSmemBytes;
 }
 
 template <typename T, int BN, int STAGES, class Epi>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, Epi epi, DevStatus* status, uint64_t limit_ns) {
   using Sh = GemmShape<BN>;
@@ -303,6 +433,8 @@ __global__ void __launch_bounds__(192, 1)
   // TMEM address slot and the CTA's abort flag
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_smem = reinterpret_cast<float*>(smem + STAGES * Sh::kStageBytes + 256);
+  static_assert(Epi::kSmemFloats * 4 <= kEpiSmemBytes, "epilogue parameters exceed their smem area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -321,7 +453,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
+      mbar_init(tempty_bar(a), 32 * (kGemmThreads / 32 - 2));
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -330,6 +462,7 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch(&tmB);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Sh::kTmemCols);
+  if (warp >= 2) epi.setup(epi_smem, threadIdx.x - 64, kGemmThreads - 64);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
@@ -436,24 +569,29 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5 (TMEM lane groups 2,3,0,1)
+    // ---------------- epilogue warps 2..9: lane quarter warp % 4, column
+    // half (warp - 2) / 4
     const int lgrp = warp & 3;
+    const int part = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(lgrp * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       int mt, nt;
-        tile_coords(tile, m_tiles, n_tiles, mt, nt);
-      // warp-uniform decision: the epilogue's TMEM loads are warp-collective
-      const bool fail = *abort_flag || !mbar_wait(tfull_bar(acc), acc_phase, limit_ns);
-      if (__any_sync(0xffffffffu, fail)) {
-        if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_EPILOGUE, tile);
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
+      tile_coords(tile, m_tiles, n_tiles, mt, nt);
       const int row = mt * Sh::BM + lgrp * 32 + lane;
-      epi(tmem_base + acc * BN + lane_off, row, nt * BN, row < M);
+      // warp-uniform: the epilogue's TMEM loads are warp-collective
+      auto wait = [&]() -> bool {
+        const bool fail = *abort_flag || !mbar_wait(tfull_bar(acc), acc_phase, limit_ns);
+        if (__any_sync(0xffffffffu, fail)) {
+          if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_EPILOGUE, tile);
+          *abort_flag = 1;
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      if (!epi(tmem_base + acc * BN + lane_off, row, nt * BN, row < M, part, wait, epi_smem)) break;
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
       if (++acc == 2) {

@@ -72,7 +72,7 @@ static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, c
   const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
-  kern<<<grid, 192, smem, s>>>(ta, tb, M, N, K, epi, device_status_ptr(), wait_limit_ns());
+  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, M, N, K, epi, device_status_ptr(), wait_limit_ns());
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return MMH3_OK;
@@ -106,31 +106,31 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
                                 const SegRows& seg, cudaStream_t s) {
   if (dtype == MMH3_BF16) {
     if (N % 256 == 0) {
-      EpiGatedResidual<256> e{x, N, mods, mods_stride, chunk_off, seg};
+      EpiGatedResidual<256> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
       return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
     }
     if (N % 224 == 0) {
-      EpiGatedResidual<224> e{x, N, mods, mods_stride, chunk_off, seg};
+      EpiGatedResidual<224> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
       return run_gemm<__nv_bfloat16, 224>(A, B, M, N, K, e, s);
     }
-    EpiGatedResidual<128> e{x, N, mods, mods_stride, chunk_off, seg};
+    EpiGatedResidual<128> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
     return run_gemm<__nv_bfloat16, 128>(A, B, M, N, K, e, s);
   }
   if (N % 256 == 0) {
-    EpiGatedResidual<256> e{x, N, mods, mods_stride, chunk_off, seg};
+    EpiGatedResidual<256> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
     return run_gemm<float, 256>(A, B, M, N, K, e, s);
   }
-  EpiGatedResidual<128> e{x, N, mods, mods_stride, chunk_off, seg};
+  EpiGatedResidual<128> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
   return run_gemm<float, 128>(A, B, M, N, K, e, s);
 }
 
 mmh3_status gemm_swiglu(int dtype, const void* A, const void* B, int M, int F, int K, void* out,
                         cudaStream_t s) {
   if (dtype == MMH3_BF16) {
-    EpiSwiGLU<__nv_bfloat16, 256> e{static_cast<__nv_bfloat16*>(out), F};
+    EpiSwiGLU<__nv_bfloat16, 256> e{{}, static_cast<__nv_bfloat16*>(out), F};
     return run_gemm<__nv_bfloat16, 256>(A, B, M, 2 * F, K, e, s);
   }
-  EpiSwiGLU<float, 256> e{static_cast<float*>(out), F};
+  EpiSwiGLU<float, 256> e{{}, static_cast<float*>(out), F};
   return run_gemm<float, 256>(A, B, M, 2 * F, K, e, s);
 }
 
@@ -138,25 +138,25 @@ mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N,
                           const float* bias, int mode, void* out, cudaStream_t s) {
   if (mode == 2) {  // output heads: fp32, negated, N = 128-wide tiles
     if (dtype == MMH3_BF16) {
-      EpiBiasAct<float, 128, 2> e{static_cast<float*>(out), N, bias};
+      EpiBiasAct<float, 128, 2> e{{}, static_cast<float*>(out), N, bias};
       return run_gemm<__nv_bfloat16, 128>(A, B, M, N, K, e, s);
     }
-    EpiBiasAct<float, 128, 2> e{static_cast<float*>(out), N, bias};
+    EpiBiasAct<float, 128, 2> e{{}, static_cast<float*>(out), N, bias};
     return run_gemm<float, 128>(A, B, M, N, K, e, s);
   }
   if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias/gelu epilogue: bf16 only");
   if (mode == 1) {
-    EpiBiasAct<__nv_bfloat16, 256, 1> e{static_cast<__nv_bfloat16*>(out), N, bias};
+    EpiBiasAct<__nv_bfloat16, 256, 1> e{{}, static_cast<__nv_bfloat16*>(out), N, bias};
     return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
   }
-  EpiBiasAct<__nv_bfloat16, 256, 0> e{static_cast<__nv_bfloat16*>(out), N, bias};
+  EpiBiasAct<__nv_bfloat16, 256, 0> e{{}, static_cast<__nv_bfloat16*>(out), N, bias};
   return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
 }
 
 mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,
                                const float* bias, float* x, cudaStream_t s) {
   if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias residual epilogue: bf16 only");
-  EpiBiasResidual<256> e{x, N, bias};
+  EpiBiasResidual<256> e{{}, x, N, nullptr, 0, 0, SegRows{}, bias};
   return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
 }
 
