@@ -1,0 +1,324 @@
+// Bidirectional flash attention on tcgen05, two query tiles per CTA.
+//
+// One CTA computes two 128-row query tiles (256 rows) of one head, so each
+// K/V tile fetched by TMA serves 256 query rows.  Tensor memory (512
+// columns) holds S0 | S1 | O0 | O1.
+//   warp 0      TMA producer: Q0 and Q1 once, then K_j / V_j (two stages)
+//   warp 1      MMA issuer: S0 = Q0 K_0^T, S1 = Q1 K_0^T, then per key tile
+//               j: O0 += P0 V_j (once P0 is written), S0 = Q0 K_{j+1}^T,
+//               O1 += P1 V_j (once P1 is written), S1 = Q1 K_{j+1}^T
+//               P_i (bf16) is read as the A operand straight from tensor
+//               memory, where softmax warpgroup i wrote it over the first 64
+//               columns of S_i.  MMAs of one thread run in issue order, so
+//               S_i(j+1) (issued after O_i += P_i V_j) cannot overwrite P_i
+//               before that product has read it; and the commit that
+//               signals S_i(j+1) also covers O_i += P_i V_j, so O_i is
+//               stable when softmax i sees S_i(j+1).
+//   warps 2..5  softmax of tile 0, warps 6..9 softmax of tile 1: thread r
+//               owns query row r; running maximum in the log2 domain, O
+//               rescaled only when the maximum grows by more than 2^8 (the
+//               final division uses the same reference maximum, so a stale
+//               maximum is exact up to rounding); late normalisation in the
+//               epilogue.
+// While softmax 1 works on S1(j) the tensor core computes O0 += P0 V_j and
+// S0(j+1); while softmax 0 works on S0(j+1) it computes O1 += P1 V_j and
+// S1(j+1).
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace mmh3 {
+
+template <int HD>
+struct Attn2Shape {
+  static constexpr int kBoxBytes = 128 * 128;   // 128 rows x 128 bytes
+  static constexpr int kHdBoxes = HD / 64;      // bf16 boxes across a head
+  static constexpr int kTileBytes = kHdBoxes * kBoxBytes;
+  static constexpr int kKV = 2;                 // K / V stages
+  static constexpr int kQOff = 0;               // Q0 then Q1
+  static constexpr int kKOff = 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kKV * kTileBytes;
+  static constexpr int kBarOff = kVOff + kKV * kTileBytes;
+  static constexpr int kSmem = kBarOff + 512 + 1024;
+  static constexpr int kThreads = 320;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(320, 1)
+    attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, __nv_bfloat16* __restrict__ out, int ldo,
+                    int seq, int inner, float scale_log2, DevStatus* status, uint64_t limit_ns) {
+  using Sh = Attn2Shape<HD>;
+  constexpr int KV = Sh::kKV;
+  constexpr uint32_t kIdescS = make_idesc(false, 128, 128, false, false);
+  constexpr uint32_t kIdescO = make_idesc(false, 128, HD, false, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::kBarOff);
+  constexpr int B_Q = 0;
+  constexpr int B_KF = 1, B_KE = B_KF + KV, B_VF = B_KE + KV, B_VE = B_VF + KV;
+  constexpr int B_SF = B_VE + KV, B_PF = B_SF + 2, B_OF = B_PF + 2, B_DRAIN = B_OF + 1;
+  constexpr int kNumBars = B_DRAIN + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(bars);
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+
+  const int head = blockIdx.y;
+  const int seq_row0 = blockIdx.z * seq;
+  const int q_row0 = seq_row0 + blockIdx.x * 256;
+  const int n_kv = (seq + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_Q), 1);
+    for (int s = 0; s < KV; ++s) {
+      mbar_init(bar(B_KF + s), 1);
+      mbar_init(bar(B_KE + s), 1);
+      mbar_init(bar(B_VF + s), 1);
+      mbar_init(bar(B_VE + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_SF + i), 1);
+      mbar_init(bar(B_PF + i), 128);
+    }
+    mbar_init(bar(B_OF), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch(&tm);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // S_i at columns 128 i, O_i at 256 + HD i
+  auto t_s = [&](int i) { return tmem + 128u * i; };
+  auto t_o = [&](int i) { return tmem + 256u + (uint32_t)HD * i; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      const int xq = head * HD, xk = inner + head * HD, xv = 2 * inner + head * HD;
+      int in_k = 0, in_v = 0;
+      bool ok = true;
+      mbar_expect_tx(bar(B_Q), 2 * Sh::kTileBytes);
+      for (int i = 0; i < 2; ++i)
+        for (int c = 0; c < Sh::kHdBoxes; ++c)
+          tma_load_2d(sbase + Sh::kQOff + i * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_Q),
+                      xq + c * 64, q_row0 + 128 * i);
+      int j = 0;
+      for (; j < n_kv && ok; ++j) {
+        const int s = j % KV;
+        const uint32_t ph = (uint32_t)((j / KV) & 1);
+        const int y = seq_row0 + j * 128;
+        if (*abort_flag || !mbar_wait(bar(B_KE + s), ph ^ 1u, limit_ns)) { ok = false; break; }
+        mbar_expect_tx(bar(B_KF + s), Sh::kTileBytes);
+        for (int c = 0; c < Sh::kHdBoxes; ++c)
+          tma_load_2d(sbase + Sh::kKOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_KF + s),
+                      xk + c * 64, y);
+        in_k = j + 1;
+        if (*abort_flag || !mbar_wait(bar(B_VE + s), ph ^ 1u, limit_ns)) { ok = false; break; }
+        mbar_expect_tx(bar(B_VF + s), Sh::kTileBytes);
+        for (int c = 0; c < Sh::kHdBoxes; ++c)
+          tma_load_2d(sbase + Sh::kVOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_VF + s),
+                      xv + c * 64, y);
+        in_v = j + 1;
+      }
+      if (!ok) {
+        if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, j);
+        *abort_flag = 1;
+        mbar_wait(bar(B_Q), 0, limit_ns);
+        for (int i = (in_k > KV ? in_k - KV : 0); i < in_k; ++i)
+          mbar_wait(bar(B_KF + i % KV), (uint32_t)((i / KV) & 1), limit_ns);
+        for (int i = (in_v > KV ? in_v - KV : 0); i < in_v; ++i)
+          mbar_wait(bar(B_VF + i % KV), (uint32_t)((i / KV) & 1), limit_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      // Order: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+      // S_i(j+1) goes right after PV_i(j), so the tensor core computes
+      // S0(j+1) while softmax 1 still works on S1(j).
+      auto issue_s = [&](int i, int j) {
+        const uint32_t ka = sbase + Sh::kKOff + (j % KV) * Sh::kTileBytes;
+        const uint32_t qa = sbase + Sh::kQOff + i * Sh::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t off = (ks / 4) * Sh::kBoxBytes + (ks % 4) * 32;
+          umma_ss<false>(t_s(i), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), kIdescS,
+                         ks > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(B_SF + i));
+      };
+      auto issue_pv = [&](int i, int j) {
+        const uint32_t va = sbase + Sh::kVOff + (j % KV) * Sh::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < 128 / 16; ++ks) {
+          const uint64_t bd = sdesc_sw128(va + ks * 16 * 128, Sh::kBoxBytes, 1024);
+          umma_ts(t_o(i), t_s(i) + ks * 8, bd, kIdescO, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_kf = [&](int j) {
+        return !*abort_flag && mbar_wait(bar(B_KF + j % KV), (uint32_t)((j / KV) & 1), limit_ns);
+      };
+      bool ok = mbar_wait(bar(B_Q), 0, limit_ns) && wait_kf(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(bar(B_KE + 0));
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j % KV;
+        const uint32_t pj = (uint32_t)(j & 1);
+        const bool more = j + 1 < n_kv;
+        if (*abort_flag || !mbar_wait(bar(B_VF + s), (uint32_t)((j / KV) & 1), limit_ns)) { ok = false; break; }
+        if (*abort_flag || !mbar_wait(bar(B_PF + 0), pj, limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!wait_kf(j + 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (*abort_flag || !mbar_wait(bar(B_PF + 1), pj, limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(bar(B_VE + s));
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(bar(B_KE + (j + 1) % KV));
+        }
+      }
+      if (ok) umma_commit(bar(B_OF));
+      if (!ok) {
+        if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, blockIdx.x);
+        *abort_flag = 1;
+        umma_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, limit_ns);
+      }
+    }
+  } else {
+    // -------------------------------------------------- softmax warpgroups
+    const int wg = (warp - 2) >> 2;       // query tile
+    const int lgrp = warp & 3;            // TMEM lane quarter
+    const int r = lgrp * 32 + lane;       // row within the tile
+    const uint32_t lane_off = (uint32_t)(lgrp * 32) << 16;
+    const uint32_t ts = t_s(wg) + lane_off;
+    const uint32_t to = t_o(wg) + lane_off;
+    float m_ref = 0.f, l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      {
+        const bool fail = *abort_flag || !mbar_wait(bar(B_SF + wg), (uint32_t)(j & 1), limit_ns);
+        if (__any_sync(0xffffffffu, fail)) { ok = false; break; }
+      }
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tmem_ld32(ts + 0, u0);
+        tmem_ld32(ts + 32, u1);
+        tmem_ld32(ts + 64, u2);
+        tmem_ld32(ts + 96, u3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(u0[i]);
+          s[32 + i] = __uint_as_float(u1[i]);
+          s[64 + i] = __uint_as_float(u2[i]);
+          s[96 + i] = __uint_as_float(u3[i]);
+        }
+      }
+      const int valid = seq - j * 128;
+      if (valid < 128) {
+#pragma unroll
+        for (int k = 0; k < 128; ++k)
+          if (k >= valid) s[k] = -INFINITY;
+      }
+      float pm[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pm[i] = s[i];
+#pragma unroll
+      for (int k = 8; k < 128; ++k) pm[k & 7] = fmaxf(pm[k & 7], s[k]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      const float m_tile = mx * scale_log2;
+      if (j == 0) {
+        m_ref = m_tile;
+      } else {
+        const bool need = m_tile > m_ref + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          // O_i holds every earlier product (see the kernel comment).
+          const float m_new = need ? m_tile : m_ref;
+          const float f = ex2_approx(m_ref - m_new);
+          l_sum *= f;
+          m_ref = m_new;
+#pragma unroll 1
+          for (int c = 0; c < HD / 16; ++c) {
+            uint32_t u[16];
+            tmem_ld16(to + c * 16, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i2 = 0; i2 < 16; ++i2) u[i2] = __float_as_uint(__uint_as_float(u[i2]) * f);
+            tmem_st16(to + c * 16, u);
+          }
+        }
+      }
+      // P = 2^(s * scale * log2e - m_ref) as bf16 pairs over S_i's first 64
+      // columns, in four slices of 32 keys (16 columns).
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int k = h * 32 + 2 * q;
+          const float p0 = ex2_approx(fmaf(s[k], scale_log2, -m_ref));
+          const float p1 = ex2_approx(fmaf(s[k + 1], scale_log2, -m_ref));
+          ps[q & 3] += p0 + p1;
+          pk[q] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(ts + h * 16, pk);
+      }
+      l_sum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PF + wg));
+    }
+    if (ok) {
+      const bool fail = *abort_flag || !mbar_wait(bar(B_OF), 0, limit_ns);
+      if (__any_sync(0xffffffffu, fail)) ok = false;
+    }
+    if (!ok) {
+      if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_SOFTMAX, blockIdx.x);
+      *abort_flag = 1;
+    }
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
+      const int qr = blockIdx.x * 256 + wg * 128 + r;
+      const bool row_ok = qr < seq;
+      __nv_bfloat16* dst = out + (size_t)(seq_row0 + qr) * ldo + head * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float v[32];
+        ld_acc32(to + c * 32, v);
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) v[i2] *= inv;
+        if (row_ok) store32(dst + c * 32, v);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace mmh3
