@@ -2,10 +2,8 @@
 // attention: full bidirectional softmax attention per head over the packed
 // sequence; "ffai-argus 0.7.0 src/siglip.rs": attention inside each image).
 #include <cmath>
-#include <cstdlib>
 
 #include "attn2_tc.cuh"
-#include "attn_tc.cuh"
 #include "mmh3_internal.h"
 
 namespace mmh3 {
@@ -72,28 +70,6 @@ static mmh3_status run_attn_f32(const void* qkv, int n_seq, int seq, int heads, 
   return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "fp32 attention launch");
 }
 
-template <typename T, int HD, int KV, int PB>
-static mmh3_status run_attn(const void* qkv, int n_seq, int seq, int heads, float scale, void* out,
-                            cudaStream_t s) {
-  using Sh = AttnShape<T, HD, KV, PB>;
-  static_assert(Sh::kSmem <= 232448, "attention shared memory above the per-CTA limit");
-  const int inner = heads * HD;
-  const int rows = n_seq * seq;
-  CUtensorMap tm;
-  if (!make_tmap_2d(&tm, qkv, (int)sizeof(T), (uint64_t)(3 * inner), (uint64_t)rows, 128))
-    return fail(MMH3_ERR_CUDA, "attention: cuTensorMapEncodeTiled failed");
-  auto kern = attn_tc_kernel<T, HD, KV, PB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmem);
-  if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
-  dim3 grid((seq + 127) / 128, heads, n_seq);
-  const float scale_log2 = scale * 1.4426950408889634f;
-  kern<<<grid, 192, Sh::kSmem, s>>>(tm, static_cast<T*>(out), inner, seq, inner, scale_log2,
-                                    device_status_ptr(), wait_limit_ns());
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-  return MMH3_OK;
-}
-
 template <int HD>
 static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, int heads, float scale, void* out,
                              cudaStream_t s) {
@@ -119,16 +95,8 @@ mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads,
   if (n_seq <= 0 || seq <= 0) return MMH3_OK;
   if ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "attention: pointer not 16-byte aligned");
-  static const bool v1 = [] {
-    const char* e = std::getenv("MMH3_ATTN_V1");
-    return e != nullptr && e[0] == '1';
-  }();
-  if (dtype == MMH3_BF16 && head_dim == 128)
-    return v1 ? run_attn<__nv_bfloat16, 128, 2, 2>(qkv, n_seq, seq, heads, scale, out, s)
-              : run_attn2<128>(qkv, n_seq, seq, heads, scale, out, s);
-  if (dtype == MMH3_BF16 && head_dim == 64)
-    return v1 ? run_attn<__nv_bfloat16, 64, 2, 2>(qkv, n_seq, seq, heads, scale, out, s)
-              : run_attn2<64>(qkv, n_seq, seq, heads, scale, out, s);
+  if (dtype == MMH3_BF16 && head_dim == 128) return run_attn2<128>(qkv, n_seq, seq, heads, scale, out, s);
+  if (dtype == MMH3_BF16 && head_dim == 64) return run_attn2<64>(qkv, n_seq, seq, heads, scale, out, s);
   if (dtype == MMH3_F32 && head_dim == 64) return run_attn_f32<64>(qkv, n_seq, seq, heads, scale, out, s);
   return fail(MMH3_ERR_SHAPE, "attention: dtype %d head_dim %d unsupported", dtype, head_dim);
 }
