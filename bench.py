@@ -48,6 +48,10 @@ def parse():
     p.add_argument("--impl", default="b200", choices=["b200", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=128)
+    p.add_argument("--workload", default="block", choices=["block", "stack", "image", "siglip", "tiny"],
+                   help="block (default) prints the benchmark line; the others print one JSON line "
+                        "each for the remaining workloads (stack: 50 blocks + heads, image: 50 "
+                        "blocks, siglip: one encoder layer x 32 images, tiny: fp32 block)")
     return p.parse_args()
 
 
@@ -121,6 +125,24 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# -------------------------------------------------- ncu traffic of a kernel
+def measured_traffic(profile: str, source: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    recorded in a profiles/ summary, or None when the kernel source has
+    changed since that capture (the summary carries the source's sha256)."""
+    import hashlib
+    import re
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        m = re.search(r"traffic_bytes_per_launch:\s*(\d+)\s+source_sha256:\s*([0-9a-f]{64})", text)
+        digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
+        if m and m.group(2) == digest:
+            return int(m.group(1))
+    except OSError:
+        pass
+    return None
 
 
 # ------------------------------------------------------- algorithmic work
@@ -249,6 +271,10 @@ def run_gpu(args):
     per_launch = {k: v / max(1, nblocks) for k, v in phases.items() if v > 0}
     dom = max(("attention", "qkv gemm", "out gemm", "fc1 gemm", "fc2 gemm"),
               key=lambda k: per_launch.get(k, 0.0))
+    traffic = None
+    if dom == "attention":
+        traffic = measured_traffic("attn2_block_13248.md",
+                                   "packed_multimodal_diffusion_b200/csrc/attn2_tc.cuh")
     peaks = load_peaks()
     achieved = flops[dom] / (per_launch[dom] / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
@@ -266,7 +292,8 @@ def run_gpu(args):
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
-                     "traffic": None},
+                     "traffic": traffic, "traffic_unit": "bytes/launch",
+                     "algorithmic_bytes": 2 * n * 3 * 2688 + 2 * n * 2688},
         "phases_ms_per_block": {k: round(v / max(1, nblocks), 4) for k, v in phases.items()},
         "phase_frac_of_peak": {k: round(flops[k] / (per_launch[k] / 1e3) / 1e12 / peak, 4)
                                for k in flops if k in per_launch},
@@ -374,10 +401,111 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------- other workloads
+def _time(fn, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_workload(args):
+    """One JSON line for the stack, image, SigLIP or tiny workload (device-timed
+    with CUDA events, weights generated on the device from the seeded streams,
+    per-phase profile over the timed steps)."""
+    import numpy as np
+    import torch
+
+    from packed_multimodal_diffusion_b200 import api, configs
+    torch.cuda.set_device(0)
+    dev = "cuda"
+    steps, warmup = max(1, args.steps), max(1, args.warmup)
+    peaks = load_peaks()
+    line = {"workload": args.workload, "data": "synthetic", "steps": steps, "warmup": warmup}
+    if args.workload == "siglip":
+        c = configs.SIGLIP
+        d = api.vit_dims(c.hidden, c.heads, c.head_dim, c.mlp, c.ln_eps)
+        params = api.VitParams.from_host(d, configs.vit_weights(c, device=dev), device=dev)
+        x = configs.vit_inputs(c, device=dev)
+        ws = torch.empty(api.vit_workspace_size(d, c.batch, c.seq), dtype=torch.uint8, device=dev)
+        ms = _time(lambda: api.vit_layer_forward(d, params, x, c.batch, c.seq, ws), steps, warmup)
+        api.device_status()
+        rows = c.batch * c.seq
+        flop = 2.0 * rows * c.hidden * (3 * c.hidden + c.hidden + 2 * c.mlp) + 4.0 * c.batch * c.seq ** 2 * c.hidden
+        line.update(metric="SigLIP encoder layer time (bf16, 1 B200)", value=ms, unit="ms/layer",
+                    higher_is_better=False, dtype="bf16", tokens_per_s=rows / (ms / 1e3),
+                    tflops_per_s=flop / (ms / 1e3) / 1e12,
+                    config={"workload": "SigLIP layer: 32 images x 1024 tokens, hidden 768, 12x64 heads, "
+                                        "MLP 3072 tanh-GELU, LayerNorm pre-norm"},
+                    context="the pages quote 61.9 ms/layer for batch 1 on an unnamed CPU")
+        print(json.dumps(line), flush=True)
+        return
+    c = {"stack": configs.STACK, "image": configs.IMAGE, "tiny": configs.TINY}[args.workload]
+    if c.image_mode:
+        segs, pos = api.layout_image(c.text_len, c.ref_lat_h, c.ref_lat_w, c.lat_h, c.lat_w)
+    else:
+        segs, pos = api.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+    n = pos.shape[0]
+    dims = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn, act_dtype=c.act_dtype)
+    blocks = [api.BlockParams.from_host(dims, configs.block_weights(c, b, device=dev), device=dev)
+              for b in range(c.n_blocks)]
+    x0 = configs.hidden_states(c, device=dev)
+    x = x0.clone()
+    pd = torch.as_tensor(pos.astype(np.float32), device=dev)
+    ws = torch.empty(api.workspace_size(dims, n), dtype=torch.uint8, device=dev)
+    sv = c.sigma_v
+    sa = api.time_shift_sigma(max(sv, 1e-6), 12.0, 3.0)
+    heads = None
+    ov = oa = None
+    if c.heads_out or c.image_mode:
+        hc = c if c.heads_out else configs.DitConfig(c.name, c.cfg_seed, hidden=c.hidden, heads=c.heads,
+                                                       head_dim=c.head_dim, ffn=c.ffn, text_len=c.text_len,
+                                                       heads_out=128)
+        heads = api.HeadParams.from_host(configs.head_weights(hc, device=dev), device=dev)
+        vseg = [sg for sg in segs if sg[2] == 0][-1]
+        aseg = [sg for sg in segs if sg[2] == 2]
+        ov = torch.empty((vseg[1] - vseg[0], 128), device=dev)
+        oa = torch.empty((aseg[-1][1] - aseg[-1][0], 128), device=dev) if aseg else None
+
+    def step():
+        x.copy_(x0)
+        api.stack_forward(dims, blocks, heads, x, segs, pd, sv, sa, ov, oa, ws)
+
+    api.prof_reset()
+    api.prof_enable(True)
+    ms = _time(step, steps, warmup)
+    api.prof_enable(False)
+    phases, nblocks = api.prof_collect()
+    api.device_status()
+    flops = block_flops(n, c.hidden, c.heads * c.head_dim, c.ffn)
+    per_block = {k: v / max(1, nblocks) for k, v in phases.items() if v > 0}
+    peak = peaks["bf16_tflops_sustained"]
+    line.update(metric=f"{args.workload} forward time (1 B200)", value=ms, unit="ms/forward",
+                higher_is_better=False, dtype="fp32/tf32" if c.act_dtype == torch.float32 else "bf16",
+                n_tokens=n, n_blocks=c.n_blocks, heads=bool(heads),
+                tokens_per_s_per_block=n * c.n_blocks / (ms / 1e3),
+                tflops_per_s=c.n_blocks * sum(flops.values()) / (ms / 1e3) / 1e12,
+                phases_ms_per_block={k: round(v, 4) for k, v in per_block.items()},
+                phase_frac_of_peak={k: round(flops[k] / (per_block[k] / 1e3) / 1e12 / peak, 4)
+                                    for k in flops if k in per_block},
+                config={"workload": f"{c.name}: n {n}, hidden {c.hidden}, {c.heads}x{c.head_dim} heads, "
+                                    f"SwiGLU {c.ffn}, {c.n_blocks} blocks" + (", output heads" if heads else "")})
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload != "block":
+        run_workload(args)
     else:
         run_gpu(args)
 
