@@ -244,9 +244,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) pm[i] = s[i];
 #pragma unroll
-      for (int k = 8; k < 128; ++k) pm[k & 7] = fmaxf(pm[k & 7], s[k]);
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      for (int k = 8; k < 120; k += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], s[k + i], s[k + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pm[i] = fmaxf(pm[i], s[120 + i]);
+      const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
       const float m_tile = mx * scale_log2;
       if (j == 0) {
         m_ref = m_tile;
