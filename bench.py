@@ -127,6 +127,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------ multi-rank timing
+def max_over_ranks(ms: float, device, world: int) -> float:
+    """The slowest rank's device time (every rank gets the same value)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank runs `steps` replicas of the workload,
+    the job takes as long as its slowest rank."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 # -------------------------------------------------- ncu traffic of a kernel
 def measured_traffic(profile: str, source: str):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
@@ -224,10 +241,7 @@ def run_gpu(args):
     ms = e0.elapsed_time(e1)
     phases, nblocks = api.prof_collect()
     api.device_status()
-    ms_t = torch.tensor([ms], device=device)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, device, world)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies
     # inside the timed region
@@ -254,10 +268,7 @@ def run_gpu(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], device=device)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device, world)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -265,7 +276,7 @@ def run_gpu(args):
 
     n = W["n"]
     step_ms = ms_max / args.steps
-    value = world * n * args.steps / (ms_max / 1e3)
+    value = job_throughput(world, n, args.steps, ms_max)
     flops = block_flops(n)
     # dominant kernel from the per-phase device times (nblocks blocks)
     per_launch = {k: v / max(1, nblocks) for k, v in phases.items() if v > 0}
@@ -297,7 +308,7 @@ def run_gpu(args):
         "phases_ms_per_block": {k: round(v / max(1, nblocks), 4) for k, v in phases.items()},
         "phase_frac_of_peak": {k: round(flops[k] / (per_launch[k] / 1e3) / 1e12 / peak, 4)
                                for k in flops if k in per_launch},
-        "e2e": {"value": world * n * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": job_throughput(world, n, e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(W["x0"].numel() * 4 + W["pos_d"].numel() * 4),
                 "d2h_bytes_per_step": int(W["x0"].numel() * 4)},
         "gpu_launches": 9 * args.steps,

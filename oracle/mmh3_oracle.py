@@ -499,3 +499,72 @@ def vit_layer_forward(p: dict, x: np.ndarray, batch: int, seq: int, dims: dict,
             keep.setdefault("act", []).append(a)
         outs.append(z)
     return np.concatenate(outs)
+
+
+# --------------------------------------------------------------------------
+# token refiner  ([mmh3] ``refine_text``)
+# --------------------------------------------------------------------------
+
+def refine_text(states: np.ndarray, cond_w, cond_b, blocks: list, refiner_norm,
+                dims: dict, final_eps: float) -> np.ndarray:
+    """Text states [n, text_dim] -> refined embeddings [n, H] ([mmh3]
+    ``refine_text``): h = states cond_w^T + cond_b, then each refiner block
+    unmodulated and unrotated (plain residuals), then RMSNorm with the
+    refiner's final gain and eps."""
+    h = np.asarray(states, np.float64) @ np.asarray(cond_w, np.float64).T + np.asarray(cond_b, np.float64)
+    n = h.shape[0]
+    for p in blocks:
+        h = block_forward(p, h, None, np.zeros(n, dtype=np.int64), None, dims)
+    return rms_norm(h, refiner_norm, final_eps)
+
+
+# --------------------------------------------------------------------------
+# stream (un)packing and the embed  ([mmh3] patchify_video, pack_audio, forward "embed")
+# --------------------------------------------------------------------------
+
+def patchify_video(x: np.ndarray) -> np.ndarray:
+    """[C, T, H, W] -> [T*(H/2)*(W/2), 4C]: 2x2 spatial patches, each row
+    ordered (channel, patch row p, patch column q) ([mmh3] ``patchify_video``,
+    einsum nctrhpwq -> nthwcrpq)."""
+    C, T, H, W = x.shape
+    y = x.reshape(C, T, H // 2, 2, W // 2, 2)            # c t h p w q
+    return y.transpose(1, 2, 4, 0, 3, 5).reshape(T * (H // 2) * (W // 2), 4 * C)
+
+
+def unpatchify_video(rows: np.ndarray, C: int, T: int, H: int, W: int) -> np.ndarray:
+    """The inverse of ``patchify_video`` ([mmh3] ``unpatchify_video``)."""
+    y = np.asarray(rows).reshape(T, H // 2, W // 2, C, 2, 2)   # t h w c p q
+    return y.transpose(3, 0, 1, 4, 2, 5).reshape(C, T, H, W)
+
+
+def pack_audio(x: np.ndarray) -> np.ndarray:
+    """[C, 2, T] -> [2T, C], channel-major: stereo channel 0's frames then
+    channel 1's ([mmh3] ``pack_audio``)."""
+    C, two, T = x.shape
+    return np.asarray(x).transpose(1, 2, 0).reshape(2 * T, C)
+
+
+def unpack_audio(rows: np.ndarray, C: int, T: int) -> np.ndarray:
+    """The inverse of ``pack_audio`` ([mmh3] ``unpack_audio``)."""
+    return np.asarray(rows).reshape(2, T, C).transpose(2, 0, 1)
+
+
+def embed(layout: dict, text: np.ndarray, video: np.ndarray, audio: np.ndarray,
+          w_video, b_video, w_audio, b_audio) -> np.ndarray:
+    """The packed hidden states of one denoise evaluation ([mmh3] ``forward``
+    "embed"): text rows copied in, video latents patchified and projected
+    (+ bias), audio latents packed and projected (+ bias), each into its
+    segment."""
+    n = layout["seq_len"]
+    Hd = np.asarray(w_video).shape[0]
+    h = np.zeros((n, Hd))
+    for (a, b, tag, clock) in layout["segments"]:
+        if tag == TAG_TEXT:
+            h[a:b] = np.asarray(text, np.float64)[: b - a]
+        elif tag == TAG_VIDEO:
+            h[a:b] = patchify_video(np.asarray(video, np.float64)) @ np.asarray(w_video, np.float64).T \
+                + np.asarray(b_video, np.float64)
+        elif tag == TAG_AUDIO:
+            h[a:b] = pack_audio(np.asarray(audio, np.float64)) @ np.asarray(w_audio, np.float64).T \
+                + np.asarray(b_audio, np.float64)
+    return h

@@ -1,0 +1,50 @@
+"""The multi-rank side of bench.py on CPU: two gloo ranks (the path has no
+exchange step, so ranks are independent replicas) agree on the slowest
+rank's time, and the whole-job value counts every rank's tokens over it."""
+
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = [12.5, 40.0][rank]
+        ms = bench.max_over_ranks(local_ms, "cpu", world)
+        val = bench.job_throughput(world, 13248, 100, ms)
+        out[rank] = (ms, val)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_max_and_count_all_tokens():
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank, args=(2, port, out), nprocs=2, start_method="spawn", join=True)
+    assert out[0][0] == out[1][0] == 40.0
+    assert out[0][1] == pytest.approx(2 * 13248 * 100 / 0.040)
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.0, "cpu", 1) == 3.0
+    assert bench.job_throughput(1, 10, 5, 1000.0) == 50.0

@@ -547,3 +547,64 @@ def test_gauss_pairs_and_moments():
     # chunking does not change the stream
     assert torch.equal(synth.gauss(10, 9), synth.gauss(11, 9)[:10])
     random.seed(0)
+
+
+# ------------------------------------------------------- refiner and embed
+
+def test_patchify_and_audio_pack_round_trip_page_tests():
+    # mmh3.rs tests patchify_round_trips / audio_pack_round_trips
+    c, t, h, w = 3, 2, 4, 6
+    x = np.arange(c * t * h * w, dtype=np.float64).reshape(c, t, h, w)
+    rows = O.patchify_video(x)
+    assert rows.shape == (t * (h // 2) * (w // 2), c * 4)
+    np.testing.assert_array_equal(O.unpatchify_video(rows, c, t, h, w), x)
+    ca, ta = 5, 7
+    xa = np.arange(ca * 2 * ta, dtype=np.float64).reshape(ca, 2, ta)
+    np.testing.assert_array_equal(O.unpack_audio(O.pack_audio(xa), ca, ta), xa)
+
+
+def test_patchify_element_order_by_hand():
+    # row (t, hi, wi), column (c, p, q) holds x[c, t, 2 hi + p, 2 wi + q]
+    c, t, h, w = 2, 3, 4, 6
+    x = np.random.default_rng(13).standard_normal((c, t, h, w))
+    rows = O.patchify_video(x)
+    for (ti, hi, wi) in ((0, 0, 0), (2, 1, 2), (1, 1, 0)):
+        r = (ti * (h // 2) + hi) * (w // 2) + wi
+        for ci in range(c):
+            for p in range(2):
+                for q in range(2):
+                    assert rows[r, ci * 4 + p * 2 + q] == x[ci, ti, 2 * hi + p, 2 * wi + q]
+    xa = np.random.default_rng(14).standard_normal((4, 2, 5))
+    pa = O.pack_audio(xa)
+    assert pa[0, 3] == xa[3, 0, 0] and pa[5 + 2, 1] == xa[1, 1, 2]   # channel-major rows
+
+
+def test_refine_text_without_blocks_is_projection_then_rmsnorm():
+    rng = np.random.default_rng(15)
+    s = rng.standard_normal((5, 6))
+    w = rng.standard_normal((4, 6))
+    b = rng.standard_normal(4)
+    g = 1 + 0.1 * rng.standard_normal(4)
+    out = O.refine_text(s, w, b, [], g, dict(hidden=4), 1e-5)
+    h = np.array([[sum(s[i, k] * w[o, k] for k in range(6)) + b[o] for o in range(4)] for i in range(5)])
+    ref = h / np.sqrt((h * h).mean(-1, keepdims=True) + 1e-5) * g
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
+def test_embed_places_each_stream_in_its_segment():
+    L = O.layout_t2va(3, 2, 4, 4, 2)                 # text 3, audio 2x2, video 2x2x2
+    n = L["seq_len"]
+    rng = np.random.default_rng(16)
+    H = 5
+    text = rng.standard_normal((3, H))
+    video = rng.standard_normal((2, 2, 4, 4))        # C=2 -> 4C = 8
+    audio = rng.standard_normal((3, 2, 2))           # C=3
+    wv, bv = rng.standard_normal((H, 8)), rng.standard_normal(H)
+    wa, ba = rng.standard_normal((H, 3)), rng.standard_normal(H)
+    h = O.embed(L, text, video, audio, wv, bv, wa, ba)
+    assert h.shape == (n, H)
+    np.testing.assert_array_equal(h[:3], text)
+    # first audio row = channel 0, frame 0 of every latent channel, projected
+    np.testing.assert_allclose(h[3], wa @ audio[:, 0, 0] + ba, atol=1e-12)
+    # first video row = the 2x2 patch at the top-left of frame 0
+    np.testing.assert_allclose(h[7], wv @ video[:, 0, 0:2, 0:2].reshape(-1) + bv, atol=1e-12)
