@@ -220,6 +220,105 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                                double sigma_v, double sigma_a, float* out_video, float* out_audio,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* --------------------------------------- token refiner, embed, unpacking */
+
+/* Bytes of device workspace mmh3_refine_text needs for n text tokens: the
+ * block workspace of mmh3_workspace_size followed (256-byte aligned) by the
+ * refiner's fp32 residual stream [n, H]. */
+mmh3_status mmh3_refine_workspace_size(const mmh3_dims* dims, int n, size_t* bytes);
+
+/* The token refiner ("cortiq_engine/mmh3.rs", MiniMaxH3::refine_text):
+ *   h = states cond_w^T + cond_b;
+ *   each of the n_blocks refiner blocks, unmodulated and unrotated (plain
+ *   residuals; q/k still get their per-head RMSNorm);
+ *   out = RMSNorm(h; refiner_norm, final_eps).
+ * states [n, text_dim] and cond_w [H, text_dim] act dtype, text_dim * the
+ * element size a multiple of 16 bytes; cond_b and refiner_norm [H] fp32;
+ * blocks: host array of n_blocks weight structs (their adaLN pointers are
+ * not read and may be NULL); out [n, H] fp32.  Device pointers, 16-byte
+ * aligned.  The workspace is mmh3_refine_workspace_size bytes. */
+mmh3_status mmh3_refine_text(const mmh3_dims* dims, const void* states, int n, int text_dim,
+                             const void* cond_w, const float* cond_b,
+                             const mmh3_block_weights* blocks, int n_blocks,
+                             const float* refiner_norm, float final_eps, float* out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Stream kinds of mmh3_patch_embed (the segment tag of the rows written). */
+#define MMH3_STREAM_VIDEO 0
+#define MMH3_STREAM_AUDIO 2
+
+/* Bytes of device workspace mmh3_patch_embed needs: the staged patch rows
+ * [rows, K] in act dtype (see below for rows and K). */
+mmh3_status mmh3_patch_embed_workspace_size(const mmh3_dims* dims, int kind, int channels,
+                                            int frames, int lat_h, int lat_w, size_t* bytes);
+
+/* One stream's latents -> its rows of the packed hidden states
+ * ("cortiq_engine/mmh3.rs", forward "embed", patchify_video, pack_audio):
+ *  kind MMH3_STREAM_VIDEO: latents [C, T, lat_h, lat_w] fp32 (lat_h, lat_w
+ *    even) -> rows = T*(lat_h/2)*(lat_w/2) 2x2 patches, row (t, i, j) holding
+ *    latents[c, t, 2i+p, 2j+q] at column 4c + 2p + q; K = 4C.
+ *  kind MMH3_STREAM_AUDIO: latents [C, 2, T] fp32 -> rows = 2T, stereo
+ *    channel 0's frames then channel 1's, row (ch, t) = latents[:, ch, t];
+ *    K = C (lat_h, lat_w ignored).
+ * Then x_rows[r] = rows[r] w^T + b with w [H, K] act dtype (K * element size a
+ * multiple of 16 bytes) and b [H] fp32; x_rows is fp32 [rows, H], normally
+ * x + start*H of the stream's segment.  The patch rows are rounded to the
+ * act dtype (the projection's operand precision).  Device pointers. */
+mmh3_status mmh3_patch_embed(const mmh3_dims* dims, int kind, const float* latents, int channels,
+                             int frames, int lat_h, int lat_w, const void* w, const float* b,
+                             float* x_rows, void* workspace, size_t ws_bytes, void* stream);
+
+/* The inputs of one denoise evaluation's embed.  text: refined text rows
+ * [>= text segment rows, H] fp32 (mmh3_refine_text); video [C_v, T_v,
+ * lat_h, lat_w] and audio [C_a, 2, T_a] fp32; cond: host array of n_cond
+ * device pointers, each a condition frame [C_v, 1, lat_h, lat_w] fp32 with
+ * its noise blend already applied.  All device memory except `cond`. */
+typedef struct {
+  const float* text;
+  const float* video;
+  int video_channels, video_frames, lat_h, lat_w;
+  const float* audio;
+  int audio_channels, audio_frames;
+  const float* const* cond;
+  int n_cond;
+} mmh3_embed_inputs;
+
+/* The patch projections: w_video [H, 4*C_v], w_audio [H, C_a] act dtype;
+ * b_video, b_audio [H] fp32 (device). */
+typedef struct {
+  const void* w_video;
+  const float* b_video;
+  const void* w_audio;
+  const float* b_audio;
+} mmh3_embed_weights;
+
+/* Workspace of mmh3_embed: the largest of its mmh3_patch_embed calls. */
+mmh3_status mmh3_embed_workspace_size(const mmh3_dims* dims, const mmh3_embed_inputs* in,
+                                      size_t* bytes);
+
+/* The packed hidden states x [n, H] fp32 of one denoise evaluation
+ * ("cortiq_engine/mmh3.rs", forward "embed"): the first text-tag segment
+ * takes the first (stop - start) text rows; the LAST video-tag segment (the
+ * target) takes the video latents and the last audio-tag segment the audio
+ * latents through mmh3_patch_embed; every other video-tag segment, in order,
+ * takes the next condition frame through the video projection.  Each
+ * segment's row count must match what its stream gives (MMH3_ERR_SHAPE
+ * otherwise), and n_cond must equal the number of those other segments. */
+mmh3_status mmh3_embed(const mmh3_dims* dims, const mmh3_segment* segs, int n_seg, int n,
+                       const mmh3_embed_inputs* in, const mmh3_embed_weights* w, float* x,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* The inverse of the video patchify: rows [T*(lat_h/2)*(lat_w/2), 4C] fp32
+ * (the video head's output) -> out [C, T, lat_h, lat_w] fp32
+ * ("cortiq_engine/mmh3.rs", unpatchify_video).  Device, distinct buffers. */
+mmh3_status mmh3_unpatchify_video(const float* rows, int channels, int frames, int lat_h, int lat_w,
+                                  float* out, void* stream);
+
+/* The inverse of the audio packing: rows [2T, C] fp32 -> out [C, 2, T] fp32
+ * ("cortiq_engine/mmh3.rs", unpack_audio).  Device, distinct buffers. */
+mmh3_status mmh3_unpack_audio(const float* rows, int channels, int frames, float* out,
+                              void* stream);
+
 /* Size of the fixed device scratch that mmh3_block_forward_noalloc uses:
  * 32 MiB, reserved on every GPU where the library's device code is loaded,
  * until the process exits. */

@@ -550,21 +550,34 @@ def unpack_audio(rows: np.ndarray, C: int, T: int) -> np.ndarray:
 
 
 def embed(layout: dict, text: np.ndarray, video: np.ndarray, audio: np.ndarray,
-          w_video, b_video, w_audio, b_audio) -> np.ndarray:
+          w_video, b_video, w_audio, b_audio, cond: list = ()) -> np.ndarray:
     """The packed hidden states of one denoise evaluation ([mmh3] ``forward``
-    "embed"): text rows copied in, video latents patchified and projected
-    (+ bias), audio latents packed and projected (+ bias), each into its
-    segment."""
+    "embed").  The first text-tag segment takes the refined text rows; the
+    LAST video-tag segment (the target) takes the video latents, patchified
+    and projected (+ bias); the last audio-tag segment takes the audio
+    latents, packed and projected (+ bias).  Every other video-tag segment is
+    a condition frame: ``cond[i]`` ([C, 1, h, w], noise blend already applied
+    by the caller) goes through the same patch projection, in segment order.
+    Rows of no segment stay zero."""
     n = layout["seq_len"]
     Hd = np.asarray(w_video).shape[0]
     h = np.zeros((n, Hd))
-    for (a, b, tag, clock) in layout["segments"]:
-        if tag == TAG_TEXT:
-            h[a:b] = np.asarray(text, np.float64)[: b - a]
-        elif tag == TAG_VIDEO:
-            h[a:b] = patchify_video(np.asarray(video, np.float64)) @ np.asarray(w_video, np.float64).T \
-                + np.asarray(b_video, np.float64)
-        elif tag == TAG_AUDIO:
-            h[a:b] = pack_audio(np.asarray(audio, np.float64)) @ np.asarray(w_audio, np.float64).T \
-                + np.asarray(b_audio, np.float64)
+    segs = layout["segments"]
+    t_idx = [k for k, s in enumerate(segs) if s[2] == TAG_TEXT]
+    v_idx = [k for k, s in enumerate(segs) if s[2] == TAG_VIDEO]
+    a_idx = [k for k, s in enumerate(segs) if s[2] == TAG_AUDIO]
+    wv, bv = np.asarray(w_video, np.float64), np.asarray(b_video, np.float64)
+    if t_idx:
+        a, b = segs[t_idx[0]][:2]
+        h[a:b] = np.asarray(text, np.float64)[: b - a]
+    if v_idx:
+        a, b = segs[v_idx[-1]][:2]
+        h[a:b] = patchify_video(np.asarray(video, np.float64)) @ wv.T + bv
+        for i, k in enumerate(v_idx[:-1]):
+            a, b = segs[k][:2]
+            h[a:b] = patchify_video(np.asarray(cond[i], np.float64)) @ wv.T + bv
+    if a_idx:
+        a, b = segs[a_idx[-1]][:2]
+        h[a:b] = pack_audio(np.asarray(audio, np.float64)) @ np.asarray(w_audio, np.float64).T \
+            + np.asarray(b_audio, np.float64)
     return h

@@ -55,6 +55,19 @@ class VitWeights(C.Structure):
                                           "ln2_b", "w1", "b1", "w2", "b2")]
 
 
+class EmbedInputs(C.Structure):
+    _fields_ = [("text", C.c_void_p), ("video", C.c_void_p), ("video_channels", C.c_int),
+                ("video_frames", C.c_int), ("lat_h", C.c_int), ("lat_w", C.c_int),
+                ("audio", C.c_void_p), ("audio_channels", C.c_int), ("audio_frames", C.c_int),
+                ("cond", C.POINTER(C.c_void_p)), ("n_cond", C.c_int)]
+
+
+class EmbedWeights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("w_video", "b_video", "w_audio", "b_audio")]
+
+
+MMH3_STREAM_VIDEO, MMH3_STREAM_AUDIO = 0, 2
+
 _P = C.c_void_p
 _I = C.c_int
 _D = C.c_double
@@ -82,6 +95,19 @@ SIGNATURES = {
     "mmh3_stack_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _I,
                                 C.POINTER(HeadWeights), _P, _I, _SEGP, _I, _P, _D, _D, _P, _P, _P,
                                 C.c_size_t, _P]),
+    "mmh3_refine_workspace_size": (_I, [C.POINTER(Dims), _I, C.POINTER(C.c_size_t)]),
+    "mmh3_refine_text": (_I, [C.POINTER(Dims), _P, _I, _I, _P, _P, C.POINTER(BlockWeights), _I, _P,
+                              C.c_float, _P, _P, C.c_size_t, _P]),
+    "mmh3_patch_embed_workspace_size": (_I, [C.POINTER(Dims), _I, _I, _I, _I, _I,
+                                             C.POINTER(C.c_size_t)]),
+    "mmh3_patch_embed": (_I, [C.POINTER(Dims), _I, _P, _I, _I, _I, _I, _P, _P, _P, _P, C.c_size_t,
+                              _P]),
+    "mmh3_embed_workspace_size": (_I, [C.POINTER(Dims), C.POINTER(EmbedInputs),
+                                       C.POINTER(C.c_size_t)]),
+    "mmh3_embed": (_I, [C.POINTER(Dims), _SEGP, _I, _I, C.POINTER(EmbedInputs),
+                        C.POINTER(EmbedWeights), _P, _P, C.c_size_t, _P]),
+    "mmh3_unpatchify_video": (_I, [_P, _I, _I, _I, _I, _P, _P]),
+    "mmh3_unpack_audio": (_I, [_P, _I, _I, _P, _P]),
     "mmh3_vit_fold_qkv": (_I, [C.POINTER(VitDims), _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "mmh3_vit_workspace_size": (_I, [C.POINTER(VitDims), _I, _I, C.POINTER(C.c_size_t)]),
     "mmh3_vit_layer_forward": (_I, [C.POINTER(VitDims), C.POINTER(VitWeights), _P, _I, _I, _P,

@@ -12,13 +12,16 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import (MMH3_BF16, MMH3_F32, BlockWeights, Dims, HeadWeights, Segment, VitDims,
-                   VitWeights, check, load)
+from ._lib import (MMH3_BF16, MMH3_F32, MMH3_STREAM_AUDIO, MMH3_STREAM_VIDEO, BlockWeights, Dims,
+                   EmbedInputs, EmbedWeights, HeadWeights, Segment, VitDims, VitWeights, check,
+                   load)
 
 __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_image",
            "plan_timesteps", "time_shift_sigma", "resolve_rows", "adaln_modulation",
            "prepare_fc1", "workspace_size", "attention", "BlockParams", "HeadParams",
-           "block_forward", "stack_forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
+           "block_forward", "stack_forward", "refine_workspace_size", "refine_text",
+           "patch_embed_workspace_size", "patch_embed", "embed_workspace_size", "embed",
+           "unpatchify_video", "unpack_audio", "VitParams", "vit_fold_qkv", "vit_workspace_size",
            "vit_layer_forward", "device_status", "selftest_wait_timeout", "set_wait_limit_ns",
            "MMH3_BF16", "MMH3_F32"]
 
@@ -193,6 +196,92 @@ def stack_forward(dims: Dims, blocks: list, heads: HeadParams | None, x: torch.T
                                     segments(segs), len(segs), _ptr(pos), sigma_v, sigma_a,
                                     _ptr(out_video), _ptr(out_audio), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream()))
+
+
+# ------------------------------------------------ token refiner, embed, unpack
+def refine_workspace_size(dims: Dims, n: int) -> int:
+    b = C.c_size_t(0)
+    check(load().mmh3_refine_workspace_size(C.byref(dims), n, C.byref(b)))
+    return b.value
+
+
+def refine_text(dims: Dims, states: torch.Tensor, cond_w: torch.Tensor, cond_b: torch.Tensor,
+                blocks: list, refiner_norm: torch.Tensor, final_eps: float, out: torch.Tensor,
+                workspace: torch.Tensor) -> None:
+    """states [n, text_dim] act dtype -> out [n, H] fp32 (the token refiner)."""
+    arr = (BlockWeights * max(1, len(blocks)))(*[b.struct() for b in blocks])
+    check(load().mmh3_refine_text(C.byref(dims), _ptr(states), states.shape[0], states.shape[1],
+                                  _ptr(cond_w), _ptr(cond_b), arr, len(blocks), _ptr(refiner_norm),
+                                  final_eps, _ptr(out), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream()))
+
+
+def _stream_args(kind: int, latents: torch.Tensor):
+    if kind == MMH3_STREAM_VIDEO:
+        c, t, h, w = latents.shape
+        return c, t, h, w
+    c, two, t = latents.shape
+    if two != 2:
+        raise ValueError("audio latents must be [C, 2, T]")
+    return c, t, 0, 0
+
+
+def patch_embed_workspace_size(dims: Dims, kind: int, latents_shape) -> int:
+    b = C.c_size_t(0)
+    if kind == MMH3_STREAM_VIDEO:
+        c, t, h, w = latents_shape
+    else:
+        c, _, t = latents_shape
+        h = w = 0
+    check(load().mmh3_patch_embed_workspace_size(C.byref(dims), kind, c, t, h, w, C.byref(b)))
+    return b.value
+
+
+def patch_embed(dims: Dims, kind: int, latents: torch.Tensor, w: torch.Tensor, b: torch.Tensor,
+                x_rows: torch.Tensor, workspace: torch.Tensor) -> None:
+    """One stream's latents -> x_rows [rows, H] fp32 (patchify or pack, then
+    the projection with bias)."""
+    c, t, h, wd = _stream_args(kind, latents)
+    check(load().mmh3_patch_embed(C.byref(dims), kind, _ptr(latents), c, t, h, wd, _ptr(w), _ptr(b),
+                                  _ptr(x_rows), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream()))
+
+
+def _embed_inputs(text, video, audio, cond):
+    cond = list(cond or [])
+    arr = (C.c_void_p * max(1, len(cond)))(*[_ptr(z) for z in cond])
+    cv, tv, lh, lw = video.shape if video is not None else (1, 0, 2, 2)
+    ca, _, ta = audio.shape if audio is not None else (1, 2, 0)
+    ins = EmbedInputs(_ptr(text), _ptr(video), cv, tv, lh, lw, _ptr(audio), ca, ta,
+                      C.cast(arr, C.POINTER(C.c_void_p)), len(cond))
+    return ins, arr
+
+
+def embed_workspace_size(dims: Dims, text, video, audio, cond=()) -> int:
+    ins, _keep = _embed_inputs(text, video, audio, cond)
+    b = C.c_size_t(0)
+    check(load().mmh3_embed_workspace_size(C.byref(dims), C.byref(ins), C.byref(b)))
+    return b.value
+
+
+def embed(dims: Dims, segs, n: int, text, video, audio, w_video, b_video, w_audio, b_audio,
+          x: torch.Tensor, workspace: torch.Tensor, cond=()) -> None:
+    """The packed hidden states x [n, H] fp32 of one denoise evaluation."""
+    ins, _keep = _embed_inputs(text, video, audio, cond)
+    ew = EmbedWeights(_ptr(w_video), _ptr(b_video), _ptr(w_audio), _ptr(b_audio))
+    check(load().mmh3_embed(C.byref(dims), segments(segs), len(segs), n, C.byref(ins), C.byref(ew),
+                            _ptr(x), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            _stream()))
+
+
+def unpatchify_video(rows: torch.Tensor, channels: int, frames: int, lat_h: int, lat_w: int,
+                     out: torch.Tensor) -> None:
+    check(load().mmh3_unpatchify_video(_ptr(rows), channels, frames, lat_h, lat_w, _ptr(out),
+                                       _stream()))
+
+
+def unpack_audio(rows: torch.Tensor, channels: int, frames: int, out: torch.Tensor) -> None:
+    check(load().mmh3_unpack_audio(_ptr(rows), channels, frames, _ptr(out), _stream()))
 
 
 # -------------------------------------------------------------- encoder layer

@@ -8,7 +8,9 @@
 // MiniMaxH3::forward ("blocks", "heads"), block_forward and ffn_tail;
 // the encoder layer follows "ffai-argus 0.7.0 src/siglip.rs",
 // Layer::forward and finish_attention.
+#include <algorithm>
 #include <cmath>
+#include <cstdint>
 #include <cstring>
 #include <vector>
 
@@ -367,6 +369,220 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
     if (st != MMH3_OK) return st;
   }
   return MMH3_OK;
+}
+
+// ------------------------------------------------------------ token refiner
+static size_t refine_stream_offset(const mmh3_dims& d, int n) { return carve(d, n, nullptr).bytes; }
+
+mmh3_status mmh3_refine_workspace_size(const mmh3_dims* dims, int n, size_t* bytes) {
+  clear_error();
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (bytes == nullptr || n < 0) return fail(MMH3_ERR_ARG, "refine workspace: bytes null or n < 0");
+  *bytes = refine_stream_offset(*dims, n) + align256((size_t)n * dims->hidden * 4);
+  return MMH3_OK;
+}
+
+mmh3_status mmh3_refine_text(const mmh3_dims* dims, const void* states, int n, int text_dim, const void* cond_w,
+                             const float* cond_b, const mmh3_block_weights* blocks, int n_blocks,
+                             const float* refiner_norm, float final_eps, float* out, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  clear_error();
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (!states || !cond_w || !cond_b || !refiner_norm || !out || !workspace)
+    return fail(MMH3_ERR_ARG, "refine: null pointer");
+  if (misaligned(states) || misaligned(cond_w) || misaligned(cond_b) || misaligned(refiner_norm) ||
+      misaligned(out) || misaligned(workspace))
+    return fail(MMH3_ERR_ALIGN, "refine: pointers must be 16-byte aligned");
+  if (n < 1) return fail(MMH3_ERR_SHAPE, "refine: n = %d < 1", n);
+  const int es = esize_of(dims->act_dtype);
+  if (text_dim < 1 || ((size_t)text_dim * es) % 16 != 0)
+    return fail(MMH3_ERR_SHAPE, "refine: text_dim %d * %d bytes not a positive multiple of 16", text_dim, es);
+  if (!(final_eps > 0)) return fail(MMH3_ERR_ARG, "refine: final_eps must be positive");
+  if (n_blocks < 0 || (n_blocks > 0 && blocks == nullptr)) return fail(MMH3_ERR_ARG, "refine: blocks");
+  for (int i = 0; i < n_blocks; ++i) {
+    st = check_block(*dims, blocks + i, false);
+    if (st != MMH3_OK) return st;
+  }
+  size_t need = 0;
+  mmh3_refine_workspace_size(dims, n, &need);
+  if (ws_bytes < need) return fail(MMH3_ERR_WORKSPACE, "refine workspace %zu bytes < %zu required", ws_bytes, need);
+  const Workspace ws = carve(*dims, n, workspace);
+  float* h = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + refine_stream_offset(*dims, n));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = dims->hidden;
+  st = gemm_bias_act(dims->act_dtype, states, cond_w, n, H, text_dim, cond_b, 3, h, s);
+  if (st != MMH3_OK) return st;
+  PhaseMark pm(s, false);
+  const Plan plan{};
+  for (int i = 0; i < n_blocks; ++i) {
+    st = block_core(*dims, blocks[i], h, n, plan, nullptr, nullptr, ws, s, pm);
+    if (st != MMH3_OK) return st;
+  }
+  cudaError_t e = launch_norm_mod(MMH3_F32, h, n, H, refiner_norm, final_eps, nullptr, 0, 0, 0, SegRows{}, 0, out, s);
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "refiner final norm launch");
+}
+
+// ------------------------------------------------------------------- embed
+namespace {
+
+struct StreamShape {
+  long rows;
+  int K;
+};
+
+mmh3_status stream_shape(int kind, int C, int T, int lh, int lw, StreamShape* out) {
+  if (C < 1 || T < 0) return fail(MMH3_ERR_SHAPE, "stream: channels %d frames %d", C, T);
+  if (kind == MMH3_STREAM_VIDEO) {
+    if (lh < 2 || lw < 2 || (lh & 1) || (lw & 1))
+      return fail(MMH3_ERR_SHAPE, "video latents %d x %d: both sides must be even and >= 2", lh, lw);
+    out->rows = (long)T * (lh / 2) * (lw / 2);
+    out->K = 4 * C;
+    return MMH3_OK;
+  }
+  if (kind == MMH3_STREAM_AUDIO) {
+    out->rows = 2L * T;
+    out->K = C;
+    return MMH3_OK;
+  }
+  return fail(MMH3_ERR_ARG, "stream kind %d is neither video (0) nor audio (2)", kind);
+}
+
+}  // namespace
+
+mmh3_status mmh3_patch_embed_workspace_size(const mmh3_dims* dims, int kind, int channels, int frames, int lat_h,
+                                            int lat_w, size_t* bytes) {
+  clear_error();
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (bytes == nullptr) return fail(MMH3_ERR_ARG, "patch embed workspace: bytes null");
+  StreamShape sh;
+  st = stream_shape(kind, channels, frames, lat_h, lat_w, &sh);
+  if (st != MMH3_OK) return st;
+  *bytes = align256((size_t)sh.rows * sh.K * esize_of(dims->act_dtype));
+  return MMH3_OK;
+}
+
+mmh3_status mmh3_patch_embed(const mmh3_dims* dims, int kind, const float* latents, int channels, int frames,
+                             int lat_h, int lat_w, const void* w, const float* b, float* x_rows, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  clear_error();
+  size_t need = 0;
+  mmh3_status st = mmh3_patch_embed_workspace_size(dims, kind, channels, frames, lat_h, lat_w, &need);
+  if (st != MMH3_OK) return st;
+  StreamShape sh;
+  stream_shape(kind, channels, frames, lat_h, lat_w, &sh);
+  if (sh.rows == 0) return MMH3_OK;
+  if (!latents || !w || !b || !x_rows || !workspace) return fail(MMH3_ERR_ARG, "patch embed: null pointer");
+  if (misaligned(w) || misaligned(b) || misaligned(x_rows) || misaligned(workspace))
+    return fail(MMH3_ERR_ALIGN, "patch embed: w / b / x_rows / workspace must be 16-byte aligned");
+  const int es = esize_of(dims->act_dtype);
+  if (((size_t)sh.K * es) % 16 != 0)
+    return fail(MMH3_ERR_SHAPE, "patch embed: K = %d * %d bytes is not a multiple of 16", sh.K, es);
+  if (sh.rows > INT32_MAX) return fail(MMH3_ERR_SHAPE, "patch embed: %ld rows", sh.rows);
+  if (ws_bytes < need) return fail(MMH3_ERR_WORKSPACE, "patch embed workspace %zu < %zu", ws_bytes, need);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = kind == MMH3_STREAM_VIDEO
+                      ? launch_patchify(dims->act_dtype, latents, channels, frames, lat_h, lat_w, workspace, s)
+                      : launch_pack_audio(dims->act_dtype, latents, channels, frames, workspace, s);
+  if (e != cudaSuccess) return cuda_fail(e, "patchify / pack launch");
+  return gemm_bias_act(dims->act_dtype, workspace, w, (int)sh.rows, dims->hidden, sh.K, b, 3, x_rows, s);
+}
+
+mmh3_status mmh3_embed_workspace_size(const mmh3_dims* dims, const mmh3_embed_inputs* in, size_t* bytes) {
+  clear_error();
+  if (in == nullptr || bytes == nullptr) return fail(MMH3_ERR_ARG, "embed workspace: null");
+  size_t v = 0, c = 0, a = 0;
+  mmh3_status st = mmh3_patch_embed_workspace_size(dims, MMH3_STREAM_VIDEO, in->video_channels, in->video_frames,
+                                                   in->lat_h, in->lat_w, &v);
+  if (st != MMH3_OK) return st;
+  st = mmh3_patch_embed_workspace_size(dims, MMH3_STREAM_VIDEO, in->video_channels, 1, in->lat_h, in->lat_w, &c);
+  if (st != MMH3_OK) return st;
+  st = mmh3_patch_embed_workspace_size(dims, MMH3_STREAM_AUDIO, in->audio_channels, in->audio_frames, 0, 0, &a);
+  if (st != MMH3_OK) return st;
+  *bytes = std::max(v, std::max(in->n_cond > 0 ? c : (size_t)0, a));
+  return MMH3_OK;
+}
+
+mmh3_status mmh3_embed(const mmh3_dims* dims, const mmh3_segment* segs, int n_seg, int n,
+                       const mmh3_embed_inputs* in, const mmh3_embed_weights* w, float* x, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  clear_error();
+  if (in == nullptr || w == nullptr || x == nullptr || segs == nullptr)
+    return fail(MMH3_ERR_ARG, "embed: null pointer");
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  Plan plan;
+  st = make_plan(segs, n_seg, n, 0.5, 0.5, &plan);  // validates the segment table only
+  if (st != MMH3_OK) return st;
+  int t_seg = -1, a_seg = -1, v_last = -1, n_other = 0;
+  for (int k = 0; k < n_seg; ++k) {
+    if (segs[k].tag == 1 && t_seg < 0) t_seg = k;
+    if (segs[k].tag == 2) a_seg = k;
+    if (segs[k].tag == 0) v_last = k;
+  }
+  for (int k = 0; k < v_last; ++k) n_other += segs[k].tag == 0;
+  if (in->n_cond != n_other || (n_other > 0 && in->cond == nullptr))
+    return fail(MMH3_ERR_ARG, "embed: %d condition frames given, the segments hold %d", in->n_cond, n_other);
+  const size_t H = (size_t)dims->hidden;
+  const long frame_rows = (long)(in->lat_h / 2) * (in->lat_w / 2);
+  if (v_last >= 0 && (long)(segs[v_last].stop - segs[v_last].start) != frame_rows * in->video_frames)
+    return fail(MMH3_ERR_SHAPE, "embed: video segment of %u rows, the latents give %ld",
+                segs[v_last].stop - segs[v_last].start, frame_rows * in->video_frames);
+  if (a_seg >= 0 && (long)(segs[a_seg].stop - segs[a_seg].start) != 2L * in->audio_frames)
+    return fail(MMH3_ERR_SHAPE, "embed: audio segment of %u rows, the latents give %d",
+                segs[a_seg].stop - segs[a_seg].start, 2 * in->audio_frames);
+  for (int k = 0; k < v_last; ++k)
+    if (segs[k].tag == 0 && (long)(segs[k].stop - segs[k].start) != frame_rows)
+      return fail(MMH3_ERR_SHAPE, "embed: condition segment %d of %u rows, a frame gives %ld", k,
+                  segs[k].stop - segs[k].start, frame_rows);
+  if (t_seg >= 0 && in->text == nullptr) return fail(MMH3_ERR_ARG, "embed: text is null");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (t_seg >= 0) {
+    const size_t rows = segs[t_seg].stop - segs[t_seg].start;
+    cudaError_t e = cudaMemcpyAsync(x + segs[t_seg].start * H, in->text, rows * H * sizeof(float),
+                                    cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "embed: text copy");
+  }
+  if (v_last >= 0) {
+    st = mmh3_patch_embed(dims, MMH3_STREAM_VIDEO, in->video, in->video_channels, in->video_frames, in->lat_h,
+                          in->lat_w, w->w_video, w->b_video, x + segs[v_last].start * H, workspace, ws_bytes, s);
+    if (st != MMH3_OK) return st;
+  }
+  for (int k = 0, ci = 0; k < v_last; ++k) {
+    if (segs[k].tag != 0) continue;
+    st = mmh3_patch_embed(dims, MMH3_STREAM_VIDEO, in->cond[ci++], in->video_channels, 1, in->lat_h, in->lat_w,
+                          w->w_video, w->b_video, x + segs[k].start * H, workspace, ws_bytes, s);
+    if (st != MMH3_OK) return st;
+  }
+  if (a_seg >= 0) {
+    st = mmh3_patch_embed(dims, MMH3_STREAM_AUDIO, in->audio, in->audio_channels, in->audio_frames, 0, 0,
+                          w->w_audio, w->b_audio, x + segs[a_seg].start * H, workspace, ws_bytes, s);
+    if (st != MMH3_OK) return st;
+  }
+  return MMH3_OK;
+}
+
+mmh3_status mmh3_unpatchify_video(const float* rows, int channels, int frames, int lat_h, int lat_w, float* out,
+                                  void* stream) {
+  clear_error();
+  StreamShape sh;
+  mmh3_status st = stream_shape(MMH3_STREAM_VIDEO, channels, frames, lat_h, lat_w, &sh);
+  if (st != MMH3_OK) return st;
+  if (sh.rows == 0) return MMH3_OK;
+  if (rows == nullptr || out == nullptr) return fail(MMH3_ERR_ARG, "unpatchify: null pointer");
+  cudaError_t e = launch_unpatchify(rows, channels, frames, lat_h, lat_w, out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "unpatchify launch");
+}
+
+mmh3_status mmh3_unpack_audio(const float* rows, int channels, int frames, float* out, void* stream) {
+  clear_error();
+  if (channels < 1 || frames < 0) return fail(MMH3_ERR_SHAPE, "unpack audio: channels %d frames %d", channels, frames);
+  if (frames == 0) return MMH3_OK;
+  if (rows == nullptr || out == nullptr) return fail(MMH3_ERR_ARG, "unpack audio: null pointer");
+  cudaError_t e = launch_unpack_audio(rows, channels, frames, out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "unpack audio launch");
 }
 
 // ----------------------------------------------------------- encoder layer

@@ -342,6 +342,94 @@ cudaError_t launch_vit_fold(const void* wq, const void* wk, const void* wv, cons
   return cudaGetLastError();
 }
 
+// ---------------------------------------------- stream (un)packing
+// patchify: rows[(t*(H/2) + hi)*(W/2) + wi][c*4 + p*2 + q] = x[c][t][2hi+p][2wi+q]
+// (2x2 spatial patches, channel-major inside a row); pack audio:
+// rows[ch*T + t][c] = x[c][ch][t] (stereo channel 0's frames, then channel 1's).
+template <typename TO>
+__global__ void patchify_kernel(const float* __restrict__ x, int C, int T, int H, int W, TO* __restrict__ rows) {
+  const int hh = H / 2, ww = W / 2;
+  const long total = (long)T * hh * ww * 4 * C;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+    const int col = (int)(e % (4 * C));
+    const long r = e / (4 * C);
+    const int wi = (int)(r % ww), hi = (int)((r / ww) % hh), t = (int)(r / ((long)ww * hh));
+    const int c = col >> 2, p = (col >> 1) & 1, q = col & 1;
+    const float v = x[(((long)c * T + t) * H + 2 * hi + p) * W + 2 * wi + q];
+    if constexpr (sizeof(TO) == 2) rows[e] = __float2bfloat16_rn(v);
+    else rows[e] = v;
+  }
+}
+
+__global__ void unpatchify_kernel(const float* __restrict__ rows, int C, int T, int H, int W, float* __restrict__ x) {
+  const int hh = H / 2, ww = W / 2;
+  const long total = (long)T * hh * ww * 4 * C;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+    const int col = (int)(e % (4 * C));
+    const long r = e / (4 * C);
+    const int wi = (int)(r % ww), hi = (int)((r / ww) % hh), t = (int)(r / ((long)ww * hh));
+    const int c = col >> 2, p = (col >> 1) & 1, q = col & 1;
+    x[(((long)c * T + t) * H + 2 * hi + p) * W + 2 * wi + q] = rows[e];
+  }
+}
+
+template <typename TO>
+__global__ void pack_audio_kernel(const float* __restrict__ x, int C, int T, TO* __restrict__ rows) {
+  const long total = 2L * T * C;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+    const int c = (int)(e % C);
+    const long r = e / C;
+    const int ch = (int)(r / T), t = (int)(r % T);
+    const float v = x[((long)c * 2 + ch) * T + t];
+    if constexpr (sizeof(TO) == 2) rows[e] = __float2bfloat16_rn(v);
+    else rows[e] = v;
+  }
+}
+
+__global__ void unpack_audio_kernel(const float* __restrict__ rows, int C, int T, float* __restrict__ x) {
+  const long total = 2L * T * C;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+    const int c = (int)(e % C);
+    const long r = e / C;
+    const int ch = (int)(r / T), t = (int)(r % T);
+    x[((long)c * 2 + ch) * T + t] = rows[e];
+  }
+}
+
+static int grid_for(long total) {
+  long b = (total + 255) / 256;
+  const long cap = (long)num_sms() * 16;
+  return (int)(b < 1 ? 1 : (b > cap ? cap : b));
+}
+
+cudaError_t launch_patchify(int dtype, const float* x, int C, int T, int H, int W, void* rows, cudaStream_t s) {
+  const long total = (long)T * (H / 2) * (W / 2) * 4 * C;
+  if (dtype == MMH3_BF16)
+    patchify_kernel<__nv_bfloat16><<<grid_for(total), 256, 0, s>>>(x, C, T, H, W, static_cast<__nv_bfloat16*>(rows));
+  else
+    patchify_kernel<float><<<grid_for(total), 256, 0, s>>>(x, C, T, H, W, static_cast<float*>(rows));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpatchify(const float* rows, int C, int T, int H, int W, float* x, cudaStream_t s) {
+  unpatchify_kernel<<<grid_for((long)T * (H / 2) * (W / 2) * 4 * C), 256, 0, s>>>(rows, C, T, H, W, x);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_audio(int dtype, const float* x, int C, int T, void* rows, cudaStream_t s) {
+  const long total = 2L * T * C;
+  if (dtype == MMH3_BF16)
+    pack_audio_kernel<__nv_bfloat16><<<grid_for(total), 256, 0, s>>>(x, C, T, static_cast<__nv_bfloat16*>(rows));
+  else
+    pack_audio_kernel<float><<<grid_for(total), 256, 0, s>>>(x, C, T, static_cast<float*>(rows));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_audio(const float* rows, int C, int T, float* x, cudaStream_t s) {
+  unpack_audio_kernel<<<grid_for(2L * T * C), 256, 0, s>>>(rows, C, T, x);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------ bounded-wait self test
 // One thread initialises an mbarrier that expects one arrival which never
 // comes, waits with the given limit and records the timeout.

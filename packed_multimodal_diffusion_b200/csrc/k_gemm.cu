@@ -136,6 +136,14 @@ mmh3_status gemm_swiglu(int dtype, const void* A, const void* B, int M, int F, i
 
 mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N, int K,
                           const float* bias, int mode, void* out, cudaStream_t s) {
+  if (mode == 3) {  // fp32 output with bias (patch and condition projections)
+    if (dtype == MMH3_BF16) {
+      EpiBiasAct<float, 256, 0> e{{}, static_cast<float*>(out), N, bias};
+      return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
+    }
+    EpiBiasAct<float, 256, 0> e{{}, static_cast<float*>(out), N, bias};
+    return run_gemm<float, 256>(A, B, M, N, K, e, s);
+  }
   if (mode == 2) {  // output heads: fp32, negated, N = 128-wide tiles
     if (dtype == MMH3_BF16) {
       EpiBiasAct<float, 128, 2> e{{}, static_cast<float*>(out), N, bias};

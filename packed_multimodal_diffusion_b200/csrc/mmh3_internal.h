@@ -55,6 +55,10 @@ cudaError_t launch_vit_fold(const void* wq, const void* wk, const void* wv, cons
                             const float* bk, const float* bv, float scale, int H, void* wqkv,
                             float* bqkv, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s);
+cudaError_t launch_patchify(int dtype, const float* x, int C, int T, int H, int W, void* rows, cudaStream_t s);
+cudaError_t launch_unpatchify(const float* rows, int C, int T, int H, int W, float* x, cudaStream_t s);
+cudaError_t launch_pack_audio(int dtype, const float* x, int C, int T, void* rows, cudaStream_t s);
+cudaError_t launch_unpack_audio(const float* rows, int C, int T, float* x, cudaStream_t s);
 
 // ------------------------------------------------------------------ GEMMs
 // C = A[M,K] B[N,K]^T with a fused epilogue; dtype = mmh3_dtype of A and B.
@@ -67,7 +71,7 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
 mmh3_status gemm_swiglu(int dtype, const void* A, const void* B, int M, int F, int K, void* out,
                         cudaStream_t s);
 // mode 0: out(act dtype) = acc + bias; 1: gelu_tanh(acc + bias);
-// 2: out(fp32) = -(acc + bias)
+// 2: out(fp32) = -(acc + bias); 3: out(fp32) = acc + bias
 mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N, int K,
                           const float* bias, int mode, void* out, cudaStream_t s);
 mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,

@@ -107,3 +107,39 @@ def test_host_fault_injection(monkeypatch):
     monkeypatch.delenv("MMH3_FAULT")
     ts, rows = api.plan_timesteps([(0, 4, 1, 0)], 4, 0.5, 0.2)
     assert ts == [0.5] and rows == [1]
+
+
+def test_refine_and_embed_argument_checks():
+    lib = _lib.load()
+    d = api.make_dims(256, 2, 128, 512)
+    v = C.c_size_t()
+    # refiner workspace = block workspace + the fp32 residual stream, 256-byte aligned
+    assert lib.mmh3_workspace_size(C.byref(d), 77, C.byref(v)) == 0
+    blk = v.value
+    assert api.refine_workspace_size(d, 77) == blk + ((77 * 256 * 4 + 255) // 256) * 256
+    # patch rows staged in the act dtype: video rows T*(h/2)*(w/2) of 4C, audio rows 2T of C
+    assert api.patch_embed_workspace_size(d, api.MMH3_STREAM_VIDEO, (16, 3, 10, 14)) == \
+        ((3 * 5 * 7 * 64 * 2 + 255) // 256) * 256
+    assert api.patch_embed_workspace_size(d, api.MMH3_STREAM_AUDIO, (24, 2, 37)) == \
+        ((74 * 24 * 2 + 255) // 256) * 256
+    assert lib.mmh3_patch_embed_workspace_size(C.byref(d), 0, 4, 1, 3, 4, C.byref(v)) == 2
+    assert lib.mmh3_patch_embed_workspace_size(C.byref(d), 1, 4, 1, 2, 4, C.byref(v)) == 1
+    # K * 2 bytes = 6 is not a multiple of 16: rejected before any launch
+    rc = lib.mmh3_patch_embed(C.byref(d), 2, C.c_void_p(256), 3, 4, 0, 0, C.c_void_p(256),
+                              C.c_void_p(256), C.c_void_p(256), C.c_void_p(256), 1 << 20, None)
+    assert rc == 2 and b"K = 3" in lib.mmh3_last_error()
+    # embed: segment rows must match the streams; condition frames must match the segments
+    L = O.layout_t2va(5, 2, 6, 8, 7)
+    segs = api.segments(L["segments"])
+    fake = C.c_void_p(256)
+    ew = _lib.EmbedWeights(fake, fake, fake, fake)
+
+    def inputs(frames, n_cond=0):
+        return _lib.EmbedInputs(fake, fake, 4, frames, 6, 8, fake, 8, 7, None, n_cond)
+
+    rc = lib.mmh3_embed(C.byref(d), segs, 3, L["seq_len"], C.byref(inputs(3)), C.byref(ew), fake,
+                        fake, 1 << 20, None)
+    assert rc == 2 and b"video segment" in lib.mmh3_last_error()
+    rc = lib.mmh3_embed(C.byref(d), segs, 3, L["seq_len"], C.byref(inputs(2, 1)), C.byref(ew),
+                        fake, fake, 1 << 20, None)
+    assert rc == 1 and b"condition frames" in lib.mmh3_last_error()

@@ -608,3 +608,22 @@ def test_embed_places_each_stream_in_its_segment():
     np.testing.assert_allclose(h[3], wa @ audio[:, 0, 0] + ba, atol=1e-12)
     # first video row = the 2x2 patch at the top-left of frame 0
     np.testing.assert_allclose(h[7], wv @ video[:, 0, 0:2, 0:2].reshape(-1) + bv, atol=1e-12)
+
+
+def test_embed_condition_frames_use_the_patch_projection():
+    # a segment table [text | cond frame | target video]: the condition frame
+    # is one latent frame through the video patch projection
+    rng = np.random.default_rng(17)
+    H, C = 4, 1
+    L = {"seq_len": 2 + 4 + 8,
+         "segments": [(0, 2, O.TAG_TEXT, 0), (2, 6, O.TAG_VIDEO, 0), (6, 14, O.TAG_VIDEO, 0)]}
+    text = rng.standard_normal((2, H))
+    video = rng.standard_normal((C, 2, 4, 4))
+    cond = rng.standard_normal((C, 1, 4, 4))
+    wv, bv = rng.standard_normal((H, 4 * C)), rng.standard_normal(H)
+    h = O.embed(L, text, video, np.zeros((1, 2, 0)), wv, bv, np.zeros((H, 1)), np.zeros(H), cond=[cond])
+    # condition row 3 = patch (h=0, w=1) of the condition frame
+    np.testing.assert_allclose(h[3], wv @ cond[0, 0, 0:2, 2:4].reshape(-1) + bv, atol=1e-12)
+    # target row 6 + 4 = frame 1, patch (0, 0)
+    np.testing.assert_allclose(h[10], wv @ video[0, 1, 0:2, 0:2].reshape(-1) + bv, atol=1e-12)
+    np.testing.assert_array_equal(h[:2], text)
