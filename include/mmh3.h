@@ -319,6 +319,29 @@ mmh3_status mmh3_unpatchify_video(const float* rows, int channels, int frames, i
 mmh3_status mmh3_unpack_audio(const float* rows, int channels, int frames, float* out,
                               void* stream);
 
+/* Bytes of device workspace mmh3_forward needs: the larger of the block
+ * workspace (mmh3_workspace_size) and the embed workspace, then the video
+ * head rows [T_v*(lat_h/2)*(lat_w/2), 4*C_v] and the audio head rows
+ * [2*T_a, C_a], fp32, each 256-byte aligned. */
+mmh3_status mmh3_forward_workspace_size(const mmh3_dims* dims, int n, const mmh3_embed_inputs* in,
+                                        size_t* bytes);
+
+/* One denoise evaluation ("cortiq_engine/mmh3.rs", MiniMaxH3::forward):
+ * mmh3_embed into x [n, H] fp32, then the n_blocks blocks and both heads as
+ * in mmh3_stack_forward, then the head rows unpatchified into video_out
+ * [C_v, T_v, lat_h, lat_w] and unpacked into audio_out [C_a, 2, T_a] (fp32,
+ * device).  The results are the two velocities, each on its own clock and
+ * negated.  heads->out_video must be 4*C_v and heads->out_audio C_a
+ * (MMH3_ERR_SHAPE otherwise); a stream with no segment is skipped and its
+ * output pointer may be NULL.  x holds the last block's hidden states
+ * afterwards. */
+mmh3_status mmh3_forward(const mmh3_dims* dims, const mmh3_segment* segs, int n_seg, int n,
+                         const float* pos_dev, double sigma_v, double sigma_a,
+                         const mmh3_embed_inputs* in, const mmh3_embed_weights* ew,
+                         const mmh3_block_weights* blocks, int n_blocks,
+                         const mmh3_head_weights* heads, float* x, float* video_out,
+                         float* audio_out, void* workspace, size_t ws_bytes, void* stream);
+
 /* Size of the fixed device scratch that mmh3_block_forward_noalloc uses:
  * 32 MiB, reserved on every GPU where the library's device code is loaded,
  * until the process exits. */

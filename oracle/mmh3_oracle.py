@@ -581,3 +581,31 @@ def embed(layout: dict, text: np.ndarray, video: np.ndarray, audio: np.ndarray,
         h[a:b] = pack_audio(np.asarray(audio, np.float64)) @ np.asarray(w_audio, np.float64).T \
             + np.asarray(b_audio, np.float64)
     return h
+
+
+def denoise_forward(layout: dict, text, video, audio, embed_w: tuple, blocks: list, heads: dict,
+                    sigma_v: float, sigma_a: float, dims: dict, cond: list = ()):
+    """One denoise evaluation ([mmh3] ``forward``): the embed, every block
+    (modulated, rotated by the layout's positions), the output heads on the
+    target video and audio segments, then the head rows unpatchified /
+    unpacked.  ``embed_w`` = (w_video, b_video, w_audio, b_audio).  Returns
+    (video velocity [C, T, h, w], audio velocity [C, 2, T]), each on its own
+    clock and negated by the heads."""
+    segs, n = layout["segments"], layout["seq_len"]
+    H = dims["hidden"]
+    h = embed(layout, text, video, audio, *embed_w, cond=cond)
+    ts, slot = plan_timesteps(sigma_v, sigma_a, segs)
+    rows = token_rows(segs, slot, n)
+    for p in blocks:
+        mods = block_mods(p["adaln_w"], p["adaln_b"], p["adaln_table"], ts, H)
+        h = block_forward(p, h, mods, rows, layout["pos"], dims)
+    fm = final_mods(heads["adaln_w"], heads["adaln_b"], heads["adaln_table"], ts, H)
+    v_seg = [s for s in segs if s[2] == TAG_VIDEO][-1]
+    a_seg = [s for s in segs if s[2] == TAG_AUDIO][-1]
+    out = []
+    for (a, b, _tag, clock), key in ((v_seg, "video"), (a_seg, "audio")):
+        out.append(heads_forward(h[a:b], heads["final_norm"], fm[slot[clock]],
+                                 heads[f"w_{key}"], heads[f"b_{key}"], dims["eps"]))
+    C, T, lh, lw = np.asarray(video).shape
+    Ca, _, Ta = np.asarray(audio).shape
+    return unpatchify_video(out[0], C, T, lh, lw), unpack_audio(out[1], Ca, Ta)

@@ -106,6 +106,11 @@ SIGNATURES = {
                                        C.POINTER(C.c_size_t)]),
     "mmh3_embed": (_I, [C.POINTER(Dims), _SEGP, _I, _I, C.POINTER(EmbedInputs),
                         C.POINTER(EmbedWeights), _P, _P, C.c_size_t, _P]),
+    "mmh3_forward_workspace_size": (_I, [C.POINTER(Dims), _I, C.POINTER(EmbedInputs),
+                                         C.POINTER(C.c_size_t)]),
+    "mmh3_forward": (_I, [C.POINTER(Dims), _SEGP, _I, _I, _P, _D, _D, C.POINTER(EmbedInputs),
+                          C.POINTER(EmbedWeights), C.POINTER(BlockWeights), _I,
+                          C.POINTER(HeadWeights), _P, _P, _P, _P, C.c_size_t, _P]),
     "mmh3_unpatchify_video": (_I, [_P, _I, _I, _I, _I, _P, _P]),
     "mmh3_unpack_audio": (_I, [_P, _I, _I, _P, _P]),
     "mmh3_vit_fold_qkv": (_I, [C.POINTER(VitDims), _P, _P, _P, _P, _P, _P, _P, _P, _P]),

@@ -21,7 +21,7 @@ __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_im
            "prepare_fc1", "workspace_size", "attention", "BlockParams", "HeadParams",
            "block_forward", "stack_forward", "refine_workspace_size", "refine_text",
            "patch_embed_workspace_size", "patch_embed", "embed_workspace_size", "embed",
-           "unpatchify_video", "unpack_audio", "VitParams", "vit_fold_qkv", "vit_workspace_size",
+           "unpatchify_video", "unpack_audio", "forward_workspace_size", "forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
            "vit_layer_forward", "device_status", "selftest_wait_timeout", "set_wait_limit_ns",
            "MMH3_BF16", "MMH3_F32"]
 
@@ -272,6 +272,29 @@ def embed(dims: Dims, segs, n: int, text, video, audio, w_video, b_video, w_audi
     check(load().mmh3_embed(C.byref(dims), segments(segs), len(segs), n, C.byref(ins), C.byref(ew),
                             _ptr(x), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream()))
+
+
+def forward_workspace_size(dims: Dims, n: int, text, video, audio, cond=()) -> int:
+    ins, _keep = _embed_inputs(text, video, audio, cond)
+    b = C.c_size_t(0)
+    check(load().mmh3_forward_workspace_size(C.byref(dims), n, C.byref(ins), C.byref(b)))
+    return b.value
+
+
+def forward(dims: Dims, segs, n: int, pos, sigma_v: float, sigma_a: float, text, video, audio,
+            embed_w: tuple, blocks: list, heads: "HeadParams", x: torch.Tensor,
+            video_out: torch.Tensor | None, audio_out: torch.Tensor | None,
+            workspace: torch.Tensor, cond=()) -> None:
+    """One denoise evaluation: embed -> blocks -> heads -> unpatchify /
+    unpack.  embed_w = (w_video, b_video, w_audio, b_audio)."""
+    ins, _keep = _embed_inputs(text, video, audio, cond)
+    ew = EmbedWeights(*[_ptr(t) for t in embed_w])
+    arr = (BlockWeights * max(1, len(blocks)))(*[b.struct() for b in blocks])
+    hs = heads.struct()
+    check(load().mmh3_forward(C.byref(dims), segments(segs), len(segs), n, _ptr(pos), sigma_v,
+                              sigma_a, C.byref(ins), C.byref(ew), arr, len(blocks), C.byref(hs),
+                              _ptr(x), _ptr(video_out), _ptr(audio_out), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream()))
 
 
 def unpatchify_video(rows: torch.Tensor, channels: int, frames: int, lat_h: int, lat_w: int,

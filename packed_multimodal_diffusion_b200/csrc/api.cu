@@ -585,6 +585,81 @@ mmh3_status mmh3_unpack_audio(const float* rows, int channels, int frames, float
   return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "unpack audio launch");
 }
 
+// ------------------------------------------------- one denoise evaluation
+namespace {
+
+struct ForwardCarve {
+  size_t stage, video_rows, audio_rows, bytes;
+};
+
+mmh3_status forward_carve(const mmh3_dims* dims, int n, const mmh3_embed_inputs* in, ForwardCarve* c) {
+  size_t emb = 0;
+  mmh3_status st = mmh3_embed_workspace_size(dims, in, &emb);
+  if (st != MMH3_OK) return st;
+  const size_t stack = carve(*dims, n, nullptr).bytes;
+  const size_t nv = (size_t)in->video_frames * (in->lat_h / 2) * (in->lat_w / 2);
+  c->stage = std::max(stack, emb);
+  c->video_rows = c->stage;
+  c->audio_rows = c->video_rows + align256(nv * 4 * in->video_channels * sizeof(float));
+  c->bytes = c->audio_rows + align256(2 * (size_t)in->audio_frames * in->audio_channels * sizeof(float));
+  return MMH3_OK;
+}
+
+}  // namespace
+
+mmh3_status mmh3_forward_workspace_size(const mmh3_dims* dims, int n, const mmh3_embed_inputs* in, size_t* bytes) {
+  clear_error();
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (in == nullptr || bytes == nullptr || n < 1) return fail(MMH3_ERR_ARG, "forward workspace: null or n < 1");
+  ForwardCarve c;
+  st = forward_carve(dims, n, in, &c);
+  if (st != MMH3_OK) return st;
+  *bytes = c.bytes;
+  return MMH3_OK;
+}
+
+mmh3_status mmh3_forward(const mmh3_dims* dims, const mmh3_segment* segs, int n_seg, int n, const float* pos_dev,
+                         double sigma_v, double sigma_a, const mmh3_embed_inputs* in, const mmh3_embed_weights* ew,
+                         const mmh3_block_weights* blocks, int n_blocks, const mmh3_head_weights* heads, float* x,
+                         float* video_out, float* audio_out, void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (heads == nullptr || in == nullptr || ew == nullptr || segs == nullptr)
+    return fail(MMH3_ERR_ARG, "forward: null heads / inputs / weights / segments");
+  size_t need = 0;
+  mmh3_status st = mmh3_forward_workspace_size(dims, n, in, &need);
+  if (st != MMH3_OK) return st;
+  if (workspace == nullptr || ws_bytes < need)
+    return fail(MMH3_ERR_WORKSPACE, "forward workspace %zu bytes < %zu required", ws_bytes, need);
+  bool has_v = false, has_a = false;
+  for (int k = 0; k < n_seg && k < 64; ++k) {
+    has_v |= segs[k].tag == 0;
+    has_a |= segs[k].tag == 2;
+  }
+  if (has_v && (heads->out_video != 4 * in->video_channels || video_out == nullptr))
+    return fail(MMH3_ERR_SHAPE, "forward: video head width %d != 4 * %d latent channels, or video_out null",
+                heads->out_video, in->video_channels);
+  if (has_a && (heads->out_audio != in->audio_channels || audio_out == nullptr))
+    return fail(MMH3_ERR_SHAPE, "forward: audio head width %d != %d latent channels, or audio_out null",
+                heads->out_audio, in->audio_channels);
+  ForwardCarve c;
+  forward_carve(dims, n, in, &c);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  float* vrows = reinterpret_cast<float*>(base + c.video_rows);
+  float* arows = reinterpret_cast<float*>(base + c.audio_rows);
+  st = mmh3_embed(dims, segs, n_seg, n, in, ew, x, workspace, c.stage, stream);
+  if (st != MMH3_OK) return st;
+  st = mmh3_stack_forward(dims, blocks, n_blocks, heads, x, n, segs, n_seg, pos_dev, sigma_v, sigma_a, vrows, arows,
+                          workspace, c.stage, stream);
+  if (st != MMH3_OK) return st;
+  if (has_v) {
+    st = mmh3_unpatchify_video(vrows, in->video_channels, in->video_frames, in->lat_h, in->lat_w, video_out, stream);
+    if (st != MMH3_OK) return st;
+  }
+  if (has_a) return mmh3_unpack_audio(arows, in->audio_channels, in->audio_frames, audio_out, stream);
+  return MMH3_OK;
+}
+
 // ----------------------------------------------------------- encoder layer
 static mmh3_status check_vit(const mmh3_vit_dims* d) {
   if (d == nullptr) return fail(MMH3_ERR_ARG, "vit dims null");

@@ -155,3 +155,38 @@ def test_unpatchify_and_unpack_are_the_oracle_inverses(cuda_ok):
     aout = torch.empty((Ca, 2, Ta), device="cuda")
     api.unpack_audio(arows.cuda(), Ca, Ta, aout)
     assert torch.equal(aout.cpu(), torch.as_tensor(O.unpack_audio(arows.numpy(), Ca, Ta)))
+
+
+def test_denoise_forward_end_to_end(cuda_ok):
+    # embed -> 2 blocks -> heads -> unpatchify / unpack through one call
+    dims_o, dims_c = small_dims()
+    H, Cv, Ca = 256, 8, 32
+    L = O.layout_t2va(8, 2, 8, 12, 6)
+    segs, n = L["segments"], L["seq_len"]
+    text = configs.synth.normal((8, H), 661, 1.0)
+    video = _bf16_exact((Cv, 2, 8, 12), 662)
+    audio = _bf16_exact((Ca, 2, 6), 663)
+    ew = _embed_weights(H, Cv, Ca)
+    blocks = [small_block_weights(670 + i, H, 2, 128, 512) for i in range(2)]
+    cfg = configs.DitConfig("fwd", 68, hidden=H, heads=2, head_dim=128, ffn=512, text_len=1,
+                            heads_out=32)
+    heads = configs.head_weights(cfg)
+    heads["w_audio"] = configs.synth.normal((Ca, H), 664, 0.02).to(torch.bfloat16)
+    heads["b_audio"] = configs.synth.normal((Ca,), 665, 0.02)
+    sv, sa = 0.5, O.time_shift_sigma(0.5, 12.0, 3.0)
+    rv, ra = O.denoise_forward(L, f64(text), f64(video), f64(audio), tuple(f64(t) for t in ew),
+                               [oracle_params(w) for w in blocks], oracle_params(heads), sv, sa,
+                               dims_o)
+    bp = [api.BlockParams.from_host(dims_c, w) for w in blocks]
+    hp = api.HeadParams.from_host(heads)
+    d = [t.cuda() for t in (text, video, audio)]
+    pos = torch.as_tensor(np.asarray(L["pos"], np.float32)).cuda()
+    x = torch.empty((n, H), device="cuda")
+    vo = torch.full(video.shape, float("nan"), device="cuda")
+    ao = torch.full(audio.shape, float("nan"), device="cuda")
+    ws = torch.empty(api.forward_workspace_size(dims_c, n, *d), dtype=torch.uint8, device="cuda")
+    api.forward(dims_c, segs, n, pos, sv, sa, *d, tuple(t.cuda() for t in ew), bp, hp, x, vo, ao,
+                ws)
+    api.device_status()
+    assert_close(vo, rv, BF16_MAXABS, BF16_COS, "video velocity")
+    assert_close(ao, ra, BF16_MAXABS, BF16_COS, "audio velocity")

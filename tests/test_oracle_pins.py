@@ -627,3 +627,26 @@ def test_embed_condition_frames_use_the_patch_projection():
     # target row 6 + 4 = frame 1, patch (0, 0)
     np.testing.assert_allclose(h[10], wv @ video[0, 1, 0:2, 0:2].reshape(-1) + bv, atol=1e-12)
     np.testing.assert_array_equal(h[:2], text)
+
+
+def test_denoise_forward_identity_weights_return_the_negated_latents():
+    # H = 4 C_v = C_a; identity patch projections and head linears, no bias,
+    # zero final modulation, unit final gain, no blocks: every packed row is
+    # RMS-normalised and mapped back, so latents of +-1 (RMS exactly 1) come
+    # back negated through patchify -> heads -> unpatchify (and the audio
+    # pack / unpack) -- any transposition in the chain breaks this.
+    H, Cv, Ca = 8, 2, 8
+    L = O.layout_t2va(3, 2, 4, 6, 5)
+    rng = np.random.default_rng(21)
+    video = rng.choice([-1.0, 1.0], size=(Cv, 2, 4, 6))
+    audio = rng.choice([-1.0, 1.0], size=(Ca, 2, 5))
+    text = rng.standard_normal((3, H))
+    eye = np.eye(H)
+    heads = {"final_norm": np.ones(H), "adaln_w": np.zeros((2 * 2 * H, 24)),
+             "adaln_b": np.zeros(2 * 2 * H), "adaln_table": rng.standard_normal((1025, 24)),
+             "w_video": eye, "b_video": np.zeros(H), "w_audio": eye, "b_audio": np.zeros(H)}
+    dims = {"hidden": H, "eps": 1e-300}
+    v, a = O.denoise_forward(L, text, video, audio, (eye, np.zeros(H), eye, np.zeros(H)), [],
+                             heads, 0.5, 0.2, dims)
+    np.testing.assert_allclose(v, -video, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(a, -audio, rtol=0, atol=1e-14)
