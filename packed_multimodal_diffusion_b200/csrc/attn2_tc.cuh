@@ -273,22 +273,27 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       // P = 2^(s * scale * log2e - m_ref) as bf16 pairs over S_i's first 64
-      // columns, in four slices of 32 keys (16 columns).
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      // columns, in four slices of 32 keys (16 columns).  Scale/shift and
+      // the row sum run as packed f32x2 operations (half the issue slots of
+      // scalar ones); the exponentials stay on MUFU.
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m_ref, -m_ref);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int k = h * 32 + 2 * q;
-          const float p0 = ex2_approx(fmaf(s[k], scale_log2, -m_ref));
-          const float p1 = ex2_approx(fmaf(s[k + 1], scale_log2, -m_ref));
-          ps[q & 3] += p0 + p1;
-          pk[q] = pack_bf16x2(p0, p1);
+          const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2);
+          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if (q & 1) acc1 = __fadd2_rn(acc1, pv);
+          else acc0 = __fadd2_rn(acc0, pv);
+          pk[q] = pack_bf16x2(pv.x, pv.y);
         }
         tmem_st16(ts + h * 16, pk);
       }
-      l_sum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      l_sum += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PF + wg));
