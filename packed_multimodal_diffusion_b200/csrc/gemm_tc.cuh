@@ -607,4 +607,233 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+
+// ======================================================= CTA-pair variant
+// The same GEMM on clusters of two CTAs (one TPC): a pair computes a
+// 256 x BN tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads its
+// own 128 rows of A and half of B's BN rows (BN/2) per stage, so a CTA's
+// shared-memory operand traffic per MMA is A + B/2 instead of A + B.
+//   both CTAs   warp 0: TMA of their own A rows / B half; completion is
+//               counted on the LEADER's full barrier (the leader expects the
+//               bytes of both); each CTA waits on its own empty barrier.
+//   leader      warp 1: the MMAs, descriptors on its own shared-memory
+//               offsets (the hardware reads the same offsets in the peer);
+//               commits multicast to both CTAs' empty / accumulator-full
+//               barriers.
+//   both CTAs   warps 2..5: epilogue of their own 128 accumulator rows; the
+//               release arrives on the leader's accumulator-empty barrier
+//               (256 arrivals).
+// The tensor memory is allocated and freed by warp 1 of both CTAs
+// together.  Loads carry no multicast.  Every wait is bounded.
+template <int BN>
+struct Gemm2Shape {
+  static constexpr int BM = 128;                 // rows per CTA, 256 per pair
+  static constexpr int kABytes = BM * 128;
+  static constexpr int kBRows = BN / 2;          // B rows held by each CTA
+  static constexpr int kBBytes = kBRows * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = (2 * BN <= 256) ? 256 : 512;
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair tile width");
+};
+
+template <int BN, int STAGES>
+constexpr int gemm2_smem_bytes() {
+  return STAGES * Gemm2Shape<BN>::kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiSmemBytes;
+}
+
+template <int BN, int STAGES, class Epi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    int M, int N, int K, Epi epi, DevStatus* status, uint64_t limit_ns) {
+  using Sh = Gemm2Shape<BN>;
+  constexpr int kBK = 64;  // bf16 K elements per stage (128 bytes)
+  constexpr uint32_t kIdesc = make_idesc(false, 256, BN, false, false);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Sh::kStageBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_smem = reinterpret_cast<float*>(smem + STAGES * Sh::kStageBytes + 256);
+  static_assert(Epi::kSmemFloats * 4 <= kEpiSmemBytes, "epilogue parameters exceed their smem area");
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int st) { return bar0 + 8u * st; };
+  auto empty_bar = [&](int st) { return bar0 + 8u * (STAGES + st); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  constexpr int kEpiThreads = kGemmThreads - 64;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(full_bar(st), 1);
+      mbar_init(empty_bar(st), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * kEpiThreads);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB);
+  }
+  if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), Sh::kTmemCols);
+  if (warp >= 2) epi.setup(epi_smem, threadIdx.x - 64, kEpiThreads);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_tiles = (M + 2 * Sh::BM - 1) / (2 * Sh::BM);
+  const int n_tiles = (N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int k_blocks = (K + kBK - 1) / kBK;
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
+        int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, mt, nt);
+        const int a_row = mt * 2 * Sh::BM + (int)rank * Sh::BM;
+        const int b_row = nt * BN + (int)rank * Sh::kBRows;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (*abort_flag || !mbar_wait(empty_bar(stage), phase ^ 1u, limit_ns)) {
+            if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + stage * Sh::kStageBytes;
+          const uint32_t fb = mapa_shared(full_bar(stage), 0);
+          if (leader) mbar_expect_tx(full_bar(stage), 2 * Sh::kStageBytes);
+          tma_load_2d_pair(sa, &tmA, fb, kb * kBK, a_row);
+          tma_load_2d_pair(sa + Sh::kABytes, &tmB, fb, kb * kBK, b_row);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // The leader's full barriers count both CTAs' copies: wait (bounded)
+        // for the outstanding stages before the pair leaves.
+        int st = stage;
+        uint32_t ph = phase;
+        const int outstanding = issued < STAGES ? issued : STAGES;
+        for (int i = 0; i < outstanding; ++i) {
+          if (--st < 0) {
+            st = STAGES - 1;
+            ph ^= 1u;
+          }
+          mbar_wait(full_bar(st), ph, limit_ns);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader only)
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
+        if (*abort_flag || !mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, limit_ns)) {
+          if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, 1000 + tile);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (*abort_flag || !mbar_wait(full_bar(stage), phase, limit_ns)) {
+            if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * Sh::kStageBytes;
+          const uint32_t sb = sa + Sh::kABytes;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = sdesc_sw128(sa + ks * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sb + ks * 32, 16, 1024);
+            umma_ss_pair(d_tmem, ad, bd, kIdesc, (kb | ks) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        umma_commit_pair_local(drain_bar);
+        mbar_wait(drain_bar, 0, limit_ns);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5: this CTA's 128 rows
+    const int lgrp = warp & 3;
+    const int part = (warp - 2) >> 2;
+    const uint32_t lane_off = (uint32_t)(lgrp * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < num_tiles; tile += n_pairs) {
+      int mt, nt;
+      tile_coords(tile, m_tiles, n_tiles, mt, nt);
+      const int row = mt * 2 * Sh::BM + (int)rank * Sh::BM + lgrp * 32 + lane;
+      auto wait = [&]() -> bool {
+        const bool fail = *abort_flag || !mbar_wait_cluster(tfull_bar(acc), acc_phase, limit_ns);
+        if (__any_sync(0xffffffffu, fail)) {
+          if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_EPILOGUE, tile);
+          *abort_flag = 1;
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      if (!epi(tmem_base + acc * BN + lane_off, row, nt * BN, row < M, part, wait, epi_smem)) break;
+      tc_fence_before();
+      mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote arrive, copy or MMA of either CTA is pending
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Sh::kTmemCols);
+  }
+}
+
 }  // namespace mmh3
