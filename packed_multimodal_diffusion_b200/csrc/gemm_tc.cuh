@@ -57,7 +57,9 @@ __device__ __forceinline__ void ld_acc32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g), with the fast reciprocal division (for
+// 1 + e^-g = inf it gives 0, the limit); the result is rounded to bf16.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
@@ -132,8 +134,72 @@ __device__ __forceinline__ void store_n(float* dst, const float (&v)[N]) {
 
 struct NoSetup {
   static constexpr int kSmemFloats = 0;
+  static constexpr int kStageOut = 0;  // bytes of output staging (TMA-store epilogues)
   __device__ __forceinline__ void setup(float*, int, int) const {}
 };
+
+// Output staging for TMA-store epilogues: two buffers of one store box
+// each (128 rows x 128 bytes, 128-byte swizzle).  The epilogue threads of a
+// CTA write their row's 128 bytes into a free buffer, then one thread stores
+// the box with a tensor store.  Compared with each thread writing its own
+// row to global memory (32 cache lines per warp instruction), the tensor
+// store writes whole lines and keeps the SM's L1 / shared-memory path free
+// for the operand traffic of the MMAs.
+struct OutStage {
+  uint32_t buf0;           // shared address of buffer 0 (1024-aligned); buffer 1 at +16 KB
+  const CUtensorMap* map;  // output map: box 128 bytes x 128 rows, SWIZZLE_128B
+  int tid;                 // 0..127 within the epilogue group
+  int r;                   // accumulator row of this thread within the tile (TMEM lane)
+  int row0;                // first matrix row of the tile
+  bool rows_in;            // row0 < M (a box wholly beyond M is not stored)
+  uint32_t count;          // units issued so far (the same in every thread)
+
+  // Store this thread's 128 bytes (eight 16-byte chunks) of the unit whose
+  // first column is x (in elements of the map).
+  __device__ __forceinline__ void unit(const uint4 (&ch)[8], int x) {
+    const uint32_t buf = buf0 + ((count & 1u) << 14);
+    if (tid == 0) bulk_wait_read<1>();  // the store that last used this buffer has read it
+    named_bar_sync(1, 128);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) st_shared_v4(buf + r * 128 + ((c ^ (r & 7)) << 4), ch[c]);
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (tid == 0 && rows_in) {
+      tma_store_2d(map, buf, x, row0);
+      bulk_commit();
+    }
+    ++count;
+  }
+
+  // Both buffers as one 256-byte-wide unit (two boxes side by side), for
+  // epilogues whose row values come out of order (the rotation pairs
+  // columns j and j + 48 of a head).  begin_pair waits until the earlier
+  // stores have read the buffers; put writes the 16-byte chunk `c` (0..15)
+  // of this thread's row; end_pair stores both boxes at columns x, x + 64.
+  __device__ __forceinline__ void begin_pair() {
+    if (tid == 0) bulk_wait_read<0>();
+    named_bar_sync(1, 128);
+  }
+  __device__ __forceinline__ void put(int c, uint4 v) {
+    const uint32_t buf = buf0 + ((uint32_t)(c >> 3) << 14);
+    st_shared_v4(buf + r * 128 + (((c & 7) ^ (r & 7)) << 4), v);
+  }
+  __device__ __forceinline__ void end_pair(int x) {
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (tid == 0 && rows_in) {
+      tma_store_2d(map, buf0, x, row0);
+      tma_store_2d(map, buf0 + 16384, x + 64, row0);
+      bulk_commit();
+    }
+    count = 0;  // the next unit() starts on buffer 0 again
+  }
+};
+
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7]));
+}
 
 // qkv projection: per head of the q and k planes, RMSNorm with the q_norm /
 // k_norm weight, then the partial split-half 3-axis rotation from a per-row
@@ -152,6 +218,7 @@ struct EpiQkvNormRope {
   static constexpr int kPairs = 3 * (HD / 8);
   static constexpr int kG = HD / 8;
   static constexpr int kSmemFloats = 2 * HD;
+  static constexpr int kStageOut = 0;
 
   __device__ __forceinline__ void setup(float* sm, int tid, int nthreads) const {
     for (int i = tid; i < 2 * HD; i += nthreads) sm[i] = i < HD ? q_norm[i] : k_norm[i - HD];
@@ -236,6 +303,125 @@ struct EpiQkvNormRope {
 };
 
 
+
+// The qkv epilogue with tensor-store output (pair kernel, bf16, HD = 128):
+// each head's 128 columns go out as two 64-column boxes.
+template <int BN>
+struct EpiQkvNormRopeTma {
+  int N;
+  int inner;
+  const float* q_norm;
+  const float* k_norm;
+  const float2* cs;
+  float eps;
+  static constexpr int HD = 128;
+  static constexpr int kPairs = 3 * (HD / 8);  // 48
+  static constexpr int kG = HD / 8;            // 16
+  static constexpr int kSmemFloats = 2 * HD;
+  static constexpr int kStageOut = 32768;
+
+  __device__ __forceinline__ void setup(float* sm, int tid, int nthreads) const {
+    for (int i = tid; i < 2 * HD; i += nthreads) sm[i] = i < HD ? q_norm[i] : k_norm[i - HD];
+  }
+
+  template <class Wait>
+  __device__ __forceinline__ bool operator()(uint32_t tacc, int row, int n0, bool row_ok, int, Wait&& wait,
+                                             const float* sm, OutStage& st) const {
+    if (!wait()) return false;
+#pragma unroll 1
+    for (int g = 0; g < BN / HD; ++g) {
+      const int col0 = n0 + g * HD;
+      if (col0 >= N) break;  // uniform over the epilogue group
+      const uint32_t th = tacc + g * HD;
+      const int which = col0 / inner;  // 0 q, 1 k, 2 v
+      st.begin_pair();
+      if (which == 2) {
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          float v[32];
+          ld_acc<32>(th + c * 32, v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) st.put(c * 4 + q, pack8_bf16(v + 8 * q));
+        }
+        st.end_pair(col0);
+        continue;
+      }
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float v[32];
+        ld_acc<32>(th + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+      }
+      const float inv = rsqrtf(ss * (1.0f / HD) + eps);
+      const float* w = sm + which * HD;
+#pragma unroll 1
+      for (int a = 0; a < 3; ++a) {
+        const int j0 = a * kG;
+        float lo[kG], hi[kG];
+        ld_acc<kG>(th + j0, lo);
+        ld_acc<kG>(th + j0 + kPairs, hi);
+        const float2* c2 = cs + (size_t)(row_ok ? row : 0) * kPairs + j0;
+#pragma unroll
+        for (int i = 0; i < kG; ++i) {
+          const float2 e = cs ? __ldg(c2 + i) : make_float2(1.f, 0.f);
+          const float yl = lo[i] * inv * w[j0 + i];
+          const float yh = hi[i] * inv * w[j0 + kPairs + i];
+          lo[i] = yl * e.x - yh * e.y;
+          hi[i] = yl * e.y + yh * e.x;
+        }
+        st.put(j0 / 8, pack8_bf16(lo));
+        st.put(j0 / 8 + 1, pack8_bf16(lo + 8));
+        st.put((j0 + kPairs) / 8, pack8_bf16(hi));
+        st.put((j0 + kPairs) / 8 + 1, pack8_bf16(hi + 8));
+      }
+      float t[HD - 2 * kPairs];  // the 32 unrotated dims
+      ld_acc<32>(th + 2 * kPairs, t);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) t[i] = t[i] * inv * w[2 * kPairs + i];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) st.put(2 * kPairs / 8 + q, pack8_bf16(t + 8 * q));
+      st.end_pair(col0);
+    }
+    return true;
+  }
+};
+
+// out = act(acc + bias), bf16, with tensor-store output (pair kernel).
+template <int BN, int MODE>
+struct EpiBiasActTma : NoSetup {
+  static constexpr int kStageOut = 32768;
+  int N;
+  const float* bias;
+
+  template <class Wait>
+  __device__ __forceinline__ bool operator()(uint32_t tacc, int, int n0, bool, int, Wait&& wait, const float*,
+                                             OutStage& st) const {
+    if (!wait()) return false;
+#pragma unroll 1
+    for (int u = 0; u < BN / 64; ++u) {
+      const int col = n0 + u * 64;
+      if (col >= N) break;
+      uint4 ch[8];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float v[32];
+        ld_acc<32>(tacc + u * 64 + h * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float t = v[i] + __ldg(bias + col + h * 32 + i);
+          if (MODE == 1) t = gelu_tanh_f(t);
+          v[i] = t;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ch[h * 4 + q] = pack8_bf16(v + 8 * q);
+      }
+      st.unit(ch, col);
+    }
+    return true;
+  }
+};
 
 // x[row, :] += gate[row] * acc (the gated residual; gate = chunk of the
 // token's modulation row, found through the segment table), or x += acc when
@@ -343,6 +529,36 @@ struct EpiSwiGLU : NoSetup {
         for (int i = 0; i < 32; ++i) gt[i] = silu_f(gt[i]) * u[i];
         store_n<32>(out + (size_t)row * F + f, gt);
       }
+    }
+    return true;
+  }
+};
+
+// fc1 + SwiGLU with the output written by tensor stores (pair kernel):
+// each 256-column tile gives 128 outputs, two store units of 64 bf16.
+template <int BN>
+struct EpiSwiGLUTma : NoSetup {
+  static constexpr int kStageOut = 32768;
+  int F;
+
+  template <class Wait>
+  __device__ __forceinline__ bool operator()(uint32_t tacc, int, int n0, bool, int, Wait&& wait, const float*,
+                                             OutStage& st) const {
+    if (!wait()) return false;
+#pragma unroll 1
+    for (int u = 0; u < BN / 128; ++u) {
+      uint4 ch[8];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float gt[32], up[32];
+        ld_acc<32>(tacc + u * 64 + h * 32, gt);
+        ld_acc<32>(tacc + BN / 2 + u * 64 + h * 32, up);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) gt[i] = silu_f(gt[i]) * up[i];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ch[h * 4 + q] = pack8_bf16(gt + 8 * q);
+      }
+      st.unit(ch, n0 / 2 + u * 64);
     }
     return true;
   }
@@ -636,26 +852,31 @@ struct Gemm2Shape {
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair tile width");
 };
 
-template <int BN, int STAGES>
+// stages | output staging | barriers | epilogue parameters
+template <int BN, int STAGES, class Epi>
 constexpr int gemm2_smem_bytes() {
-  return STAGES * Gemm2Shape<BN>::kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiSmemBytes;
+  return STAGES * Gemm2Shape<BN>::kStageBytes + Epi::kStageOut + 1024 /*align*/ + 256 /*barriers*/ +
+         ((Epi::kSmemFloats * 4 + 255) / 256) * 256;
 }
 
 template <int BN, int STAGES, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    int M, int N, int K, Epi epi, DevStatus* status, uint64_t limit_ns) {
+                    const __grid_constant__ CUtensorMap tmC, int M, int N, int K, Epi epi, DevStatus* status,
+                    uint64_t limit_ns) {
   using Sh = Gemm2Shape<BN>;
   constexpr int kBK = 64;  // bf16 K elements per stage (128 bytes)
   constexpr uint32_t kIdesc = make_idesc(false, 256, BN, false, false);
+  constexpr int kOut = Epi::kStageOut;
+  static_assert(kOut == 0 || kOut == 32768, "output staging is two 16 KB boxes");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Sh::kStageBytes);
+  const uint32_t stage_out = smem_u32(smem + STAGES * Sh::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Sh::kStageBytes + kOut);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_smem = reinterpret_cast<float*>(smem + STAGES * Sh::kStageBytes + 256);
-  static_assert(Epi::kSmemFloats * 4 <= kEpiSmemBytes, "epilogue parameters exceed their smem area");
+  float* epi_smem = reinterpret_cast<float*>(smem + STAGES * Sh::kStageBytes + kOut + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -684,6 +905,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
+    if (kOut > 0) tma_prefetch(&tmC);
   }
   if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), Sh::kTmemCols);
   if (warp >= 2) epi.setup(epi_smem, threadIdx.x - 64, kEpiThreads);
@@ -802,14 +1024,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int lgrp = warp & 3;
     const int part = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(lgrp * 32) << 16;
+    OutStage ost{stage_out, &tmC, (int)threadIdx.x - 64, lgrp * 32 + lane, 0, false, 0u};
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < num_tiles; tile += n_pairs) {
       int mt, nt;
       tile_coords(tile, m_tiles, n_tiles, mt, nt);
-      const int row = mt * 2 * Sh::BM + (int)rank * Sh::BM + lgrp * 32 + lane;
+      const int row0 = mt * 2 * Sh::BM + (int)rank * Sh::BM;
+      const int row = row0 + lgrp * 32 + lane;
+      // The decision to go on is uniform over the warp (TMEM loads are
+      // warp-collective) and, for staged output, over the whole epilogue
+      // group (its named barriers need all 128 threads).
       auto wait = [&]() -> bool {
-        const bool fail = *abort_flag || !mbar_wait_cluster(tfull_bar(acc), acc_phase, limit_ns);
+        bool fail = *abort_flag || !mbar_wait_cluster(tfull_bar(acc), acc_phase, limit_ns);
+        if constexpr (kOut > 0) fail = named_bar_or(2, 128, fail);
         if (__any_sync(0xffffffffu, fail)) {
           if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_EPILOGUE, tile);
           *abort_flag = 1;
@@ -818,13 +1046,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         return true;
       };
-      if (!epi(tmem_base + acc * BN + lane_off, row, nt * BN, row < M, part, wait, epi_smem)) break;
+      bool go;
+      if constexpr (kOut > 0) {
+        ost.row0 = row0;
+        ost.rows_in = row0 < M;
+        go = epi(tmem_base + acc * BN + lane_off, row, nt * BN, row < M, part, wait, epi_smem, ost);
+      } else {
+        go = epi(tmem_base + acc * BN + lane_off, row, nt * BN, row < M, part, wait, epi_smem);
+      }
+      if (!go) break;
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
       }
+    }
+    if constexpr (kOut > 0) {
+      if (ost.tid == 0) bulk_wait_all();  // the tensor stores have written global memory
     }
   }
   tc_fence_before();

@@ -79,26 +79,40 @@ static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, c
 }
 
 // ---------------------------------------------------- CTA-pair launch
-template <int BN>
+// As many operand stages as fit beside the output staging and the
+// epilogue's parameters (at most 8).
+template <int BN, class Epi>
 constexpr int stages2_for() {
-  return BN >= 256 ? 6 : (BN >= 192 ? 7 : 8);
+  constexpr int fixed = Epi::kStageOut + 1024 + 256 + ((Epi::kSmemFloats * 4 + 255) / 256) * 256;
+  constexpr int n = (232448 - fixed) / Gemm2Shape<BN>::kStageBytes;
+  return n > 8 ? 8 : n;
 }
 
+// out / out_cols: the bf16 [M, out_cols] output of a tensor-store epilogue.
 template <int BN, class Epi>
 static mmh3_status run_gemm2(const void* A, const void* B, int M, int N, int K, const Epi& epi,
-                             cudaStream_t s) {
-  constexpr int STAGES = stages2_for<BN>();
-  constexpr int smem = gemm2_smem_bytes<BN, STAGES>();
+                             cudaStream_t s, const void* out = nullptr, int out_cols = 0) {
+  constexpr int STAGES = stages2_for<BN, Epi>();
+  constexpr int smem = gemm2_smem_bytes<BN, STAGES, Epi>();
+  static_assert(STAGES >= 4, "pair GEMM: fewer than four operand stages fit");
   static_assert(smem <= 232448, "pair GEMM shared memory above the per-CTA limit");
   if (M <= 0) return MMH3_OK;
   if (fault_injected("tensormap")) return fail(MMH3_ERR_CUDA, "injected fault at tensormap");
-  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15)
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "GEMM operand not 16-byte aligned");
   if (((size_t)K * 2) % 16 != 0) return fail(MMH3_ERR_SHAPE, "GEMM K=%d row pitch not a multiple of 16 bytes", K);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!make_tmap_2d(&ta, A, 2, (uint64_t)K, (uint64_t)M, 128) ||
       !make_tmap_2d(&tb, B, 2, (uint64_t)K, (uint64_t)N, BN / 2))
     return fail(MMH3_ERR_CUDA, "cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
+  if constexpr (Epi::kStageOut > 0) {
+    if (out == nullptr || out_cols % 64 != 0)
+      return fail(MMH3_ERR_SHAPE, "tensor-store epilogue: output width %d not a multiple of 64", out_cols);
+    if (!make_tmap_2d(&tc, out, 2, (uint64_t)out_cols, (uint64_t)M, 128))
+      return fail(MMH3_ERR_CUDA, "cuTensorMapEncodeTiled failed for the output (M=%d, %d columns)", M, out_cols);
+  } else {
+    tc = ta;  // not read
+  }
   auto kern = gemm2_tc_kernel<BN, STAGES, Epi>;
   static int max_pairs = -1;  // per instantiation, from the occupancy query
   if (max_pairs < 0) {
@@ -124,7 +138,7 @@ static mmh3_status run_gemm2(const void* A, const void* B, int M, int N, int K, 
   const int tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
-  kern<<<2 * pairs, kGemmThreads, smem, s>>>(ta, tb, M, N, K, epi, device_status_ptr(), wait_limit_ns());
+  kern<<<2 * pairs, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns());
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
   return MMH3_OK;
@@ -141,8 +155,8 @@ mmh3_status gemm_qkv(int dtype, const void* A, const void* B, int M, int N, int 
                      float eps, void* out, cudaStream_t s) {
   if (dtype == MMH3_BF16 && head_dim == 128) {
     if (use_pairs(M, N, 256)) {
-      EpiQkvNormRope<__nv_bfloat16, 128, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, eps};
-      return run_gemm2<256>(A, B, M, N, K, e, s);
+      EpiQkvNormRopeTma<256> e{N, inner, q_norm, k_norm, cs, eps};
+      return run_gemm2<256>(A, B, M, N, K, e, s, out, N);
     }
     EpiQkvNormRope<__nv_bfloat16, 128, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, eps};
     return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
@@ -199,8 +213,11 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
 mmh3_status gemm_swiglu(int dtype, const void* A, const void* B, int M, int F, int K, void* out,
                         cudaStream_t s) {
   if (dtype == MMH3_BF16) {
+    if (use_pairs(M, 2 * F, 256) && F % 64 == 0) {
+      EpiSwiGLUTma<256> et{{}, F};
+      return run_gemm2<256>(A, B, M, 2 * F, K, et, s, out, F);
+    }
     EpiSwiGLU<__nv_bfloat16, 256> e{{}, static_cast<__nv_bfloat16*>(out), F};
-    if (use_pairs(M, 2 * F, 256)) return run_gemm2<256>(A, B, M, 2 * F, K, e, s);
     return run_gemm<__nv_bfloat16, 256>(A, B, M, 2 * F, K, e, s);
   }
   EpiSwiGLU<float, 256> e{{}, static_cast<float*>(out), F};
@@ -227,12 +244,18 @@ mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N,
   }
   if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias/gelu epilogue: bf16 only");
   if (mode == 1) {
+    if (use_pairs(M, N, 256) && N % 64 == 0) {
+      EpiBiasActTma<256, 1> et{{}, N, bias};
+      return run_gemm2<256>(A, B, M, N, K, et, s, out, N);
+    }
     EpiBiasAct<__nv_bfloat16, 256, 1> e{{}, static_cast<__nv_bfloat16*>(out), N, bias};
-    if (use_pairs(M, N, 256)) return run_gemm2<256>(A, B, M, N, K, e, s);
     return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
   }
+  if (use_pairs(M, N, 256) && N % 64 == 0) {
+    EpiBiasActTma<256, 0> et{{}, N, bias};
+    return run_gemm2<256>(A, B, M, N, K, et, s, out, N);
+  }
   EpiBiasAct<__nv_bfloat16, 256, 0> e{{}, static_cast<__nv_bfloat16*>(out), N, bias};
-  if (use_pairs(M, N, 256)) return run_gemm2<256>(A, B, M, N, K, e, s);
   return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
 }
 
