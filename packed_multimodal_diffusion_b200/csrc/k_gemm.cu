@@ -43,27 +43,42 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, ui
 }
 
 // ---------------------------------------------------------------- launch
-template <int BN>
+template <int BN, int OUT>
 constexpr int stages_for() {
-  return BN >= 256 ? 4 : (BN >= 224 ? 5 : 6);
+  constexpr int base = BN >= 256 ? 4 : (BN >= 224 ? 5 : 6);
+  constexpr int fit = (232448 - OUT - 1024 - 256 - kEpiSmemBytes) / GemmShape<BN>::kStageBytes;
+  return base < fit ? base : fit;
 }
 
+// out / out_esize / out_cols: the [M, out_cols] tensor a staged epilogue
+// loads and stores with TMA (bf16 or fp32).
 template <typename T, int BN, class Epi>
 static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, const Epi& epi,
-                            cudaStream_t s) {
-  constexpr int STAGES = stages_for<BN>();
-  constexpr int smem = gemm_smem_bytes<BN, STAGES>();
+                            cudaStream_t s, const void* out = nullptr, int out_esize = 0, int out_cols = 0) {
+  constexpr int OUT = Epi::kStageOut;
+  constexpr int STAGES = stages_for<BN, OUT>();
+  constexpr int smem = gemm_smem_bytes<BN, STAGES, OUT>();
+  static_assert(STAGES >= 4, "GEMM: fewer than four operand stages fit");
   static_assert(smem <= 232448, "GEMM shared memory above the per-CTA limit");
   if (M <= 0) return MMH3_OK;
   if (fault_injected("tensormap")) return fail(MMH3_ERR_CUDA, "injected fault at tensormap");
   const int es = (int)sizeof(T);
-  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15)
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "GEMM operand not 16-byte aligned");
   if (((size_t)K * es) % 16 != 0) return fail(MMH3_ERR_SHAPE, "GEMM K=%d row pitch not a multiple of 16 bytes", K);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!make_tmap_2d(&ta, A, es, (uint64_t)K, (uint64_t)M, 128) ||
       !make_tmap_2d(&tb, B, es, (uint64_t)K, (uint64_t)N, BN))
     return fail(MMH3_ERR_CUDA, "cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
+  if constexpr (OUT > 0) {
+    if (out == nullptr || (out_cols * out_esize) % 128 != 0)
+      return fail(MMH3_ERR_SHAPE, "staged epilogue: output row of %d x %d bytes not a multiple of 128", out_cols,
+                  out_esize);
+    if (!make_tmap_2d(&tc, out, out_esize, (uint64_t)out_cols, (uint64_t)M, 128))
+      return fail(MMH3_ERR_CUDA, "cuTensorMapEncodeTiled failed for the output (M=%d, %d columns)", M, out_cols);
+  } else {
+    tc = ta;  // not read
+  }
   auto kern = gemm_tc_kernel<T, BN, STAGES, Epi>;
   {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -72,7 +87,7 @@ static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, c
   const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
-  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, M, N, K, epi, device_status_ptr(), wait_limit_ns());
+  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns());
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return MMH3_OK;
@@ -88,10 +103,11 @@ constexpr int stages2_for() {
   return n > 8 ? 8 : n;
 }
 
-// out / out_cols: the bf16 [M, out_cols] output of a tensor-store epilogue.
+// out / out_cols / out_esize: the [M, out_cols] tensor (bf16 or fp32) a
+// staged epilogue loads and stores with TMA.
 template <int BN, class Epi>
 static mmh3_status run_gemm2(const void* A, const void* B, int M, int N, int K, const Epi& epi,
-                             cudaStream_t s, const void* out = nullptr, int out_cols = 0) {
+                             cudaStream_t s, const void* out = nullptr, int out_cols = 0, int out_esize = 2) {
   constexpr int STAGES = stages2_for<BN, Epi>();
   constexpr int smem = gemm2_smem_bytes<BN, STAGES, Epi>();
   static_assert(STAGES >= 4, "pair GEMM: fewer than four operand stages fit");
@@ -106,9 +122,10 @@ static mmh3_status run_gemm2(const void* A, const void* B, int M, int N, int K, 
       !make_tmap_2d(&tb, B, 2, (uint64_t)K, (uint64_t)N, BN / 2))
     return fail(MMH3_ERR_CUDA, "cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
   if constexpr (Epi::kStageOut > 0) {
-    if (out == nullptr || out_cols % 64 != 0)
-      return fail(MMH3_ERR_SHAPE, "tensor-store epilogue: output width %d not a multiple of 64", out_cols);
-    if (!make_tmap_2d(&tc, out, 2, (uint64_t)out_cols, (uint64_t)M, 128))
+    if (out == nullptr || (out_cols * out_esize) % 128 != 0)
+      return fail(MMH3_ERR_SHAPE, "staged epilogue: output row of %d x %d bytes not a multiple of 128", out_cols,
+                  out_esize);
+    if (!make_tmap_2d(&tc, out, out_esize, (uint64_t)out_cols, (uint64_t)M, 128))
       return fail(MMH3_ERR_CUDA, "cuTensorMapEncodeTiled failed for the output (M=%d, %d columns)", M, out_cols);
   } else {
     tc = ta;  // not read
@@ -181,15 +198,21 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
                                 const SegRows& seg, cudaStream_t s) {
   if (dtype == MMH3_BF16) {
     // Pairs for the out projection; the long-K fc2 (K = 4H) measured about
-    // 4% faster on single CTAs with 224-wide tiles, so it stays there.
+    // 4% faster on single CTAs with 224-wide tiles, so it stays there.  x is
+    // moved by TMA (staged read-modify-write) when N is a multiple of 32.
     const bool pair_ok = K <= 4096;
-    if (pair_ok && N % 192 == 0 && use_pairs(M, N, 192)) {
-      EpiGatedResidual<192> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
-      return run_gemm2<192>(A, B, M, N, K, e, s);
+    const bool staged = N % 32 == 0;
+    if (pair_ok && staged && N % 192 == 0 && use_pairs(M, N, 192)) {
+      EpiResidualTma<192, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
+      return run_gemm2<192>(A, B, M, N, K, e, s, x, N, 4);
     }
-    if (pair_ok && use_pairs(M, N, 256)) {
-      EpiGatedResidual<256> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
-      return run_gemm2<256>(A, B, M, N, K, e, s);
+    if (pair_ok && staged && use_pairs(M, N, 256)) {
+      EpiResidualTma<256, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
+      return run_gemm2<256>(A, B, M, N, K, e, s, x, N, 4);
+    }
+    if (staged && N % 224 == 0) {
+      EpiResidualTma<224, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
+      return run_gemm<__nv_bfloat16, 224>(A, B, M, N, K, e, s, x, 4, N);
     }
     if (N % 256 == 0) {
       EpiGatedResidual<256> e{{}, x, N, mods, mods_stride, chunk_off, seg, nullptr};
@@ -262,8 +285,11 @@ mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N,
 mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,
                                const float* bias, float* x, cudaStream_t s) {
   if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias residual epilogue: bf16 only");
+  if (use_pairs(M, N, 256) && N % 32 == 0) {
+    EpiResidualTma<256, true> et{{}, N, nullptr, 0, 0, SegRows{}, bias};
+    return run_gemm2<256>(A, B, M, N, K, et, s, x, N, 4);
+  }
   EpiBiasResidual<256> e{{}, x, N, nullptr, 0, 0, SegRows{}, bias};
-  if (use_pairs(M, N, 256)) return run_gemm2<256>(A, B, M, N, K, e, s);
   return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
 }
 
