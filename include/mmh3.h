@@ -220,6 +220,38 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                                double sigma_v, double sigma_a, float* out_video, float* out_audio,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------- block over a sequence shard */
+
+/* The block split at its one exchange step, for a packed sequence whose
+ * rows are divided over ranks in contiguous shards (context parallelism;
+ * "cortiq_engine/mmh3.rs", block_forward, with attention over the whole
+ * sequence).  Each rank calls begin on its shard, the caller all-gathers
+ * the K|V rows of all shards in sequence order (for example NCCL
+ * all-gather on the same stream), then each rank calls end.  Shard
+ * arguments: x [n, H] fp32 holds the shard's rows; segs are the shard's
+ * segments with rows counted from the shard's first row (the tags and
+ * clocks of the segments it intersects); pos_dev [n, 3] the shard's
+ * positions.  bf16 activations only (MMH3_ERR_UNSUPPORTED otherwise).
+ *
+ * begin: adaLN, rotation table, norm1 + modulate, qkv GEMM with q/k norm and
+ * rotation; then the shard's K|V rows (bf16, k then v, [n, 2*inner]) are
+ * copied to kv_out (device, 16-byte aligned).  The workspace
+ * (mmh3_workspace_size for n rows) keeps the modulation, the rotation
+ * table and q for end: pass the same workspace to end, untouched. */
+mmh3_status mmh3_block_cp_begin(const mmh3_dims* dims, const mmh3_block_weights* w, const float* x,
+                                int n, const mmh3_segment* segs, int n_seg, const float* pos_dev,
+                                double sigma_v, double sigma_a, int modulated, void* kv_out,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* end: attention of the shard's n queries against kv_all [n_kv, 2*inner]
+ * (the gathered K|V of the whole sequence, rows in sequence order; rows
+ * beyond n_kv are never read), then out GEMM + gated residual, norm2 +
+ * modulate, fc1 + SwiGLU, fc2 + gated residual, in place on x. */
+mmh3_status mmh3_block_cp_end(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
+                              const mmh3_segment* segs, int n_seg, double sigma_v, double sigma_a,
+                              int modulated, const void* kv_all, int n_kv, void* workspace,
+                              size_t ws_bytes, void* stream);
+
 /* --------------------------------------- token refiner, embed, unpacking */
 
 /* Bytes of device workspace mmh3_refine_text needs for n text tokens: the

@@ -95,6 +95,10 @@ SIGNATURES = {
     "mmh3_stack_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _I,
                                 C.POINTER(HeadWeights), _P, _I, _SEGP, _I, _P, _D, _D, _P, _P, _P,
                                 C.c_size_t, _P]),
+    "mmh3_block_cp_begin": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _P,
+                                 _D, _D, _I, _P, _P, C.c_size_t, _P]),
+    "mmh3_block_cp_end": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _D, _D,
+                               _I, _P, _I, _P, C.c_size_t, _P]),
     "mmh3_refine_workspace_size": (_I, [C.POINTER(Dims), _I, C.POINTER(C.c_size_t)]),
     "mmh3_refine_text": (_I, [C.POINTER(Dims), _P, _I, _I, _P, _P, C.POINTER(BlockWeights), _I, _P,
                               C.c_float, _P, _P, C.c_size_t, _P]),

@@ -19,7 +19,7 @@ from ._lib import (MMH3_BF16, MMH3_F32, MMH3_STREAM_AUDIO, MMH3_STREAM_VIDEO, Bl
 __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_image",
            "plan_timesteps", "time_shift_sigma", "resolve_rows", "adaln_modulation",
            "prepare_fc1", "workspace_size", "attention", "BlockParams", "HeadParams",
-           "block_forward", "stack_forward", "refine_workspace_size", "refine_text",
+           "block_forward", "stack_forward", "block_cp_begin", "block_cp_end", "refine_workspace_size", "refine_text",
            "patch_embed_workspace_size", "patch_embed", "embed_workspace_size", "embed",
            "unpatchify_video", "unpack_audio", "forward_workspace_size", "forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
            "vit_layer_forward", "device_status", "selftest_wait_timeout", "set_wait_limit_ns",
@@ -196,6 +196,31 @@ def stack_forward(dims: Dims, blocks: list, heads: HeadParams | None, x: torch.T
                                     segments(segs), len(segs), _ptr(pos), sigma_v, sigma_a,
                                     _ptr(out_video), _ptr(out_audio), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream()))
+
+
+# ------------------------------------------------ block over a sequence shard
+def block_cp_begin(dims: Dims, params: BlockParams, x: torch.Tensor, segs, pos, sigma_v: float,
+                   sigma_a: float, kv_out: torch.Tensor, workspace: torch.Tensor,
+                   modulated: bool = True) -> None:
+    """The shard's block up to the qkv GEMM; its K|V rows go to kv_out
+    [n, 2*inner] bf16.  segs are the shard's (rows from its first row)."""
+    st = params.struct()
+    check(load().mmh3_block_cp_begin(C.byref(dims), C.byref(st), _ptr(x), x.shape[0], segments(segs),
+                                     len(segs), _ptr(pos), sigma_v, sigma_a, 1 if modulated else 0,
+                                     _ptr(kv_out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream()))
+
+
+def block_cp_end(dims: Dims, params: BlockParams, x: torch.Tensor, segs, sigma_v: float,
+                 sigma_a: float, kv_all: torch.Tensor, n_kv: int, workspace: torch.Tensor,
+                 modulated: bool = True) -> None:
+    """The rest of the shard's block against the gathered K|V rows (the first
+    n_kv rows of kv_all); in place on x.  Same workspace as begin."""
+    st = params.struct()
+    check(load().mmh3_block_cp_end(C.byref(dims), C.byref(st), _ptr(x), x.shape[0], segments(segs),
+                                   len(segs), sigma_v, sigma_a, 1 if modulated else 0, _ptr(kv_all),
+                                   n_kv, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream()))
 
 
 # ------------------------------------------------ token refiner, embed, unpack

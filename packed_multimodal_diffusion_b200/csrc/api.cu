@@ -149,12 +149,10 @@ mmh3_status check_block(const mmh3_dims& d, const mmh3_block_weights* w, bool mo
   return MMH3_OK;
 }
 
-// norm1-modulate -> qkv+qknorm+rope -> attention -> out+gated residual ->
-// norm2-modulate -> fc1+SwiGLU -> fc2+gated residual
-mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x, int n,
-                       const Plan& plan, const float* mods, const float2* cs, const Workspace& ws,
-                       cudaStream_t s, PhaseMark& pm) {
-  const int H = d.hidden, I = d.heads * d.head_dim, F = d.ffn;
+// norm1-modulate -> qkv+qknorm+rope (the part before attention)
+mmh3_status block_pre(const mmh3_dims& d, const mmh3_block_weights& w, const float* x, int n, const Plan& plan,
+                      const float* mods, const float2* cs, const Workspace& ws, cudaStream_t s, PhaseMark& pm) {
+  const int H = d.hidden, I = d.heads * d.head_dim;
   const int dt = d.act_dtype;
   const int stride = 6 * H;
   cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm1, d.eps, mods, stride, 0 * H, 1 * H, plan.block_rows, 0,
@@ -165,13 +163,29 @@ mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x
                             ws.qkv, s);
   if (st != MMH3_OK) return st;
   pm.mark(1);
-  st = attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, 1.0f / std::sqrt((float)d.head_dim), ws.attn, s);
+  return MMH3_OK;
+}
+
+// attention -> out+gated residual -> norm2-modulate -> fc1+SwiGLU -> fc2+gated
+// residual.  kv_all == nullptr: keys and values from this call's own qkv
+// panel; otherwise from kv_all [n_kv, 2*inner] (the gathered K|V rows).
+mmh3_status block_post(const mmh3_dims& d, const mmh3_block_weights& w, float* x, int n, const Plan& plan,
+                       const float* mods, const Workspace& ws, cudaStream_t s, PhaseMark& pm,
+                       const void* kv_all, int n_kv) {
+  const int H = d.hidden, I = d.heads * d.head_dim, F = d.ffn;
+  const int dt = d.act_dtype;
+  const int stride = 6 * H;
+  const float scale = 1.0f / std::sqrt((float)d.head_dim);
+  mmh3_status st = kv_all == nullptr
+                       ? attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, scale, ws.attn, s)
+                       : attention_kv(dt, ws.qkv, n, kv_all, n_kv, d.heads, d.head_dim, scale, ws.attn, s);
   if (st != MMH3_OK) return st;
   pm.mark(3);
   st = gemm_gated_residual(dt, ws.attn, w.wout, n, H, I, x, mods, stride, 2 * H, plan.block_rows, s);
   if (st != MMH3_OK) return st;
   pm.mark(4);
-  e = launch_norm_mod(dt, x, n, H, w.norm2, d.eps, mods, stride, 3 * H, 4 * H, plan.block_rows, 0, ws.xn2, s);
+  cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm2, d.eps, mods, stride, 3 * H, 4 * H, plan.block_rows, 0,
+                                  ws.xn2, s);
   if (e != cudaSuccess) return cuda_fail(e, "norm2/modulate launch");
   pm.mark(0);
   st = gemm_swiglu(dt, ws.xn2, w.wfc1, n, F, H, ws.act, s);
@@ -182,6 +196,15 @@ mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x
   pm.mark(7);
   if (pm.on) ++g_prof_blocks;
   return MMH3_OK;
+}
+
+// The whole block on one GPU.
+mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x, int n,
+                       const Plan& plan, const float* mods, const float2* cs, const Workspace& ws,
+                       cudaStream_t s, PhaseMark& pm) {
+  mmh3_status st = block_pre(d, w, x, n, plan, mods, cs, ws, s, pm);
+  if (st != MMH3_OK) return st;
+  return block_post(d, w, x, n, plan, mods, ws, s, pm, nullptr, 0);
 }
 
 mmh3_status common_checks(const mmh3_dims* dims, float* x, int n, const float* pos, void* ws,
@@ -369,6 +392,65 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
     if (st != MMH3_OK) return st;
   }
   return MMH3_OK;
+}
+
+// ------------------------------------------- block over a sequence shard
+mmh3_status mmh3_block_cp_begin(const mmh3_dims* dims, const mmh3_block_weights* w, const float* x, int n,
+                                const mmh3_segment* segs, int n_seg, const float* pos_dev, double sigma_v,
+                                double sigma_a, int modulated, void* kv_out, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  clear_error();
+  Workspace ws;
+  mmh3_status st = common_checks(dims, const_cast<float*>(x), n, pos_dev, workspace, ws_bytes, &ws);
+  if (st != MMH3_OK) return st;
+  if (dims->act_dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "sequence shards: bf16 activations only");
+  if (kv_out == nullptr || misaligned(kv_out)) return fail(MMH3_ERR_ARG, "kv_out null or not 16-byte aligned");
+  st = check_block(*dims, w, modulated != 0);
+  if (st != MMH3_OK) return st;
+  Plan plan;
+  if (modulated) {
+    st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+    if (st != MMH3_OK) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PhaseMark pm(s, false);
+  if (modulated) {
+    cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * dims->hidden,
+                                 plan, ws.mods, s);
+    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
+  }
+  if (pos_dev) {
+    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  }
+  st = block_pre(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s, pm);
+  if (st != MMH3_OK) return st;
+  const size_t I = (size_t)dims->heads * dims->head_dim;
+  cudaError_t e = cudaMemcpy2DAsync(kv_out, 2 * I * 2, static_cast<const uint8_t*>(ws.qkv) + I * 2, 3 * I * 2,
+                                    2 * I * 2, (size_t)n, cudaMemcpyDeviceToDevice, s);
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "K|V export copy");
+}
+
+mmh3_status mmh3_block_cp_end(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
+                              const mmh3_segment* segs, int n_seg, double sigma_v, double sigma_a, int modulated,
+                              const void* kv_all, int n_kv, void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  Workspace ws;
+  mmh3_status st = common_checks(dims, x, n, nullptr, workspace, ws_bytes, &ws);
+  if (st != MMH3_OK) return st;
+  if (dims->act_dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "sequence shards: bf16 activations only");
+  if (kv_all == nullptr || misaligned(kv_all)) return fail(MMH3_ERR_ARG, "kv_all null or not 16-byte aligned");
+  if (n_kv < n) return fail(MMH3_ERR_SHAPE, "n_kv = %d keys < the shard's %d rows", n_kv, n);
+  st = check_block(*dims, w, modulated != 0);
+  if (st != MMH3_OK) return st;
+  Plan plan;
+  if (modulated) {
+    st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+    if (st != MMH3_OK) return st;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PhaseMark pm(s, false);
+  return block_post(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, ws, s, pm, kv_all, n_kv);
 }
 
 // ------------------------------------------------------------ token refiner

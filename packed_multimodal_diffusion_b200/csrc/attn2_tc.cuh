@@ -45,8 +45,9 @@ struct Attn2Shape {
 
 template <int HD>
 __global__ void __launch_bounds__(320, 1)
-    attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, __nv_bfloat16* __restrict__ out, int ldo,
-                    int seq, int inner, float scale_log2, DevStatus* status, uint64_t limit_ns) {
+    attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tmkv,
+                    __nv_bfloat16* __restrict__ out, int ldo, int seq, int seq_kv, int k_off, int v_off,
+                    float scale_log2, DevStatus* status, uint64_t limit_ns) {
   using Sh = Attn2Shape<HD>;
   constexpr int KV = Sh::kKV;
   constexpr uint32_t kIdescS = make_idesc(false, 128, 128, false, false);
@@ -67,10 +68,15 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t bar0 = smem_u32(bars);
   auto bar = [&](int i) { return bar0 + 8u * i; };
 
+  // Queries: rows [z*seq, (z+1)*seq) of the panel `tm` (q at column 0).
+  // Keys / values: rows [z*seq_kv, (z+1)*seq_kv) of `tmkv`, k at column
+  // k_off, v at v_off (the same panel for a whole sequence on one GPU; the
+  // gathered K|V rows of all ranks for a sequence split over ranks).
   const int head = blockIdx.y;
   const int seq_row0 = blockIdx.z * seq;
+  const int kv_row0 = blockIdx.z * seq_kv;
   const int q_row0 = seq_row0 + blockIdx.x * 256;
-  const int n_kv = (seq + 127) / 128;
+  const int n_kv = (seq_kv + 127) / 128;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q), 1);
@@ -89,6 +95,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch(&tm);
+    tma_prefetch(&tmkv);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
   __syncthreads();
@@ -101,7 +108,7 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      const int xq = head * HD, xk = inner + head * HD, xv = 2 * inner + head * HD;
+      const int xq = head * HD, xk = k_off + head * HD, xv = v_off + head * HD;
       int in_k = 0, in_v = 0;
       bool ok = true;
       mbar_expect_tx(bar(B_Q), 2 * Sh::kTileBytes);
@@ -113,17 +120,17 @@ __global__ void __launch_bounds__(320, 1)
       for (; j < n_kv && ok; ++j) {
         const int s = j % KV;
         const uint32_t ph = (uint32_t)((j / KV) & 1);
-        const int y = seq_row0 + j * 128;
+        const int y = kv_row0 + j * 128;
         if (*abort_flag || !mbar_wait(bar(B_KE + s), ph ^ 1u, limit_ns)) { ok = false; break; }
         mbar_expect_tx(bar(B_KF + s), Sh::kTileBytes);
         for (int c = 0; c < Sh::kHdBoxes; ++c)
-          tma_load_2d(sbase + Sh::kKOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_KF + s),
+          tma_load_2d(sbase + Sh::kKOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tmkv, bar(B_KF + s),
                       xk + c * 64, y);
         in_k = j + 1;
         if (*abort_flag || !mbar_wait(bar(B_VE + s), ph ^ 1u, limit_ns)) { ok = false; break; }
         mbar_expect_tx(bar(B_VF + s), Sh::kTileBytes);
         for (int c = 0; c < Sh::kHdBoxes; ++c)
-          tma_load_2d(sbase + Sh::kVOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_VF + s),
+          tma_load_2d(sbase + Sh::kVOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tmkv, bar(B_VF + s),
                       xv + c * 64, y);
         in_v = j + 1;
       }
@@ -234,7 +241,7 @@ __global__ void __launch_bounds__(320, 1)
           s[96 + i] = __uint_as_float(u3[i]);
         }
       }
-      const int valid = seq - j * 128;
+      const int valid = seq_kv - j * 128;
       if (valid < 128) {
 #pragma unroll
         for (int k = 0; k < 128; ++k)

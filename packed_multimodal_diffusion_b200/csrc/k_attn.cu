@@ -70,21 +70,36 @@ static mmh3_status run_attn_f32(const void* qkv, int n_seq, int seq, int heads, 
   return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "fp32 attention launch");
 }
 
+// kv == nullptr: keys and values come from the qkv panel itself (columns
+// inner and 2*inner).  Otherwise from kv [n_seq*seq_kv, 2*inner] (k at
+// column 0, v at inner); the map covers exactly n_seq*seq_kv rows, so rows
+// a caller padded beyond them are never read.
 template <int HD>
-static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, int heads, float scale, void* out,
-                             cudaStream_t s) {
+static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv, int seq_kv, int heads,
+                             float scale, void* out, cudaStream_t s) {
   using Sh = Attn2Shape<HD>;
   static_assert(Sh::kSmem <= 232448, "attention shared memory above the per-CTA limit");
   const int inner = heads * HD;
-  CUtensorMap tm;
+  CUtensorMap tm, tkv;
   if (!make_tmap_2d(&tm, qkv, 2, (uint64_t)(3 * inner), (uint64_t)n_seq * seq, 128))
     return fail(MMH3_ERR_CUDA, "attention: cuTensorMapEncodeTiled failed");
+  int k_off = inner, v_off = 2 * inner;
+  if (kv != nullptr) {
+    if (!make_tmap_2d(&tkv, kv, 2, (uint64_t)(2 * inner), (uint64_t)n_seq * seq_kv, 128))
+      return fail(MMH3_ERR_CUDA, "attention: cuTensorMapEncodeTiled failed for K|V");
+    k_off = 0;
+    v_off = inner;
+  } else {
+    tkv = tm;
+    seq_kv = seq;
+  }
   auto kern = attn2_tc_kernel<HD>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmem);
   if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
   dim3 grid((seq + 255) / 256, heads, n_seq);
-  kern<<<grid, Sh::kThreads, Sh::kSmem, s>>>(tm, static_cast<__nv_bfloat16*>(out), inner, seq, inner,
-                                             scale * 1.4426950408889634f, device_status_ptr(), wait_limit_ns());
+  kern<<<grid, Sh::kThreads, Sh::kSmem, s>>>(tm, tkv, static_cast<__nv_bfloat16*>(out), inner, seq, seq_kv, k_off,
+                                             v_off, scale * 1.4426950408889634f, device_status_ptr(),
+                                             wait_limit_ns());
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return MMH3_OK;
@@ -95,10 +110,22 @@ mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads,
   if (n_seq <= 0 || seq <= 0) return MMH3_OK;
   if ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "attention: pointer not 16-byte aligned");
-  if (dtype == MMH3_BF16 && head_dim == 128) return run_attn2<128>(qkv, n_seq, seq, heads, scale, out, s);
-  if (dtype == MMH3_BF16 && head_dim == 64) return run_attn2<64>(qkv, n_seq, seq, heads, scale, out, s);
+  if (dtype == MMH3_BF16 && head_dim == 128) return run_attn2<128>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, s);
+  if (dtype == MMH3_BF16 && head_dim == 64) return run_attn2<64>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, s);
   if (dtype == MMH3_F32 && head_dim == 64) return run_attn_f32<64>(qkv, n_seq, seq, heads, scale, out, s);
   return fail(MMH3_ERR_SHAPE, "attention: dtype %d head_dim %d unsupported", dtype, head_dim);
+}
+
+mmh3_status attention_kv(int dtype, const void* q_panel, int n_q, const void* kv, int n_kv, int heads,
+                         int head_dim, float scale, void* out, cudaStream_t s) {
+  if (n_q <= 0) return MMH3_OK;
+  if (n_kv <= 0) return fail(MMH3_ERR_SHAPE, "attention: %d keys", n_kv);
+  if ((reinterpret_cast<uintptr_t>(q_panel) | reinterpret_cast<uintptr_t>(kv) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return fail(MMH3_ERR_ALIGN, "attention: pointer not 16-byte aligned");
+  if (dtype == MMH3_BF16 && head_dim == 128) return run_attn2<128>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, s);
+  if (dtype == MMH3_BF16 && head_dim == 64) return run_attn2<64>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, s);
+  return fail(MMH3_ERR_UNSUPPORTED, "attention over gathered K|V: bf16 only (dtype %d, head_dim %d)", dtype,
+              head_dim);
 }
 
 }  // namespace mmh3

@@ -78,6 +78,8 @@ mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, i
                                const float* bias, float* x, cudaStream_t s);
 mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads, int head_dim,
                       float scale, void* out, cudaStream_t s);
+mmh3_status attention_kv(int dtype, const void* q_panel, int n_q, const void* kv, int n_kv, int heads,
+                         int head_dim, float scale, void* out, cudaStream_t s);
 
 // The block on a caller-provided scratch region (see mmh3_workspace_size);
 // profile = false records no phase-profile events.

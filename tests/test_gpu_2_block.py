@@ -124,3 +124,18 @@ def test_block_workload_full_size_sampled_rows(cuda_ok):
     assert_close(reg["attn"][sample], keep["attn"], what="attn rows", rel=BF16_STORE_REL)
     assert_close(reg["xn2"][sample], keep["xn2"], what="xn2 rows", rel=BF16_STORE_REL)
     assert_close(reg["act"][sample], keep["act"], what="act rows", rel=BF16_STORE_REL)
+
+
+@pytest.mark.parametrize("layout", [(16, 2, 20, 20, 20), (17, 2, 20, 20, 20), (16, 2, 8, 82, 20),
+                                    (17, 2, 24, 38, 20)])
+def test_block_pair_tile_boundaries(cuda_ok, layout):
+    # n = 256, 257, 384, 513: one exact 256-row pair tile; a second pair tile
+    # whose upper CTA holds no row (its loads and stores are skipped); a
+    # second tile whose lower CTA is full; a single valid row in the last tile
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(*layout)
+    n = int(pos.shape[0])
+    w = small_block_weights(35, 256, 2, 128, 512)
+    x = configs.synth.normal((n, 256), 85, 1.0)
+    sv, sa = sigma_pair(0.5)
+    _check_block(dims_o, dims_c, w, x, segs, pos, sv, sa, (BF16_MAXABS, BF16_COS, BF16_STORE_REL))
