@@ -220,6 +220,33 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                                double sigma_v, double sigma_a, float* out_video, float* out_audio,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* ----------------------------------------------------- block on host data */
+
+/* One modulated block whose input and result live in host memory, with the
+ * copies overlapped with other calls' compute.  Per call, ordered by events:
+ *   copy_in_stream:  x_in_host -> x_dev and pos_host -> pos_dev (after the
+ *                    previous call on the same slot has copied its result
+ *                    out of x_dev);
+ *   stream:          mmh3_block_forward on x_dev / pos_dev (workspace as
+ *                    there);
+ *   copy_out_stream: x_dev -> x_out_host.
+ * The call returns at once.  Alternate slot 0 and 1 with two sets of
+ * device buffers (x_dev [n, H] fp32 and pos_dev [n, 3] fp32 per slot): the
+ * copies of one call then overlap the block of the other.  Host buffers
+ * must be pinned (cudaHostAlloc / cudaHostRegister) for the copies to be
+ * asynchronous, and stay untouched until the call's copy-out has finished
+ * (synchronize copy_out_stream).  pos_host / pos_dev may both be NULL (no
+ * rotation).  The events are the library's, one set per device: calls on
+ * one device must come from one host thread at a time.  No counterpart in
+ * the pages; this is how a caller keeps the host transfers off the
+ * critical path. */
+mmh3_status mmh3_block_forward_host(const mmh3_dims* dims, const mmh3_block_weights* w,
+                                    const float* x_in_host, float* x_out_host, int n,
+                                    const mmh3_segment* segs, int n_seg, const float* pos_host,
+                                    double sigma_v, double sigma_a, int slot, float* x_dev,
+                                    float* pos_dev, void* workspace, size_t ws_bytes, void* stream,
+                                    void* copy_in_stream, void* copy_out_stream);
+
 /* ------------------------------------------- block over a sequence shard */
 
 /* The block split at its one exchange step, for a packed sequence whose

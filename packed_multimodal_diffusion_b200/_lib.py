@@ -95,6 +95,8 @@ SIGNATURES = {
     "mmh3_stack_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _I,
                                 C.POINTER(HeadWeights), _P, _I, _SEGP, _I, _P, _D, _D, _P, _P, _P,
                                 C.c_size_t, _P]),
+    "mmh3_block_forward_host": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _P, _I, _SEGP, _I,
+                                     _P, _D, _D, _I, _P, _P, _P, C.c_size_t, _P, _P, _P]),
     "mmh3_block_cp_begin": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _P,
                                  _D, _D, _I, _P, _P, C.c_size_t, _P]),
     "mmh3_block_cp_end": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _D, _D,

@@ -19,7 +19,7 @@ from ._lib import (MMH3_BF16, MMH3_F32, MMH3_STREAM_AUDIO, MMH3_STREAM_VIDEO, Bl
 __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_image",
            "plan_timesteps", "time_shift_sigma", "resolve_rows", "adaln_modulation",
            "prepare_fc1", "workspace_size", "attention", "BlockParams", "HeadParams",
-           "block_forward", "stack_forward", "block_cp_begin", "block_cp_end", "refine_workspace_size", "refine_text",
+           "block_forward", "stack_forward", "block_forward_host", "block_cp_begin", "block_cp_end", "refine_workspace_size", "refine_text",
            "patch_embed_workspace_size", "patch_embed", "embed_workspace_size", "embed",
            "unpatchify_video", "unpack_audio", "forward_workspace_size", "forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
            "vit_layer_forward", "device_status", "selftest_wait_timeout", "set_wait_limit_ns",
@@ -196,6 +196,30 @@ def stack_forward(dims: Dims, blocks: list, heads: HeadParams | None, x: torch.T
                                     segments(segs), len(segs), _ptr(pos), sigma_v, sigma_a,
                                     _ptr(out_video), _ptr(out_audio), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream()))
+
+
+# ---------------------------------------------------- block on host buffers
+def _host_ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_contiguous() or not t.is_pinned():
+        raise ValueError("expected a contiguous pinned host tensor")
+    return t.data_ptr()
+
+
+def block_forward_host(dims: Dims, params: BlockParams, x_in: torch.Tensor, x_out: torch.Tensor,
+                       segs, pos: torch.Tensor | None, sigma_v: float, sigma_a: float, slot: int,
+                       x_dev: torch.Tensor, pos_dev: torch.Tensor | None, workspace: torch.Tensor,
+                       copy_in: torch.cuda.Stream, copy_out: torch.cuda.Stream) -> None:
+    """One block from pinned host x_in (and pos) to pinned host x_out,
+    through device slot `slot` (x_dev, pos_dev); copies on copy_in /
+    copy_out, the block on the current stream.  Returns without waiting."""
+    st = params.struct()
+    check(load().mmh3_block_forward_host(C.byref(dims), C.byref(st), _host_ptr(x_in), _host_ptr(x_out),
+                                         x_in.shape[0], segments(segs), len(segs), _host_ptr(pos),
+                                         sigma_v, sigma_a, slot, _ptr(x_dev), _ptr(pos_dev),
+                                         _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _stream(), copy_in.cuda_stream, copy_out.cuda_stream))
 
 
 # ------------------------------------------------ block over a sequence shard

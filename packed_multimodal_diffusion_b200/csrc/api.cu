@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "mmh3_internal.h"
@@ -392,6 +393,85 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
     if (st != MMH3_OK) return st;
   }
   return MMH3_OK;
+}
+
+// ----------------------------------------------- block on host buffers
+namespace {
+
+// Per device: the events that order the copy-in, compute and copy-out
+// streams of the two staging slots.
+struct HostSlots {
+  bool ready = false;
+  cudaEvent_t in_done[2], compute_done[2], out_done[2];
+};
+constexpr int kMaxHostDevices = 64;
+HostSlots g_host_slots[kMaxHostDevices];
+std::mutex g_host_mu;
+
+mmh3_status host_slots(HostSlots** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "host pipeline: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxHostDevices) return fail(MMH3_ERR_UNSUPPORTED, "host pipeline: device %d", dev);
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostSlots& h = g_host_slots[dev];
+  if (!h.ready) {
+    for (int k = 0; k < 2; ++k) {
+      cudaEvent_t* evs[3] = {&h.in_done[k], &h.compute_done[k], &h.out_done[k]};
+      for (cudaEvent_t* ev : evs) {
+        e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_fail(e, "host pipeline: event");
+      }
+      // a never-used slot counts as free: record the "copied out" event once
+      e = cudaEventRecord(h.out_done[k], 0);
+      if (e != cudaSuccess) return cuda_fail(e, "host pipeline: event record");
+    }
+    h.ready = true;
+  }
+  *out = &h;
+  return MMH3_OK;
+}
+
+}  // namespace
+
+mmh3_status mmh3_block_forward_host(const mmh3_dims* dims, const mmh3_block_weights* w, const float* x_in_host,
+                                    float* x_out_host, int n, const mmh3_segment* segs, int n_seg,
+                                    const float* pos_host, double sigma_v, double sigma_a, int slot,
+                                    float* x_dev, float* pos_dev, void* workspace, size_t ws_bytes, void* stream,
+                                    void* copy_in_stream, void* copy_out_stream) {
+  clear_error();
+  mmh3_status st = check_dims(dims);
+  if (st != MMH3_OK) return st;
+  if (slot != 0 && slot != 1) return fail(MMH3_ERR_ARG, "host block: slot %d is neither 0 nor 1", slot);
+  if (!x_in_host || !x_out_host || !x_dev) return fail(MMH3_ERR_ARG, "host block: null x buffer");
+  if ((pos_host == nullptr) != (pos_dev == nullptr))
+    return fail(MMH3_ERR_ARG, "host block: pos_host and pos_dev must both be given or both be null");
+  if (n < 1) return fail(MMH3_ERR_SHAPE, "host block: n = %d < 1", n);
+  HostSlots* h = nullptr;
+  st = host_slots(&h);
+  if (st != MMH3_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t si = static_cast<cudaStream_t>(copy_in_stream);
+  cudaStream_t so = static_cast<cudaStream_t>(copy_out_stream);
+  const size_t xb = (size_t)n * dims->hidden * sizeof(float), pb = (size_t)n * 3 * sizeof(float);
+  // 1. copy in, once the slot's previous result has left the device
+  cudaError_t e = cudaStreamWaitEvent(si, h->out_done[slot], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(x_dev, x_in_host, xb, cudaMemcpyHostToDevice, si);
+  if (e == cudaSuccess && pos_host) e = cudaMemcpyAsync(pos_dev, pos_host, pb, cudaMemcpyHostToDevice, si);
+  if (e == cudaSuccess) e = cudaEventRecord(h->in_done[slot], si);
+  if (e != cudaSuccess) return cuda_fail(e, "host block: copy in");
+  // 2. the block, after its input arrived
+  e = cudaStreamWaitEvent(s, h->in_done[slot], 0);
+  if (e != cudaSuccess) return cuda_fail(e, "host block: wait for the input");
+  st = mmh3::block_forward_impl(dims, w, x_dev, n, segs, n_seg, pos_dev, sigma_v, sigma_a, 1, workspace, ws_bytes,
+                                stream, /*profile=*/false);
+  if (st != MMH3_OK) return st;
+  e = cudaEventRecord(h->compute_done[slot], s);
+  // 3. copy the result out
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(so, h->compute_done[slot], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(x_out_host, x_dev, xb, cudaMemcpyDeviceToHost, so);
+  if (e == cudaSuccess) e = cudaEventRecord(h->out_done[slot], so);
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "host block: copy out");
 }
 
 // ------------------------------------------- block over a sequence shard
