@@ -1,11 +1,14 @@
 // The C ABI entry points that run the hot path: adaLN modulation, the
-// modulated block, the 50-block stack with its output heads, and the SigLIP
-// encoder layer.  Each entry point validates everything before the first
-// launch and then enqueues a fixed sequence of kernels on the caller's
-// stream (no host synchronisation, no allocation).
+// modulated block, the 50-block stack with its output heads, the SigLIP
+// encoder layer, and around them the token refiner, the embed and output
+// unpacking, one whole denoise evaluation, the block over a sequence shard
+// and the block on host buffers.  Each entry point validates everything
+// before the first launch and then enqueues a fixed sequence of kernels on
+// the caller's stream(s) (no host synchronisation, no allocation).
 //
 // Step order follows "cortiq_engine/mmh3.rs" (cortiq-engine 0.5.72):
-// MiniMaxH3::forward ("blocks", "heads"), block_forward and ffn_tail;
+// MiniMaxH3::forward ("embed", "blocks", "heads"), refine_text,
+// block_forward and ffn_tail;
 // the encoder layer follows "ffai-argus 0.7.0 src/siglip.rs",
 // Layer::forward and finish_attention.
 #include <algorithm>

@@ -1,4 +1,4 @@
-// Persistent, warp-specialised tcgen05 GEMM  C[M, N] = A[M, K] * B[N, K]^T
+// Persistent, warp-specialised tcgen05 GEMMs  C[M, N] = A[M, K] * B[N, K]^T
 // with the block's epilogues fused in.
 //
 // Roles (192 threads, one CTA per SM):
@@ -7,8 +7,12 @@
 //   warps 2..5  epilogue: tcgen05.ld the accumulator rows, apply the fused
 //               epilogue, store; the second TMEM buffer lets the next tile's
 //               MMAs run under this tile's epilogue.
-// Tiles are 128 x BN x (128 bytes of K); operands are bf16 (kind::f16) or
-// fp32 read as tf32 (kind::tf32).  Every wait is bounded (mbar_wait) and a
+// gemm_tc_kernel: one CTA per 128 x BN tile, operands bf16 (kind::f16) or
+// fp32 read as tf32 (kind::tf32).  gemm2_tc_kernel (further down): CTA pairs
+// on one TPC computing 256 x BN tiles with tcgen05.mma.cta_group::2, bf16.
+// Epilogues either store each thread's row directly or (kStageOut > 0) stage
+// 128-row x 128-byte boxes in shared memory and move them with TMA tensor
+// loads / stores (OutStage).  Every wait is bounded (mbar_wait) and a
 // timeout leaves the loops, drains in-flight copies and frees TMEM.
 #pragma once
 

@@ -1,9 +1,12 @@
 // Host launchers of the tcgen05 GEMM instantiations and the TMA tensor-map
 // encoder.  The block's four projections ("cortiq_engine/mmh3.rs",
-// block_forward / ffn_tail: qkv, out, fc1, fc2, and the output heads of
-// forward) and the encoder layer's four biased projections ("ffai-argus
-// 0.7.0 src/siglip.rs", Layer::forward / finish_attention) all go through
-// gemm_tc_kernel with the matching fused epilogue.
+// block_forward / ffn_tail: qkv, out, fc1, fc2), the output heads and the
+// patch / condition projections of forward and refine_text, and the encoder
+// layer's four biased projections ("ffai-argus 0.7.0 src/siglip.rs",
+// Layer::forward / finish_attention) all go through gemm_tc_kernel or its
+// CTA-pair form gemm2_tc_kernel with the matching fused epilogue.  Which one
+// runs is fixed per call shape (use_pairs and the dispatch below), not
+// switched at run time.
 #include <cudaTypedefs.h>
 
 #include <mutex>
