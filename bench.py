@@ -361,17 +361,28 @@ class OracleSample:
         mods = O.block_mods(p["adaln_w"], p["adaln_b"], p["adaln_table"], self.ts, c.hidden)
         O.block_forward(p, self.x, mods, self.rows_of, self.L["pos"], c.dims(), sample_rows=rows)
 
-    def calibrate(self):
+    def calibrate(self, rows: int = 192, reps: int = 2):
         """Per-row cost of the block (attention over all keys, projections,
-        FFN) from two runs that differ only in the number of query rows."""
-        t0 = time.perf_counter()
-        self._block(self.sample[:1])
-        t_one = time.perf_counter() - t0
-        t0 = time.perf_counter()
-        self._block(self.sample)
-        t_s = time.perf_counter() - t0
-        self.t_row = max(0.0, (t_s - t_one) / (len(self.sample) - 1))
-        return t_one + t_s
+        FFN): the difference between a `rows`-row and a 1-row run, each the
+        best of `reps`.  Both runs share the fixed cost of k and v for all
+        tokens (seconds on the host), so the row count must be large enough
+        for the marginal cost to stand well above that cost's run-to-run
+        noise."""
+        import numpy as np
+        big = np.linspace(0, self.n - 1, rows).astype(int)
+
+        def best(r):
+            ts = []
+            for _ in range(reps):
+                t0 = time.perf_counter()
+                self._block(r)
+                ts.append(time.perf_counter() - t0)
+            return min(ts)
+
+        t_one = best(self.sample[:1])
+        t_big = best(big)
+        self.t_row = max(0.0, (t_big - t_one) / (len(big) - 1))
+        self.calib_rows = len(big)
 
     def run(self):
         """Time one sample; -> (seconds, extrapolated full-block seconds)."""
@@ -386,7 +397,7 @@ class OracleSample:
         return (f"block workload: k/v for all {self.n} tokens + {len(self.sample)} sampled query "
                 f"rows through the whole block ({t_s:.2f} s); full {self.n}-row block "
                 f"extrapolated with the per-row cost measured between 1 and "
-                f"{len(self.sample)} rows ({t_full:.1f} s)")
+                f"{self.calib_rows} rows, best of 2 ({t_full:.1f} s)")
 
 
 def cpu_baseline(rows_sample):
