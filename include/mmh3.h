@@ -191,6 +191,20 @@ mmh3_status mmh3_workspace_size(const mmh3_dims* dims, int n, size_t* bytes);
 mmh3_status mmh3_attention(const void* qkv, int n_seq, int seq, int heads, int head_dim,
                            int act_dtype, float scale, void* out, void* stream);
 
+/* mmh3_attention with a scratch region for the last wave (bf16 only).
+ * Work units of 256 query rows of one head fill the SMs in waves; when
+ * the last wave would hold at most half as many units as there are SMs,
+ * each of its units is split along the keys over f = min(SMs / units, 4,
+ * key tiles) CTAs whose partial results (unnormalised O, running maximum,
+ * row sum: 256 x (head_dim + 4) fp32 per CTA) go to scratch and are then
+ * merged.  Without room in scratch (or with scratch NULL) nothing is split.
+ * The result equals mmh3_attention's up to the order of the softmax sums.
+ * The block entry points give attention this region from their workspace
+ * (the head scratch, unused inside a block). */
+mmh3_status mmh3_attention_ws(const void* qkv, int n_seq, int seq, int heads, int head_dim,
+                              int act_dtype, float scale, void* out, void* scratch,
+                              size_t scratch_bytes, void* stream);
+
 /* One modulated block, in place on x [n, H] fp32 (device)
  * ("cortiq_engine/mmh3.rs", block_forward + ffn_tail):
  *   mods = adaLN(ts); xn1 = RMSNorm(x; norm1)(1+scale_msa)+shift_msa;

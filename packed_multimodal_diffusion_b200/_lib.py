@@ -88,6 +88,7 @@ SIGNATURES = {
     "mmh3_prepare_fc1": (_I, [C.POINTER(Dims), _P, _P, _P]),
     "mmh3_workspace_size": (_I, [C.POINTER(Dims), _I, C.POINTER(C.c_size_t)]),
     "mmh3_attention": (_I, [_P, _I, _I, _I, _I, _I, C.c_float, _P, _P]),
+    "mmh3_attention_ws": (_I, [_P, _I, _I, _I, _I, _I, C.c_float, _P, _P, C.c_size_t, _P]),
     "mmh3_block_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _P,
                                 _D, _D, _I, _P, C.c_size_t, _P]),
     "mmh3_block_forward_noalloc": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I,

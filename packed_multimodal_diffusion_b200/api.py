@@ -18,7 +18,7 @@ from ._lib import (MMH3_BF16, MMH3_F32, MMH3_STREAM_AUDIO, MMH3_STREAM_VIDEO, Bl
 
 __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_image",
            "plan_timesteps", "time_shift_sigma", "resolve_rows", "adaln_modulation",
-           "prepare_fc1", "workspace_size", "attention", "BlockParams", "HeadParams",
+           "prepare_fc1", "workspace_size", "attention", "attention_ws", "BlockParams", "HeadParams",
            "block_forward", "stack_forward", "block_forward_host", "block_cp_begin", "block_cp_end", "refine_workspace_size", "refine_text",
            "patch_embed_workspace_size", "patch_embed", "embed_workspace_size", "embed",
            "unpatchify_video", "unpack_audio", "forward_workspace_size", "forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
@@ -124,6 +124,14 @@ def attention(qkv: torch.Tensor, n_seq: int, seq: int, heads: int, head_dim: int
               out: torch.Tensor) -> None:
     check(load().mmh3_attention(_ptr(qkv), n_seq, seq, heads, head_dim, _dtype_code(qkv.dtype),
                                 scale, _ptr(out), _stream()))
+
+
+def attention_ws(qkv: torch.Tensor, n_seq: int, seq: int, heads: int, head_dim: int, scale: float,
+                 out: torch.Tensor, scratch: torch.Tensor | None) -> None:
+    """attention with a scratch region that lets the last wave be split."""
+    nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
+    check(load().mmh3_attention_ws(_ptr(qkv), n_seq, seq, heads, head_dim, _dtype_code(qkv.dtype), scale,
+                                   _ptr(out), _ptr(scratch), nbytes, _stream()))
 
 
 @dataclass

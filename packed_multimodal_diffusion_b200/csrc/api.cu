@@ -180,9 +180,12 @@ mmh3_status block_post(const mmh3_dims& d, const mmh3_block_weights& w, float* x
   const int dt = d.act_dtype;
   const int stride = 6 * H;
   const float scale = 1.0f / std::sqrt((float)d.head_dim);
+  // the head region is free during a block: it holds split-attention partials
+  const size_t head_bytes = (size_t)n * H * esize_of(dt);
   mmh3_status st = kv_all == nullptr
-                       ? attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, scale, ws.attn, s)
-                       : attention_kv(dt, ws.qkv, n, kv_all, n_kv, d.heads, d.head_dim, scale, ws.attn, s);
+                       ? attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, scale, ws.attn, s, ws.head, head_bytes)
+                       : attention_kv(dt, ws.qkv, n, kv_all, n_kv, d.heads, d.head_dim, scale, ws.attn, s, ws.head,
+                                      head_bytes);
   if (st != MMH3_OK) return st;
   pm.mark(3);
   st = gemm_gated_residual(dt, ws.attn, w.wout, n, H, I, x, mods, stride, 2 * H, plan.block_rows, s);

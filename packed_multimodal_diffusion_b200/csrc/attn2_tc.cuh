@@ -41,13 +41,17 @@ struct Attn2Shape {
   static constexpr int kBarOff = kVOff + kKV * kTileBytes;
   static constexpr int kSmem = kBarOff + 512 + 1024;
   static constexpr int kThreads = 320;
+  // floats per query row of a partial result: O[HD], m, l, padded to 16 bytes
+  static constexpr int kPartStride = HD + 4;
+  static constexpr size_t kPartBytesPerCta = (size_t)256 * kPartStride * 4;
 };
 
 template <int HD>
 __global__ void __launch_bounds__(320, 1)
     attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tmkv,
                     __nv_bfloat16* __restrict__ out, int ldo, int seq, int seq_kv, int k_off, int v_off,
-                    float scale_log2, DevStatus* status, uint64_t limit_ns) {
+                    float scale_log2, int heads, int unit0, int split, float* __restrict__ part,
+                    DevStatus* status, uint64_t limit_ns) {
   using Sh = Attn2Shape<HD>;
   constexpr int KV = Sh::kKV;
   constexpr uint32_t kIdescS = make_idesc(false, 128, 128, false, false);
@@ -72,11 +76,22 @@ __global__ void __launch_bounds__(320, 1)
   // Keys / values: rows [z*seq_kv, (z+1)*seq_kv) of `tmkv`, k at column
   // k_off, v at v_off (the same panel for a whole sequence on one GPU; the
   // gathered K|V rows of all ranks for a sequence split over ranks).
-  const int head = blockIdx.y;
-  const int seq_row0 = blockIdx.z * seq;
-  const int kv_row0 = blockIdx.z * seq_kv;
-  const int q_row0 = seq_row0 + blockIdx.x * 256;
-  const int n_kv = (seq_kv + 127) / 128;
+  // Work unit u = unit0 + blockIdx.x / split: 256 query rows (q pair) of one
+  // head of one sequence.  With split > 1 the unit's key tiles are divided
+  // into `split` contiguous ranges, one per CTA, and each CTA writes its
+  // unnormalised partial result to `part` for attn_merge_kernel.
+  const int nq = (seq + 255) / 256;
+  const int u = unit0 + (int)blockIdx.x / split;
+  const int piece = (int)blockIdx.x % split;
+  const int qpair = u % nq;
+  const int head = (u / nq) % heads;
+  const int zseq = u / (nq * heads);
+  const int seq_row0 = zseq * seq;
+  const int kv_row0 = zseq * seq_kv;
+  const int q_row0 = seq_row0 + qpair * 256;
+  const int kv_tiles = (seq_kv + 127) / 128;
+  const int j0 = piece * kv_tiles / split;              // first key tile of this CTA
+  const int n_kv = (piece + 1) * kv_tiles / split - j0;  // key tiles of this CTA (>= 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q), 1);
@@ -120,7 +135,7 @@ __global__ void __launch_bounds__(320, 1)
       for (; j < n_kv && ok; ++j) {
         const int s = j % KV;
         const uint32_t ph = (uint32_t)((j / KV) & 1);
-        const int y = kv_row0 + j * 128;
+        const int y = kv_row0 + (j0 + j) * 128;
         if (*abort_flag || !mbar_wait(bar(B_KE + s), ph ^ 1u, limit_ns)) { ok = false; break; }
         mbar_expect_tx(bar(B_KF + s), Sh::kTileBytes);
         for (int c = 0; c < Sh::kHdBoxes; ++c)
@@ -241,7 +256,7 @@ __global__ void __launch_bounds__(320, 1)
           s[96 + i] = __uint_as_float(u3[i]);
         }
       }
-      const int valid = seq_kv - j * 128;
+      const int valid = seq_kv - (j0 + j) * 128;
       if (valid < 128) {
 #pragma unroll
         for (int k = 0; k < 128; ++k)
@@ -315,17 +330,32 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
-      const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
-      const int qr = blockIdx.x * 256 + wg * 128 + r;
+      const int qr = qpair * 256 + wg * 128 + r;
       const bool row_ok = qr < seq;
-      __nv_bfloat16* dst = out + (size_t)(seq_row0 + qr) * ldo + head * HD;
+      if (split == 1) {
+        const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
+        __nv_bfloat16* dst = out + (size_t)(seq_row0 + qr) * ldo + head * HD;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
-        float v[32];
-        ld_acc32(to + c * 32, v);
+        for (int c = 0; c < HD / 32; ++c) {
+          float v[32];
+          ld_acc32(to + c * 32, v);
 #pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) v[i2] *= inv;
-        if (row_ok) store32(dst + c * 32, v);
+          for (int i2 = 0; i2 < 32; ++i2) v[i2] *= inv;
+          if (row_ok) store32(dst + c * 32, v);
+        }
+      } else {
+        // partial: O unnormalised (relative to m_ref), then m_ref and l_sum
+        float* dst = part + ((size_t)blockIdx.x * 256 + wg * 128 + r) * Attn2Shape<HD>::kPartStride;
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          float v[32];
+          ld_acc32(to + c * 32, v);
+          if (row_ok) store32(dst + c * 32, v);
+        }
+        if (row_ok) {
+          dst[HD] = m_ref;
+          dst[HD + 1] = l_sum;
+        }
       }
     }
   }
@@ -333,6 +363,45 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Combine the `split` partial results of each tail unit (unnormalised O,
+// reference maximum m in the log2 domain, row sum l):
+//   m* = max_p m_p,  w_p = 2^(m_p - m*),  O = sum_p w_p O_p / sum_p w_p l_p.
+// One thread per query row of the unit.
+template <int HD>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ part, int split,
+                                                         __nv_bfloat16* __restrict__ out, int ldo, int seq,
+                                                         int heads, int unit0) {
+  const int nq = (seq + 255) / 256;
+  const int t = blockIdx.x;
+  const int u = unit0 + t;
+  const int qpair = u % nq;
+  const int head = (u / nq) % heads;
+  const int zseq = u / (nq * heads);
+  const int r = threadIdx.x;
+  const int qr = qpair * 256 + r;
+  if (qr >= seq) return;
+  auto row = [&](int p) { return part + ((size_t)(t * split + p) * 256 + r) * Attn2Shape<HD>::kPartStride; };
+  float m = -INFINITY;
+  for (int p = 0; p < split; ++p) m = fmaxf(m, row(p)[HD]);
+  float l = 0.f;
+  for (int p = 0; p < split; ++p) l += ex2_approx(row(p)[HD] - m) * row(p)[HD + 1];
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
+  __nv_bfloat16* dst = out + (size_t)(zseq * seq + qr) * ldo + head * HD;
+#pragma unroll 1
+  for (int c = 0; c < HD / 32; ++c) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    for (int p = 0; p < split; ++p) {
+      const float* o = row(p) + c * 32;
+      const float wgt = ex2_approx(row(p)[HD] - m) * inv;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaf(wgt, o[i], v[i]);
+    }
+    store32(dst + c * 32, v);
   }
 }
 

@@ -74,9 +74,16 @@ static mmh3_status run_attn_f32(const void* qkv, int n_seq, int seq, int heads, 
 // inner and 2*inner).  Otherwise from kv [n_seq*seq_kv, 2*inner] (k at
 // column 0, v at inner); the map covers exactly n_seq*seq_kv rows, so rows
 // a caller padded beyond them are never read.
+//
+// Work units (256 query rows of one head) fill the SMs in waves, one CTA per
+// SM.  When the last wave would hold at most half as many units as there
+// are SMs, and `scratch` has room, each of those tail units is split over
+// f = min(SMs / tail, 4, key tiles) CTAs along the keys; their partial
+// results are merged by attn_merge_kernel, so the tail takes about 1/f of a
+// wave.
 template <int HD>
 static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv, int seq_kv, int heads,
-                             float scale, void* out, cudaStream_t s) {
+                             float scale, void* out, void* scratch, size_t scratch_bytes, cudaStream_t s) {
   using Sh = Attn2Shape<HD>;
   static_assert(Sh::kSmem <= 232448, "attention shared memory above the per-CTA limit");
   const int inner = heads * HD;
@@ -96,34 +103,62 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
   auto kern = attn2_tc_kernel<HD>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmem);
   if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
-  dim3 grid((seq + 255) / 256, heads, n_seq);
-  kern<<<grid, Sh::kThreads, Sh::kSmem, s>>>(tm, tkv, static_cast<__nv_bfloat16*>(out), inner, seq, seq_kv, k_off,
-                                             v_off, scale * 1.4426950408889634f, device_status_ptr(),
-                                             wait_limit_ns());
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  const float sl2 = scale * 1.4426950408889634f;
+  const int nq = (seq + 255) / 256;
+  const int units = n_seq * heads * nq;
+  const int sms = num_sms();
+  const int tail = units % sms;
+  const int kv_tiles = (seq_kv + 127) / 128;
+  int f = tail > 0 ? sms / tail : 1;
+  f = f < 4 ? f : 4;
+  f = f < kv_tiles ? f : kv_tiles;
+  const bool split = f >= 2 && scratch != nullptr &&
+                     (size_t)tail * f * Sh::kPartBytesPerCta <= scratch_bytes &&
+                     (reinterpret_cast<uintptr_t>(scratch) & 15) == 0;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  const int whole = split ? units - tail : units;
+  if (whole > 0) {
+    kern<<<whole, Sh::kThreads, Sh::kSmem, s>>>(tm, tkv, o, inner, seq, seq_kv, k_off, v_off, sl2, heads, 0, 1,
+                                               nullptr, device_status_ptr(), wait_limit_ns());
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  }
+  if (split) {
+    float* part = static_cast<float*>(scratch);
+    kern<<<tail * f, Sh::kThreads, Sh::kSmem, s>>>(tm, tkv, o, inner, seq, seq_kv, k_off, v_off, sl2, heads,
+                                                   units - tail, f, part, device_status_ptr(), wait_limit_ns());
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "attention (split tail) launch");
+    attn_merge_kernel<HD><<<tail, 256, 0, s>>>(part, f, o, inner, seq, heads, units - tail);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
+  }
   return MMH3_OK;
 }
 
 mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads, int head_dim,
-                      float scale, void* out, cudaStream_t s) {
+                      float scale, void* out, cudaStream_t s, void* scratch, size_t scratch_bytes) {
   if (n_seq <= 0 || seq <= 0) return MMH3_OK;
   if ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "attention: pointer not 16-byte aligned");
-  if (dtype == MMH3_BF16 && head_dim == 128) return run_attn2<128>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, s);
-  if (dtype == MMH3_BF16 && head_dim == 64) return run_attn2<64>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, s);
+  if (dtype == MMH3_BF16 && head_dim == 128)
+    return run_attn2<128>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, scratch, scratch_bytes, s);
+  if (dtype == MMH3_BF16 && head_dim == 64)
+    return run_attn2<64>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, scratch, scratch_bytes, s);
   if (dtype == MMH3_F32 && head_dim == 64) return run_attn_f32<64>(qkv, n_seq, seq, heads, scale, out, s);
   return fail(MMH3_ERR_SHAPE, "attention: dtype %d head_dim %d unsupported", dtype, head_dim);
 }
 
 mmh3_status attention_kv(int dtype, const void* q_panel, int n_q, const void* kv, int n_kv, int heads,
-                         int head_dim, float scale, void* out, cudaStream_t s) {
+                         int head_dim, float scale, void* out, cudaStream_t s, void* scratch, size_t scratch_bytes) {
   if (n_q <= 0) return MMH3_OK;
   if (n_kv <= 0) return fail(MMH3_ERR_SHAPE, "attention: %d keys", n_kv);
   if ((reinterpret_cast<uintptr_t>(q_panel) | reinterpret_cast<uintptr_t>(kv) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "attention: pointer not 16-byte aligned");
-  if (dtype == MMH3_BF16 && head_dim == 128) return run_attn2<128>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, s);
-  if (dtype == MMH3_BF16 && head_dim == 64) return run_attn2<64>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, s);
+  if (dtype == MMH3_BF16 && head_dim == 128)
+    return run_attn2<128>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, scratch, scratch_bytes, s);
+  if (dtype == MMH3_BF16 && head_dim == 64)
+    return run_attn2<64>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, scratch, scratch_bytes, s);
   return fail(MMH3_ERR_UNSUPPORTED, "attention over gathered K|V: bf16 only (dtype %d, head_dim %d)", dtype,
               head_dim);
 }
@@ -139,4 +174,12 @@ extern "C" mmh3_status mmh3_attention(const void* qkv, int n_seq, int seq, int h
   if (heads < 1 || n_seq < 0 || seq < 0) return fail(MMH3_ERR_SHAPE, "attention: bad sizes");
   if (act_dtype != MMH3_BF16 && act_dtype != MMH3_F32) return fail(MMH3_ERR_ARG, "attention: bad dtype");
   return attention(act_dtype, qkv, n_seq, seq, heads, head_dim, scale, out, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" mmh3_status mmh3_attention_ws(const void* qkv, int n_seq, int seq, int heads, int head_dim,
+                                         int act_dtype, float scale, void* out, void* scratch,
+                                         size_t scratch_bytes, void* stream) {
+  clear_error();
+  return attention(act_dtype, qkv, n_seq, seq, heads, head_dim, scale, out, static_cast<cudaStream_t>(stream),
+                   scratch, scratch_bytes);
 }

@@ -77,9 +77,11 @@ mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N,
 mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,
                                const float* bias, float* x, cudaStream_t s);
 mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads, int head_dim,
-                      float scale, void* out, cudaStream_t s);
+                      float scale, void* out, cudaStream_t s, void* scratch = nullptr,
+                      size_t scratch_bytes = 0);
 mmh3_status attention_kv(int dtype, const void* q_panel, int n_q, const void* kv, int n_kv, int heads,
-                         int head_dim, float scale, void* out, cudaStream_t s);
+                         int head_dim, float scale, void* out, cudaStream_t s, void* scratch = nullptr,
+                         size_t scratch_bytes = 0);
 
 // The block on a caller-provided scratch region (see mmh3_workspace_size);
 // profile = false records no phase-profile events.

@@ -115,3 +115,28 @@ def test_bounded_wait_returns_timeout_and_context_survives(cuda_ok):
     api.attention(qkv.cuda(), 1, n, heads, hd, 1 / math.sqrt(hd), out)
     api.device_status()
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("n_seq,seq,heads,hd", [(1, 700, 5, 128), (1, 300, 1, 128), (3, 200, 2, 64),
+                                                (1, 13248, 21, 128)])
+def test_attention_split_tail(cuda_ok, n_seq, seq, heads, hd):
+    # last-wave units split along the keys (partials + merge) against the
+    # oracle and against the unsplit kernel; the full-size case is the block
+    # workload's 1092 units (56 in the last wave, split in two)
+    n = n_seq * seq
+    qkv = _qkv(n, heads, hd, 300 + seq).cuda()
+    scale = 1 / math.sqrt(hd)
+    out = torch.full((n, heads * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    scratch = torch.empty(160 * 256 * (hd + 4) * 4, dtype=torch.uint8, device="cuda")
+    api.attention_ws(qkv, n_seq, seq, heads, hd, scale, out, scratch)
+    plain = torch.empty_like(out)
+    api.attention(qkv, n_seq, seq, heads, hd, scale, plain)
+    api.device_status()
+    assert_close(out, plain, 4e-3, 0.99999, "split tail vs unsplit", rel=2.0 ** -8)
+    rows = range(n) if n <= 1000 else range(0, n, 97)
+    for b in range(n_seq):
+        part = qkv[b * seq:(b + 1) * seq].cpu()
+        q, k, v = (f64(t).reshape(seq, heads, hd) for t in part.split(heads * hd, dim=1))
+        sel = [r - b * seq for r in rows if b * seq <= r < (b + 1) * seq]
+        ref = O.attention(q, k, v, scale, q_rows=np.asarray(sel)).reshape(len(sel), -1)
+        assert_close(out[b * seq:(b + 1) * seq][sel], ref, what=f"split tail sequence {b}")
