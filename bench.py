@@ -231,12 +231,14 @@ def run_gpu(args):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = api.launch_count()
     with ClockSampler(torch.cuda.current_device()) as clk:
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+    launches = api.launch_count() - launches0
     barrier()
     api.prof_enable(False)
     ms = e0.elapsed_time(e1)
@@ -319,7 +321,7 @@ def run_gpu(args):
         "e2e": {"value": job_throughput(world, n, e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(W["x0"].numel() * 4 + W["pos_d"].numel() * 4),
                 "d2h_bytes_per_step": int(W["x0"].numel() * 4)},
-        "gpu_launches": 9 * args.steps,
+        "gpu_launches": launches,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples": clocks["samples"]},
     }

@@ -526,6 +526,10 @@ void mmh3_prof_reset(void);
 /* Message of the last failing call on this thread ("" if none). */
 const char* mmh3_last_error(void);
 
+/* Number of kernels the library has launched in this process so far (all
+ * devices, all threads).  Host only, never fails. */
+long long mmh3_launch_count(void);
+
 /* Library version string. */
 const char* mmh3_version(void);
 

@@ -131,6 +131,7 @@ SIGNATURES = {
     "mmh3_prof_collect": (_I, [C.POINTER(C.c_double), _I, C.POINTER(C.c_long)]),
     "mmh3_prof_reset": (None, []),
     "mmh3_last_error": (C.c_char_p, []),
+    "mmh3_launch_count": (C.c_longlong, []),
     "mmh3_version": (C.c_char_p, []),
 }
 

@@ -442,6 +442,11 @@ def prof_collect() -> tuple[dict, int]:
     return dict(zip(PROF_SLOTS, list(ms))), nb.value
 
 
+def launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(load().mmh3_launch_count())
+
+
 def set_wait_limit_ns(ns: int) -> None:
     load().mmh3_set_wait_limit_ns(ns)
 

@@ -6,6 +6,7 @@
 // flow-schedule remap (time_shift_sigma), the packed layout
 // (axis_from_sqrt_area, push_audio_grid, Layout::build_full) and the
 // timestep / row assembly at the top of MiniMaxH3::forward.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -16,6 +17,9 @@
 #include "mmh3_internal.h"
 
 namespace mmh3 {
+
+static std::atomic<long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ errors
 static thread_local char g_msg[512] = "";
@@ -248,3 +252,5 @@ extern "C" mmh3_status mmh3_plan_timesteps(const mmh3_segment* segs, int n_seg, 
   for (int k = 0; k < n_seg; ++k) seg_rows[k] = p.block_rows.row[k];
   return MMH3_OK;
 }
+
+extern "C" long long mmh3_launch_count(void) { return mmh3::g_launches.load(std::memory_order_relaxed); }

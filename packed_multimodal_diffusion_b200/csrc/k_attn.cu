@@ -65,7 +65,7 @@ static mmh3_status run_attn_f32(const void* qkv, int n_seq, int seq, int heads, 
                                 cudaStream_t s) {
   dim3 grid((seq + 63) / 64, heads, n_seq);
   attn_f32_simt_kernel<HD><<<grid, 64, 0, s>>>(static_cast<const float*>(qkv), static_cast<float*>(out), seq,
-                                                heads * HD, scale);
+                                                heads * HD, scale); count_launch();
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "fp32 attention launch");
 }
@@ -119,17 +119,17 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
   const int whole = split ? units - tail : units;
   if (whole > 0) {
     kern<<<whole, Sh::kThreads, Sh::kSmem, s>>>(tm, tkv, o, inner, seq, seq_kv, k_off, v_off, sl2, heads, 0, 1,
-                                               nullptr, device_status_ptr(), wait_limit_ns());
+                                               nullptr, device_status_ptr(), wait_limit_ns()); count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   }
   if (split) {
     float* part = static_cast<float*>(scratch);
     kern<<<tail * f, Sh::kThreads, Sh::kSmem, s>>>(tm, tkv, o, inner, seq, seq_kv, k_off, v_off, sl2, heads,
-                                                   units - tail, f, part, device_status_ptr(), wait_limit_ns());
+                                                   units - tail, f, part, device_status_ptr(), wait_limit_ns()); count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "attention (split tail) launch");
-    attn_merge_kernel<HD><<<tail, 256, 0, s>>>(part, f, o, inner, seq, heads, units - tail);
+    attn_merge_kernel<HD><<<tail, 256, 0, s>>>(part, f, o, inner, seq, heads, units - tail); count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
   }

@@ -94,7 +94,7 @@ cudaError_t launch_adaln(const float* w, const float* b, const float* table, int
   int blocks = (total + 255) / 256;
   const int cap = num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  adaln_kernel<<<blocks, 256, 0, s>>>(w, b, table, rank, rows_per_slot, plan.n_ts, ca, out);
+  adaln_kernel<<<blocks, 256, 0, s>>>(w, b, table, rank, rows_per_slot, plan.n_ts, ca, out); count_launch();
   return cudaGetLastError();
 }
 
@@ -125,7 +125,7 @@ cudaError_t launch_rope_table(const float* pos, int n, int k, float theta, float
   const long total = (long)n * 3 * k;
   long blocks = (total + 255) / 256;
   if (blocks > num_sms() * 16) blocks = num_sms() * 16;
-  rope_table_kernel<<<(int)blocks, 256, 0, s>>>(pos, n, k, inv, cs);
+  rope_table_kernel<<<(int)blocks, 256, 0, s>>>(pos, n, k, inv, cs); count_launch();
   return cudaGetLastError();
 }
 
@@ -194,7 +194,7 @@ static cudaError_t norm_mod_dispatch(const float* x, int n, int H, const float* 
   switch (H / 128) {
 #define MMH3_NM(V) \
   case V:          \
-    norm_mod_kernel<TO, V><<<blocks, 256, 0, s>>>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out); break;
+    norm_mod_kernel<TO, V><<<blocks, 256, 0, s>>>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out); count_launch(); break;
     MMH3_NM(1) MMH3_NM(2) MMH3_NM(4) MMH3_NM(6) MMH3_NM(8) MMH3_NM(16) MMH3_NM(21) MMH3_NM(24)
     MMH3_NM(32)
 #undef MMH3_NM
@@ -265,7 +265,7 @@ cudaError_t launch_layernorm(const float* x, int n, int H, const float* g, const
   const int blocks = (n + 7) / 8;
   switch (H / 128) {
 #define MMH3_LN(V) \
-  case V: layernorm_kernel<V><<<blocks, 256, 0, s>>>(x, n, H, g, b, eps, out); break;
+  case V: layernorm_kernel<V><<<blocks, 256, 0, s>>>(x, n, H, g, b, eps, out); count_launch(); break;
     MMH3_LN(2) MMH3_LN(4) MMH3_LN(6) MMH3_LN(8) MMH3_LN(16) MMH3_LN(21)
 #undef MMH3_LN
     default:
@@ -283,7 +283,7 @@ __global__ void rows_kernel(SegRows seg, int n, int32_t* __restrict__ rows) {
 cudaError_t launch_rows(const SegRows& seg, int n, int32_t* rows, cudaStream_t s) {
   int blocks = (n + 255) / 256;
   if (blocks > 4096) blocks = 4096;
-  rows_kernel<<<blocks, 256, 0, s>>>(seg, n, rows);
+  rows_kernel<<<blocks, 256, 0, s>>>(seg, n, rows); count_launch();
   return cudaGetLastError();
 }
 
@@ -307,7 +307,7 @@ cudaError_t launch_fc1_tile(int esize, const void* in, void* out, int F, int H, 
   long blocks = (total + 255) / 256;
   if (blocks > num_sms() * 32) blocks = num_sms() * 32;
   fc1_tile_kernel<<<(int)blocks, 256, 0, s>>>(static_cast<const uint4*>(in), static_cast<uint4*>(out), F,
-                                              words);
+                                              words); count_launch();
   return cudaGetLastError();
 }
 
@@ -338,7 +338,7 @@ cudaError_t launch_vit_fold(const void* wq, const void* wk, const void* wv, cons
   if (blocks > num_sms() * 32) blocks = num_sms() * 32;
   vit_fold_kernel<<<(int)blocks, 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(wq), static_cast<const __nv_bfloat16*>(wk),
-      static_cast<const __nv_bfloat16*>(wv), bq, bk, bv, scale, H, static_cast<__nv_bfloat16*>(wqkv), bqkv);
+      static_cast<const __nv_bfloat16*>(wv), bq, bk, bv, scale, H, static_cast<__nv_bfloat16*>(wqkv), bqkv); count_launch();
   return cudaGetLastError();
 }
 
@@ -408,11 +408,12 @@ cudaError_t launch_patchify(int dtype, const float* x, int C, int T, int H, int 
     patchify_kernel<__nv_bfloat16><<<grid_for(total), 256, 0, s>>>(x, C, T, H, W, static_cast<__nv_bfloat16*>(rows));
   else
     patchify_kernel<float><<<grid_for(total), 256, 0, s>>>(x, C, T, H, W, static_cast<float*>(rows));
+  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpatchify(const float* rows, int C, int T, int H, int W, float* x, cudaStream_t s) {
-  unpatchify_kernel<<<grid_for((long)T * (H / 2) * (W / 2) * 4 * C), 256, 0, s>>>(rows, C, T, H, W, x);
+  unpatchify_kernel<<<grid_for((long)T * (H / 2) * (W / 2) * 4 * C), 256, 0, s>>>(rows, C, T, H, W, x); count_launch();
   return cudaGetLastError();
 }
 
@@ -422,11 +423,12 @@ cudaError_t launch_pack_audio(int dtype, const float* x, int C, int T, void* row
     pack_audio_kernel<__nv_bfloat16><<<grid_for(total), 256, 0, s>>>(x, C, T, static_cast<__nv_bfloat16*>(rows));
   else
     pack_audio_kernel<float><<<grid_for(total), 256, 0, s>>>(x, C, T, static_cast<float*>(rows));
+  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpack_audio(const float* rows, int C, int T, float* x, cudaStream_t s) {
-  unpack_audio_kernel<<<grid_for(2L * T * C), 256, 0, s>>>(rows, C, T, x);
+  unpack_audio_kernel<<<grid_for(2L * T * C), 256, 0, s>>>(rows, C, T, x); count_launch();
   return cudaGetLastError();
 }
 
@@ -444,7 +446,7 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns, DevStatus* st) {
 }
 
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s) {
-  selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns, device_status_ptr());
+  selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns, device_status_ptr()); count_launch();
   return cudaGetLastError();
 }
 

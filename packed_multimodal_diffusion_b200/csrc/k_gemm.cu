@@ -90,7 +90,7 @@ static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, c
   const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
-  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns());
+  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns()); count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return MMH3_OK;
@@ -158,7 +158,7 @@ static mmh3_status run_gemm2(const void* A, const void* B, int M, int N, int K, 
   const int tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
-  kern<<<2 * pairs, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns());
+  kern<<<2 * pairs, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns()); count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
   return MMH3_OK;

@@ -55,6 +55,8 @@ cudaError_t launch_vit_fold(const void* wq, const void* wk, const void* wv, cons
                             const float* bk, const float* bv, float scale, int H, void* wqkv,
                             float* bqkv, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t s);
+// Every kernel launch the library makes is counted (mmh3_launch_count).
+void count_launch();
 cudaError_t launch_patchify(int dtype, const float* x, int C, int T, int H, int W, void* rows, cudaStream_t s);
 cudaError_t launch_unpatchify(const float* rows, int C, int T, int H, int W, float* x, cudaStream_t s);
 cudaError_t launch_pack_audio(int dtype, const float* x, int C, int T, void* rows, cudaStream_t s);

@@ -21,7 +21,7 @@ def declared_symbols():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        for m in re.finditer(r"^\s*(?:mmh3_status|double|void|const char\s*\*)\s*(mmh3_\w+)\s*\(",
+        for m in re.finditer(r"^\s*(?:mmh3_status|double|void|long long|const char\s*\*)\s*(mmh3_\w+)\s*\(",
                              text, flags=re.M):
             names.add(m.group(1))
     return names

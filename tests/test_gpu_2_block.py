@@ -168,3 +168,20 @@ def test_block_forward_host_pipelined_matches_device_calls(cuda_ok):
         ref = xs[k].cuda()
         api.block_forward(dims_c, params, ref, segs, pd, sv, sa, ws)
         assert torch.equal(outs[k], ref.cpu()), f"call {k}"
+
+
+def test_launch_count_of_one_block(cuda_ok):
+    # adaLN, rotation table, 2 x norm/modulate, 4 GEMMs, attention: 9 kernels
+    # (attention adds a split launch and a merge when its last wave is split)
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    n = int(pos.shape[0])
+    w = small_block_weights(37, 256, 2, 128, 512)
+    x = configs.synth.normal((n, 256), 97, 1.0)
+    params = api.BlockParams.from_host(dims_c, w)
+    xd = x.cuda()
+    pd = torch.as_tensor(np.asarray(pos, np.float32)).cuda()
+    ws = torch.empty(api.workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
+    c0 = api.launch_count()
+    api.block_forward(dims_c, params, xd, segs, pd, *sigma_pair(0.5), ws)
+    assert api.launch_count() - c0 == 9
