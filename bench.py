@@ -146,14 +146,15 @@ def job_throughput(world: int, tokens_per_rank: int, steps: int, ms_max: float) 
 
 # -------------------------------------------------- ncu traffic of a kernel
 def measured_traffic(profile: str, source: str):
-    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
-    recorded in a profiles/ summary, or None when the kernel source has
-    changed since that capture (the summary carries the source's sha256)."""
+    """DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+    attention step recorded in a profiles/ summary, or None when the kernel
+    source has changed since that capture (the summary carries the source's
+    sha256)."""
     import hashlib
     import re
     try:
         text = open(os.path.join(ROOT, "profiles", profile)).read()
-        m = re.search(r"traffic_bytes_per_launch:\s*(\d+)\s+source_sha256:\s*([0-9a-f]{64})", text)
+        m = re.search(r"traffic_bytes_per_step:\s*(\d+)\s+source_sha256:\s*([0-9a-f]{64})", text)
         digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
         if m and m.group(2) == digest:
             return int(m.group(1))
@@ -313,7 +314,10 @@ def run_gpu(args):
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
-                     "traffic": traffic, "traffic_unit": "bytes/launch",
+                     "traffic": traffic,
+                     "traffic_unit": ("bytes per attention step (whole-unit launch, split-tail launch and "
+                                      "merge when the last wave is split)" if dom == "attention"
+                                      else "bytes/launch"),
                      "algorithmic_bytes": 2 * n * 3 * 2688 + 2 * n * 2688},
         "phases_ms_per_block": {k: round(v / max(1, nblocks), 4) for k, v in phases.items()},
         "phase_frac_of_peak": {k: round(flops[k] / (per_launch[k] / 1e3) / 1e12 / peak, 4)

@@ -369,39 +369,50 @@ __global__ void __launch_bounds__(320, 1)
 // Combine the `split` partial results of each tail unit (unnormalised O,
 // reference maximum m in the log2 domain, row sum l):
 //   m* = max_p m_p,  w_p = 2^(m_p - m*),  O = sum_p w_p O_p / sum_p w_p l_p.
-// One thread per query row of the unit.
+// One warp per query row (each lane four of the head's columns, so a warp
+// reads a partial row as whole lines); a CTA of 8 warps covers 8 rows of a
+// unit, 32 CTAs a unit.
 template <int HD>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ part, int split,
                                                          __nv_bfloat16* __restrict__ out, int ldo, int seq,
                                                          int heads, int unit0) {
+  static_assert(HD == 128 || HD == 64, "head_dim");
+  constexpr int kLaneCols = HD / 32;  // 4 or 2
   const int nq = (seq + 255) / 256;
-  const int t = blockIdx.x;
+  const int t = blockIdx.x / 32;
   const int u = unit0 + t;
   const int qpair = u % nq;
   const int head = (u / nq) % heads;
   const int zseq = u / (nq * heads);
-  const int r = threadIdx.x;
+  const int r = (blockIdx.x % 32) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   const int qr = qpair * 256 + r;
   if (qr >= seq) return;
-  auto row = [&](int p) { return part + ((size_t)(t * split + p) * 256 + r) * Attn2Shape<HD>::kPartStride; };
+  auto row = [&](int p) {
+    return part + ((size_t)(t * split + p) * 256 + r) * Attn2Shape<HD>::kPartStride;
+  };
   float m = -INFINITY;
   for (int p = 0; p < split; ++p) m = fmaxf(m, row(p)[HD]);
   float l = 0.f;
-  for (int p = 0; p < split; ++p) l += ex2_approx(row(p)[HD] - m) * row(p)[HD + 1];
+  float acc[kLaneCols];
+#pragma unroll
+  for (int i = 0; i < kLaneCols; ++i) acc[i] = 0.f;
+  for (int p = 0; p < split; ++p) {
+    const float* rp = row(p);
+    const float wgt = ex2_approx(rp[HD] - m);
+    l = fmaf(wgt, rp[HD + 1], l);
+#pragma unroll
+    for (int i = 0; i < kLaneCols; ++i) acc[i] = fmaf(wgt, rp[lane * kLaneCols + i], acc[i]);
+  }
   const float inv = l > 0.f ? 1.0f / l : 0.f;
-  __nv_bfloat16* dst = out + (size_t)(zseq * seq + qr) * ldo + head * HD;
-#pragma unroll 1
-  for (int c = 0; c < HD / 32; ++c) {
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = 0.f;
-    for (int p = 0; p < split; ++p) {
-      const float* o = row(p) + c * 32;
-      const float wgt = ex2_approx(row(p)[HD] - m) * inv;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fmaf(wgt, o[i], v[i]);
-    }
-    store32(dst + c * 32, v);
+  __nv_bfloat16* dst = out + (size_t)(zseq * seq + qr) * ldo + head * HD + lane * kLaneCols;
+  if constexpr (kLaneCols == 4) {
+    uint2 v;
+    v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = v;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }
 }
 

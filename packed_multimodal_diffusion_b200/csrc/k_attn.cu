@@ -129,7 +129,7 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
                                                    units - tail, f, part, device_status_ptr(), wait_limit_ns()); count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "attention (split tail) launch");
-    attn_merge_kernel<HD><<<tail, 256, 0, s>>>(part, f, o, inner, seq, heads, units - tail); count_launch();
+    attn_merge_kernel<HD><<<tail * 32, 256, 0, s>>>(part, f, o, inner, seq, heads, units - tail); count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
   }
