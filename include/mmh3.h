@@ -192,15 +192,18 @@ mmh3_status mmh3_attention(const void* qkv, int n_seq, int seq, int heads, int h
                            int act_dtype, float scale, void* out, void* stream);
 
 /* mmh3_attention with a scratch region for the last wave (bf16 only).
- * Work units of 256 query rows of one head fill the SMs in waves; when
- * the last wave would hold at most half as many units as there are SMs,
- * each of its units is split along the keys over f = min(SMs / units, 4,
- * key tiles) CTAs whose partial results (unnormalised O, running maximum,
- * row sum: 256 x (head_dim + 4) fp32 per CTA) go to scratch and are then
- * merged.  Without room in scratch (or with scratch NULL) nothing is split.
- * The result equals mmh3_attention's up to the order of the softmax sums.
- * The block entry points give attention this region from their workspace
- * (the head scratch, unused inside a block). */
+ * Work units of 256 query rows of one head fill the SMs in waves.  The
+ * units of the last, partial wave are split along the keys over f CTAs
+ * when that shortens the wave enough: f in 2..8 minimises
+ * ceil(tail * f / SMs) / f, each piece keeps at least 32 key tiles of 128,
+ * and the split is made only if the tail's time drops to 0.6 of a unit or
+ * less.  The CTAs' partial results (unnormalised O,
+ * running maximum, row sum: 256 x (head_dim + 4) fp32 per CTA) go to scratch
+ * and are then merged.  Without room in scratch (or with scratch NULL)
+ * nothing is split.  The result equals mmh3_attention's up to the order of
+ * the softmax sums.  The block entry points give attention this region from
+ * their workspace (the SwiGLU activation region, free until fc1; the
+ * encoder layer its LayerNorm output, free between qkv and LN2). */
 mmh3_status mmh3_attention_ws(const void* qkv, int n_seq, int seq, int heads, int head_dim,
                               int act_dtype, float scale, void* out, void* scratch,
                               size_t scratch_bytes, void* stream);

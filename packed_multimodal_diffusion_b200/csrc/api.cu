@@ -180,12 +180,13 @@ mmh3_status block_post(const mmh3_dims& d, const mmh3_block_weights& w, float* x
   const int dt = d.act_dtype;
   const int stride = 6 * H;
   const float scale = 1.0f / std::sqrt((float)d.head_dim);
-  // the head region is free during a block: it holds split-attention partials
-  const size_t head_bytes = (size_t)n * H * esize_of(dt);
+  // the SwiGLU activation region is free until fc1: it holds the partial
+  // results of split attention units
+  const size_t act_bytes = (size_t)n * F * esize_of(dt);
   mmh3_status st = kv_all == nullptr
-                       ? attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, scale, ws.attn, s, ws.head, head_bytes)
-                       : attention_kv(dt, ws.qkv, n, kv_all, n_kv, d.heads, d.head_dim, scale, ws.attn, s, ws.head,
-                                      head_bytes);
+                       ? attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, scale, ws.attn, s, ws.act, act_bytes)
+                       : attention_kv(dt, ws.qkv, n, kv_all, n_kv, d.heads, d.head_dim, scale, ws.attn, s, ws.act,
+                                      act_bytes);
   if (st != MMH3_OK) return st;
   pm.mark(3);
   st = gemm_gated_residual(dt, ws.attn, w.wout, n, H, I, x, mods, stride, 2 * H, plan.block_rows, s);
@@ -903,7 +904,9 @@ mmh3_status mmh3_vit_layer_forward(const mmh3_vit_dims* dims, const mmh3_vit_wei
   if (e != cudaSuccess) return cuda_fail(e, "ln1 launch");
   st = gemm_bias_act(MMH3_BF16, h, w->wqkv, M, 3 * H, H, w->bqkv, 0, qkv, s);
   if (st != MMH3_OK) return st;
-  st = attention(MMH3_BF16, qkv, batch, seq, dims->heads, dims->head_dim, 1.0f, attn, s);
+  // h is free between the qkv projection and LN2: it holds the partial
+  // results of split attention units
+  st = attention(MMH3_BF16, qkv, batch, seq, dims->heads, dims->head_dim, 1.0f, attn, s, h, rows * H * 2);
   if (st != MMH3_OK) return st;
   st = gemm_bias_residual(MMH3_BF16, attn, w->wo, M, H, H, w->bo, x, s);
   if (st != MMH3_OK) return st;

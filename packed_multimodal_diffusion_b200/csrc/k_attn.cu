@@ -76,11 +76,10 @@ static mmh3_status run_attn_f32(const void* qkv, int n_seq, int seq, int heads, 
 // a caller padded beyond them are never read.
 //
 // Work units (256 query rows of one head) fill the SMs in waves, one CTA per
-// SM.  When the last wave would hold at most half as many units as there
-// are SMs, and `scratch` has room, each of those tail units is split over
-// f = min(SMs / tail, 4, key tiles) CTAs along the keys; their partial
-// results are merged by attn_merge_kernel, so the tail takes about 1/f of a
-// wave.
+// SM.  When splitting the units of the last, partial wave along the keys
+// shortens it (and `scratch` has room for the partial results), each tail
+// unit runs as f CTAs over contiguous key ranges and attn_merge_kernel
+// combines their results.
 template <int HD>
 static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv, int seq_kv, int heads,
                              float scale, void* out, void* scratch, size_t scratch_bytes, cudaStream_t s) {
@@ -109,12 +108,29 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
   const int sms = num_sms();
   const int tail = units % sms;
   const int kv_tiles = (seq_kv + 127) / 128;
-  int f = tail > 0 ? sms / tail : 1;
-  f = f < 4 ? f : 4;
-  f = f < kv_tiles ? f : kv_tiles;
-  const bool split = f >= 2 && scratch != nullptr &&
-                     (size_t)tail * f * Sh::kPartBytesPerCta <= scratch_bytes &&
-                     (reinterpret_cast<uintptr_t>(scratch) & 15) == 0;
+  // f pieces per tail unit: the tail then takes ceil(tail * f / sms) rounds
+  // of 1/f of a unit's time.  Take the f (at most 8, partials fitting in
+  // scratch) with the fewest rounds x 1/f, the smaller f on ties, but only
+  // when each piece keeps at least 32 key tiles and the tail's time drops
+  // to at most 0.6 of a unit: a CTA's fixed cost (Q load, pipeline fill,
+  // the partial write and the merge) eats the gain of shorter pieces.
+  // Measured at 13248 keys, f = 2: -3%; at 8448 keys f = 4 (16 tiles a
+  // piece): +6%; at 26496 keys f = 5 (0.8 of a unit): +1%; 32 x 1024 keys
+  // f = 2 (4 tiles a piece): +7%.
+  int f = 1;
+  if (tail > 0 && scratch != nullptr && (reinterpret_cast<uintptr_t>(scratch) & 15) == 0) {
+    double best = 1.0;
+    for (int c = 2; c <= 8 && kv_tiles / c >= 32; ++c) {
+      if ((size_t)tail * c * Sh::kPartBytesPerCta > scratch_bytes) break;
+      const double rounds = (double)((tail * c + sms - 1) / sms) / c;
+      if (rounds < best - 1e-9) {
+        best = rounds;
+        f = c;
+      }
+    }
+    if (best > 0.6) f = 1;
+  }
+  const bool split = f >= 2;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   const int whole = split ? units - tail : units;
   if (whole > 0) {

@@ -117,12 +117,14 @@ def test_bounded_wait_returns_timeout_and_context_survives(cuda_ok):
     assert torch.isfinite(out.float()).all()
 
 
-@pytest.mark.parametrize("n_seq,seq,heads,hd", [(1, 700, 5, 128), (1, 300, 1, 128), (3, 200, 2, 64),
+@pytest.mark.parametrize("n_seq,seq,heads,hd", [(1, 700, 5, 128), (1, 12288, 1, 128), (2, 8192, 1, 64),
                                                 (1, 13248, 21, 128)])
 def test_attention_split_tail(cuda_ok, n_seq, seq, heads, hd):
     # last-wave units split along the keys (partials + merge) against the
-    # oracle and against the unsplit kernel; the full-size case is the block
-    # workload's 1092 units (56 in the last wave, split in two)
+    # oracle and against the unsplit kernel: 700 keys are too few to split;
+    # 12288 keys x 1 head (48 units) split in three; two sequences of 8192
+    # (64 units, head_dim 64) in two; the block workload's 1092 units (56 in
+    # the last wave) in two
     n = n_seq * seq
     qkv = _qkv(n, heads, hd, 300 + seq).cuda()
     scale = 1 / math.sqrt(hd)
