@@ -201,7 +201,8 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
                                 const SegRows& seg, cudaStream_t s) {
   if (dtype == MMH3_BF16) {
     // Pairs for the out projection; the long-K fc2 (K = 4H) measured 7-9%
-    // faster on single CTAs with 224-wide tiles, so it stays there.  x is
+    // faster on single CTAs with 224-wide tiles, so it stays there (192-wide
+    // single-CTA tiles, which fill the last wave better, measured 7% slower).  x is
     // moved by TMA (staged read-modify-write) when N is a multiple of 32.
     const bool pair_ok = K <= 4096;
     const bool staged = N % 32 == 0;
