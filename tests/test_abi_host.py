@@ -9,6 +9,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import mmh3_oracle as O
 from packed_multimodal_diffusion_b200 import _lib, api, configs
@@ -143,3 +144,48 @@ def test_refine_and_embed_argument_checks():
     rc = lib.mmh3_embed(C.byref(d), segs, 3, L["seq_len"], C.byref(inputs(2, 1)), C.byref(ew),
                         fake, fake, 1 << 20, None)
     assert rc == 1 and b"condition frames" in lib.mmh3_last_error()
+
+
+def test_new_entry_points_reject_bad_arguments_before_launch():
+    lib = _lib.load()
+    d = api.make_dims(256, 2, 128, 512)
+    fake = C.c_void_p(256)
+    segs = api.segments([(0, 10, 1, 0)])
+    # host-buffer block: slot must be 0 or 1; pos_host / pos_dev both or neither
+    rc = lib.mmh3_block_forward_host(C.byref(d), None, fake, fake, 10, segs, 1, fake, 0.5, 0.2, 2, fake,
+                                     fake, fake, 1 << 20, None, None, None)
+    assert rc == 1 and b"slot" in lib.mmh3_last_error()
+    rc = lib.mmh3_block_forward_host(C.byref(d), None, fake, fake, 10, segs, 1, fake, 0.5, 0.2, 0, fake,
+                                     None, fake, 1 << 20, None, None, None)
+    assert rc == 1 and b"pos_host" in lib.mmh3_last_error()
+    # shard block: fp32 activations are not supported; kv pointers are required
+    d32 = api.make_dims(256, 4, 64, 512, act_dtype=torch.float32)
+    v = C.c_size_t()
+    lib.mmh3_workspace_size(C.byref(d32), 10, C.byref(v))
+    rc = lib.mmh3_block_cp_begin(C.byref(d32), None, fake, 10, segs, 1, None, 0.5, 0.2, 1, fake, fake,
+                                 v.value, None)
+    assert rc == 5
+    lib.mmh3_workspace_size(C.byref(d), 10, C.byref(v))
+    rc = lib.mmh3_block_cp_end(C.byref(d), None, fake, 10, segs, 1, 0.5, 0.2, 1, None, 10, fake, v.value,
+                               None)
+    assert rc == 1 and b"kv_all" in lib.mmh3_last_error()
+    rc = lib.mmh3_block_cp_end(C.byref(d), None, fake, 10, segs, 1, 0.5, 0.2, 1, fake, 9, fake, v.value,
+                               None)
+    assert rc == 2 and b"n_kv" in lib.mmh3_last_error()
+    # refiner: text_dim * 2 bytes must be a multiple of 16
+    lib.mmh3_refine_workspace_size(C.byref(d), 10, C.byref(v))
+    rc = lib.mmh3_refine_text(C.byref(d), fake, 10, 12, fake, fake, None, 0, fake, 1e-6, fake, fake, v.value,
+                              None)
+    assert rc == 2 and b"text_dim" in lib.mmh3_last_error()
+    # forward: the video head width must be 4 x the latent channels
+    L = O.layout_t2va(5, 2, 6, 8, 7)
+    fsegs = api.segments(L["segments"])
+    ins = _lib.EmbedInputs(fake, fake, 4, 2, 6, 8, fake, 8, 7, None, 0)
+    ew = _lib.EmbedWeights(fake, fake, fake, fake)
+    hw = _lib.HeadWeights(fake, fake, fake, fake, fake, fake, fake, fake, 32, 8)
+    lib.mmh3_forward_workspace_size(C.byref(d), L["seq_len"], C.byref(ins), C.byref(v))
+    rc = lib.mmh3_forward(C.byref(d), fsegs, 3, L["seq_len"], None, 0.5, 0.2, C.byref(ins), C.byref(ew), None, 0,
+                          C.byref(hw), fake, fake, fake, fake, v.value, None)
+    assert rc == 2 and b"video head width" in lib.mmh3_last_error()
+    # the launch counter exists and never goes backwards
+    assert lib.mmh3_launch_count() >= 0
