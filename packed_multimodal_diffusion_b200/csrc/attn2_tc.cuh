@@ -9,7 +9,9 @@
 //               O1 += P1 V_j (once P1 is written), S1 = Q1 K_{j+1}^T
 //               P_i (bf16) is read as the A operand straight from tensor
 //               memory, where softmax warpgroup i wrote it over the first 64
-//               columns of S_i.  MMAs of one thread run in issue order, so
+//               columns of S_i.  P_i arrives in two halves of 64 keys, and
+//               the first half of O_i += P_i V_j is issued as soon as the
+//               softmax has released it.  MMAs of one thread run in issue order, so
 //               S_i(j+1) (issued after O_i += P_i V_j) cannot overwrite P_i
 //               before that product has read it; and the commit that
 //               signals S_i(j+1) also covers O_i += P_i V_j, so O_i is
@@ -19,11 +21,17 @@
 //               rescaled only when the maximum grows by more than 2^8 (the
 //               final division uses the same reference maximum, so a stale
 //               maximum is exact up to rounding); late normalisation in the
-//               epilogue.
+//               epilogue.  After the first key tile the exponentials are
+//               computed against the current reference maximum while the
+//               tile's own maximum is found; a row whose maximum outgrew the
+//               reference by more than 2^8 makes its warp rescale and redo
+//               the first half before it is released.
 // While softmax 1 works on S1(j) the tensor core computes O0 += P0 V_j and
 // S0(j+1); while softmax 0 works on S0(j+1) it computes O1 += P1 V_j and
 // S1(j+1).
 #pragma once
+
+#include <type_traits>
 
 #include "gemm_tc.cuh"
 
@@ -46,6 +54,55 @@ struct Attn2Shape {
   static constexpr size_t kPartBytesPerCta = (size_t)256 * kPartStride * 4;
 };
 
+// Eight partial maxima of a 128-score row (three-input max).
+__device__ __forceinline__ void attn_row_max(const float (&s)[128], float (&pm)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pm[i] = s[i];
+#pragma unroll
+  for (int k = 8; k < 120; k += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], s[k + i], s[k + 8 + i]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pm[i] = fmaxf(pm[i], s[120 + i]);
+}
+
+__device__ __forceinline__ float attn_max8(const float (&pm)[8]) {
+  return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+}
+
+// P = 2^(s * scale_log2 - m) for the keys of slices [H0, H1) (32 keys a
+// slice) as bf16 pairs over the first 64 columns of S (16 columns a slice);
+// the row sum accumulates in acc0 / acc1.  Scale/shift and the sum run as
+// packed f32x2 operations; the exponentials stay on MUFU.  With kMax (two
+// slices), the maximum of all 128 scores is folded into pm alongside, two
+// three-input maxima per pair of exponentials.
+template <int H0, int H1, bool kMax>
+__device__ __forceinline__ void attn_exp_slices(const float (&s)[128], uint32_t ts, float scale_log2, float m,
+                                                float2& acc0, float2& acc1, float (&pm)[8]) {
+  static_assert(!kMax || H1 - H0 == 2, "the folded maximum spans two slices");
+  const float2 sc2 = make_float2(scale_log2, scale_log2);
+  const float2 nm2 = make_float2(-m, -m);
+#pragma unroll
+  for (int h = H0; h < H1; ++h) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      if constexpr (kMax) {
+        const int g = (h - H0) * 16 + q;
+        pm[g & 7] = fmax3(pm[g & 7], s[4 * g], s[4 * g + 1]);
+        pm[g & 7] = fmax3(pm[g & 7], s[4 * g + 2], s[4 * g + 3]);
+      }
+      const int k = h * 32 + 2 * q;
+      const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2);
+      const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      if (q & 1) acc1 = __fadd2_rn(acc1, pv);
+      else acc0 = __fadd2_rn(acc0, pv);
+      pk[q] = pack_bf16x2(pv.x, pv.y);
+    }
+    tmem_st16(ts + h * 16, pk);
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(320, 1)
     attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tmkv,
@@ -62,7 +119,7 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::kBarOff);
   constexpr int B_Q = 0;
   constexpr int B_KF = 1, B_KE = B_KF + KV, B_VF = B_KE + KV, B_VE = B_VF + KV;
-  constexpr int B_SF = B_VE + KV, B_PF = B_SF + 2, B_OF = B_PF + 2, B_DRAIN = B_OF + 1;
+  constexpr int B_SF = B_VE + KV, B_PF = B_SF + 2, B_PH = B_PF + 2, B_OF = B_PH + 2, B_DRAIN = B_OF + 1;
   constexpr int kNumBars = B_DRAIN + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -104,6 +161,7 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SF + i), 1);
       mbar_init(bar(B_PF + i), 128);
+      mbar_init(bar(B_PH + i), 128);
     }
     mbar_init(bar(B_OF), 1);
     mbar_init(bar(B_DRAIN), 1);
@@ -136,13 +194,13 @@ __global__ void __launch_bounds__(320, 1)
         const int s = j % KV;
         const uint32_t ph = (uint32_t)((j / KV) & 1);
         const int y = kv_row0 + (j0 + j) * 128;
-        if (*abort_flag || !mbar_wait(bar(B_KE + s), ph ^ 1u, limit_ns)) { ok = false; break; }
+        if (!mbar_wait_ab(bar(B_KE + s), ph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
         mbar_expect_tx(bar(B_KF + s), Sh::kTileBytes);
         for (int c = 0; c < Sh::kHdBoxes; ++c)
           tma_load_2d(sbase + Sh::kKOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tmkv, bar(B_KF + s),
                       xk + c * 64, y);
         in_k = j + 1;
-        if (*abort_flag || !mbar_wait(bar(B_VE + s), ph ^ 1u, limit_ns)) { ok = false; break; }
+        if (!mbar_wait_ab(bar(B_VE + s), ph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
         mbar_expect_tx(bar(B_VF + s), Sh::kTileBytes);
         for (int c = 0; c < Sh::kHdBoxes; ++c)
           tma_load_2d(sbase + Sh::kVOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tmkv, bar(B_VF + s),
@@ -160,69 +218,89 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      // Order: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
-      // S_i(j+1) goes right after PV_i(j), so the tensor core computes
-      // S0(j+1) while softmax 1 still works on S1(j).
-      auto issue_s = [&](int i, int j) {
-        const uint32_t ka = sbase + Sh::kKOff + (j % KV) * Sh::kTileBytes;
-        const uint32_t qa = sbase + Sh::kQOff + i * Sh::kTileBytes;
+    // -------------------------------------------------- MMA issuer
+    // The whole warp runs this loop and its waits, so descriptors and
+    // tensor-memory addresses are warp-uniform; one elected lane (always the
+    // same) issues every MMA and commit.  Stage indices are compile-time
+    // (the loop body is instantiated per K/V stage), so each descriptor is a
+    // base plus a constant.
+    // Order: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+    // S_i(j+1) goes right after PV_i(j), so the tensor core computes
+    // S0(j+1) while softmax 1 still works on S1(j).  Each PV_i(j) is issued
+    // in two halves of 64 keys, the first once P_i's first half is released.
+    static_assert(KV == 2, "the issue loop is written for two K/V stages");
+    const uint64_t dk_major = sdesc_sw128(sbase, 16, 1024);           // Q, K: K-major
+    const uint64_t dv_major = sdesc_sw128(sbase, Sh::kBoxBytes, 1024);  // V: MN-major
+    auto wait = [&](int b, uint32_t ph) {
+      return __all_sync(0xffffffffu, mbar_wait_ab(bar(b), ph, limit_ns, abort_flag));
+    };
+    auto issue_s = [&](int i, auto stage) {
+      constexpr int st = decltype(stage)::value;
 #pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t off = (ks / 4) * Sh::kBoxBytes + (ks % 4) * 32;
-          umma_ss<false>(t_s(i), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), kIdescS,
-                         ks > 0 ? 1u : 0u);
-        }
-        umma_commit(bar(B_SF + i));
-      };
-      auto issue_pv = [&](int i, int j) {
-        const uint32_t va = sbase + Sh::kVOff + (j % KV) * Sh::kTileBytes;
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t off = (ks / 4) * Sh::kBoxBytes + (ks % 4) * 32;
+        umma_ss_elect(t_s(i), dk_major + ((Sh::kQOff + i * Sh::kTileBytes + off) >> 4),
+                      dk_major + ((Sh::kKOff + st * Sh::kTileBytes + off) >> 4), kIdescS, ks > 0 ? 1u : 0u);
+      }
+      umma_commit_elect(bar(B_SF + i));
+    };
+    auto issue_pv = [&](int i, int half, bool first, auto stage) {
+      constexpr int st = decltype(stage)::value;
 #pragma unroll
-        for (int ks = 0; ks < 128 / 16; ++ks) {
-          const uint64_t bd = sdesc_sw128(va + ks * 16 * 128, Sh::kBoxBytes, 1024);
-          umma_ts(t_o(i), t_s(i) + ks * 8, bd, kIdescO, (j > 0 || ks > 0) ? 1u : 0u);
-        }
-      };
-      auto wait_kf = [&](int j) {
-        return !*abort_flag && mbar_wait(bar(B_KF + j % KV), (uint32_t)((j / KV) & 1), limit_ns);
-      };
-      bool ok = mbar_wait(bar(B_Q), 0, limit_ns) && wait_kf(0);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        umma_commit(bar(B_KE + 0));
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int ks = half * 4 + k4;
+        umma_ts_elect(t_o(i), t_s(i) + ks * 8, dv_major + ((Sh::kVOff + st * Sh::kTileBytes + ks * 16 * 128) >> 4),
+                      kIdescO, (!first || ks > 0) ? 1u : 0u);
       }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int s = j % KV;
-        const uint32_t pj = (uint32_t)(j & 1);
-        const bool more = j + 1 < n_kv;
-        if (*abort_flag || !mbar_wait(bar(B_VF + s), (uint32_t)((j / KV) & 1), limit_ns)) { ok = false; break; }
-        if (*abort_flag || !mbar_wait(bar(B_PF + 0), pj, limit_ns)) { ok = false; break; }
+    };
+    // One key tile j in stage st: PV0(j) [S0(j+1)] PV1(j) [S1(j+1)].
+    auto step = [&](int j, auto stage) -> bool {
+      constexpr int st = decltype(stage)::value;
+      const std::integral_constant<int, 1 - st> next{};
+      const uint32_t pj = (uint32_t)(j & 1);
+      const uint32_t pv = (uint32_t)((j / KV) & 1);
+      const bool more = j + 1 < n_kv;
+      if (!wait(B_VF + st, pv) || !wait(B_PH + 0, pj)) return false;
+      tc_fence_after();
+      issue_pv(0, 0, j == 0, stage);
+      if (!wait(B_PF + 0, pj)) return false;
+      tc_fence_after();
+      issue_pv(0, 1, j == 0, stage);
+      if (more) {
+        if (!wait(B_KF + 1 - st, (uint32_t)(((j + 1) / KV) & 1))) return false;
         tc_fence_after();
-        issue_pv(0, j);
-        if (more) {
-          if (!wait_kf(j + 1)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(0, j + 1);
-        }
-        if (*abort_flag || !mbar_wait(bar(B_PF + 1), pj, limit_ns)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(1, j);
-        umma_commit(bar(B_VE + s));
-        if (more) {
-          issue_s(1, j + 1);
-          umma_commit(bar(B_KE + (j + 1) % KV));
-        }
+        issue_s(0, next);
       }
-      if (ok) umma_commit(bar(B_OF));
-      if (!ok) {
-        if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, blockIdx.x);
-        *abort_flag = 1;
-        umma_commit(bar(B_DRAIN));
-        mbar_wait(bar(B_DRAIN), 0, limit_ns);
+      if (!wait(B_PH + 1, pj)) return false;
+      tc_fence_after();
+      issue_pv(1, 0, j == 0, stage);
+      if (!wait(B_PF + 1, pj)) return false;
+      tc_fence_after();
+      issue_pv(1, 1, j == 0, stage);
+      umma_commit_elect(bar(B_VE + st));
+      if (more) {
+        issue_s(1, next);
+        umma_commit_elect(bar(B_KE + 1 - st));
       }
+      return true;
+    };
+    const std::integral_constant<int, 0> stage0{};
+    const std::integral_constant<int, 1> stage1{};
+    bool ok = wait(B_Q, 0) && wait(B_KF + 0, 0);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, stage0);
+      issue_s(1, stage0);
+      umma_commit_elect(bar(B_KE + 0));
+    }
+    for (int j = 0; j < n_kv && ok; ++j) ok = (j & 1) ? step(j, stage1) : step(j, stage0);
+    if (ok) umma_commit_elect(bar(B_OF));
+    if (!ok) {
+      if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_MMA, blockIdx.x);
+      __syncwarp();
+      *abort_flag = 1;
+      umma_commit_elect(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, limit_ns);
     }
   } else {
     // -------------------------------------------------- softmax warpgroups
@@ -236,7 +314,7 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       {
-        const bool fail = *abort_flag || !mbar_wait(bar(B_SF + wg), (uint32_t)(j & 1), limit_ns);
+        const bool fail = !mbar_wait_ab(bar(B_SF + wg), (uint32_t)(j & 1), limit_ns, abort_flag);
         if (__any_sync(0xffffffffu, fail)) { ok = false; break; }
       }
       tc_fence_after();
@@ -262,20 +340,20 @@ __global__ void __launch_bounds__(320, 1)
         for (int k = 0; k < 128; ++k)
           if (k >= valid) s[k] = -INFINITY;
       }
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
       float pm[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) pm[i] = s[i];
-#pragma unroll
-      for (int k = 8; k < 120; k += 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], s[k + i], s[k + 8 + i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) pm[i] = fmaxf(pm[i], s[120 + i]);
-      const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-      const float m_tile = mx * scale_log2;
       if (j == 0) {
-        m_ref = m_tile;
+        // first key tile: the row maximum before any exponential
+        attn_row_max(s, pm);
+        m_ref = attn_max8(pm) * scale_log2;
+        attn_exp_slices<0, 2, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
       } else {
+        // keys 0..63 against the current reference, with the row maximum
+        // of all 128 keys folded in
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
+        attn_exp_slices<0, 2, true>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
+        const float m_tile = attn_max8(pm) * scale_log2;
         const bool need = m_tile > m_ref + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           // O_i holds every earlier product (see the kernel comment).
@@ -292,36 +370,23 @@ __global__ void __launch_bounds__(320, 1)
             for (int i2 = 0; i2 < 16; ++i2) u[i2] = __float_as_uint(__uint_as_float(u[i2]) * f);
             tmem_st16(to + c * 16, u);
           }
+          tmem_wait_st();
+          acc0 = make_float2(0.f, 0.f);
+          acc1 = make_float2(0.f, 0.f);
+          attn_exp_slices<0, 2, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
         }
       }
-      // P = 2^(s * scale * log2e - m_ref) as bf16 pairs over S_i's first 64
-      // columns, in four slices of 32 keys (16 columns).  Scale/shift and
-      // the row sum run as packed f32x2 operations (half the issue slots of
-      // scalar ones); the exponentials stay on MUFU.
-      const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(-m_ref, -m_ref);
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int k = h * 32 + 2 * q;
-          const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2);
-          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if (q & 1) acc1 = __fadd2_rn(acc1, pv);
-          else acc0 = __fadd2_rn(acc0, pv);
-          pk[q] = pack_bf16x2(pv.x, pv.y);
-        }
-        tmem_st16(ts + h * 16, pk);
-      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PH + wg));
+      attn_exp_slices<2, 4, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
       l_sum += (acc0.x + acc0.y) + (acc1.x + acc1.y);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PF + wg));
     }
     if (ok) {
-      const bool fail = *abort_flag || !mbar_wait(bar(B_OF), 0, limit_ns);
+      const bool fail = !mbar_wait_ab(bar(B_OF), 0, limit_ns, abort_flag);
       if (__any_sync(0xffffffffu, fail)) ok = false;
     }
     if (!ok) {

@@ -82,6 +82,28 @@ def test_attention_large_scores_exercise_rescale(cuda_ok):
     assert_close(out, ref, what="attention large scores")
 
 
+def test_attention_growing_maximum_every_tile(cuda_ok):
+    # Scores that climb with the key index: along k's first dimension the
+    # log2-domain score of an even query row rises by about 11 per key tile,
+    # so its running maximum outgrows the reference on every tile, while odd
+    # rows (a twentieth of the slope) rarely do.  Rows of both kinds share
+    # each warp.
+    n, heads, hd = 1000, 1, 128
+    gen = torch.Generator().manual_seed(5)
+    q = 0.05 * torch.randn((n, hd), generator=gen)
+    k = 0.05 * torch.randn((n, hd), generator=gen)
+    v = torch.randn((n, hd), generator=gen)
+    q[:, 0] = torch.where(torch.arange(n) % 2 == 0, 1.0, 0.05)
+    k[:, 0] = 0.06 * math.sqrt(hd) * torch.arange(n, dtype=torch.float32)
+    qkv = torch.cat([q, k, v], dim=1).to(torch.bfloat16).contiguous()
+    out = torch.empty((n, hd), dtype=torch.bfloat16, device="cuda")
+    api.attention(qkv.cuda(), 1, n, heads, hd, 1 / math.sqrt(hd), out)
+    api.device_status()
+    q64, k64, v64 = (f64(t).reshape(n, heads, hd) for t in qkv.split(hd, dim=1))
+    ref = O.attention(q64, k64, v64, 1 / math.sqrt(hd)).reshape(n, -1)
+    assert_close(out, ref, what="attention growing maximum")
+
+
 def test_attention_multi_sequence(cuda_ok):
     n_seq, seq, heads, hd = 3, 200, 2, 64
     qkv = _qkv(n_seq * seq, heads, hd, 11)
