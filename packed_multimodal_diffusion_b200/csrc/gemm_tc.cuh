@@ -859,57 +859,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (*abort_flag || !mbar_wait(tempty_bar(acc), acc_phase ^ 1u, limit_ns)) {
-          if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, 1000 + tile);
-          *abort_flag = 1;
+    // ---------------- MMA issuer: the whole warp runs the loop and its
+    // waits (warp-uniform descriptors and addresses); the lane elect.sync
+    // picks, always the same, issues every MMA and commit.
+    const uint64_t d_base = sdesc_sw128(sbase, 16, 1024);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      if (!__all_sync(0xffffffffu, mbar_wait_ab(tempty_bar(acc), acc_phase ^ 1u, limit_ns, abort_flag))) {
+        if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_MMA, 1000 + tile);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait_ab(full_bar(stage), phase, limit_ns, abort_flag))) {
+          if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_MMA, tile);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < k_blocks; ++kb) {
-          if (*abort_flag || !mbar_wait(full_bar(stage), phase, limit_ns)) {
-            if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, tile);
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = sbase + stage * Sh::kStageBytes;
-          const uint32_t sb = sa + Sh::kABytes;
+        const uint64_t ad = d_base + (uint64_t)((stage * Sh::kStageBytes) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = sdesc_sw128(sa + ks * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sb + ks * 32, 16, 1024);
-            umma_ss<kTf32>(d_tmem, ad, bd, kIdesc, (kb | ks) != 0 ? 1u : 0u);
-          }
-          umma_commit(empty_bar(stage));
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        umma_commit(tfull_bar(acc));
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
+        for (int ks = 0; ks < 4; ++ks)
+          umma_ss_elect<kTf32>(d_tmem, ad + 2 * ks, ad + (Sh::kABytes >> 4) + 2 * ks, kIdesc,
+                               (kb | ks) != 0 ? 1u : 0u);
+        umma_commit_elect(empty_bar(stage));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      // Drain: wait until every MMA this thread issued has completed before
-      // TMEM is released (a commit tracks all prior MMAs of the thread).
-      if (!ok) {
-        umma_commit(drain_bar);
-        mbar_wait(drain_bar, 0, limit_ns);
+      if (!ok) break;
+      umma_commit_elect(tfull_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
       }
+    }
+    // Drain: wait until every MMA this warp issued has completed before
+    // TMEM is released (a commit tracks all prior MMAs of the thread).
+    if (!ok) {
+      __syncwarp();
+      *abort_flag = 1;
+      umma_commit_elect(drain_bar);
+      mbar_wait(drain_bar, 0, limit_ns);
     }
   } else {
     // ---------------- epilogue warps 2..5: lane quarter warp % 4
@@ -1113,53 +1111,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      // ---------------- MMA issuer (leader only)
+    if (leader) {
+      // ---------------- MMA issuer (leader only): the whole warp runs the
+      // loop and its waits; the lane elect.sync picks issues (as in the
+      // single-CTA kernel).
+      const uint64_t d_base = sdesc_sw128(sbase, 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
-        if (*abort_flag || !mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, limit_ns)) {
-          if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, 1000 + tile);
-          *abort_flag = 1;
+        const bool got = !*abort_flag && mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, limit_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_MMA, 1000 + tile);
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < k_blocks; ++kb) {
-          if (*abort_flag || !mbar_wait(full_bar(stage), phase, limit_ns)) {
-            if (!*abort_flag) record_error(status, DEV_TIMEOUT_MMA, tile);
-            *abort_flag = 1;
+          if (!__all_sync(0xffffffffu, mbar_wait_ab(full_bar(stage), phase, limit_ns, abort_flag))) {
+            if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_MMA, tile);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = sbase + stage * Sh::kStageBytes;
-          const uint32_t sb = sa + Sh::kABytes;
+          const uint64_t ad = d_base + (uint64_t)((stage * Sh::kStageBytes) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = sdesc_sw128(sa + ks * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sb + ks * 32, 16, 1024);
-            umma_ss_pair(d_tmem, ad, bd, kIdesc, (kb | ks) != 0 ? 1u : 0u);
-          }
-          umma_commit_pair(empty_bar(stage));
+          for (int ks = 0; ks < 4; ++ks)
+            umma_ss_pair_elect(d_tmem, ad + 2 * ks, ad + (Sh::kABytes >> 4) + 2 * ks, kIdesc,
+                               (kb | ks) != 0 ? 1u : 0u);
+          umma_commit_pair_elect(empty_bar(stage));
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit_pair(tfull_bar(acc));
+        umma_commit_pair_elect(tfull_bar(acc));
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       if (!ok) {
-        umma_commit_pair_local(drain_bar);
+        __syncwarp();
+        *abort_flag = 1;
+        if (lane == 0) umma_commit_pair_local(drain_bar);
         mbar_wait(drain_bar, 0, limit_ns);
       }
     }
