@@ -200,17 +200,17 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
                                 float* x, const float* mods, int mods_stride, int chunk_off,
                                 const SegRows& seg, cudaStream_t s) {
   if (dtype == MMH3_BF16) {
-    // Pairs for the out projection; the long-K fc2 (K = 4H) measured 7-9%
-    // faster on single CTAs with 224-wide tiles, so it stays there (192-wide
-    // single-CTA tiles, which fill the last wave better, measured 7% slower).  x is
-    // moved by TMA (staged read-modify-write) when N is a multiple of 32.
-    const bool pair_ok = K <= 4096;
+    // CTA pairs with 192-wide tiles for the out projection and for fc2
+    // (K = 4H): with the warp-wide MMA issue, fc2 on pairs measured 0.545 ms
+    // against 0.642 on single CTAs with 224-wide tiles, and 256-wide pair
+    // tiles 0.560.  x is moved by TMA (staged read-modify-write) when N is a
+    // multiple of 32.
     const bool staged = N % 32 == 0;
-    if (pair_ok && staged && N % 192 == 0 && use_pairs(M, N, 192)) {
+    if (staged && N % 192 == 0 && use_pairs(M, N, 192)) {
       EpiResidualTma<192, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
       return run_gemm2<192>(A, B, M, N, K, e, s, x, N, 4);
     }
-    if (pair_ok && staged && use_pairs(M, N, 256)) {
+    if (staged && use_pairs(M, N, 256)) {
       EpiResidualTma<256, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
       return run_gemm2<256>(A, B, M, N, K, e, s, x, N, 4);
     }
