@@ -249,19 +249,19 @@ def run_gpu(args):
 
     # ---- end to end through the C ABI with host buffers (pinned), copies
     # inside the timed region: each step copies its input in and its result
-    # out (mmh3_block_forward_host); two device slots let one step's copies
-    # overlap the next step's block
+    # out (mmh3_block_forward_host); three device slots let a step's
+    # copy-out and a later step's copy-in overlap the blocks between them
     x_host = W["x0"].cpu().pin_memory()
     pos_host = torch.as_tensor(np.asarray(W["pos"], np.float32)).pin_memory()
-    out_host = [torch.empty_like(x_host).pin_memory() for _ in range(2)]
-    xd = [torch.empty_like(W["x0"]) for _ in range(2)]
-    pd = [torch.empty_like(W["pos_d"]) for _ in range(2)]
+    out_host = [torch.empty_like(x_host).pin_memory() for _ in range(api.HOST_SLOTS)]
+    xd = [torch.empty_like(W["x0"]) for _ in range(api.HOST_SLOTS)]
+    pd = [torch.empty_like(W["pos_d"]) for _ in range(api.HOST_SLOTS)]
     copy_in, copy_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
     e2e_steps = max(10, args.steps // 4)
     e2e_count = [0]
 
     def e2e_step():
-        k = e2e_count[0] & 1
+        k = e2e_count[0] % api.HOST_SLOTS
         e2e_count[0] += 1
         api.block_forward_host(W["dims"], W["params"], x_host, out_host[k], W["segs"], pos_host, W["sv"],
                                W["sa"], k, xd[k], pd[k], W["ws"], copy_in, copy_out)

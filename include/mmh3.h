@@ -239,6 +239,9 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
 
 /* ----------------------------------------------------- block on host data */
 
+/* Device slots of the host-buffer block (below). */
+#define MMH3_HOST_SLOTS 3
+
 /* One modulated block whose input and result live in host memory, with the
  * copies overlapped with other calls' compute.  Per call, ordered by events:
  *   copy_in_stream:  x_in_host -> x_dev and pos_host -> pos_dev (after the
@@ -247,9 +250,13 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
  *   stream:          mmh3_block_forward on x_dev / pos_dev (workspace as
  *                    there);
  *   copy_out_stream: x_dev -> x_out_host.
- * The call returns at once.  Alternate slot 0 and 1 with two sets of
- * device buffers (x_dev [n, H] fp32 and pos_dev [n, 3] fp32 per slot): the
- * copies of one call then overlap the block of the other.  Host buffers
+ * The call returns at once.  Rotate the slots 0, 1, 2 (MMH3_HOST_SLOTS) with
+ * one set of device buffers per slot (x_dev [n, H] fp32 and pos_dev [n, 3]
+ * fp32): a call's copy-in then waits only for the copy-out of the call three
+ * back, so the copy-out of call i and the copy-in of call i + 3 overlap the
+ * blocks of calls i + 1 and i + 2.  With two slots the two copies would
+ * have to fit within one block's time.  slot outside [0, MMH3_HOST_SLOTS)
+ * returns MMH3_ERR_ARG.  Host buffers
  * must be pinned (cudaHostAlloc / cudaHostRegister) for the copies to be
  * asynchronous, and stay untouched until the call's copy-out has finished
  * (synchronize copy_out_stream).  pos_host / pos_dev may both be NULL (no

@@ -215,13 +215,18 @@ def _host_ptr(t: torch.Tensor | None) -> int | None:
     return t.data_ptr()
 
 
+# Device slots of the host-buffer block (MMH3_HOST_SLOTS in mmh3.h).
+HOST_SLOTS = 3
+
+
 def block_forward_host(dims: Dims, params: BlockParams, x_in: torch.Tensor, x_out: torch.Tensor,
                        segs, pos: torch.Tensor | None, sigma_v: float, sigma_a: float, slot: int,
                        x_dev: torch.Tensor, pos_dev: torch.Tensor | None, workspace: torch.Tensor,
                        copy_in: torch.cuda.Stream, copy_out: torch.cuda.Stream) -> None:
     """One block from pinned host x_in (and pos) to pinned host x_out,
-    through device slot `slot` (x_dev, pos_dev); copies on copy_in /
-    copy_out, the block on the current stream.  Returns without waiting."""
+    through device slot `slot` (0 .. HOST_SLOTS - 1, one x_dev / pos_dev per
+    slot; rotate them); copies on copy_in / copy_out, the block on the
+    current stream.  Returns without waiting."""
     st = params.struct()
     check(load().mmh3_block_forward_host(C.byref(dims), C.byref(st), _host_ptr(x_in), _host_ptr(x_out),
                                          x_in.shape[0], segments(segs), len(segs), _host_ptr(pos),

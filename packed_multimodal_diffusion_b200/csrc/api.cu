@@ -406,10 +406,10 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
 namespace {
 
 // Per device: the events that order the copy-in, compute and copy-out
-// streams of the two staging slots.
+// streams of the staging slots.
 struct HostSlots {
   bool ready = false;
-  cudaEvent_t in_done[2], compute_done[2], out_done[2];
+  cudaEvent_t in_done[MMH3_HOST_SLOTS], compute_done[MMH3_HOST_SLOTS], out_done[MMH3_HOST_SLOTS];
 };
 constexpr int kMaxHostDevices = 64;
 HostSlots g_host_slots[kMaxHostDevices];
@@ -423,7 +423,7 @@ mmh3_status host_slots(HostSlots** out) {
   std::lock_guard<std::mutex> lock(g_host_mu);
   HostSlots& h = g_host_slots[dev];
   if (!h.ready) {
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < MMH3_HOST_SLOTS; ++k) {
       cudaEvent_t* evs[3] = {&h.in_done[k], &h.compute_done[k], &h.out_done[k]};
       for (cudaEvent_t* ev : evs) {
         e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
@@ -449,7 +449,8 @@ mmh3_status mmh3_block_forward_host(const mmh3_dims* dims, const mmh3_block_weig
   clear_error();
   mmh3_status st = check_dims(dims);
   if (st != MMH3_OK) return st;
-  if (slot != 0 && slot != 1) return fail(MMH3_ERR_ARG, "host block: slot %d is neither 0 nor 1", slot);
+  if (slot < 0 || slot >= MMH3_HOST_SLOTS)
+    return fail(MMH3_ERR_ARG, "host block: slot %d outside [0, %d)", slot, MMH3_HOST_SLOTS);
   if (!x_in_host || !x_out_host || !x_dev) return fail(MMH3_ERR_ARG, "host block: null x buffer");
   if ((pos_host == nullptr) != (pos_dev == nullptr))
     return fail(MMH3_ERR_ARG, "host block: pos_host and pos_dev must both be given or both be null");

@@ -151,10 +151,11 @@ def test_new_entry_points_reject_bad_arguments_before_launch():
     d = api.make_dims(256, 2, 128, 512)
     fake = C.c_void_p(256)
     segs = api.segments([(0, 10, 1, 0)])
-    # host-buffer block: slot must be 0 or 1; pos_host / pos_dev both or neither
-    rc = lib.mmh3_block_forward_host(C.byref(d), None, fake, fake, 10, segs, 1, fake, 0.5, 0.2, 2, fake,
-                                     fake, fake, 1 << 20, None, None, None)
-    assert rc == 1 and b"slot" in lib.mmh3_last_error()
+    # host-buffer block: slot in [0, HOST_SLOTS); pos_host / pos_dev both or neither
+    for bad in (-1, api.HOST_SLOTS):
+        rc = lib.mmh3_block_forward_host(C.byref(d), None, fake, fake, 10, segs, 1, fake, 0.5, 0.2, bad, fake,
+                                         fake, fake, 1 << 20, None, None, None)
+        assert rc == 1 and b"slot" in lib.mmh3_last_error()
     rc = lib.mmh3_block_forward_host(C.byref(d), None, fake, fake, 10, segs, 1, fake, 0.5, 0.2, 0, fake,
                                      None, fake, 1 << 20, None, None, None)
     assert rc == 1 and b"pos_host" in lib.mmh3_last_error()
@@ -189,3 +190,9 @@ def test_new_entry_points_reject_bad_arguments_before_launch():
     assert rc == 2 and b"video head width" in lib.mmh3_last_error()
     # the launch counter exists and never goes backwards
     assert lib.mmh3_launch_count() >= 0
+
+
+def test_host_slot_count_matches_header():
+    text = open(os.path.join(ROOT, "include", "mmh3.h")).read()
+    m = re.search(r"#define MMH3_HOST_SLOTS (\d+)", text)
+    assert m and int(m.group(1)) == api.HOST_SLOTS

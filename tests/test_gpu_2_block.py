@@ -142,8 +142,8 @@ def test_block_pair_tile_boundaries(cuda_ok, layout):
 
 
 def test_block_forward_host_pipelined_matches_device_calls(cuda_ok):
-    # four calls on alternating slots with different inputs: each result is
-    # the device block's on the same input, bit for bit
+    # seven calls rotating over the slots with different inputs: each result
+    # is the device block's on the same input, bit for bit
     dims_o, dims_c = small_dims()
     segs, pos = t2va(20, 3, 16, 20, 20)
     n = int(pos.shape[0])
@@ -152,19 +152,21 @@ def test_block_forward_host_pipelined_matches_device_calls(cuda_ok):
     sv, sa = sigma_pair(0.5)
     ws = torch.empty(api.workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
     pos_h = torch.as_tensor(np.asarray(pos, np.float32)).pin_memory()
-    xs = [configs.synth.normal((n, 256), 95 + k, 1.0).pin_memory() for k in range(4)]
+    calls = 7
+    xs = [configs.synth.normal((n, 256), 95 + k, 1.0).pin_memory() for k in range(calls)]
     outs = [torch.empty_like(x).pin_memory() for x in xs]
-    x_dev = [torch.empty((n, 256), device="cuda") for _ in range(2)]
-    p_dev = [torch.empty((n, 3), device="cuda") for _ in range(2)]
+    x_dev = [torch.empty((n, 256), device="cuda") for _ in range(api.HOST_SLOTS)]
+    p_dev = [torch.empty((n, 3), device="cuda") for _ in range(api.HOST_SLOTS)]
     cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
-    for k in range(4):
-        api.block_forward_host(dims_c, params, xs[k], outs[k], segs, pos_h, sv, sa, k & 1, x_dev[k & 1],
-                               p_dev[k & 1], ws, cin, cout)
+    for k in range(calls):
+        slot = k % api.HOST_SLOTS
+        api.block_forward_host(dims_c, params, xs[k], outs[k], segs, pos_h, sv, sa, slot, x_dev[slot],
+                               p_dev[slot], ws, cin, cout)
     cout.synchronize()
     torch.cuda.synchronize()
     api.device_status()
     pd = pos_h.cuda()
-    for k in range(4):
+    for k in range(calls):
         ref = xs[k].cuda()
         api.block_forward(dims_c, params, ref, segs, pd, sv, sa, ws)
         assert torch.equal(outs[k], ref.cpu()), f"call {k}"
