@@ -164,3 +164,26 @@ def test_attention_split_tail(cuda_ok, n_seq, seq, heads, hd):
         sel = [r - b * seq for r in rows if b * seq <= r < (b + 1) * seq]
         ref = O.attention(q, k, v, scale, q_rows=np.asarray(sel)).reshape(len(sel), -1)
         assert_close(out[b * seq:(b + 1) * seq][sel], ref, what=f"split tail sequence {b}")
+
+
+def test_attention_split_tail_with_rescales(cuda_ok):
+    # 12288 keys x 1 head split in three with scores of std ~5: rows rescale
+    # inside each piece, the pieces end with different reference maxima, and
+    # the merge weighs them by 2^(m_p - max m); sampled rows against the
+    # oracle, every row against the unsplit kernel
+    n, heads, hd = 12288, 1, 128
+    qkv = _qkv(n, heads, hd, 41, qscale=5.0).cuda()
+    scale = 1 / math.sqrt(hd)
+    out = torch.full((n, heads * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    scratch = torch.empty(160 * 256 * (hd + 4) * 4, dtype=torch.uint8, device="cuda")
+    api.attention_ws(qkv, 1, n, heads, hd, scale, out, scratch)
+    plain = torch.empty_like(out)
+    api.attention(qkv, 1, n, heads, hd, scale, plain)
+    api.device_status()
+    # P is rounded to bf16 against each piece's own reference maximum, so the
+    # two kernels differ by more than rounding order: the oracle's bf16 bar
+    assert_close(out, plain, BF16_MAXABS, BF16_COS, "split tail with rescales vs unsplit")
+    rows = np.arange(0, n, 89)
+    q, k, v = (f64(t).reshape(n, heads, hd) for t in qkv.cpu().split(heads * hd, dim=1))
+    ref = O.attention(q, k, v, scale, q_rows=rows).reshape(len(rows), -1)
+    assert_close(out[rows.tolist()], ref, what="split tail with rescales")
