@@ -4,7 +4,8 @@
 // K/V tile fetched by TMA serves 256 query rows.  Tensor memory (512
 // columns) holds S0 | S1 | O0 | O1.
 //   warp 0      TMA producer: Q0 and Q1 once, then K_j / V_j (two stages)
-//   warp 1      MMA issuer: S0 = Q0 K_0^T, S1 = Q1 K_0^T, then per key tile
+//   warp 1      MMA issuer (the whole warp runs the loop, one elected lane
+//               issues): S0 = Q0 K_0^T, S1 = Q1 K_0^T, then per key tile
 //               j: O0 += P0 V_j (once P0 is written), S0 = Q0 K_{j+1}^T,
 //               O1 += P1 V_j (once P1 is written), S1 = Q1 K_{j+1}^T
 //               P_i (bf16) is read as the A operand straight from tensor

@@ -4,6 +4,7 @@
 // Roles (192 threads, one CTA per SM):
 //   warp 0      TMA producer: A and B tiles into a STAGES-deep smem ring
 //   warp 1      MMA issuer: tcgen05.mma into one of two TMEM accumulators
+//               (the whole warp runs the loop, one elected lane issues)
 //   warps 2..5  epilogue: tcgen05.ld the accumulator rows, apply the fused
 //               epilogue, store; the second TMEM buffer lets the next tile's
 //               MMAs run under this tile's epilogue.
