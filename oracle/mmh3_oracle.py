@@ -25,7 +25,7 @@ rounded to the device storage type.  Library primitives used as steps:
 ``numpy.cos``, ``numpy.tanh``.  There is no blocking, fusion or reordering
 beyond what the definitions state.
 
-Readings of points the pages leave open (each is listed in the design doc):
+Readings of points the pages leave open (numbered as in the design notes):
 
 R1  adaLN output layout: the basis rows are [timestep slot][tag][chunk][H];
     slot s is evaluated at ts[s].
