@@ -1,4 +1,4 @@
-"""The multi-rank side of bench.py on CPU: two gloo ranks (the path has no
+"""Host logic of bench.py on CPU: two gloo ranks (the path has no
 exchange step, so ranks are independent replicas) agree on the slowest
 rank's time, and the whole-job value counts every rank's tokens over it."""
 
@@ -48,3 +48,23 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.0, "cpu", 1) == 3.0
     assert bench.job_throughput(1, 10, 5, 1000.0) == 50.0
+
+
+def test_measured_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    # the bench's roofline traffic comes from a profiles/ summary only while
+    # the kernel source still has the sha256 recorded with the capture
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    src = tmp_path / "kern.cuh"
+    src.write_bytes(b"// kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()
+    (tmp_path / "profiles" / "p.md").write_text(
+        f"summary\n\ntraffic_bytes_per_step: 123456 source_sha256: {digest}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("p.md", "kern.cuh") == 123456
+    src.write_bytes(b"// kernel v2\n")
+    assert bench.measured_traffic("p.md", "kern.cuh") is None
+    assert bench.measured_traffic("missing.md", "kern.cuh") is None
+
