@@ -1,6 +1,8 @@
-"""Host logic of bench.py on CPU: two gloo ranks (the path has no
-exchange step, so ranks are independent replicas) agree on the slowest
-rank's time, and the whole-job value counts every rank's tokens over it."""
+"""Host logic of bench.py on CPU.  Two gloo ranks (the path has no exchange
+step, so ranks are independent replicas) agree on the slowest rank's time,
+and the whole-job value counts every rank's tokens over it.  The roofline's
+ncu traffic is read from a profile summary only while the kernel source
+still matches the capture."""
 
 import os
 import socket
