@@ -301,9 +301,14 @@ def rope_inv_freq(k: int, theta: float = 10000.0) -> np.ndarray:
 
 def rope_angles(pos: np.ndarray, inv_freq: np.ndarray) -> np.ndarray:
     """[n, 3k] angles, axis-major: angle[axis * k + j] = pos[axis] *
-    inv_freq[j] ([mmh3] ``rope_angles``)."""
+    inv_freq[j] ([mmh3] ``rope_angles``).  As on that page, the frequencies
+    are the model's f32 tensor (``dit.rope_inv_freq`` is read as f32), the
+    product is taken in f64 from the f64 position, and each angle is stored
+    as f32; the returned array holds those f32 values widened to f64."""
     pos = np.asarray(pos, dtype=np.float64)
-    return (pos[:, :, None] * inv_freq[None, None, :]).reshape(pos.shape[0], -1)
+    inv32 = np.asarray(inv_freq, dtype=np.float32).astype(np.float64)
+    prod = pos[:, :, None] * inv32[None, None, :]
+    return prod.astype(np.float32).astype(np.float64).reshape(pos.shape[0], -1)
 
 
 def qk_norm_rope(v: np.ndarray, w: np.ndarray, angles: np.ndarray,

@@ -194,6 +194,28 @@ def test_adaln_zero_basis_gives_bias_and_one_hot_picks_coordinate():
     assert m1.shape == (3, 6 * H) and m1.reshape(-1)[5] == table[512, 3]
 
 
+def test_final_mods_one_hot_picks_its_slots_timestep():
+    # Final layer: rows_per_slot = 2H (chunks shift, scale), row = slot.  A
+    # one-hot basis row in slot 1 picks coordinate k of ts[1]; slot 0's rows
+    # come from ts[0].  A swapped slot order or a transposed [T_s, 2H]
+    # reshape moves the ones.
+    H, R = 5, 24
+    rps = 2 * H
+    table = np.arange(1025 * R, dtype=np.float64).reshape(1025, R) * 0.5
+    ts = [128 / 1024, 896 / 1024]
+    w = np.zeros((2 * rps, R))
+    w[3, 7] = 1.0              # slot 0, shift chunk, element 3
+    w[rps + H + 1, 19] = 1.0   # slot 1, scale chunk, element 1
+    fm = O.final_mods(w, np.zeros(2 * rps), table, ts, H)
+    assert fm.shape == (2, 2 * H)
+    assert fm[0, 3] == table[128, 7]
+    assert fm[1, H + 1] == table[896, 19]
+    assert np.count_nonzero(fm) == 2
+    # with a single timestep only slot 0 is evaluated
+    fm1 = O.final_mods(w, np.zeros(2 * rps), table, [896 / 1024], H)
+    assert fm1.shape == (1, 2 * H) and fm1[0, 3] == table[896, 7] and np.count_nonzero(fm1) == 1
+
+
 def test_block_mods_row_and_chunk_addressing():
     # row = slot*3 + tag; chunk e of that row starts at e*H (modulate doc)
     H = 2
@@ -303,12 +325,44 @@ def test_rope_norm_identity_relative_position_and_untouched_tail():
     y = O.qk_norm_rope(v, g, O.rope_angles(pos, inv), 1e-5)
     np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(y0, axis=-1), rtol=1e-12)
     np.testing.assert_array_equal(y[..., 96:], y0[..., 96:])              # dims >= 96 untouched
-    # q.k depends only on the position difference: shift every axis by delta
+
+    # q.k depends only on the position difference: shift every axis by
+    # delta.  The rotation is checked with exact (unrounded) angles, which
+    # are linear in the position; rope_angles' f32 rounding is pinned on its
+    # own below.
+    def exact_angles(p):
+        return (p[:, :, None] * inv[None, None, :]).reshape(p.shape[0], -1)
+
+    ye = O.qk_norm_rope(v, g, exact_angles(pos), 1e-5)
     for delta in ([7.0, 0, 0], [0, -3.5, 0], [0, 0, 11.25]):
-        ys = O.qk_norm_rope(v, g, O.rope_angles(pos + np.array(delta), inv), 1e-5)
-        dots = np.einsum("ahd,bhd->abh", y, y)
+        ys = O.qk_norm_rope(v, g, exact_angles(pos + np.array(delta)), 1e-5)
+        dots = np.einsum("ahd,bhd->abh", ye, ye)
         dots_s = np.einsum("ahd,bhd->abh", ys, ys)
         np.testing.assert_allclose(dots, dots_s, atol=1e-9)
+
+
+def test_rope_angles_are_f32_roundings_of_the_product():
+    # The page stores the frequencies as an f32 tensor and every angle as
+    # f32: each angle must be an f32 value, within half an f32 ulp of the
+    # exact product of the position and the f32 frequency, and the angles
+    # of integer positions on the first frequency (1.0) stay exact.
+    rng = np.random.default_rng(9)
+    k = 16
+    inv = O.rope_inv_freq(k)
+    pos = np.concatenate([rng.uniform(0, 700, (50, 3)), np.arange(12.0).reshape(4, 3)])
+    ang = O.rope_angles(pos, inv)
+    assert np.array_equal(ang.astype(np.float32).astype(np.float64), ang)
+    inv32 = np.array([float(np.float32(f)) for f in inv])
+    for i in range(pos.shape[0]):
+        for a in range(3):
+            for j in range(k):
+                exact = pos[i, a] * inv32[j]
+                got = ang[i, a * k + j]
+                ulp = float(np.spacing(np.float32(abs(exact)))) if exact != 0 else 0.0
+                assert abs(got - exact) <= 0.5 * ulp
+    np.testing.assert_array_equal(ang[-4:, 0::k], pos[-4:])
+    # the f32 frequencies differ from the fp64 formula by at most half an f32 ulp
+    assert np.all(np.abs(inv32 - inv) <= 0.5 * np.spacing(inv.astype(np.float32)).astype(np.float64))
 
 
 # --------------------------------------------------------------- attention
@@ -373,7 +427,8 @@ def _block_loops(p, dims, x, mods, rows, pos):
     n = x.shape[0]
     kf = dims["rope_k"]
     P = 3 * kf
-    inv = [dims["rope_theta"] ** (-i / kf) for i in range(kf)]
+    # the page's rope_angles: f32 frequencies, f64 product, f32 angle
+    inv = [float(np.float32(dims["rope_theta"] ** (-i / kf))) for i in range(kf)]
 
     def rms(vec, g, eps):
         ss = sum(t * t for t in vec) / len(vec)
@@ -394,7 +449,7 @@ def _block_loops(p, dims, x, mods, rows, pos):
     qkv = [matvec(p["wqkv"], xn[r]) for r in range(n)]
     Q = np.zeros((n, nh, hd)); K = np.zeros((n, nh, hd)); V = np.zeros((n, nh, hd))
     for r in range(n):
-        ang = [pos[r][a] * inv[j] for a in range(3) for j in range(kf)]
+        ang = [float(np.float32(pos[r][a] * inv[j])) for a in range(3) for j in range(kf)]
         for h in range(nh):
             for which, dst, w in ((0, Q, p["q_norm"]), (1, K, p["k_norm"])):
                 seg = qkv[r][which * I + h * hd: which * I + (h + 1) * hd]
@@ -650,3 +705,31 @@ def test_denoise_forward_identity_weights_return_the_negated_latents():
                              heads, 0.5, 0.2, dims)
     np.testing.assert_allclose(v, -video, rtol=0, atol=1e-14)
     np.testing.assert_allclose(a, -audio, rtol=0, atol=1e-14)
+
+
+def test_denoise_forward_each_stream_reads_its_own_clocks_final_row():
+    # Same identity chain, now with a final-layer bias whose scale chunk is
+    # 1 in slot 0 and 3 in slot 1 (zero basis).  sigma_v 0.5 and sigma_a 0.2
+    # give ts = [0.5, 0.8]: the video clock owns slot 0 (x * 2) and the audio
+    # clock slot 1 (x * 4).  Swapping the streams' final rows, or the slot
+    # order inside final_mods, swaps the factors.
+    H, Cv, Ca = 8, 2, 8
+    L = O.layout_t2va(3, 2, 4, 6, 5)
+    rng = np.random.default_rng(22)
+    video = rng.choice([-1.0, 1.0], size=(Cv, 2, 4, 6))
+    audio = rng.choice([-1.0, 1.0], size=(Ca, 2, 5))
+    text = rng.standard_normal((3, H))
+    eye = np.eye(H)
+    b = np.zeros(2 * 2 * H)
+    b[H:2 * H] = 1.0            # slot 0 scale
+    b[3 * H:4 * H] = 3.0        # slot 1 scale
+    heads = {"final_norm": np.ones(H), "adaln_w": np.zeros((2 * 2 * H, 24)),
+             "adaln_b": b, "adaln_table": rng.standard_normal((1025, 24)),
+             "w_video": eye, "b_video": np.zeros(H), "w_audio": eye, "b_audio": np.zeros(H)}
+    dims = {"hidden": H, "eps": 1e-300}
+    ts, slot = O.plan_timesteps(0.5, 0.2, L["segments"])
+    assert ts == [0.5, 0.8] and slot == {O.CLOCK_VIDEO: 0, O.CLOCK_AUDIO: 1}
+    v, a = O.denoise_forward(L, text, video, audio, (eye, np.zeros(H), eye, np.zeros(H)), [],
+                             heads, 0.5, 0.2, dims)
+    np.testing.assert_allclose(v, -2.0 * video, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(a, -4.0 * audio, rtol=0, atol=1e-14)
