@@ -14,8 +14,8 @@ residual.
 With N > 1 (torchrun, one rank per GPU) every rank runs an independent
 replica of the workload (the path has no exchange step); the reported time
 is the maximum over ranks and the value is all ranks' tokens over it.
-`--impl reference` times the CPU oracle on the host cores instead (a bounded
-sample of the same workload per step).
+`--impl reference` times the CPU oracle on the host cores instead (one whole
+block of the same workload per step).
 """
 
 from __future__ import annotations
@@ -47,7 +47,6 @@ def parse():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="b200", choices=["b200", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-rows", type=int, default=128)
     p.add_argument("--workload", default="block", choices=["block", "stack", "image", "siglip", "tiny"],
                    help="block (default) prints the benchmark line; the others print one JSON line "
                         "each for the remaining workloads (stack: 50 blocks + heads, image: 50 "
@@ -71,60 +70,103 @@ def load_peaks():
 
 # --------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock and clock-event (throttle) reasons sampled every few
+    milliseconds while the timed region runs: read-only NVML queries on a
+    background thread (nvidia-smi as a fallback when NVML cannot be loaded).
+    The GPU is found by its PCI bus id, so CUDA_VISIBLE_DEVICES remapping does
+    not matter."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_device: int, period_s: float = 0.005):
+        self.dev = cuda_device
+        self.period = period_s
+        self.samples = []          # (sm_mhz, reasons bitmask)
+        self.sm_max = None
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+
+    def _nvml_handle(self):
+        import pynvml as N
+        import torch
+        N.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            h = N.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            h = N.nvmlDeviceGetHandleByIndex(self.dev)
+        return N, h
+
+    def _run_nvml(self, N, h):
+        get_reasons = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            N.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)), int(get_reasons(h))))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def _run_smi(self):
+        for line in self._proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            try:
+                mhz, mx = float(parts[0]), float(parts[1])
+            except (ValueError, IndexError):
+                continue
+            self.sm_max = mx
+            bits = 0
+            for (name, bit), v in zip(self.REASONS.items(), parts[2:6]):
+                if v.lower().startswith("active"):
+                    bits |= bit
+            self.samples.append((mhz, bits))
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            N, h = self._nvml_handle()
+            self.sm_max = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+            self.source = "nvml"
+            self._thread = threading.Thread(target=self._run_nvml, args=(N, h), daemon=True)
         except Exception:
-            self.proc = None
+            try:
+                self._proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.dev}",
+                     "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.sw_power_cap,"
+                     "clocks_event_reasons.hw_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                     "clocks_event_reasons.hw_thermal_slowdown",
+                     "--format=csv,noheader,nounits", "-lms", "20"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi"
+                self._thread = threading.Thread(target=self._run_smi, daemon=True)
+            except Exception:
+                self._thread = None
+        if self._thread is not None:
+            self._thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 3.0:   # the first sample before the timed region
+                time.sleep(0.002)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except Exception:
-                self.proc.kill()
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [m for m, _ in self.samples]
+        reasons = sorted({name for _, bits in self.samples for name, bit in self.REASONS.items() if bits & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.sm_max,
+                "reasons": reasons, "samples": len(sm), "source": self.source}
 
 
 # ------------------------------------------------------ multi-rank timing
@@ -145,22 +187,23 @@ def job_throughput(world: int, tokens_per_rank: int, steps: int, ms_max: float) 
 
 
 # -------------------------------------------------- ncu traffic of a kernel
-def measured_traffic(profile: str, source: str):
-    """DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
-    attention step recorded in a profiles/ summary, or None when the kernel
-    source has changed since that capture (the summary carries the source's
-    sha256)."""
+def measured_traffic(record: str):
+    """DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per step of
+    the dominant kernel from a JSON record under profiles/ that
+    profile_summary.py wrote from an ncu capture, or None when the record is
+    missing or any source file it lists has changed since (its sha256 no
+    longer matches)."""
     import hashlib
-    import re
     try:
-        text = open(os.path.join(ROOT, "profiles", profile)).read()
-        m = re.search(r"traffic_bytes_per_step:\s*(\d+)\s+source_sha256:\s*([0-9a-f]{64})", text)
-        digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
-        if m and m.group(2) == digest:
-            return int(m.group(1))
-    except OSError:
-        pass
-    return None
+        with open(os.path.join(ROOT, "profiles", record)) as f:
+            rec = json.load(f)
+        for path, digest in rec["sources"].items():
+            with open(os.path.join(ROOT, path), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        return int(rec["traffic_bytes_per_step"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 # ------------------------------------------------------- algorithmic work
@@ -169,6 +212,44 @@ def block_flops(n, H=2688, I=2688, F=10752):
             "fc1 gemm": 2.0 * n * H * 2 * F, "fc2 gemm": 2.0 * n * F * H}
     gemm["attention"] = 4.0 * n * n * I
     return gemm
+
+
+def hbm_bytes(n, H=2688, k=16, t_s=2, rank=24):
+    """Algorithmic HBM bytes per launch of the memory-bound kernels:
+    RMSNorm + modulate reads x (fp32) and writes xn (bf16); the adaLN curve
+    reads its basis [T_s*18H, R] and bias and writes the modulation (fp32);
+    the rotation table reads the positions and writes (cos, sin) fp32 pairs."""
+    norm = n * H * 4 + n * H * 2
+    return {"norm1": norm, "norm2": norm,
+            "adaln": t_s * 18 * H * (rank * 4 + 4 + 4),
+            "rope_table": n * 3 * 4 + n * 3 * k * 8}
+
+
+def percentile(v, q):
+    """Linear-interpolation percentile of a list (q in [0, 100])."""
+    v = sorted(v)
+    if not v:
+        return None
+    x = (len(v) - 1) * q / 100.0
+    lo = int(math.floor(x))
+    hi = min(lo + 1, len(v) - 1)
+    return v[lo] + (v[hi] - v[lo]) * (x - lo)
+
+
+def choose_peak(peaks, clocks, timed_s):
+    """The bf16 peak the timed region ran against: the burst figure while the
+    SM clock stayed at its maximum (a short run, not power-capped), the
+    sustained (power-capped) figure otherwise.  Without clock samples the
+    length of the timed region decides (under one second: burst)."""
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm and mx:
+        burst = sm >= 0.97 * mx
+        why = f"median SM clock {sm:.0f} of max {mx:.0f} MHz under load"
+    else:
+        burst = timed_s < 1.0
+        why = f"no clock samples; timed region {timed_s:.2f} s"
+    kind = "burst" if burst else "sustained"
+    return (peaks["bf16_tflops"] if burst else peaks["bf16_tflops_sustained"]), kind, why
 
 
 # ------------------------------------------------------------- GPU arm
@@ -226,24 +307,28 @@ def run_gpu(args):
         step()
     api.device_status()
 
-    # ---- device-timed region
+    # ---- device-timed region: one event before every step and one after
+    # the last (the per-step distribution); the phase profiler records its
+    # per-kernel events on the same stream
     api.prof_reset()
     api.prof_enable(True)
     barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     launches0 = api.launch_count()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
+        ev[0].record(stream)
+        for i in range(args.steps):
             step()
-        e1.record(stream)
+            ev[i + 1].record(stream)
         torch.cuda.synchronize()
     launches = api.launch_count() - launches0
     barrier()
     api.prof_enable(False)
-    ms = e0.elapsed_time(e1)
+    ms = ev[0].elapsed_time(ev[-1])
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     phases, nblocks = api.prof_collect()
+    kernels = api.prof_collect_kernels()
     api.device_status()
     ms_max = max_over_ranks(ms, device, world)
 
@@ -270,6 +355,7 @@ def run_gpu(args):
         e2e_step()
     barrier()
     torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     copy_in.wait_event(e0)
     copy_out.wait_event(e0)
@@ -289,31 +375,40 @@ def run_gpu(args):
     step_ms = ms_max / args.steps
     value = job_throughput(world, n, args.steps, ms_max)
     flops = block_flops(n)
-    # dominant kernel from the per-phase device times (nblocks blocks)
     per_launch = {k: v / max(1, nblocks) for k, v in phases.items() if v > 0}
     dom = max(("attention", "qkv gemm", "out gemm", "fc1 gemm", "fc2 gemm"),
               key=lambda k: per_launch.get(k, 0.0))
-    traffic = None
-    if dom == "attention":
-        traffic = measured_traffic("attn2_block_13248.md",
-                                   "packed_multimodal_diffusion_b200/csrc/attn2_tc.cuh")
+    traffic = measured_traffic("attn2_block_13248.traffic.json") if dom == "attention" else None
     peaks = load_peaks()
-    achieved = flops[dom] / (per_launch[dom] / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
     clocks = clk.summary()
+    peak, peak_kind, peak_why = choose_peak(peaks, clocks, ms / 1e3)
+    achieved = flops[dom] / (per_launch[dom] / 1e3) / 1e12
     total_flop = sum(flops.values())
+    hb = hbm_bytes(n)
+    hbm_kernels = {}
+    for name, nbytes in hb.items():
+        kms, calls = kernels[name]
+        if calls:
+            t = kms / calls
+            gbs = nbytes / (t / 1e3) / 1e9
+            hbm_kernels[name] = {"ms_per_launch": round(t, 5), "launches": calls, "bytes_per_launch": nbytes,
+                                 "achieved_gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_tokens": n, "hidden": 2688, "heads": 21, "head_dim": 128,
-                   "ffn": 10752, "timesteps": 2,
-                   "l2": "inputs larger than L2 (x 142 MB fp32, weights 231 MB bf16), no flush",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": config_dict(world),
+        "step_ms": {"median": statistics.median(per_step), "p10": percentile(per_step, 10),
+                    "p90": percentile(per_step, 90), "mean": ms / args.steps},
         "tflops_per_s": total_flop / (step_ms / 1e3) / 1e12,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
+                     "peak_source": f"{peaks['source']} bf16 {peak_kind} (MEASURED_PEAKS.json)"
+                                    if peaks["source"] == "measured" else
+                                    f"fallback bf16 {peak_kind} (profiling recipe; MEASURED_PEAKS.json absent)",
+                     "peak_kind": peak_kind, "peak_reason": peak_why,
+                     "frac_burst": achieved / peaks["bf16_tflops"],
+                     "frac_sustained": achieved / peaks["bf16_tflops_sustained"],
                      "traffic": traffic,
                      "traffic_unit": ("bytes per attention step (whole-unit launch, split-tail launch and "
                                       "merge when the last wave is split)" if dom == "attention"
@@ -322,27 +417,36 @@ def run_gpu(args):
         "phases_ms_per_block": {k: round(v / max(1, nblocks), 4) for k, v in phases.items()},
         "phase_frac_of_peak": {k: round(flops[k] / (per_launch[k] / 1e3) / 1e12 / peak, 4)
                                for k in flops if k in per_launch},
+        "hbm_kernels": {"peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"], **hbm_kernels},
         "e2e": {"value": job_throughput(world, n, e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(W["x0"].numel() * 4 + W["pos_d"].numel() * 4),
                 "d2h_bytes_per_step": int(W["x0"].numel() * 4)},
         "gpu_launches": launches,
-        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
+        "clocks": clocks,
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_rows)
+        line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
 
 
+def config_dict(world: int) -> dict:
+    return {"workload": WORKLOAD, "n_tokens": N_TOKENS, "hidden": 2688, "heads": 21, "head_dim": 128,
+            "ffn": 10752, "timesteps": 2,
+            "l2": "inputs larger than L2 (x 142 MB fp32, weights 231 MB bf16), no flush",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 # -------------------------------------------------------------- CPU oracle
-class OracleSample:
-    """The oracle on a bounded sample of the block workload: k and v for all
-    tokens (attention reads every key) plus `rows` query rows through the
-    whole block.  Inputs are generated once; run() times one sample."""
+class OracleBlock:
+    """The oracle (fp64 numpy, as it stands) on the whole block workload,
+    timed as one whole block cut into `parts` contiguous chunks of query
+    rows: the first chunk's call also evaluates the adaLN modulation and k
+    and v of every token (the oracle's k/v cache hands them to the later
+    chunks), so the chunks together do exactly one block's work, and their
+    times add up to one measured block.  Inputs are generated and widened
+    before any timing."""
 
-    def __init__(self, rows: int):
-        import numpy as np
-
+    def __init__(self):
         from oracle import mmh3_oracle as O
         from packed_multimodal_diffusion_b200 import configs
         self.O = O
@@ -354,101 +458,83 @@ class OracleSample:
         self.x = configs.hidden_states(c).double().numpy()
         sa = O.time_shift_sigma(c.sigma_v, 12.0, 3.0)
         self.ts, slot = O.plan_timesteps(c.sigma_v, sa, L["segments"])
-        self.rows_of = O.token_rows(L["segments"], slot, self.n)
-        self.sample = np.linspace(0, self.n - 1, max(2, rows)).astype(int)
+        self.rows = O.token_rows(L["segments"], slot, self.n)
         try:
             from threadpoolctl import threadpool_info
             self.cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
         except Exception:
             self.cores = os.cpu_count()
 
-    def _block(self, rows):
-        O, c, p = self.O, self.c, self.p
-        mods = O.block_mods(p["adaln_w"], p["adaln_b"], p["adaln_table"], self.ts, c.hidden)
-        O.block_forward(p, self.x, mods, self.rows_of, self.L["pos"], c.dims(), sample_rows=rows)
-
-    def calibrate(self, rows: int = 192, reps: int = 2):
-        """Per-row cost of the block (attention over all keys, projections,
-        FFN): the difference between a `rows`-row and a 1-row run, each the
-        best of `reps`.  Both runs share the fixed cost of k and v for all
-        tokens (seconds on the host), so the row count must be large enough
-        for the marginal cost to stand well above that cost's run-to-run
-        noise."""
+    def block_in_parts(self, parts: int) -> list:
+        """Seconds of each of the `parts` chunks of one whole block."""
         import numpy as np
-        big = np.linspace(0, self.n - 1, rows).astype(int)
+        O, c, p = self.O, self.c, self.p
+        bounds = np.linspace(0, self.n, max(1, min(parts, self.n)) + 1).astype(int)
+        cache, mods, times = {}, None, []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            t0 = time.perf_counter()
+            if mods is None:
+                mods = O.block_mods(p["adaln_w"], p["adaln_b"], p["adaln_table"], self.ts, c.hidden)
+            O.block_forward(p, self.x, mods, self.rows, self.L["pos"], c.dims(),
+                            sample_rows=np.arange(a, b), kv_cache=cache)
+            times.append(time.perf_counter() - t0)
+        return times
 
-        def best(r):
-            ts = []
-            for _ in range(reps):
-                t0 = time.perf_counter()
-                self._block(r)
-                ts.append(time.perf_counter() - t0)
-            return min(ts)
-
-        t_one = best(self.sample[:1])
-        t_big = best(big)
-        self.t_row = max(0.0, (t_big - t_one) / (len(big) - 1))
-        self.calib_rows = len(big)
-
-    def run(self):
-        """Time one sample; -> (seconds, extrapolated full-block seconds)."""
-        if not hasattr(self, "t_row"):
-            self.calibrate()
-        t0 = time.perf_counter()
-        self._block(self.sample)
-        t_s = time.perf_counter() - t0
-        return t_s, t_s + (self.n - len(self.sample)) * self.t_row
-
-    def describe(self, t_s, t_full):
-        return (f"block workload: k/v for all {self.n} tokens + {len(self.sample)} sampled query "
-                f"rows through the whole block ({t_s:.2f} s); full {self.n}-row block "
-                f"extrapolated with the per-row cost measured between 1 and "
-                f"{self.calib_rows} rows, best of 2 ({t_full:.1f} s)")
+    def describe(self, times) -> str:
+        return (f"one whole block of the block workload ({self.n} tokens: adaLN modulation, k/v of every "
+                f"token and all {self.n} query rows through the block, fp64 numpy) in {len(times)} "
+                f"timed chunk(s) of query rows, {sum(times):.1f} s in total")
 
 
-def cpu_baseline(rows_sample):
-    o = OracleSample(rows_sample)
-    t_s, t_full = o.run()
-    return {"value": N_TOKENS / t_full, "unit": UNIT, "cores": o.cores, "kind": "oracle",
-            "sample": o.describe(t_s, t_full)}
+def cpu_baseline():
+    o = OracleBlock()
+    times = o.block_in_parts(1)
+    return {"value": o.n / sum(times), "unit": UNIT, "cores": o.cores, "kind": "oracle",
+            "sample": o.describe(times)}
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle.  The `steps` timed steps together
+    compute one whole block (each a contiguous chunk of the query rows, the
+    first also the modulation and k/v of every token), so the value is the
+    block's tokens over the measured time of one block.  The oracle keeps no
+    state between blocks, so there is nothing to warm up and no warm-up block
+    runs (the line records the requested count).  Only rank 0 runs it."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    o = OracleSample(max(2, min(args.cpu_rows, 64)))
-    fulls, samples = [], []
-    for i in range(args.warmup + args.steps):
-        t_s, t_full = o.run()
-        if i >= args.warmup:
-            fulls.append(t_full)
-            samples.append(t_s)
-    t_full = statistics.mean(fulls)
-    value = N_TOKENS / t_full
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * t_full, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": WORKLOAD, "n_tokens": N_TOKENS},
+    o = OracleBlock()
+    times = o.block_in_parts(args.steps)
+    total = sum(times)
+    value = o.n / total
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": len(times),
+            "warmup": 0, "warmup_requested": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference", "config": config_dict(1),
+            "step_ms": {"median": 1e3 * statistics.median(times), "p10": 1e3 * percentile(times, 10),
+                        "p90": 1e3 * percentile(times, 90), "mean": 1e3 * total / len(times)},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": o.cores, "kind": "oracle",
-                             "sample": o.describe(statistics.mean(samples), t_full)},
+                             "sample": o.describe(times)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------- other workloads
 def _time(fn, steps, warmup):
+    """Mean ms per call of fn over `steps` calls after `warmup`, CUDA events
+    on the current stream, with the clocks sampled meanwhile."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        fn()
-    e1.record()
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+    _time.clocks = clk.summary()
     return e0.elapsed_time(e1) / steps
 
 
@@ -480,7 +566,8 @@ def run_workload(args):
                     tflops_per_s=flop / (ms / 1e3) / 1e12,
                     config={"workload": "SigLIP layer: 32 images x 1024 tokens, hidden 768, 12x64 heads, "
                                         "MLP 3072 tanh-GELU, LayerNorm pre-norm"},
-                    context="the pages quote 61.9 ms/layer for batch 1 on an unnamed CPU")
+                    context="the pages quote 61.9 ms/layer for batch 1 on an unnamed CPU",
+                    clocks=_time.clocks)
         print(json.dumps(line), flush=True)
         return
     c = {"stack": configs.STACK, "image": configs.IMAGE, "tiny": configs.TINY}[args.workload]
@@ -522,7 +609,8 @@ def run_workload(args):
     api.device_status()
     flops = block_flops(n, c.hidden, c.heads * c.head_dim, c.ffn)
     per_block = {k: v / max(1, nblocks) for k, v in phases.items() if v > 0}
-    peak = peaks["bf16_tflops_sustained"]
+    peak, peak_kind, _ = choose_peak(peaks, _time.clocks, ms * steps / 1e3)
+    line.update(clocks=_time.clocks, peak_tflops=peak, peak_kind=peak_kind)
     line.update(metric=f"{args.workload} forward time (1 B200)", value=ms, unit="ms/forward",
                 higher_is_better=False, dtype="fp32/tf32" if c.act_dtype == torch.float32 else "bf16",
                 n_tokens=n, n_blocks=c.n_blocks, heads=bool(heads),

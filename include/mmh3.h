@@ -169,7 +169,14 @@ mmh3_status mmh3_adaln_modulation(const mmh3_dims* dims, const float* w, const f
 
 /* Rewrites fc1 [2F, H] from the checkpoint order [gate | up] into the tile
  * order the fused fc1+SwiGLU kernel reads: blocks of 256 rows, 128 gate rows
- * then the 128 matching up rows.  Device in/out, act dtype, distinct. */
+ * then the 128 matching up rows ("cortiq_engine/mmh3.rs", ffn_tail: fc1's
+ * output is [gate | up]).  Device in/out, act dtype, distinct buffers
+ * (MMH3_ERR_ARG if null or equal, MMH3_ERR_ALIGN unless 16-byte aligned).
+ * The one preparation a block's weights need; run it once per block. */
+mmh3_status mmh3_prepare_block_weights(const mmh3_dims* dims, const void* fc1_gate_up,
+                                       void* fc1_interleaved, void* stream);
+
+/* The same call under its older name. */
 mmh3_status mmh3_prepare_fc1(const mmh3_dims* dims, const void* fc1_gate_up, void* fc1_tiled,
                              void* stream);
 
@@ -218,11 +225,21 @@ mmh3_status mmh3_attention_ws(const void* qkv, int n_seq, int seq, int heads, in
  * The modulation row of token i is given by its segment (mmh3_segment).
  * pos_dev: device fp32 [n, 3] (t, h, w), or NULL for no rotation.
  * modulated = 0 runs the unmodulated form (plain residuals, no adaLN; the
- * weights' adaln pointers may be NULL).  workspace: mmh3_workspace_size. */
+ * weights' adaln pointers may be NULL).
+ * mods_or_null: NULL evaluates the block's adaLN curve (Adaln::eval) at the
+ * segments' timesteps; otherwise a device fp32 [T_s*3, 6H] modulation
+ * buffer, 16-byte aligned, laid out as mmh3_adaln_modulation writes it
+ * (row slot*3 + tag, chunks shift_msa, scale_msa, gate_msa, shift_mlp,
+ * scale_mlp, gate_mlp), used as is: the adaLN launch is skipped and the
+ * weights' adaln pointers may be NULL.  T_s and the slots still come from
+ * the segments and sigmas.  Only read by the call's kernels, so it must stay
+ * valid until they finish.  MMH3_ERR_ARG if given with modulated = 0.
+ * workspace: mmh3_workspace_size. */
 mmh3_status mmh3_block_forward(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
                                const mmh3_segment* segs, int n_seg, const float* pos_dev,
-                               double sigma_v, double sigma_a, int modulated, void* workspace,
-                               size_t ws_bytes, void* stream);
+                               double sigma_v, double sigma_a, int modulated,
+                               const float* mods_or_null, void* workspace, size_t ws_bytes,
+                               void* stream);
 
 /* n_blocks blocks (blocks: host array of n_blocks weight structs) then,
  * if heads != NULL, the two output heads ("cortiq_engine/mmh3.rs", forward
@@ -447,8 +464,12 @@ mmh3_status mmh3_forward(const mmh3_dims* dims, const mmh3_segment* segs, int n_
  *  - All calls share the array, which keeps the last call's contents; calls
  *    whose kernels overlap on the GPU race on it.  Nothing in it needs to
  *    start at zero.  The phase profile is not recorded by this entry point.
+ *  - The cached address belongs to the CUDA context that was current at the
+ *    lookup; a call made under another context on the same device (after
+ *    cudaDeviceReset, for example) looks it up again.
  * Arguments and results are those of mmh3_block_forward without the
- * workspace. */
+ * workspace; the modulation is always the block's own adaLN curve (no
+ * mods_or_null). */
 mmh3_status mmh3_block_forward_noalloc(const mmh3_dims* dims, const mmh3_block_weights* w, float* x,
                                        int n, const mmh3_segment* segs, int n_seg,
                                        const float* pos_dev, double sigma_v, double sigma_a,
@@ -510,6 +531,13 @@ mmh3_status mmh3_vit_layer_forward(const mmh3_vit_dims* dims, const mmh3_vit_wei
  * returns MMH3_ERR_TIMEOUT if one was recorded. */
 mmh3_status mmh3_device_status(void* stream, int* code, int* site);
 
+/* Synchronises `stream` and reads and clears the device status word, as
+ * mmh3_device_status does without the site: *device_status receives the
+ * first device error code (0 = none; may be NULL); returns MMH3_ERR_TIMEOUT
+ * if a kernel gave up waiting, MMH3_ERR_CUDA if the synchronisation failed.
+ * The one entry point besides mmh3_device_status that waits for the GPU. */
+mmh3_status mmh3_status_sync(void* stream, int* device_status);
+
 /* Bound on every in-kernel wait, in nanoseconds (0 restores the default). */
 void mmh3_set_wait_limit_ns(uint64_t ns);
 
@@ -532,6 +560,28 @@ mmh3_status mmh3_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 void mmh3_prof_enable(int on);
 mmh3_status mmh3_prof_collect(double* ms, int n_slots, long* n_blocks);
 void mmh3_prof_reset(void);
+
+/* The same intervals by kernel (a finer split of the phase slots: slot 0
+ * holds the adaLN curve, the rotation table and both RMSNorm + modulate
+ * launches).  Attention counts its whole step (the main launch and, when
+ * its last wave is split, the tail launch and the merge). */
+#define MMH3_PROF_K_ADALN 0   /* adaLN curve -> modulation */
+#define MMH3_PROF_K_ROPE 1    /* rotation (cos, sin) table */
+#define MMH3_PROF_K_NORM1 2   /* segment gather + RMSNorm(norm1) + modulate */
+#define MMH3_PROF_K_QKV 3     /* qkv GEMM + qk-norm + rotation */
+#define MMH3_PROF_K_ATTN 4    /* attention step */
+#define MMH3_PROF_K_OUT 5     /* out GEMM + gated residual */
+#define MMH3_PROF_K_NORM2 6   /* segment gather + RMSNorm(norm2) + modulate */
+#define MMH3_PROF_K_FC1 7     /* fc1 GEMM + SwiGLU */
+#define MMH3_PROF_K_FC2 8     /* fc2 GEMM + gated residual */
+#define MMH3_PROF_KERNELS 9
+
+/* Waits for the recorded events like mmh3_prof_collect (which it calls, so
+ * the phase totals are folded in too) and writes, for each kernel id below
+ * n_kernels, the cumulative device time in ms[id] and, if calls is not
+ * NULL, the number of timed launches in calls[id].  Reset by
+ * mmh3_prof_reset. */
+mmh3_status mmh3_prof_collect_kernels(double* ms, long* calls, int n_kernels);
 
 /* Message of the last failing call on this thread ("" if none). */
 const char* mmh3_last_error(void);

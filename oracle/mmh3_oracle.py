@@ -367,7 +367,8 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
 # --------------------------------------------------------------------------
 
 def block_forward(p: dict, x: np.ndarray, mods, rows, pos, dims: dict,
-                  sample_rows=None, keep: dict | None = None) -> np.ndarray:
+                  sample_rows=None, keep: dict | None = None,
+                  kv_cache: dict | None = None) -> np.ndarray:
     """One modulated DiT block ([mmh3] ``block_forward`` + ``ffn_tail``).
 
     ``p``: norm1, norm2 [H]; wqkv [3I, H] (rows [q | k | v], heads
@@ -382,6 +383,11 @@ def block_forward(p: dict, x: np.ndarray, mods, rows, pos, dims: dict,
     are still computed for every token, since attention reads all keys).
     ``keep``: if a dict, intermediates (xn1, q, k, v, attn, xmid, xn2, act)
     for the computed rows are stored in it.
+    ``kv_cache``: if a dict, k (after qk-norm and rotation) and v of every
+    token are stored in it by the first call and read back by later calls on
+    the same x, so that a block can be computed in chunks of query rows with
+    k and v computed once (the values are the same either way, up to the
+    summation order the matrix product picks for a given row count).
 
     Returns x_out for the computed rows ([len(rows)] x H)."""
     H, nh, hd, F = dims["hidden"], dims["heads"], dims["head_dim"], dims["ffn"]
@@ -392,26 +398,37 @@ def block_forward(p: dict, x: np.ndarray, mods, rows, pos, dims: dict,
     sel = np.arange(n) if sample_rows is None else np.asarray(sample_rows)
     f64 = lambda a: np.asarray(a, dtype=np.float64)  # noqa: E731
     wqkv, wout, wfc1, wfc2 = f64(p["wqkv"]), f64(p["wout"]), f64(p["wfc1"]), f64(p["wfc2"])
-    m = None if mods is None else f64(mods)[np.asarray(rows)]  # [n, 6H]
+    cached = kv_cache is not None and "k" in kv_cache
+    # each token's modulation row [6H]: every token for k and v, or only the
+    # computed rows when k and v come from the cache
+    rows = np.asarray(rows)
+    mr = None if mods is None else f64(mods)[rows[sel] if cached else rows]
+    ms = None if mr is None else (mr if cached else mr[sel])
 
     # norm1 -> modulate(shift 0, scale 1)
-    xn1 = rms_norm(x, p["norm1"], eps)
-    if m is not None:
-        xn1 = modulate(xn1, chunk(m, 0, H), chunk(m, 1, H))
-    # qkv projection: q only where needed, k and v for every token
-    q = (xn1[sel] @ wqkv[:I].T).reshape(-1, nh, hd)
-    k = (xn1 @ wqkv[I:2 * I].T).reshape(n, nh, hd)
-    v = (xn1 @ wqkv[2 * I:].T).reshape(n, nh, hd)
+    xr = x[sel] if cached else x
+    xn1 = rms_norm(xr, p["norm1"], eps)
+    if mr is not None:
+        xn1 = modulate(xn1, chunk(mr, 0, H), chunk(mr, 1, H))
+    xn1_sel = xn1 if cached else xn1[sel]
     if pos is None:
         ang_all = np.zeros((n, 0))
     else:
         ang_all = rope_angles(pos, rope_inv_freq(dims["rope_k"], dims["rope_theta"]))
+    # qkv projection: q only where needed, k and v for every token
+    q = (xn1_sel @ wqkv[:I].T).reshape(-1, nh, hd)
     q = qk_norm_rope(q, p["q_norm"], ang_all[sel], qk_eps)
-    k = qk_norm_rope(k, p["k_norm"], ang_all, qk_eps)
+    if cached:
+        k, v = kv_cache["k"], kv_cache["v"]
+    else:
+        k = (xn1 @ wqkv[I:2 * I].T).reshape(n, nh, hd)
+        v = (xn1 @ wqkv[2 * I:].T).reshape(n, nh, hd)
+        k = qk_norm_rope(k, p["k_norm"], ang_all, qk_eps)
+        if kv_cache is not None:
+            kv_cache["k"], kv_cache["v"] = k, v
     o = attention(q, k, v, 1.0 / math.sqrt(hd)).reshape(-1, I)
     proj = o @ wout.T
     xs = x[sel]
-    ms = None if m is None else m[sel]
     xmid = xs + (proj if ms is None else chunk(ms, 2, H) * proj)
     # ffn tail: norm2 -> modulate(3, 4) -> fc1 -> SwiGLU -> fc2 -> gate 5
     xn2 = rms_norm(xmid, p["norm2"], eps)
@@ -422,7 +439,7 @@ def block_forward(p: dict, x: np.ndarray, mods, rows, pos, dims: dict,
     down = act @ wfc2.T
     xout = xmid + (down if ms is None else chunk(ms, 5, H) * down)
     if keep is not None:
-        keep.update(xn1=xn1[sel], q=q, k=k[sel], v=v[sel], attn=o, xmid=xmid,
+        keep.update(xn1=xn1_sel, q=q, k=k[sel], v=v[sel], attn=o, xmid=xmid,
                     xn2=xn2, act=act, rows=sel)
     return xout
 

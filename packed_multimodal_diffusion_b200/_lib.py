@@ -85,12 +85,13 @@ SIGNATURES = {
     "mmh3_resolve_rows": (_I, [_SEGP, _I, _I, _D, _D, _P, _P]),
     "mmh3_adaln_modulation": (_I, [C.POINTER(Dims), _P, _P, _P, _I, _SEGP, _I, _I, _D, _D, _P,
                                    C.POINTER(_I), _P]),
+    "mmh3_prepare_block_weights": (_I, [C.POINTER(Dims), _P, _P, _P]),
     "mmh3_prepare_fc1": (_I, [C.POINTER(Dims), _P, _P, _P]),
     "mmh3_workspace_size": (_I, [C.POINTER(Dims), _I, C.POINTER(C.c_size_t)]),
     "mmh3_attention": (_I, [_P, _I, _I, _I, _I, _I, C.c_float, _P, _P]),
     "mmh3_attention_ws": (_I, [_P, _I, _I, _I, _I, _I, C.c_float, _P, _P, C.c_size_t, _P]),
     "mmh3_block_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I, _P,
-                                _D, _D, _I, _P, C.c_size_t, _P]),
+                                _D, _D, _I, _P, _P, C.c_size_t, _P]),
     "mmh3_block_forward_noalloc": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _P, _I, _SEGP, _I,
                                         _P, _D, _D, _I, _P]),
     "mmh3_stack_forward": (_I, [C.POINTER(Dims), C.POINTER(BlockWeights), _I,
@@ -125,11 +126,13 @@ SIGNATURES = {
     "mmh3_vit_layer_forward": (_I, [C.POINTER(VitDims), C.POINTER(VitWeights), _P, _I, _I, _P,
                                     C.c_size_t, _P]),
     "mmh3_device_status": (_I, [_P, C.POINTER(_I), C.POINTER(_I)]),
+    "mmh3_status_sync": (_I, [_P, C.POINTER(_I)]),
     "mmh3_set_wait_limit_ns": (None, [C.c_uint64]),
     "mmh3_selftest_wait_timeout": (_I, [C.c_uint64, _P]),
     "mmh3_prof_enable": (None, [_I]),
     "mmh3_prof_collect": (_I, [C.POINTER(C.c_double), _I, C.POINTER(C.c_long)]),
     "mmh3_prof_reset": (None, []),
+    "mmh3_prof_collect_kernels": (_I, [C.POINTER(C.c_double), C.POINTER(C.c_long), _I]),
     "mmh3_last_error": (C.c_char_p, []),
     "mmh3_launch_count": (C.c_longlong, []),
     "mmh3_version": (C.c_char_p, []),

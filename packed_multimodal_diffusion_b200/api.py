@@ -18,7 +18,7 @@ from ._lib import (MMH3_BF16, MMH3_F32, MMH3_STREAM_AUDIO, MMH3_STREAM_VIDEO, Bl
 
 __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_image",
            "plan_timesteps", "time_shift_sigma", "resolve_rows", "adaln_modulation",
-           "prepare_fc1", "workspace_size", "attention", "attention_ws", "BlockParams", "HeadParams",
+           "prepare_block_weights", "prepare_fc1", "workspace_size", "attention", "attention_ws", "BlockParams", "HeadParams",
            "block_forward", "stack_forward", "block_forward_host", "block_cp_begin", "block_cp_end", "refine_workspace_size", "refine_text",
            "patch_embed_workspace_size", "patch_embed", "embed_workspace_size", "embed",
            "unpatchify_video", "unpack_audio", "forward_workspace_size", "forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
@@ -110,6 +110,11 @@ def adaln_modulation(dims: Dims, w, b, table, rows_per_slot, segs, n, sigma_v, s
     return nts.value
 
 
+def prepare_block_weights(dims: Dims, fc1_gate_up: torch.Tensor, out: torch.Tensor) -> None:
+    """fc1 [gate | up] -> the fused fc1+SwiGLU kernel's tile order."""
+    check(load().mmh3_prepare_block_weights(C.byref(dims), _ptr(fc1_gate_up), _ptr(out), _stream()))
+
+
 def prepare_fc1(dims: Dims, fc1_gate_up: torch.Tensor, out: torch.Tensor) -> None:
     check(load().mmh3_prepare_fc1(C.byref(dims), _ptr(fc1_gate_up), _ptr(out), _stream()))
 
@@ -153,7 +158,7 @@ class BlockParams:
         t = {k: v.to(device).contiguous() for k, v in w.items() if k != "wfc1"}
         fc1 = w["wfc1"].to(device).contiguous()
         t["wfc1_tiled"] = torch.empty_like(fc1)
-        prepare_fc1(dims, fc1, t["wfc1_tiled"])
+        prepare_block_weights(dims, fc1, t["wfc1_tiled"])
         return BlockParams(t)
 
 
@@ -175,12 +180,13 @@ class HeadParams:
 
 def block_forward(dims: Dims, params: BlockParams, x: torch.Tensor, segs, pos: torch.Tensor | None,
                   sigma_v: float, sigma_a: float, workspace: torch.Tensor,
-                  modulated: bool = True) -> None:
-    """In place on x [n, H] fp32."""
+                  modulated: bool = True, mods: torch.Tensor | None = None) -> None:
+    """In place on x [n, H] fp32.  ``mods``: an optional [T_s*3, 6H] fp32
+    device modulation used instead of the block's adaLN curve."""
     st = params.struct()
     check(load().mmh3_block_forward(C.byref(dims), C.byref(st), _ptr(x), x.shape[0],
                                     segments(segs), len(segs), _ptr(pos), sigma_v, sigma_a,
-                                    1 if modulated else 0, _ptr(workspace),
+                                    1 if modulated else 0, _ptr(mods), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream()))
 
 
@@ -422,6 +428,14 @@ def device_status() -> tuple[int, int]:
     return code.value, site.value
 
 
+def status_sync() -> int:
+    """Synchronise the current stream and return the device status code
+    (0 = none), raising Mmh3Error(MMH3_ERR_TIMEOUT) if a kernel gave up."""
+    code = C.c_int()
+    check(load().mmh3_status_sync(_stream(), C.byref(code)))
+    return code.value
+
+
 def selftest_wait_timeout(limit_ns: int) -> int:
     """Run the bounded-wait self test; returns the status code (7 expected)."""
     return load().mmh3_selftest_wait_timeout(limit_ns, _stream())
@@ -445,6 +459,20 @@ def prof_collect() -> tuple[dict, int]:
     nb = C.c_long()
     check(load().mmh3_prof_collect(ms, 9, C.byref(nb)))
     return dict(zip(PROF_SLOTS, list(ms))), nb.value
+
+
+PROF_KERNELS = ("adaln", "rope_table", "norm1", "qkv gemm", "attention", "out gemm", "norm2",
+                "fc1 gemm", "fc2 gemm")
+
+
+def prof_collect_kernels() -> dict:
+    """Cumulative device milliseconds and launch counts per kernel id
+    (MMH3_PROF_K_*): {name: (ms, calls)}."""
+    n = len(PROF_KERNELS)
+    ms = (C.c_double * n)()
+    calls = (C.c_long * n)()
+    check(load().mmh3_prof_collect_kernels(ms, calls, n))
+    return {k: (ms[i], calls[i]) for i, k in enumerate(PROF_KERNELS)}
 
 
 def launch_count() -> int:

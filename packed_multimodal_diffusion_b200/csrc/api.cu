@@ -32,14 +32,19 @@ using namespace mmh3;
 // the gated residual (slot 8 stays 0).  Enabled by mmh3_prof_enable(1);
 // events are recorded on the caller's stream between the launches, so the
 // phases never overlap and are never counted twice.
+// Each interval also carries the kernel it times (MMH3_PROF_K_*), so the
+// memory-bound kernels that share slot 0 get their own device times.
 struct ProfRec {
   int slot;
+  int kernel;
   cudaEvent_t a, b;
 };
 static bool g_prof_on = false;
 static std::vector<ProfRec> g_prof_recs;
 static std::vector<cudaEvent_t> g_prof_free;
 static double g_prof_ms[9] = {0};
+static double g_prof_kms[MMH3_PROF_KERNELS] = {0};
+static long g_prof_kcalls[MMH3_PROF_KERNELS] = {0};
 static long g_prof_blocks = 0;
 
 static cudaEvent_t prof_event() {
@@ -60,13 +65,14 @@ struct PhaseMark {
   PhaseMark(cudaStream_t st, bool enabled) : s(st), on(enabled && g_prof_on) {
     if (on && (last = prof_event()) != nullptr) cudaEventRecord(last, s);
   }
-  // closes the running phase as `slot` and opens the next one
-  void mark(int slot) {
+  // closes the running interval as phase `slot`, kernel `kernel`, and opens
+  // the next one
+  void mark(int slot, int kernel) {
     if (!on || last == nullptr) return;
     cudaEvent_t e = prof_event();
     if (e == nullptr) return;
     cudaEventRecord(e, s);
-    g_prof_recs.push_back({slot, last, e});
+    g_prof_recs.push_back({slot, kernel, last, e});
     cudaEvent_t next = prof_event();
     if (next) cudaEventRecord(next, s);
     last = next;
@@ -162,11 +168,11 @@ mmh3_status block_pre(const mmh3_dims& d, const mmh3_block_weights& w, const flo
   cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm1, d.eps, mods, stride, 0 * H, 1 * H, plan.block_rows, 0,
                                   ws.xn1, s);
   if (e != cudaSuccess) return cuda_fail(e, "norm1/modulate launch");
-  pm.mark(0);
+  pm.mark(0, MMH3_PROF_K_NORM1);
   mmh3_status st = gemm_qkv(dt, ws.xn1, w.wqkv, n, 3 * I, H, d.head_dim, I, w.q_norm, w.k_norm, cs, d.qk_eps,
                             ws.qkv, s);
   if (st != MMH3_OK) return st;
-  pm.mark(1);
+  pm.mark(1, MMH3_PROF_K_QKV);
   return MMH3_OK;
 }
 
@@ -188,20 +194,20 @@ mmh3_status block_post(const mmh3_dims& d, const mmh3_block_weights& w, float* x
                        : attention_kv(dt, ws.qkv, n, kv_all, n_kv, d.heads, d.head_dim, scale, ws.attn, s, ws.act,
                                       act_bytes);
   if (st != MMH3_OK) return st;
-  pm.mark(3);
+  pm.mark(3, MMH3_PROF_K_ATTN);
   st = gemm_gated_residual(dt, ws.attn, w.wout, n, H, I, x, mods, stride, 2 * H, plan.block_rows, s);
   if (st != MMH3_OK) return st;
-  pm.mark(4);
+  pm.mark(4, MMH3_PROF_K_OUT);
   cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm2, d.eps, mods, stride, 3 * H, 4 * H, plan.block_rows, 0,
                                   ws.xn2, s);
   if (e != cudaSuccess) return cuda_fail(e, "norm2/modulate launch");
-  pm.mark(0);
+  pm.mark(0, MMH3_PROF_K_NORM2);
   st = gemm_swiglu(dt, ws.xn2, w.wfc1, n, F, H, ws.act, s);
   if (st != MMH3_OK) return st;
-  pm.mark(5);
+  pm.mark(5, MMH3_PROF_K_FC1);
   st = gemm_gated_residual(dt, ws.act, w.wfc2, n, H, F, x, mods, stride, 5 * H, plan.block_rows, s);
   if (st != MMH3_OK) return st;
-  pm.mark(7);
+  pm.mark(7, MMH3_PROF_K_FC2);
   if (pm.on) ++g_prof_blocks;
   return MMH3_OK;
 }
@@ -239,13 +245,19 @@ mmh3_status common_checks(const mmh3_dims* dims, float* x, int n, const float* p
 // phase events.
 mmh3_status mmh3::block_forward_impl(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
                                      const mmh3_segment* segs, int n_seg, const float* pos_dev, double sigma_v,
-                                     double sigma_a, int modulated, void* workspace, size_t ws_bytes,
-                                     void* stream, bool profile) {
+                                     double sigma_a, int modulated, const float* mods_or_null, void* workspace,
+                                     size_t ws_bytes, void* stream, bool profile) {
   Workspace ws;
   mmh3_status st = common_checks(dims, x, n, pos_dev, workspace, ws_bytes, &ws);
   if (st != MMH3_OK) return st;
-  st = check_block(*dims, w, modulated != 0);
+  // with the caller's modulation the block reads no adaLN weights
+  const bool own_mods = modulated && mods_or_null == nullptr;
+  st = check_block(*dims, w, own_mods);
   if (st != MMH3_OK) return st;
+  if (mods_or_null != nullptr && !modulated)
+    return fail(MMH3_ERR_ARG, "mods_or_null given to an unmodulated block");
+  if (mods_or_null != nullptr && misaligned(mods_or_null))
+    return fail(MMH3_ERR_ALIGN, "mods_or_null is not 16-byte aligned");
   Plan plan;
   if (modulated) {
     st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
@@ -254,17 +266,19 @@ mmh3_status mmh3::block_forward_impl(const mmh3_dims* dims, const mmh3_block_wei
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden;
   PhaseMark pm(s, profile);
-  if (modulated) {
+  if (own_mods) {
     cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * H, plan,
                                  ws.mods, s);
     if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
+    pm.mark(0, MMH3_PROF_K_ADALN);
   }
   if (pos_dev) {
     cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+    pm.mark(0, MMH3_PROF_K_ROPE);
   }
-  pm.mark(0);
-  return block_core(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s, pm);
+  const float* mods = !modulated ? nullptr : (mods_or_null ? mods_or_null : ws.mods);
+  return block_core(*dims, *w, x, n, plan, mods, pos_dev ? ws.cs : nullptr, ws, s, pm);
 }
 
 extern "C" {
@@ -309,6 +323,11 @@ mmh3_status mmh3_adaln_modulation(const mmh3_dims* dims, const float* w, const f
   return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "adaln launch");
 }
 
+mmh3_status mmh3_prepare_block_weights(const mmh3_dims* dims, const void* fc1_gate_up, void* fc1_interleaved,
+                                       void* stream) {
+  return mmh3_prepare_fc1(dims, fc1_gate_up, fc1_interleaved, stream);
+}
+
 mmh3_status mmh3_prepare_fc1(const mmh3_dims* dims, const void* fc1_gate_up, void* fc1_tiled, void* stream) {
   clear_error();
   mmh3_status st = check_dims(dims);
@@ -323,11 +342,11 @@ mmh3_status mmh3_prepare_fc1(const mmh3_dims* dims, const void* fc1_gate_up, voi
 
 mmh3_status mmh3_block_forward(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
                                const mmh3_segment* segs, int n_seg, const float* pos_dev, double sigma_v,
-                               double sigma_a, int modulated, void* workspace, size_t ws_bytes,
-                               void* stream) {
+                               double sigma_a, int modulated, const float* mods_or_null, void* workspace,
+                               size_t ws_bytes, void* stream) {
   clear_error();
-  return block_forward_impl(dims, w, x, n, segs, n_seg, pos_dev, sigma_v, sigma_a, modulated, workspace,
-                            ws_bytes, stream, /*profile=*/true);
+  return block_forward_impl(dims, w, x, n, segs, n_seg, pos_dev, sigma_v, sigma_a, modulated, mods_or_null,
+                            workspace, ws_bytes, stream, /*profile=*/true);
 }
 
 mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* blocks, int n_blocks,
@@ -372,13 +391,14 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
   if (pos_dev) {
     cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+    pm.mark(0, MMH3_PROF_K_ROPE);
   }
   for (int i = 0; i < n_blocks; ++i) {
     const mmh3_block_weights& w = blocks[i];
     cudaError_t e = launch_adaln(w.adaln_w, w.adaln_b, w.adaln_table, dims->rank, dims->grid, 18 * H, plan,
                                  ws.mods, s);
     if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
-    pm.mark(0);
+    pm.mark(0, MMH3_PROF_K_ADALN);
     st = block_core(*dims, w, x, n, plan, ws.mods, pos_dev ? ws.cs : nullptr, ws, s, pm);
     if (st != MMH3_OK) return st;
   }
@@ -471,8 +491,8 @@ mmh3_status mmh3_block_forward_host(const mmh3_dims* dims, const mmh3_block_weig
   // 2. the block, after its input arrived
   e = cudaStreamWaitEvent(s, h->in_done[slot], 0);
   if (e != cudaSuccess) return cuda_fail(e, "host block: wait for the input");
-  st = mmh3::block_forward_impl(dims, w, x_dev, n, segs, n_seg, pos_dev, sigma_v, sigma_a, 1, workspace, ws_bytes,
-                                stream, /*profile=*/false);
+  st = mmh3::block_forward_impl(dims, w, x_dev, n, segs, n_seg, pos_dev, sigma_v, sigma_a, 1, nullptr, workspace,
+                                ws_bytes, stream, /*profile=*/false);
   if (st != MMH3_OK) return st;
   e = cudaEventRecord(h->compute_done[slot], s);
   // 3. copy the result out
@@ -929,6 +949,10 @@ mmh3_status mmh3_prof_collect(double* ms, int n_slots, long* n_blocks) {
     if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
     if (e != cudaSuccess) return cuda_fail(e, "prof: event");
     g_prof_ms[r.slot] += t;
+    if (r.kernel >= 0 && r.kernel < MMH3_PROF_KERNELS) {
+      g_prof_kms[r.kernel] += t;
+      ++g_prof_kcalls[r.kernel];
+    }
     g_prof_free.push_back(r.a);
     g_prof_free.push_back(r.b);
   }
@@ -938,8 +962,23 @@ mmh3_status mmh3_prof_collect(double* ms, int n_slots, long* n_blocks) {
   return MMH3_OK;
 }
 
+mmh3_status mmh3_prof_collect_kernels(double* ms, long* calls, int n_kernels) {
+  clear_error();
+  if (n_kernels < 0 || (n_kernels > 0 && ms == nullptr)) return fail(MMH3_ERR_ARG, "prof: ms is null");
+  double phases[9];
+  mmh3_status st = mmh3_prof_collect(phases, 9, nullptr);
+  if (st != MMH3_OK) return st;
+  for (int i = 0; i < n_kernels && i < MMH3_PROF_KERNELS; ++i) {
+    ms[i] = g_prof_kms[i];
+    if (calls) calls[i] = g_prof_kcalls[i];
+  }
+  return MMH3_OK;
+}
+
 void mmh3_prof_reset(void) {
   for (double& v : g_prof_ms) v = 0.0;
+  for (double& v : g_prof_kms) v = 0.0;
+  for (long& v : g_prof_kcalls) v = 0;
   g_prof_blocks = 0;
 }
 

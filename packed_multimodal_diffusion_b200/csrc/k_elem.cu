@@ -475,6 +475,10 @@ extern "C" mmh3_status mmh3_device_status(void* stream, int* code, int* site) {
   return MMH3_OK;
 }
 
+extern "C" mmh3_status mmh3_status_sync(void* stream, int* device_status) {
+  return mmh3_device_status(stream, device_status, nullptr);
+}
+
 extern "C" mmh3_status mmh3_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   clear_error();
   cudaStream_t s = static_cast<cudaStream_t>(stream);

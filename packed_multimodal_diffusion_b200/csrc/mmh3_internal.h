@@ -86,11 +86,12 @@ mmh3_status attention_kv(int dtype, const void* q_panel, int n_q, const void* kv
                          size_t scratch_bytes = 0);
 
 // The block on a caller-provided scratch region (see mmh3_workspace_size);
-// profile = false records no phase-profile events.
+// mods_or_null: the caller's modulation [T_s*3, 6H] fp32 (device) in place
+// of the adaLN evaluation; profile = false records no phase-profile events.
 mmh3_status block_forward_impl(const mmh3_dims* dims, const mmh3_block_weights* w, float* x, int n,
                                const mmh3_segment* segs, int n_seg, const float* pos_dev, double sigma_v,
-                               double sigma_a, int modulated, void* workspace, size_t ws_bytes, void* stream,
-                               bool profile);
+                               double sigma_a, int modulated, const float* mods_or_null, void* workspace,
+                               size_t ws_bytes, void* stream, bool profile);
 
 // 2-D row-major tensor map, 128-byte swizzle, box {128 bytes, box_rows}.
 bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, uint64_t rows,

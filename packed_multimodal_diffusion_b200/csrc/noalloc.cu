@@ -14,11 +14,16 @@
 // loaded and stays reserved until the process exits.  Its device address is
 // looked up once per device (the first call on that device, with the device
 // current), so that first call should be made before any stream capture.
+// The address is kept together with the CUDA context that was current at
+// the lookup; a call under another context on that device (after
+// cudaDeviceReset, say, when the module is loaded again and the array may
+// move) looks the address up again.
 // All calls share the array: two calls whose kernels overlap on the GPU (for
 // example on two streams without ordering) race on it and give wrong
 // results.  Nothing in the array has to start at zero -- every region the
 // block reads is written earlier in the same call.
 #include <cstring>
+#include <mutex>
 
 #include "mmh3_internal.h"
 
@@ -31,7 +36,32 @@ constexpr size_t kScratchBytes = MMH3_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-static void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+// Per device: the context of the last lookup and the address found there.
+struct ScratchSlot {
+  void* ctx;
+  void* addr;
+};
+static ScratchSlot g_scratch[kMaxDevices] = {};
+static std::mutex g_scratch_mu;
+
+// The current CUDA context (the driver's cuCtxGetCurrent, reached through
+// the runtime's entry-point query), or null if it cannot be asked.
+void* current_context() {
+  using GetCtx = int (*)(void**);
+  static GetCtx fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCtx>(p);
+  });
+  void* ctx = nullptr;
+  if (fn != nullptr && fn(&ctx) != 0) ctx = nullptr;
+  return ctx;
+}
 
 // Device address of the scratch array on the current device, or null with
 // the error recorded.
@@ -46,16 +76,20 @@ void* scratch_address(mmh3_status* st) {
     *st = mmh3::fail(MMH3_ERR_UNSUPPORTED, "noalloc: device ordinal %d above %d", dev, kMaxDevices - 1);
     return nullptr;
   }
-  if (g_scratch_addr[dev] == nullptr) {
+  void* ctx = current_context();
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchSlot& slot = g_scratch[dev];
+  if (slot.addr == nullptr || slot.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) {
       *st = mmh3::cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "noalloc: cudaGetSymbolAddress");
       return nullptr;
     }
-    g_scratch_addr[dev] = p;
+    slot.ctx = ctx;
+    slot.addr = p;
   }
-  return g_scratch_addr[dev];
+  return slot.addr;
 }
 
 }  // namespace
@@ -84,6 +118,6 @@ extern "C" mmh3_status mmh3_block_forward_noalloc(const mmh3_dims* dims, const m
   }
   void* scratch = scratch_address(&st);
   if (scratch == nullptr) return st;
-  return mmh3::block_forward_impl(dims, w, x, n, segs, n_seg, pos_dev, sigma_v, sigma_a, modulated, scratch,
-                                  kScratchBytes, stream, /*profile=*/false);
+  return mmh3::block_forward_impl(dims, w, x, n, segs, n_seg, pos_dev, sigma_v, sigma_a, modulated, nullptr,
+                                  scratch, kScratchBytes, stream, /*profile=*/false);
 }

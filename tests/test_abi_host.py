@@ -36,6 +36,12 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, n), n
     assert set(_lib.SIGNATURES) == names
     assert lib.mmh3_version().startswith(b"mmh3-b200")
+    # the boundary's calls under the names the design fixes
+    for n in ("mmh3_time_shift_sigma", "mmh3_workspace_size", "mmh3_prepare_block_weights",
+              "mmh3_resolve_rows", "mmh3_adaln_modulation", "mmh3_block_forward", "mmh3_stack_forward",
+              "mmh3_vit_layer_forward", "mmh3_status_sync", "mmh3_last_error", "mmh3_layout_t2va",
+              "mmh3_layout_image"):
+        assert n in names, n
 
 
 def test_time_shift_matches_oracle():
@@ -92,7 +98,7 @@ def test_argument_errors_are_reported_before_launch():
     segs = api.segments([(0, 10, 1, 0)])
     ws = C.c_void_p(256)  # never dereferenced: validation fails first
     rc = lib.mmh3_block_forward(C.byref(d), None, C.c_void_p(256), 10, segs, 1, None, 0.5, 0.2, 1,
-                                ws, v.value, None)
+                                None, ws, v.value, None)
     assert rc in (1, 4)
     # segments with a gap
     with pytest.raises(_lib.Mmh3Error) as e:

@@ -187,3 +187,33 @@ def test_launch_count_of_one_block(cuda_ok):
     c0 = api.launch_count()
     api.block_forward(dims_c, params, xd, segs, pd, *sigma_pair(0.5), ws)
     assert api.launch_count() - c0 == 9
+
+
+def test_block_caller_modulation_replaces_the_adaln_curve(cuda_ok):
+    # mods_or_null: the oracle's modulation at timesteps other than the
+    # plan's (so the block's own curve would give different rows) is passed
+    # in, with the adaLN weights left out of the weight struct; the block
+    # must match the oracle block run on exactly those rows.
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    n = int(pos.shape[0])
+    w = small_block_weights(35, 256, 2, 128, 512)
+    x = configs.synth.normal((n, 256), 81, 1.0)
+    sv, sa = sigma_pair(0.5)
+    ts, slot = O.plan_timesteps(sv, sa, segs)
+    rows = O.token_rows(segs, slot, n)
+    mods = O.block_mods(f64(w["adaln_w"]), f64(w["adaln_b"]), f64(w["adaln_table"]), [0.15, 0.85], 256)
+    ref = O.block_forward({k: f64(v) for k, v in w.items()}, f64(x), mods, rows, f64(pos), dims_o)
+    params = api.BlockParams.from_host(dims_c, {k: v for k, v in w.items() if not k.startswith("adaln")})
+    xd = x.cuda().clone()
+    pd = torch.as_tensor(np.asarray(pos, dtype=np.float32)).cuda()
+    ws = torch.empty(api.workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
+    md = torch.as_tensor(mods.astype(np.float32)).cuda()
+    api.block_forward(dims_c, params, xd, segs, pd, sv, sa, ws, mods=md)
+    assert api.status_sync() == 0
+    assert_close(xd, ref, what="x_out with caller modulation")
+    assert_close(xd.cpu().double() - x.double(), ref - f64(x), what="block delta with caller modulation")
+    # the block's own curve gives other rows: its delta would fail the bar
+    own, _, _ = oracle_block(w, x, segs, pos, sv, sa, dims_o)
+    from gpu_common import cosine
+    assert cosine(own - f64(x), ref - f64(x)) < BF16_COS

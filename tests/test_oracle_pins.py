@@ -495,6 +495,20 @@ def test_block_zero_gates_is_identity_and_sampled_rows_agree():
                                full[[5, 0, 3]], atol=1e-13)
 
 
+def test_block_in_chunks_with_kv_cache_equals_the_whole_block():
+    # the block computed in chunks of query rows, k and v computed once by
+    # the first chunk and read back by the others, gives the whole block
+    p, dims, x, mods, rows, pos = _tiny_block_inputs()
+    full = O.block_forward(p, x, mods, rows, pos, dims)
+    cache = {}
+    n = x.shape[0]
+    parts = [O.block_forward(p, x, mods, rows, pos, dims, sample_rows=np.arange(a, min(a + 5, n)),
+                             kv_cache=cache) for a in range(0, n, 5)]
+    assert set(cache) == {"k", "v"} and cache["k"].shape[0] == n
+    # equal up to the summation order the matrix product picks for a row count
+    np.testing.assert_allclose(np.concatenate(parts), full, rtol=0, atol=1e-12)
+
+
 def test_block_zero_shift_scale_reduces_to_plain_rmsnorm():
     p, dims, x, mods, rows, pos = _tiny_block_inputs(seed=9)
     H = dims["hidden"]

@@ -21,6 +21,18 @@ from packed_multimodal_diffusion_b200 import _lib
 pytestmark = pytest.mark.gpu
 
 
+def _poison(dims, seed):
+    """A no-alloc call on other data and a larger size, so that the shared
+    scratch holds stale values everywhere the next call could read."""
+    segs, pos = t2va(30, 4, 16, 24, 40)          # 30 + 80 + 384 = 494 tokens
+    n = int(pos.shape[0])
+    params = api.BlockParams.from_host(dims, small_block_weights(seed, 256, 2, 128, 512))
+    x = configs.synth.normal((n, 256), seed + 1, 3.0).cuda()
+    pd = torch.as_tensor(np.asarray(pos, np.float32)).cuda()
+    api.block_forward_noalloc(dims, params, x, segs, pd, *sigma_pair(0.9))
+    api.device_status()
+
+
 def test_noalloc_block_matches_workspace_block_twice(cuda_ok):
     dims = api.make_dims(256, 2, 128, 512)
     segs, pos = t2va(20, 3, 16, 20, 20)          # 300 tokens, ragged last tile
@@ -37,11 +49,16 @@ def test_noalloc_block_matches_workspace_block_twice(cuda_ok):
     api.device_status()
 
     for call in range(2):                           # two calls in a row share the scratch
+        # another workload leaves different values in the scratch first, so a
+        # read of a region before this call writes it would show
+        _poison(dims, 400 + call)
         got = x.clone()
         api.block_forward_noalloc(dims, params, got, segs, pd, sv, sa)
         api.device_status()
         assert_close(got, ref, BF16_MAXABS, BF16_COS, what=f"no-alloc call {call}")
         assert_close(got - x, ref - x, BF16_MAXABS, BF16_COS, what=f"no-alloc call {call} delta")
+        # the same kernels on the same inputs: identical to the last bit
+        assert torch.equal(got, ref), f"no-alloc call {call} differs from the workspace block"
 
 
 def test_noalloc_rejects_sizes_beyond_the_fixed_scratch(cuda_ok):
