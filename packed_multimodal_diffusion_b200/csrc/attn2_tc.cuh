@@ -74,13 +74,13 @@ __device__ __forceinline__ float attn_max8(const float (&pm)[8]) {
 // P = 2^(s * scale_log2 - m) for the keys of slices [H0, H1) (32 keys a
 // slice) as bf16 pairs over the first 64 columns of S (16 columns a slice);
 // the row sum accumulates in acc0 / acc1.  Scale/shift and the sum run as
-// packed f32x2 operations; the exponentials stay on MUFU.  With kMax (two
-// slices), the maximum of all 128 scores is folded into pm alongside, two
-// three-input maxima per pair of exponentials.
-template <int H0, int H1, bool kMax>
+// packed f32x2 operations; the exponentials stay on MUFU.  With kMaxHi (two
+// slices), the maximum of the upper 64 scores (keys 64..127) is folded into
+// pm alongside, one three-input maximum per pair of exponentials.
+template <int H0, int H1, bool kMaxHi>
 __device__ __forceinline__ void attn_exp_slices(const float (&s)[128], uint32_t ts, float scale_log2, float m,
                                                 float2& acc0, float2& acc1, float (&pm)[8]) {
-  static_assert(!kMax || H1 - H0 == 2, "the folded maximum spans two slices");
+  static_assert(!kMaxHi || (H0 == 0 && H1 == 2), "the folded maximum runs alongside the lower half");
   const float2 sc2 = make_float2(scale_log2, scale_log2);
   const float2 nm2 = make_float2(-m, -m);
 #pragma unroll
@@ -88,10 +88,9 @@ __device__ __forceinline__ void attn_exp_slices(const float (&s)[128], uint32_t 
     uint32_t pk[16];
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
-      if constexpr (kMax) {
-        const int g = (h - H0) * 16 + q;
-        pm[g & 7] = fmax3(pm[g & 7], s[4 * g], s[4 * g + 1]);
-        pm[g & 7] = fmax3(pm[g & 7], s[4 * g + 2], s[4 * g + 3]);
+      if constexpr (kMaxHi) {
+        const int g = h * 16 + q;
+        pm[g & 7] = fmax3(pm[g & 7], s[64 + 2 * g], s[64 + 2 * g + 1]);
       }
       const int k = h * 32 + 2 * q;
       const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2);
@@ -349,16 +348,23 @@ __global__ void __launch_bounds__(320, 1)
         m_ref = attn_max8(pm) * scale_log2;
         attn_exp_slices<0, 2, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
       } else {
-        // keys 0..63 against the current reference, with the row maximum
-        // of all 128 keys folded in
+        // keys 0..63 against the current reference, with the maximum of
+        // keys 64..127 folded in.  The lower half needs no maximum of its
+        // own: its exponentials are non-negative, so a lower-half sum of at
+        // most 2^8 bounds each of them by 2^8, i.e. no lower score exceeds
+        // the reference by more than 8 (log2 domain).  A row whose lower
+        // sum or upper maximum fails that bound rescales to its full row
+        // maximum and redoes the lower half.
 #pragma unroll
         for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
         attn_exp_slices<0, 2, true>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
-        const float m_tile = attn_max8(pm) * scale_log2;
-        const bool need = m_tile > m_ref + 8.0f;
+        const float m_hi = attn_max8(pm) * scale_log2;
+        const float lo_sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        const bool need = lo_sum > 256.0f || m_hi > m_ref + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           // O_i holds every earlier product (see the kernel comment).
-          const float m_new = need ? m_tile : m_ref;
+          attn_row_max(s, pm);
+          const float m_new = need ? fmaxf(attn_max8(pm) * scale_log2, m_ref) : m_ref;
           const float f = ex2_approx(m_ref - m_new);
           l_sum *= f;
           m_ref = m_new;

@@ -719,16 +719,16 @@ struct EpiBiasAct : NoSetup {
 };
 
 // ------------------------------------------------------------------ kernel
-// Tile order: groups of kGroupM row tiles, all column tiles of a group
-// before the next group, so the A rows of a group and all of B stay in L2
-// while the group is processed (A is read from DRAM about once).
-constexpr int kGroupM = 16;
-
-__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mt, int& nt) {
-  const int per_group = kGroupM * n_tiles;
+// Tile order: groups of group_m row tiles, all column tiles of a group
+// before the next group, row tiles fastest within a group.  The persistent
+// CTAs work on a window of consecutive tiles, so a group's A panel is
+// reused from L2 by all its column tiles while B is swept once per group;
+// the host sizes the group (group_m_for).
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group_m, int& mt, int& nt) {
+  const int per_group = group_m * n_tiles;
   const int g = tile / per_group;
-  const int first_m = g * kGroupM;
-  const int gm = (m_tiles - first_m) < kGroupM ? (m_tiles - first_m) : kGroupM;
+  const int first_m = g * group_m;
+  const int gm = (m_tiles - first_m) < group_m ? (m_tiles - first_m) : group_m;
   const int t = tile - g * per_group;
   mt = first_m + t % gm;
   nt = t / gm;
@@ -756,8 +756,8 @@ constexpr int gemm_smem_bytes() {
 template <typename T, int BN, int STAGES, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, int M, int N, int K, Epi epi, DevStatus* status,
-                   uint64_t limit_ns) {
+                   const __grid_constant__ CUtensorMap tmC, int M, int N, int K, int group_m, Epi epi,
+                   DevStatus* status, uint64_t limit_ns) {
   using Sh = GemmShape<BN>;
   constexpr bool kTf32 = ElemTraits<T>::kTf32;
   constexpr int kOut = Epi::kStageOut;
@@ -825,7 +825,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         int mt, nt;
-        tile_coords(tile, m_tiles, n_tiles, mt, nt);
+        tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (*abort_flag || !mbar_wait(empty_bar(stage), phase ^ 1u, limit_ns)) {
             if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, tile);
@@ -920,7 +920,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       int mt, nt;
-      tile_coords(tile, m_tiles, n_tiles, mt, nt);
+      tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
       const int row = mt * Sh::BM + lgrp * 32 + lane;
       // warp-uniform (the TMEM loads are warp-collective); group-uniform for
       // staged output (its named barriers need all 128 threads)
@@ -1002,7 +1002,8 @@ constexpr int gemm2_smem_bytes() {
 template <int BN, int STAGES, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC, int M, int N, int K, Epi epi, DevStatus* status,
+                    const __grid_constant__ CUtensorMap tmC, int M, int N, int K, int group_m, Epi epi,
+                    DevStatus* status,
                     uint64_t limit_ns) {
   using Sh = Gemm2Shape<BN>;
   constexpr int kBK = 64;  // bf16 K elements per stage (128 bytes)
@@ -1074,7 +1075,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
         int mt, nt;
-        tile_coords(tile, m_tiles, n_tiles, mt, nt);
+        tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
         const int a_row = mt * 2 * Sh::BM + (int)rank * Sh::BM;
         const int b_row = nt * BN + (int)rank * Sh::kBRows;
         for (int kb = 0; kb < k_blocks; ++kb) {
@@ -1173,7 +1174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < num_tiles; tile += n_pairs) {
       int mt, nt;
-      tile_coords(tile, m_tiles, n_tiles, mt, nt);
+      tile_coords(tile, m_tiles, n_tiles, group_m, mt, nt);
       const int row0 = mt * 2 * Sh::BM + (int)rank * Sh::BM;
       const int row = row0 + lgrp * 32 + lane;
       // The decision to go on is uniform over the warp (TMEM loads are

@@ -9,6 +9,8 @@
 // switched at run time.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "gemm_tc.cuh"
@@ -46,6 +48,30 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, int esize, uint64_t cols, ui
 }
 
 // ---------------------------------------------------------------- launch
+// Row tiles per group of the persistent tile order (see tile_coords).  A
+// group's A panel (group_m row tiles x K) is reused by every column tile of
+// the group, and B is swept once per group; the L2 that a working set can
+// count on is about one die's half (whole-operand residency of 58-71 MB
+// thrashed: A or B re-read 6-12 times), so the panel is kept to about
+// 24 MB.  With few column tiles (N <= 16 tiles) a group of at most 8 row
+// tiles measured best (the out and fc2 GEMMs of the block workload).
+// Measured at that workload, group sizes 1..52, two alternating rounds:
+// qkv 0.42 ms for 8..26, fc1 0.943-0.955 ms at 26 (1.06 at 1), fc2 0.53 ms
+// for 1..16 (0.62 at 52), out 0.147-0.150 ms for 2..8.  MMH3_GEMM_GROUP_M=<g>
+// (g >= 1) overrides the choice, for such measurements.
+static int group_m_for(int K, int n_tiles, int m_tiles, int bm) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* v = std::getenv("MMH3_GEMM_GROUP_M");
+    forced = v ? std::max(0, std::atoi(v)) : 0;
+  }
+  if (forced > 0) return std::min(forced, m_tiles);
+  const int64_t row_tile_bytes = (int64_t)bm * K * 2;
+  int g = (int)std::max<int64_t>(1, ((int64_t)24 << 20) / row_tile_bytes);
+  if (n_tiles <= 16) g = std::min(g, 8);
+  return std::min(g, m_tiles);
+}
+
 template <int BN, int OUT>
 constexpr int stages_for() {
   constexpr int base = BN >= 256 ? 4 : (BN >= 224 ? 5 : 6);
@@ -87,10 +113,13 @@ static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, c
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM smem attribute");
   }
-  const int tiles = ((M + 127) / 128) * ((N + BN - 1) / BN);
+  const int m_tiles = (M + 127) / 128;
+  const int tiles = m_tiles * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
-  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns()); count_launch();
+  const int gm = group_m_for(K, (N + BN - 1) / BN, m_tiles, 128);
+  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, gm, epi, device_status_ptr(), wait_limit_ns());
+  count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return MMH3_OK;
@@ -155,10 +184,13 @@ static mmh3_status run_gemm2(const void* A, const void* B, int M, int N, int K, 
     if (n < 1) return fail(MMH3_ERR_CUDA, "pair GEMM: no CTA pair fits on this device");
     max_pairs = n;
   }
-  const int tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
+  const int m_tiles = (M + 255) / 256;
+  const int tiles = m_tiles * ((N + BN - 1) / BN);
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
-  kern<<<2 * pairs, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, epi, device_status_ptr(), wait_limit_ns()); count_launch();
+  const int gm = group_m_for(K, (N + BN - 1) / BN, m_tiles, 256);
+  kern<<<2 * pairs, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, gm, epi, device_status_ptr(), wait_limit_ns());
+  count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
   return MMH3_OK;

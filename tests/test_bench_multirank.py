@@ -70,7 +70,7 @@ def test_measured_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
         '"0","attn2_tc_kernel(args)","gpu__time_duration.sum","msecond","1.5"',
         '"1","attn_merge_kernel(args)","dram__bytes_read.sum","byte","1000"',
         '"1","attn_merge_kernel(args)","dram__bytes_write.sum","byte","24"',
-        '"1","attn_merge_kernel(args)","gpu__time_duration.sum","usecond","8"',
+        '"1","attn_merge_kernel(args)","gpu__time_duration.sum","us","8"',
         '"2","gemm_tc_kernel(args)","dram__bytes_read.sum","byte","77"',
     ]) + "\n"
     (tmp_path / "cap.csv").write_text(csv_text)
