@@ -214,15 +214,29 @@ def block_flops(n, H=2688, I=2688, F=10752):
     return gemm
 
 
-def hbm_bytes(n, H=2688, k=16, t_s=2, rank=24):
+def hbm_bytes(n, H=2688, k=16, t_s=2, rank=24, blocks_per_prologue=1, act_bytes=2):
     """Algorithmic HBM bytes per launch of the memory-bound kernels:
-    RMSNorm + modulate reads x (fp32) and writes xn (bf16); the adaLN curve
-    reads its basis [T_s*18H, R] and bias and writes the modulation (fp32);
-    the rotation table reads the positions and writes (cos, sin) fp32 pairs."""
-    norm = n * H * 4 + n * H * 2
+    RMSNorm + modulate reads x (fp32) and writes xn (act dtype); the
+    prologue reads each block's adaLN basis [T_s*18H, R] and bias and writes
+    its modulation (fp32), and writes the rotation table ((cos, sin) fp32
+    pairs from the positions)."""
+    norm = n * H * 4 + n * H * act_bytes
     return {"norm1": norm, "norm2": norm,
-            "adaln": t_s * 18 * H * (rank * 4 + 4 + 4),
-            "rope_table": n * 3 * 4 + n * 3 * k * 8}
+            "prologue": blocks_per_prologue * t_s * 18 * H * (rank * 4 + 4 + 4) + n * 3 * 4 + n * 3 * k * 8}
+
+
+def hbm_fractions(kernels, hb, peak_gbs):
+    """Per memory-bound kernel: mean event time per launch, bytes, GB/s and
+    the fraction of the HBM peak."""
+    out = {}
+    for name, nbytes in hb.items():
+        kms, calls = kernels.get(name, (0.0, 0))
+        if calls:
+            t = kms / calls
+            gbs = nbytes / (t / 1e3) / 1e9
+            out[name] = {"ms_per_launch": round(t, 5), "launches": calls, "bytes_per_launch": nbytes,
+                         "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak_gbs, 4)}
+    return out
 
 
 def percentile(v, q):
@@ -384,15 +398,7 @@ def run_gpu(args):
     peak, peak_kind, peak_why = choose_peak(peaks, clocks, ms / 1e3)
     achieved = flops[dom] / (per_launch[dom] / 1e3) / 1e12
     total_flop = sum(flops.values())
-    hb = hbm_bytes(n)
-    hbm_kernels = {}
-    for name, nbytes in hb.items():
-        kms, calls = kernels[name]
-        if calls:
-            t = kms / calls
-            gbs = nbytes / (t / 1e3) / 1e9
-            hbm_kernels[name] = {"ms_per_launch": round(t, 5), "launches": calls, "bytes_per_launch": nbytes,
-                                 "achieved_gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    hbm_kernels = hbm_fractions(kernels, hbm_bytes(n), peaks["hbm_gbs"])
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": step_ms, "higher_is_better": True,
@@ -606,6 +612,7 @@ def run_workload(args):
     ms = _time(step, steps, warmup)
     api.prof_enable(False)
     phases, nblocks = api.prof_collect()
+    kernels = api.prof_collect_kernels()
     api.device_status()
     flops = block_flops(n, c.hidden, c.heads * c.head_dim, c.ffn)
     per_block = {k: v / max(1, nblocks) for k, v in phases.items() if v > 0}
@@ -619,6 +626,11 @@ def run_workload(args):
                 phases_ms_per_block={k: round(v, 4) for k, v in per_block.items()},
                 phase_frac_of_peak={k: round(flops[k] / (per_block[k] / 1e3) / 1e12 / peak, 4)
                                     for k in flops if k in per_block},
+                hbm_kernels={"peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                             **hbm_fractions(kernels, hbm_bytes(
+                                 n, c.hidden, c.rope_k, len(api.plan_timesteps(segs, n, sv, sa)[0]), c.rank,
+                                 blocks_per_prologue=min(c.n_blocks, 64),
+                                 act_bytes=4 if c.act_dtype == torch.float32 else 2), peaks["hbm_gbs"])},
                 config={"workload": f"{c.name}: n {n}, hidden {c.hidden}, {c.heads}x{c.head_dim} heads, "
                                     f"SwiGLU {c.ffn}, {c.n_blocks} blocks" + (", output heads" if heads else "")})
     print(json.dumps(line), flush=True)

@@ -562,19 +562,20 @@ mmh3_status mmh3_prof_collect(double* ms, int n_slots, long* n_blocks);
 void mmh3_prof_reset(void);
 
 /* The same intervals by kernel (a finer split of the phase slots: slot 0
- * holds the adaLN curve, the rotation table and both RMSNorm + modulate
- * launches).  Attention counts its whole step (the main launch and, when
- * its last wave is split, the tail launch and the merge). */
-#define MMH3_PROF_K_ADALN 0   /* adaLN curve -> modulation */
-#define MMH3_PROF_K_ROPE 1    /* rotation (cos, sin) table */
-#define MMH3_PROF_K_NORM1 2   /* segment gather + RMSNorm(norm1) + modulate */
-#define MMH3_PROF_K_QKV 3     /* qkv GEMM + qk-norm + rotation */
-#define MMH3_PROF_K_ATTN 4    /* attention step */
-#define MMH3_PROF_K_OUT 5     /* out GEMM + gated residual */
-#define MMH3_PROF_K_NORM2 6   /* segment gather + RMSNorm(norm2) + modulate */
-#define MMH3_PROF_K_FC1 7     /* fc1 GEMM + SwiGLU */
-#define MMH3_PROF_K_FC2 8     /* fc2 GEMM + gated residual */
-#define MMH3_PROF_KERNELS 9
+ * holds the prologue and both RMSNorm + modulate launches).  The prologue
+ * is one launch that evaluates the adaLN curve of one block (of up to 64
+ * blocks at once in mmh3_stack_forward) and writes the rotation table.
+ * Attention counts its whole step (the main launch and, when its last wave
+ * is split, the tail launch and the merge). */
+#define MMH3_PROF_K_PROLOGUE 0 /* adaLN curve -> modulation, rotation table */
+#define MMH3_PROF_K_NORM1 1    /* segment gather + RMSNorm(norm1) + modulate */
+#define MMH3_PROF_K_QKV 2      /* qkv GEMM + qk-norm + rotation */
+#define MMH3_PROF_K_ATTN 3     /* attention step */
+#define MMH3_PROF_K_OUT 4      /* out GEMM + gated residual */
+#define MMH3_PROF_K_NORM2 5    /* segment gather + RMSNorm(norm2) + modulate */
+#define MMH3_PROF_K_FC1 6      /* fc1 GEMM + SwiGLU */
+#define MMH3_PROF_K_FC2 7      /* fc2 GEMM + gated residual */
+#define MMH3_PROF_KERNELS 8
 
 /* Waits for the recorded events like mmh3_prof_collect (which it calls, so
  * the phase totals are folded in too) and writes, for each kernel id below

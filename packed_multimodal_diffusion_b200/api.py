@@ -461,8 +461,8 @@ def prof_collect() -> tuple[dict, int]:
     return dict(zip(PROF_SLOTS, list(ms))), nb.value
 
 
-PROF_KERNELS = ("adaln", "rope_table", "norm1", "qkv gemm", "attention", "out gemm", "norm2",
-                "fc1 gemm", "fc2 gemm")
+PROF_KERNELS = ("prologue", "norm1", "qkv gemm", "attention", "out gemm", "norm2", "fc1 gemm",
+                "fc2 gemm")
 
 
 def prof_collect_kernels() -> dict:

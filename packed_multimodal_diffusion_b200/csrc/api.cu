@@ -221,6 +221,22 @@ mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x
   return block_post(d, w, x, n, plan, mods, ws, s, pm, nullptr, 0);
 }
 
+// adaLN modulation of one block (when own_mods) into ws.mods and the
+// rotation table (when pos != null) into ws.cs, in one launch.
+mmh3_status prologue(const mmh3_dims& d, const mmh3_block_weights* w, bool own_mods, const Plan& plan,
+                     const Workspace& ws, const float* pos, int n, cudaStream_t s) {
+  if (!own_mods && pos == nullptr) return MMH3_OK;
+  AdalnBatch ab{};
+  if (own_mods) {
+    ab.w[0] = w->adaln_w;
+    ab.b[0] = w->adaln_b;
+    ab.table[0] = w->adaln_table;
+  }
+  cudaError_t e = launch_prologue(ab, own_mods ? 1 : 0, d.rank, d.grid, 18 * d.hidden, plan, ws.mods, 0, pos, n,
+                                  d.rope_k, d.rope_theta, ws.cs, s);
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "prologue launch");
+}
+
 mmh3_status common_checks(const mmh3_dims* dims, float* x, int n, const float* pos, void* ws,
                           size_t ws_bytes, Workspace* out_ws) {
   mmh3_status st = check_dims(dims);
@@ -266,17 +282,9 @@ mmh3_status mmh3::block_forward_impl(const mmh3_dims* dims, const mmh3_block_wei
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden;
   PhaseMark pm(s, profile);
-  if (own_mods) {
-    cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * H, plan,
-                                 ws.mods, s);
-    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
-    pm.mark(0, MMH3_PROF_K_ADALN);
-  }
-  if (pos_dev) {
-    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
-    pm.mark(0, MMH3_PROF_K_ROPE);
-  }
+  st = prologue(*dims, w, own_mods, plan, ws, pos_dev, n, s);
+  if (st != MMH3_OK) return st;
+  if (own_mods || pos_dev) pm.mark(0, MMH3_PROF_K_PROLOGUE);
   const float* mods = !modulated ? nullptr : (mods_or_null ? mods_or_null : ws.mods);
   return block_core(*dims, *w, x, n, plan, mods, pos_dev ? ws.cs : nullptr, ws, s, pm);
 }
@@ -388,18 +396,38 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   PhaseMark pm(s, true);
-  if (pos_dev) {
-    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
-    pm.mark(0, MMH3_PROF_K_ROPE);
+  // Every block's modulation is evaluated up front, up to kAdalnBatch blocks
+  // per launch, into the head-scratch region (unused until the heads); the
+  // first launch also writes the rotation table.  When that region cannot
+  // hold one block's rows, each block's modulation goes to ws.mods just
+  // before the block.
+  const long long mods_floats = (long long)plan.n_ts * 18 * H;
+  const size_t head_bytes = (size_t)n * H * esize_of(dims->act_dtype);
+  long long fit = (long long)(head_bytes / ((size_t)mods_floats * 4));
+  const int per_launch = (int)std::max(1ll, std::min<long long>(kAdalnBatch, fit));
+  float* mbase = fit >= 1 ? static_cast<float*>(ws.head) : ws.mods;
+  if (n_blocks == 0 && pos_dev) {
+    cudaError_t e = launch_prologue(AdalnBatch{}, 0, dims->rank, dims->grid, 18 * H, plan, mbase, mods_floats,
+                                    pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+    pm.mark(0, MMH3_PROF_K_PROLOGUE);
   }
   for (int i = 0; i < n_blocks; ++i) {
-    const mmh3_block_weights& w = blocks[i];
-    cudaError_t e = launch_adaln(w.adaln_w, w.adaln_b, w.adaln_table, dims->rank, dims->grid, 18 * H, plan,
-                                 ws.mods, s);
-    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
-    pm.mark(0, MMH3_PROF_K_ADALN);
-    st = block_core(*dims, w, x, n, plan, ws.mods, pos_dev ? ws.cs : nullptr, ws, s, pm);
+    if (i % per_launch == 0) {
+      const int cnt = std::min(per_launch, n_blocks - i);
+      AdalnBatch ab{};
+      for (int b = 0; b < cnt; ++b) {
+        ab.w[b] = blocks[i + b].adaln_w;
+        ab.b[b] = blocks[i + b].adaln_b;
+        ab.table[b] = blocks[i + b].adaln_table;
+      }
+      cudaError_t e = launch_prologue(ab, cnt, dims->rank, dims->grid, 18 * H, plan, mbase, mods_floats,
+                                      i == 0 ? pos_dev : nullptr, n, dims->rope_k, dims->rope_theta, ws.cs, s);
+      if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+      pm.mark(0, MMH3_PROF_K_PROLOGUE);
+    }
+    const float* mods = mbase + (i % per_launch) * mods_floats;
+    st = block_core(*dims, blocks[i], x, n, plan, mods, pos_dev ? ws.cs : nullptr, ws, s, pm);
     if (st != MMH3_OK) return st;
   }
   if (heads == nullptr) return MMH3_OK;
@@ -522,15 +550,8 @@ mmh3_status mmh3_block_cp_begin(const mmh3_dims* dims, const mmh3_block_weights*
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   PhaseMark pm(s, false);
-  if (modulated) {
-    cudaError_t e = launch_adaln(w->adaln_w, w->adaln_b, w->adaln_table, dims->rank, dims->grid, 18 * dims->hidden,
-                                 plan, ws.mods, s);
-    if (e != cudaSuccess) return cuda_fail(e, "adaln launch");
-  }
-  if (pos_dev) {
-    cudaError_t e = launch_rope_table(pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
-  }
+  st = prologue(*dims, w, modulated != 0, plan, ws, pos_dev, n, s);
+  if (st != MMH3_OK) return st;
   st = block_pre(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s, pm);
   if (st != MMH3_OK) return st;
   const size_t I = (size_t)dims->heads * dims->head_dim;

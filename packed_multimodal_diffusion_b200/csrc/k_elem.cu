@@ -1,5 +1,6 @@
-// Memory-bound kernels of the block: the adaLN curve evaluation, the fused
-// segment-gather RMSNorm + modulate, the rotary (cos, sin) table, the
+// Memory-bound kernels of the block: the prologue (adaLN curve evaluation
+// and the rotary (cos, sin) table in one launch), the fused
+// segment-gather RMSNorm + modulate, the
 // encoder layer's LayerNorm and the weight-preparation copies; plus the
 // device status word written by bounded waits.
 //
@@ -86,47 +87,167 @@ __global__ void __launch_bounds__(256) adaln_kernel(const float* __restrict__ w,
   }
 }
 
-cudaError_t launch_adaln(const float* w, const float* b, const float* table, int rank, int grid,
-                         int rows_per_slot, const Plan& plan, float* out, cudaStream_t s) {
-  CurveArgs ca{};
-  for (int i = 0; i < plan.n_ts; ++i) curve_coords(plan.ts[i], grid, &ca.i0[i], &ca.f[i]);
-  const int total = plan.n_ts * rows_per_slot;
-  int blocks = (total + 255) / 256;
-  const int cap = num_sms() * 8;
-  if (blocks > cap) blocks = cap;
-  adaln_kernel<<<blocks, 256, 0, s>>>(w, b, table, rank, rows_per_slot, plan.n_ts, ca, out); count_launch();
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------- rotary (cos, sin)
-// cs[i, j] = (cos a, sin a), a = pos[i, j / k] * inv_freq[j % k], the
-// product taken in fp64 and rounded to fp32 as rope_angles does.
+// ------------------------------------------------ the block's prologue
+// One launch computes what a block (or a whole stack) reads before its
+// first RMSNorm: the adaLN modulation rows of up to kAdalnBatch blocks and
+// the rotation (cos, sin) table.  Work items are one warp each: the first
+// n_ab * (n_ts * rows_per_slot / 32) items evaluate 32 consecutive
+// modulation rows of one block; the rest fill 256 table entries.
+//  - adaLN ("cortiq_engine/mmh3.rs", Adaln::eval): the warp's 32 basis rows
+//    are one contiguous run of 32 * rank floats, read as float4 at
+//    lane + 32 q (coalesced); each float4 is dotted with its four curve
+//    coordinates, and a row's rank / 4 partial dots are added from shared
+//    memory, then the bias; the 32 results are one coalesced store.
+//  - rotation table ("cortiq_engine/mmh3.rs", rope_angles): cs[i, j] =
+//    (cos a, sin a), a = pos[i, j / K] * inv_freq[j % K], the product taken
+//    in fp64 and rounded to fp32, then CUDA's sincosf.
 struct InvFreq {
   float v[32];
 };
 
-__global__ void rope_table_kernel(const float* __restrict__ pos, int n, int k, InvFreq inv,
-                                  float2* __restrict__ cs) {
-  const int np = 3 * k;
-  const long total = (long)n * np;
-  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
-    const int i = (int)(e / np), j = (int)(e % np);
-    const float a = (float)((double)pos[i * 3 + j / k] * (double)inv.v[j % k]);
-    float sv, cv;
-    sincosf(a, &sv, &cv);
-    cs[e] = make_float2(cv, sv);
+template <int K>  // rotation frequencies per axis (8 or 16); 0: no table
+__global__ void __launch_bounds__(256, 4)
+    prologue_kernel(AdalnBatch ab, int n_ab, int rank, int rows_per_slot, int n_ts, CurveArgs ca,
+                    float* __restrict__ mods, long long mods_stride, const float* __restrict__ pos, int n,
+                    InvFreq inv, float2* __restrict__ cs) {
+  __shared__ __align__(16) float part[8][32 * 8];
+  __shared__ __align__(16) float coord[8][32];
+  __shared__ float sinv[K > 0 ? K : 1];
+  if constexpr (K > 0) {
+    if (threadIdx.x == 0) {
+#pragma unroll
+      for (int i = 0; i < K; ++i) sinv[i] = inv.v[i];  // static indices: no local copy of the parameter
+    }
+    __syncthreads();
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nq = rank >> 2;
+  const int row_items = (n_ts * rows_per_slot) >> 5;  // per block
+  const int ad_items = n_ab * row_items;              // < 2^31 (checked by the host)
+  const int n_warps = gridDim.x * 8;
+  const int gw = blockIdx.x * 8 + warp;
+  float* pw = part[warp];
+  float* cw = coord[warp];
+  // adaLN: each warp walks its own contiguous range of items, so the curve
+  // coordinates (one block, one slot) are recomputed only where the range
+  // crosses a slot, and consecutive items read consecutive basis rows.
+  const int chunk = (ad_items + n_warps - 1) / n_warps;
+  const int it_end = min(ad_items, (gw + 1) * chunk);
+  int cur = -1;  // bb * 2 + slot of the coordinates in cw
+  for (int it = gw * chunk; it < it_end; ++it) {
+    const int bb = it / row_items;
+    const int row0 = (it - bb * row_items) << 5;
+    const float4* w4 = reinterpret_cast<const float4*>(ab.w[bb] + (size_t)row0 * rank);
+    float4 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < nq) v[q] = __ldcs(w4 + lane + 32 * q);
+    const float bias = __ldg(ab.b[bb] + row0 + lane);
+    const int sl = row0 / rows_per_slot;
+    if (bb * 2 + sl != cur) {
+      cur = bb * 2 + sl;
+      __syncwarp();
+      if (lane < rank) {
+        const float* tb = ab.table[bb];
+        const float a = __ldg(tb + ca.i0[sl] * rank + lane);
+        const float b2 = __ldg(tb + (ca.i0[sl] + 1) * rank + lane);
+        cw[lane] = (1.0f - ca.f[sl]) * a + ca.f[sl] * b2;
+      }
+      __syncwarp();
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < nq) {
+        const int idx = lane + 32 * q;
+        const float4 c = *reinterpret_cast<const float4*>(cw + 4 * (idx % nq));
+        pw[idx] = fmaf(v[q].w, c.w, fmaf(v[q].z, c.z, fmaf(v[q].y, c.y, v[q].x * c.x)));
+      }
+    }
+    __syncwarp();
+    float acc = 0.f;
+    for (int q = 0; q < nq; ++q) acc += pw[lane * nq + q];
+    __stcs(mods + bb * mods_stride + row0 + lane, acc + bias);
+    __syncwarp();
+  }
+  if constexpr (K > 0) {
+    // rotation table: 256 entries per warp item, grid-stride
+    const unsigned cs_total = (unsigned)n * 3u * K;  // < 2^31 (checked by the host)
+    for (unsigned e0 = (unsigned)gw * 256u; e0 < cs_total; e0 += (unsigned)n_warps * 256u) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const unsigned e = e0 + u * 32 + lane;
+        if (e < cs_total) {
+          const unsigned i = e / (3u * K), j = e % (3u * K);
+          const float a = (float)((double)pos[i * 3 + j / K] * (double)sinv[j % K]);
+          float sv, cv;
+          sincosf(a, &sv, &cv);
+          cs[e] = make_float2(cv, sv);
+        }
+      }
+    }
   }
 }
 
-cudaError_t launch_rope_table(const float* pos, int n, int k, float theta, float2* cs,
-                              cudaStream_t s) {
+// The adaLN rows of ab's first n_ab blocks into mods + b * mods_stride
+// (floats) and, when pos != null, the rotation table of n rows into cs.
+// The fast path needs rank % 4 == 0 (16-byte basis rows) and
+// rows_per_slot % 32 == 0; other shapes run the per-row adaln_kernel once
+// per block, and the table alone through the prologue kernel.
+cudaError_t launch_prologue(const AdalnBatch& ab, int n_ab, int rank, int grid, int rows_per_slot,
+                            const Plan& plan, float* mods, long long mods_stride, const float* pos, int n,
+                            int k, float theta, float2* cs, cudaStream_t s) {
+  CurveArgs ca{};
+  for (int i = 0; i < plan.n_ts; ++i) curve_coords(plan.ts[i], grid, &ca.i0[i], &ca.f[i]);
+  if (n_ab < 0 || n_ab > kAdalnBatch || (pos != nullptr && (long long)n * 3 * k >= (1ll << 31)) ||
+      (long long)n_ab * plan.n_ts * rows_per_slot >= (1ll << 31))
+    return cudaErrorInvalidValue;
+  bool fast = rank % 4 == 0 && rank <= 32 && rows_per_slot % 32 == 0;
+  for (int i = 0; i < n_ab && fast; ++i)
+    if (reinterpret_cast<uintptr_t>(ab.w[i]) & 15) fast = false;
+  if (!fast) {
+    for (int i = 0; i < n_ab; ++i) {
+      const int total = plan.n_ts * rows_per_slot;
+      int blocks = (total + 255) / 256;
+      if (blocks > num_sms() * 8) blocks = num_sms() * 8;
+      adaln_kernel<<<blocks, 256, 0, s>>>(ab.w[i], ab.b[i], ab.table[i], rank, rows_per_slot, plan.n_ts, ca,
+                                          mods + i * mods_stride);
+      count_launch();
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    n_ab = 0;
+  }
   InvFreq inv{};
   for (int i = 0; i < k && i < 32; ++i) inv.v[i] = (float)std::pow((double)theta, -(double)i / (double)k);
-  const long total = (long)n * 3 * k;
-  long blocks = (total + 255) / 256;
-  if (blocks > num_sms() * 16) blocks = num_sms() * 16;
-  rope_table_kernel<<<(int)blocks, 256, 0, s>>>(pos, n, k, inv, cs); count_launch();
+  const int kk = pos ? k : 0;
+  const long long items = (long long)n_ab * ((long long)plan.n_ts * rows_per_slot / 32) +
+                          ((long long)n * 3 * kk + 255) / 256;
+  if (items == 0) return cudaSuccess;
+  long long blocks = (items + 7) / 8;
+  if (blocks > (long long)num_sms() * 4) blocks = (long long)num_sms() * 4;  // 32 warps per SM
+  const int g = (int)blocks;
+  if (kk == 16)
+    prologue_kernel<16><<<g, 256, 0, s>>>(ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods, mods_stride, pos, n,
+                                          inv, cs);
+  else if (kk == 8)
+    prologue_kernel<8><<<g, 256, 0, s>>>(ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods, mods_stride, pos, n,
+                                         inv, cs);
+  else if (kk == 0)
+    prologue_kernel<0><<<g, 256, 0, s>>>(ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods, mods_stride, pos, n,
+                                         inv, cs);
+  else
+    return cudaErrorInvalidValue;
+  count_launch();
   return cudaGetLastError();
+}
+
+cudaError_t launch_adaln(const float* w, const float* b, const float* table, int rank, int grid,
+                         int rows_per_slot, const Plan& plan, float* out, cudaStream_t s) {
+  AdalnBatch ab{};
+  ab.w[0] = w;
+  ab.b[0] = b;
+  ab.table[0] = table;
+  return launch_prologue(ab, 1, rank, grid, rows_per_slot, plan, out, 0, nullptr, 0, 0, 0.f, nullptr, s);
 }
 
 // ------------------------------------------- K2 RMSNorm + modulate gather

@@ -42,8 +42,19 @@ void curve_coords(double t, int grid, int* i0, float* f);
 // -------------------------------------------------------------- launches
 cudaError_t launch_adaln(const float* w, const float* b, const float* table, int rank, int grid,
                          int rows_per_slot, const Plan& plan, float* out, cudaStream_t s);
-cudaError_t launch_rope_table(const float* pos, int n, int k, float theta, float2* cs,
-                              cudaStream_t s);
+// The adaLN bases of up to kAdalnBatch blocks for one prologue launch.
+constexpr int kAdalnBatch = 64;
+struct AdalnBatch {
+  const float* w[kAdalnBatch];
+  const float* b[kAdalnBatch];
+  const float* table[kAdalnBatch];
+};
+// One launch: the modulation of ab's first n_ab blocks (block i's rows at
+// mods + i * mods_stride floats) and, if pos != null, the rotation (cos,
+// sin) table of n rows with k frequencies per axis.
+cudaError_t launch_prologue(const AdalnBatch& ab, int n_ab, int rank, int grid, int rows_per_slot,
+                            const Plan& plan, float* mods, long long mods_stride, const float* pos, int n,
+                            int k, float theta, float2* cs, cudaStream_t s);
 cudaError_t launch_norm_mod(int dtype, const float* x, int n, int H, const float* g, float eps,
                             const float* mods, int mods_stride, int shift_off, int scale_off,
                             const SegRows& seg, int row_base, void* out, cudaStream_t s);

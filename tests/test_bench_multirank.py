@@ -104,4 +104,6 @@ def test_peak_choice_and_percentiles():
     assert bench.percentile(v, 50) == 3.0 and bench.percentile(v, 10) == pytest.approx(1.4)
     assert bench.percentile(v, 90) == pytest.approx(4.6)
     hb = bench.hbm_bytes(13248)
-    assert hb["norm1"] == 13248 * 2688 * 6 and hb["adaln"] == 2 * 18 * 2688 * 104
+    assert hb["norm1"] == 13248 * 2688 * 6
+    assert hb["prologue"] == 2 * 18 * 2688 * 104 + 13248 * 12 + 13248 * 48 * 8
+    assert bench.hbm_bytes(64, blocks_per_prologue=50)["prologue"] == 50 * 2 * 18 * 2688 * 104 + 64 * 12 + 64 * 384

@@ -49,6 +49,31 @@ def test_adaln_modulation(cuda_ok, name, sigma_v):
     np.testing.assert_allclose(got, ref, rtol=1e-4, atol=1e-6)
 
 
+@pytest.mark.parametrize("rank", [6, 24, 32])
+def test_adaln_modulation_ranks(cuda_ok, rank):
+    # rank 24 and 32 take the coalesced prologue path (16-byte basis rows);
+    # rank 6 (24-byte rows) takes the per-row kernel
+    H = 256
+    cfg = configs.DitConfig("r", 9, hidden=H, heads=2, head_dim=128, ffn=512, text_len=1, rank=rank)
+    w = configs.block_weights(cfg, 0, keys=("adaln_w", "adaln_b", "adaln_table"))
+    segs, _ = t2va_layout(20, 3, 16, 20, 20)
+    n = segs[-1][1]
+    sv, sa = sigma_pair(0.4)
+    ts, _ = O.plan_timesteps(sv, sa, segs)
+    ref = O.block_mods(f64(w["adaln_w"]), f64(w["adaln_b"]), f64(w["adaln_table"]), ts, H)
+    out = torch.full((2 * 18 * H,), float("nan"), device="cuda")
+    dims = api.make_dims(H, 2, 128, 512, rank=rank)
+    nts = api.adaln_modulation(dims, w["adaln_w"].cuda(), w["adaln_b"].cuda(), w["adaln_table"].cuda(),
+                               18 * H, segs, n, sv, sa, out)
+    assert nts == 2
+    np.testing.assert_allclose(f64(out[: nts * 18 * H]).reshape(6, 6 * H), ref, rtol=1e-4, atol=1e-6)
+
+
+def t2va_layout(*a):
+    L = O.layout_t2va(*a)
+    return L["segments"], L["pos"]
+
+
 def _qkv(n, heads, hd, seed, dtype=torch.bfloat16, qscale=1.0):
     I = heads * hd
     q = synth.normal((n, I), seed, qscale, dtype=dtype)

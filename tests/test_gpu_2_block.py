@@ -173,8 +173,9 @@ def test_block_forward_host_pipelined_matches_device_calls(cuda_ok):
 
 
 def test_launch_count_of_one_block(cuda_ok):
-    # adaLN, rotation table, 2 x norm/modulate, 4 GEMMs, attention: 9 kernels
-    # (attention adds a split launch and a merge when its last wave is split)
+    # prologue (adaLN curve + rotation table), 2 x norm/modulate, 4 GEMMs,
+    # attention: 8 kernels (attention adds a split launch and a merge when
+    # its last wave is split)
     dims_o, dims_c = small_dims()
     segs, pos = t2va(20, 3, 16, 20, 20)
     n = int(pos.shape[0])
@@ -186,7 +187,7 @@ def test_launch_count_of_one_block(cuda_ok):
     ws = torch.empty(api.workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
     c0 = api.launch_count()
     api.block_forward(dims_c, params, xd, segs, pd, *sigma_pair(0.5), ws)
-    assert api.launch_count() - c0 == 9
+    assert api.launch_count() - c0 == 8
 
 
 def test_block_caller_modulation_replaces_the_adaln_curve(cuda_ok):

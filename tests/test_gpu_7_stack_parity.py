@@ -129,3 +129,33 @@ def test_tiny_shape_fifty_block_chain(cuda_ok, act):
     else:
         assert_close(xd, h, what="50-block chain x (bf16 storage)")
         assert_close(xd.cpu().double() - x.double(), h - f64(x), what="50-block chain delta (bf16 storage)")
+
+
+@pytest.mark.parametrize("n_blocks,layout", [(5, (2, 1, 4, 4, 1)), (7, (20, 3, 16, 20, 20))])
+def test_stack_modulation_batches(cuda_ok, n_blocks, layout):
+    # The stack evaluates its blocks' modulation in batches placed in the
+    # head-scratch region: 8 tokens leave no room there (one block at a time
+    # through the block's own modulation region), 300 tokens hold four
+    # blocks' rows (batches of four and three).  Both against the oracle.
+    from gpu_common import small_block_weights, small_dims, t2va
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(*layout)
+    n = int(pos.shape[0])
+    ws_ = [small_block_weights(70 + b, 256, 2, 128, 512) for b in range(n_blocks)]
+    x = configs.synth.normal((n, 256), 83, 1.0)
+    sv, sa = sigma_pair(0.5)
+    bp = [api.BlockParams.from_host(dims_c, w) for w in ws_]
+    xd = x.cuda().clone()
+    pd = torch.as_tensor(np.asarray(pos, np.float32)).cuda()
+    ws = torch.empty(api.workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
+    api.stack_forward(dims_c, bp, None, xd, segs, pd, sv, sa, None, None, ws)
+    api.device_status()
+    ts, slot = O.plan_timesteps(sv, sa, segs)
+    rows = O.token_rows(segs, slot, n)
+    h = f64(x)
+    for w in ws_:
+        p = {k: f64(v) for k, v in w.items()}
+        h = O.block_forward(p, h, O.block_mods(p["adaln_w"], p["adaln_b"], p["adaln_table"], ts, 256), rows,
+                            f64(pos), dims_o)
+    assert_close(xd, h, what=f"{n_blocks}-block stack x")
+    assert_close(xd.cpu().double() - x.double(), h - f64(x), what=f"{n_blocks}-block stack delta")
