@@ -65,11 +65,20 @@ typedef struct {
   int act_dtype;     /* mmh3_dtype of activations and projection weights */
 } mmh3_dims;
 
-/* One contiguous run of tokens sharing a modality tag and a flow clock.
+/* One contiguous run of tokens sharing a modality tag and a clock.
  * tag: 0 video, 1 text, 2 audio (adaLN row order).  clock: 0 = the video
  * clock (t_v = 1 - max(sigma_v, 1e-6)), 1 = the audio clock
- * (t_a = 1 - sigma_a).  Text uses the video clock.  Segments must be sorted,
- * contiguous and cover [0, n) exactly; at most 8. */
+ * (t_a = 1 - sigma_a), 2 = the visual condition clock (keyframe and
+ * reference-image rows: max(t_v, 0.999)), 3 = the audio condition clock
+ * (reference audio rows: max(t_a, 1)) ("cortiq_engine/mmh3.rs", forward:
+ * VISUAL_COND_TIMESTEP, AUDIO_COND_TIMESTEP).  Text uses the video clock.
+ * Segments must be sorted, contiguous and cover [0, n) exactly; at most
+ * 16.  A token's adaLN row is slot*3 + tag, slot the index of its clock's
+ * timestep among the distinct timesteps of the clocks in use (ascending).
+ * The block's own adaLN basis holds two slots: more than two distinct
+ * timesteps need the caller's modulation (mmh3_block_forward's
+ * mods_or_null); every other entry point then returns
+ * MMH3_ERR_UNSUPPORTED. */
 typedef struct {
   uint32_t start, stop;
   uint8_t tag, clock;
@@ -133,6 +142,59 @@ mmh3_status mmh3_layout_t2va(int text_len, int latent_t, int lat_h, int lat_w, i
                              mmh3_segment* segs, int* n_seg, float* pos, int pos_capacity,
                              int* n_out);
 
+/* A keyframe of fl2va: the pixel frame it stands for and the clip's frame
+ * count.  Only the first (pixel_index 0) and the last (frame_count - 1)
+ * frame can anchor one. */
+typedef struct {
+  int pixel_index, frame_count;
+} mmh3_keyframe;
+
+/* A reference block of ref2va, in the order given.
+ *  MMH3_REF_IMAGE: a still of lat_h x lat_w latents (even);
+ *  MMH3_REF_AUDIO: audio_t standalone audio frames (stereo);
+ *  MMH3_REF_VIDEO: latent_t frames of lat_h x lat_w latents with an
+ *                  optional soundtrack of audio_t frames packed before
+ *                  them from the same origin. */
+#define MMH3_REF_IMAGE 0
+#define MMH3_REF_AUDIO 1
+#define MMH3_REF_VIDEO 2
+typedef struct {
+  int kind;
+  int lat_h, lat_w;
+  int latent_t;
+  int audio_t;
+} mmh3_ref;
+
+/* fl2va ("cortiq_engine/mmh3.rs", Layout::fl2va / build_full):
+ * [text | keyframes | audio | video].  Keyframe rows take the target's
+ * 2x2-patch grid at the time of the frame they stand for -- the first frame
+ * at the text's end, the last one at text_len + spans - 5/3 (spans = the
+ * target's summed 5/3 x [1,4,4,4,4] frame spans) -- and never move the
+ * cursor, so the audio and the video start where t2va puts them.  Keyframe
+ * segments are tag video on clock 2.  text_tags (host, text_len entries, or
+ * NULL = all text) gives each prompt token's modality tag; runs of one tag
+ * become separate text segments on clock 0.  Host buffers: segs
+ * [seg_capacity], pos [pos_capacity * 3] (pos may be NULL to query n).
+ * MMH3_ERR_ARG for a keyframe that is neither the first nor the last
+ * frame; MMH3_ERR_SHAPE if the segments exceed seg_capacity or 16. */
+mmh3_status mmh3_layout_fl2va(int text_len, int latent_t, int lat_h, int lat_w, int audio_t,
+                              const mmh3_keyframe* frames, int n_frames, const uint8_t* text_tags,
+                              mmh3_segment* segs, int seg_capacity, int* n_seg, float* pos,
+                              int pos_capacity, int* n_out);
+
+/* ref2va ("cortiq_engine/mmh3.rs", Layout::ref2va / build_full):
+ * [text | references | audio | video].  Each reference advances the cursor:
+ * a still puts its own h/w grid at the cursor, +1; standalone audio its
+ * stereo frames from the cursor, +audio_t; a clip its soundtrack (w at its
+ * own grid's extremes) and then its frames (t stepping by the frame
+ * spans), + max(audio_t, spans).  The target audio and video start at the
+ * final cursor.  Reference frames are tag video on clock 2, reference audio
+ * tag audio on clock 3.  Buffers and errors as mmh3_layout_fl2va. */
+mmh3_status mmh3_layout_ref2va(int text_len, int latent_t, int lat_h, int lat_w, int audio_t,
+                               const mmh3_ref* refs, int n_refs, const uint8_t* text_tags,
+                               mmh3_segment* segs, int seg_capacity, int* n_seg, float* pos,
+                               int pos_capacity, int* n_out);
+
 /* Image mode [text | reference image | target image]: the reference image is
  * placed like a reference still of "cortiq_engine/mmh3.rs" build_full (rows
  * at the cursor t with their own h/w grid, cursor + 1), the target at the
@@ -143,8 +205,8 @@ mmh3_status mmh3_layout_image(int text_len, int ref_lat_h, int ref_lat_w, int la
 
 /* Distinct timesteps (ascending, de-duplicated) of the clocks the segments
  * use, and each segment's block adaLN row slot(clock)*3 + tag
- * ("cortiq_engine/mmh3.rs", forward).  Host buffers: ts [2], seg_rows
- * [n_seg].  MMH3_ERR_UNSUPPORTED if the clocks give > 2 timesteps. */
+ * ("cortiq_engine/mmh3.rs", forward).  Host buffers: ts [4], seg_rows
+ * [n_seg].  Up to four timesteps (the four clocks). */
 mmh3_status mmh3_plan_timesteps(const mmh3_segment* segs, int n_seg, int n, double sigma_v,
                                 double sigma_a, double* ts, int* n_ts, int* seg_rows);
 
@@ -403,7 +465,11 @@ mmh3_status mmh3_embed_workspace_size(const mmh3_dims* dims, const mmh3_embed_in
  * latents through mmh3_patch_embed; every other video-tag segment, in order,
  * takes the next condition frame through the video projection.  Each
  * segment's row count must match what its stream gives (MMH3_ERR_SHAPE
- * otherwise), and n_cond must equal the number of those other segments. */
+ * otherwise), and n_cond must equal the number of those other segments.
+ * This places fl2va keyframes (frames on the target grid) and image-mode
+ * references; reference audio (clock 3) has no input here
+ * (MMH3_ERR_UNSUPPORTED), and a reference still or clip of another grid
+ * fails the row-count check. */
 mmh3_status mmh3_embed(const mmh3_dims* dims, const mmh3_segment* segs, int n_seg, int n,
                        const mmh3_embed_inputs* in, const mmh3_embed_weights* w, float* x,
                        void* workspace, size_t ws_bytes, void* stream);

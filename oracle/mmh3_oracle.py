@@ -63,8 +63,14 @@ EXPAND = 6
 #: Rows of the timestep-curve table ([mmh3] CURVE_GRID).
 CURVE_GRID = 1025
 
-#: Clocks: 0 = the video flow clock, 1 = the audio flow clock.
-CLOCK_VIDEO, CLOCK_AUDIO = 0, 1
+#: Clocks: 0 = the video flow clock, 1 = the audio flow clock, 2 = the
+#: visual condition clock (keyframe and reference-image rows), 3 = the audio
+#: condition clock (reference audio rows).
+CLOCK_VIDEO, CLOCK_AUDIO, CLOCK_COND, CLOCK_COND_AUDIO = 0, 1, 2, 3
+#: Where condition rows sit on the schedule ([mmh3] VISUAL_COND_TIMESTEP,
+#: AUDIO_COND_TIMESTEP; the model's cond_aug and cond_aug_audio).
+VISUAL_COND_TIMESTEP = 0.999
+AUDIO_COND_TIMESTEP = 1.0
 
 
 # --------------------------------------------------------------------------
@@ -112,38 +118,139 @@ def _audio_rows(cursor: float, t: int, w_low: float, w_high: float) -> list[tupl
     return rows
 
 
-def layout_t2va(text_len: int, latent_t: int, lat_h: int, lat_w: int,
-                audio_t: int) -> dict:
-    """The text-to-video+audio layout ``[text | audio | video]``
-    ([mmh3] ``Layout::t2va`` / ``build_full`` with no keyframes or refs).
+def layout_build_full(text_len: int, latent_t: int, lat_h: int, lat_w: int, audio_t: int,
+                      frames=(), refs=(), text_tags=None) -> dict:
+    """The packed layout ([mmh3] ``Layout::build_full``), step by step:
 
-    Returns ``seq_len``, ``frame_rows``, ``segments`` as a list of
-    (start, stop, tag, clock) and ``pos`` as an [n, 3] float64 array of
-    (t, h, w).  Text uses the video clock ([mmh3] ``forward``: text rows use
-    t_v's index), audio the audio clock, video the video clock."""
+    * text rows (i, 0, 0); the segment table splits the prompt into runs of
+      one modality tag (``text_tags``, default all TEXT), all on the video
+      clock ([mmh3] ``forward``: text rows use t_v's index and their own tag);
+    * the cursor starts at text_len; each reference, in order, advances it:
+      ``("image", h, w)`` puts its own grid (``axis_from_sqrt_area`` of its
+      own area) at the cursor, cursor + 1; ``("audio", t)`` puts t stereo
+      frames at the cursor (w at the TARGET grid's extremes), cursor + t;
+      ``("video", latent_t, h, w, audio_t)`` puts its soundtrack first (w at
+      its own grid's extremes), then its frames with t stepping by
+      5/3 * [1,4,4,4,4][k % 5], cursor + max(audio_t, summed spans);
+    * keyframes ``(pixel_index, frame_count)`` on the target grid, not moving
+      the cursor: the first frame at the cursor, the last one at cursor +
+      spans - 5/3 (spans summed over the target's latent frames); any other
+      frame is an error;
+    * the target audio (stereo, target w extremes) and video from the cursor.
+
+    Reference and keyframe rows are conditions ([mmh3] ``forward``):
+    frames tag VIDEO on the visual condition clock, reference audio tag AUDIO
+    on the audio condition clock.  Returns seq_len, frame_rows, segments
+    (start, stop, tag, clock), kinds (the page's segment kind per segment)
+    and pos [n, 3] float64."""
     area = math.sqrt(lat_h * lat_w)
     h_axis = axis_from_sqrt_area(lat_h, 2, area)
     w_axis = axis_from_sqrt_area(lat_w, 2, area)
-    pos: list[tuple] = [(float(i), 0.0, 0.0) for i in range(text_len)]
-    segments = [(0, text_len, TAG_TEXT, CLOCK_VIDEO)]
+    pos: list[tuple] = []
+    segments, kinds = [], []
+
+    def seg(start, tag, clock, kind):
+        segments.append((start, len(pos), tag, clock))
+        kinds.append(kind)
+
+    tags = [TAG_TEXT] * text_len if text_tags is None else list(text_tags)
+    run0 = 0
+    for i in range(text_len):
+        if i > 0 and tags[i] != tags[i - 1]:
+            seg(run0, tags[i - 1], CLOCK_VIDEO, "Text")
+            run0 = len(pos)
+        pos.append((float(i), 0.0, 0.0))
+    seg(run0, tags[-1], CLOCK_VIDEO, "Text")
     cursor = float(text_len)
+    w_low_t, w_high_t = w_axis[0], w_axis[-1]
+    for r in refs:
+        if r[0] == "image":
+            _, rh_, rw_ = r
+            a = math.sqrt(rh_ * rw_)
+            rh, rw = axis_from_sqrt_area(rh_, 2, a), axis_from_sqrt_area(rw_, 2, a)
+            s0 = len(pos)
+            pos += [(cursor, h, w) for h in rh for w in rw]
+            seg(s0, TAG_VIDEO, CLOCK_COND, "RefImg")
+            cursor += 1.0
+        elif r[0] == "audio":
+            t = r[1]
+            if t > 0:
+                s0 = len(pos)
+                pos += _audio_rows(cursor, t, w_low_t, w_high_t)
+                seg(s0, TAG_AUDIO, CLOCK_COND_AUDIO, "RefAudio")
+            cursor += float(t)
+        elif r[0] == "video":
+            _, vt, rh_, rw_, rt = r
+            a = math.sqrt(rh_ * rw_)
+            rh, rw = axis_from_sqrt_area(rh_, 2, a), axis_from_sqrt_area(rw_, 2, a)
+            if rt > 0:
+                s0 = len(pos)
+                pos += _audio_rows(cursor, rt, rw[0], rw[-1])
+                seg(s0, TAG_AUDIO, CLOCK_COND_AUDIO, "RefAudio")
+            s0 = len(pos)
+            t_coord = cursor
+            for k in range(vt):
+                pos += [(t_coord, h, w) for h in rh for w in rw]
+                t_coord += FRAME_RESCALE * FRAME_PER_TOKEN[k % 5]
+            seg(s0, TAG_VIDEO, CLOCK_COND, "RefImg")
+            spans = 0.0
+            for k in range(vt):
+                spans += FRAME_RESCALE * FRAME_PER_TOKEN[k % 5]
+            cursor += max(float(rt), spans)
+        else:
+            raise ValueError(f"reference kind {r[0]!r}")
+    spans = 0.0
+    for k in range(latent_t):
+        spans += FRAME_RESCALE * FRAME_PER_TOKEN[k % 5]
+    for (pixel_index, frame_count) in frames:
+        if pixel_index == 0:
+            cond_t = cursor
+        elif frame_count > 0 and pixel_index == frame_count - 1:
+            cond_t = cursor + spans - FRAME_RESCALE
+        else:
+            raise ValueError("only the first and last frame can anchor a keyframe")
+        s0 = len(pos)
+        pos += [(cond_t, h, w) for h in h_axis for w in w_axis]
+        seg(s0, TAG_VIDEO, CLOCK_COND, "Cond")
     a0 = len(pos)
-    pos += _audio_rows(cursor, audio_t, w_axis[0], w_axis[-1])
-    segments.append((a0, len(pos), TAG_AUDIO, CLOCK_AUDIO))
+    pos += _audio_rows(cursor, audio_t, w_low_t, w_high_t)
+    seg(a0, TAG_AUDIO, CLOCK_AUDIO, "Audio")
     v0 = len(pos)
     t_coord = cursor
     for k in range(latent_t):
-        for h in h_axis:
-            for w in w_axis:
-                pos.append((t_coord, h, w))
+        pos += [(t_coord, h, w) for h in h_axis for w in w_axis]
         t_coord += FRAME_RESCALE * FRAME_PER_TOKEN[k % 5]
-    segments.append((v0, len(pos), TAG_VIDEO, CLOCK_VIDEO))
+    seg(v0, TAG_VIDEO, CLOCK_VIDEO, "Video")
     return {
         "seq_len": len(pos),
         "frame_rows": len(h_axis) * len(w_axis),
         "segments": segments,
+        "kinds": kinds,
         "pos": np.asarray(pos, dtype=np.float64).reshape(-1, 3),
     }
+
+
+def layout_t2va(text_len: int, latent_t: int, lat_h: int, lat_w: int,
+                audio_t: int) -> dict:
+    """The text-to-video+audio layout ``[text | audio | video]``
+    ([mmh3] ``Layout::t2va``: ``build_full`` with no keyframes or
+    references).  Text uses the video clock, audio the audio clock, video the
+    video clock."""
+    return layout_build_full(text_len, latent_t, lat_h, lat_w, audio_t)
+
+
+def layout_fl2va(text_len: int, latent_t: int, lat_h: int, lat_w: int, audio_t: int,
+                 frames, text_tags=None) -> dict:
+    """Keyframes between the text and the audio ([mmh3] ``Layout::fl2va``)."""
+    return layout_build_full(text_len, latent_t, lat_h, lat_w, audio_t, frames=frames,
+                             text_tags=text_tags)
+
+
+def layout_ref2va(text_len: int, latent_t: int, lat_h: int, lat_w: int, audio_t: int,
+                  refs, text_tags=None) -> dict:
+    """References ahead of the target streams ([mmh3] ``Layout::ref2va``)."""
+    return layout_build_full(text_len, latent_t, lat_h, lat_w, audio_t, refs=refs,
+                             text_tags=text_tags)
 
 
 def layout_image(text_len: int, ref_lat_h: int, ref_lat_w: int,
@@ -183,12 +290,17 @@ def plan_timesteps(sigma_v: float, sigma_a: float, segments) -> tuple[list, dict
     """Distinct timesteps in ascending order and the slot of each clock.
 
     [mmh3] ``forward``: sigma_v is clamped to >= 1e-6, t_v = 1 - sigma_v,
-    t_a = 1 - sigma_a; the list of distinct timesteps is sorted and
-    de-duplicated, and a row's adaLN slot is the position of its clock's
-    timestep in that list.  Only clocks that some segment uses enter the list
-    (image mode has one clock)."""
+    t_a = 1 - sigma_a; keyframe and reference-image rows sit at
+    t_cond = max(t_v, VISUAL_COND_TIMESTEP), reference audio rows at
+    t_cond_a = max(t_a, AUDIO_COND_TIMESTEP); the list of distinct timesteps
+    is sorted and de-duplicated, and a row's adaLN slot is the position of
+    its clock's timestep in that list.  Only clocks that some segment uses
+    enter the list (image mode has one clock)."""
     sigma_v = max(sigma_v, 1e-6)
-    t_of_clock = {CLOCK_VIDEO: 1.0 - sigma_v, CLOCK_AUDIO: 1.0 - sigma_a}
+    t_v, t_a = 1.0 - sigma_v, 1.0 - sigma_a
+    t_of_clock = {CLOCK_VIDEO: t_v, CLOCK_AUDIO: t_a,
+                  CLOCK_COND: max(t_v, VISUAL_COND_TIMESTEP),
+                  CLOCK_COND_AUDIO: max(t_a, AUDIO_COND_TIMESTEP)}
     used = sorted({seg[3] for seg in segments})
     ts = sorted({t_of_clock[c] for c in used})
     slot = {c: ts.index(t_of_clock[c]) for c in used}

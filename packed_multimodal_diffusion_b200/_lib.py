@@ -34,6 +34,18 @@ class Segment(C.Structure):
                 ("clock", C.c_uint8), ("pad", C.c_uint8 * 2)]
 
 
+class Keyframe(C.Structure):
+    _fields_ = [("pixel_index", C.c_int), ("frame_count", C.c_int)]
+
+
+class Ref(C.Structure):
+    _fields_ = [("kind", C.c_int), ("lat_h", C.c_int), ("lat_w", C.c_int), ("latent_t", C.c_int),
+                ("audio_t", C.c_int)]
+
+
+MMH3_REF_IMAGE, MMH3_REF_AUDIO, MMH3_REF_VIDEO = 0, 1, 2
+
+
 class BlockWeights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("norm1", "norm2", "wqkv", "wout", "q_norm", "k_norm",
                                           "wfc1", "wfc2", "adaln_w", "adaln_b", "adaln_table")]
@@ -80,6 +92,10 @@ SIGNATURES = {
                               C.POINTER(_I)]),
     "mmh3_layout_image": (_I, [_I, _I, _I, _I, _I, _SEGP, C.POINTER(_I), C.POINTER(C.c_float), _I,
                                C.POINTER(_I)]),
+    "mmh3_layout_fl2va": (_I, [_I, _I, _I, _I, _I, C.POINTER(Keyframe), _I, C.POINTER(C.c_uint8), _SEGP, _I,
+                               C.POINTER(_I), C.POINTER(C.c_float), _I, C.POINTER(_I)]),
+    "mmh3_layout_ref2va": (_I, [_I, _I, _I, _I, _I, C.POINTER(Ref), _I, C.POINTER(C.c_uint8), _SEGP, _I,
+                                C.POINTER(_I), C.POINTER(C.c_float), _I, C.POINTER(_I)]),
     "mmh3_plan_timesteps": (_I, [_SEGP, _I, _I, _D, _D, C.POINTER(_D), C.POINTER(_I),
                                  C.POINTER(_I)]),
     "mmh3_resolve_rows": (_I, [_SEGP, _I, _I, _D, _D, _P, _P]),

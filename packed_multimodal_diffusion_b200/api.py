@@ -12,9 +12,9 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import (MMH3_BF16, MMH3_F32, MMH3_STREAM_AUDIO, MMH3_STREAM_VIDEO, BlockWeights, Dims,
-                   EmbedInputs, EmbedWeights, HeadWeights, Segment, VitDims, VitWeights, check,
-                   load)
+from ._lib import (MMH3_BF16, MMH3_F32, MMH3_REF_AUDIO, MMH3_REF_IMAGE, MMH3_REF_VIDEO, MMH3_STREAM_AUDIO,
+                   MMH3_STREAM_VIDEO, BlockWeights, Dims, EmbedInputs, EmbedWeights, HeadWeights, Keyframe, Ref,
+                   Segment, VitDims, VitWeights, check, load)
 
 __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_image",
            "plan_timesteps", "time_shift_sigma", "resolve_rows", "adaln_modulation",
@@ -69,7 +69,7 @@ def time_shift_sigma(sigma: float, from_shift: float, to_shift: float) -> float:
 
 
 def _layout(fn, *args):
-    segs = (Segment * 8)()
+    segs = (Segment * 16)()
     nseg, n = C.c_int(), C.c_int()
     check(fn(*args, segs, C.byref(nseg), None, 0, C.byref(n)))
     pos = np.zeros((n.value, 3), dtype=np.float32)
@@ -87,9 +87,48 @@ def layout_image(text_len, ref_lat_h, ref_lat_w, lat_h, lat_w):
     return _layout(load().mmh3_layout_image, text_len, ref_lat_h, ref_lat_w, lat_h, lat_w)
 
 
+def _layout_cap(fn, *args):
+    """Layouts whose segment count varies (keyframes, references): segment
+    capacity 16, positions queried first."""
+    segs = (Segment * 16)()
+    nseg, n = C.c_int(), C.c_int()
+    check(fn(*args, segs, 16, C.byref(nseg), None, 0, C.byref(n)))
+    pos = np.zeros((n.value, 3), dtype=np.float32)
+    check(fn(*args, segs, 16, C.byref(nseg), pos.ctypes.data_as(C.POINTER(C.c_float)), n.value, C.byref(n)))
+    return _seg_tuples(segs, nseg.value), pos
+
+
+def _tags(text_tags):
+    if text_tags is None:
+        return None
+    return (C.c_uint8 * len(text_tags))(*text_tags)
+
+
+def layout_fl2va(text_len, latent_t, lat_h, lat_w, audio_t, frames, text_tags=None):
+    """frames: [(pixel_index, frame_count)]; text_tags: per-token modality
+    tags of the prompt (None: all text)."""
+    kf = (Keyframe * max(1, len(frames)))(*[Keyframe(a, b) for a, b in frames])
+    return _layout_cap(load().mmh3_layout_fl2va, text_len, latent_t, lat_h, lat_w, audio_t, kf, len(frames),
+                       _tags(text_tags))
+
+
+def layout_ref2va(text_len, latent_t, lat_h, lat_w, audio_t, refs, text_tags=None):
+    """refs: [("image", lat_h, lat_w) | ("audio", t) | ("video", latent_t, lat_h, lat_w, audio_t)]."""
+    arr = (Ref * max(1, len(refs)))()
+    for i, r in enumerate(refs):
+        if r[0] == "image":
+            arr[i] = Ref(MMH3_REF_IMAGE, r[1], r[2], 0, 0)
+        elif r[0] == "audio":
+            arr[i] = Ref(MMH3_REF_AUDIO, 0, 0, 0, r[1])
+        else:
+            arr[i] = Ref(MMH3_REF_VIDEO, r[2], r[3], r[1], r[4])
+    return _layout_cap(load().mmh3_layout_ref2va, text_len, latent_t, lat_h, lat_w, audio_t, arr, len(refs),
+                       _tags(text_tags))
+
+
 def plan_timesteps(segs, n, sigma_v, sigma_a):
     arr = segments(segs)
-    ts = (C.c_double * 2)()
+    ts = (C.c_double * 4)()
     nts = C.c_int()
     rows = (C.c_int * len(segs))()
     check(load().mmh3_plan_timesteps(arr, len(segs), n, sigma_v, sigma_a, ts, C.byref(nts), rows))

@@ -221,6 +221,18 @@ mmh3_status block_core(const mmh3_dims& d, const mmh3_block_weights& w, float* x
   return block_post(d, w, x, n, plan, mods, ws, s, pm, nullptr, 0);
 }
 
+// The block's own adaLN basis has two timestep slots (rows [slot][tag]
+// [chunk][H], slot s at ts[s]); how a third or fourth distinct timestep
+// (keyframe or reference rows on their condition clocks) maps onto it is
+// not fixed, so such plans run only with a caller's modulation.
+mmh3_status own_curve_slots(const Plan& plan) {
+  if (plan.n_ts > 2)
+    return fail(MMH3_ERR_UNSUPPORTED,
+                "%d distinct timesteps: the adaLN basis holds two slots; pass the modulation (mods_or_null)",
+                plan.n_ts);
+  return MMH3_OK;
+}
+
 // adaLN modulation of one block (when own_mods) into ws.mods and the
 // rotation table (when pos != null) into ws.cs, in one launch.
 mmh3_status prologue(const mmh3_dims& d, const mmh3_block_weights* w, bool own_mods, const Plan& plan,
@@ -278,6 +290,10 @@ mmh3_status mmh3::block_forward_impl(const mmh3_dims* dims, const mmh3_block_wei
   if (modulated) {
     st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
     if (st != MMH3_OK) return st;
+    if (own_mods) {
+      st = own_curve_slots(plan);
+      if (st != MMH3_OK) return st;
+    }
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden;
@@ -326,6 +342,8 @@ mmh3_status mmh3_adaln_modulation(const mmh3_dims* dims, const float* w, const f
   mmh3_status st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
   if (st != MMH3_OK) return st;
   if (n_ts) *n_ts = plan.n_ts;
+  st = own_curve_slots(plan);
+  if (st != MMH3_OK) return st;
   cudaError_t e = launch_adaln(w, b, table, dims->rank, dims->grid, rows_per_slot, plan, out,
                                static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "adaln launch");
@@ -373,6 +391,8 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
   }
   Plan plan;
   st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+  if (st != MMH3_OK) return st;
+  st = own_curve_slots(plan);
   if (st != MMH3_OK) return st;
   const int H = dims->hidden;
   // output streams: the last video-tag segment and the last audio-tag segment
@@ -547,6 +567,8 @@ mmh3_status mmh3_block_cp_begin(const mmh3_dims* dims, const mmh3_block_weights*
   if (modulated) {
     st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
     if (st != MMH3_OK) return st;
+    st = own_curve_slots(plan);
+    if (st != MMH3_OK) return st;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   PhaseMark pm(s, false);
@@ -575,6 +597,8 @@ mmh3_status mmh3_block_cp_end(const mmh3_dims* dims, const mmh3_block_weights* w
   Plan plan;
   if (modulated) {
     st = make_plan(segs, n_seg, n, sigma_v, sigma_a, &plan);
+    if (st != MMH3_OK) return st;
+    st = own_curve_slots(plan);
     if (st != MMH3_OK) return st;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -729,6 +753,8 @@ mmh3_status mmh3_embed(const mmh3_dims* dims, const mmh3_segment* segs, int n_se
   if (st != MMH3_OK) return st;
   int t_seg = -1, a_seg = -1, v_last = -1, n_other = 0;
   for (int k = 0; k < n_seg; ++k) {
+    if (segs[k].clock == 3)
+      return fail(MMH3_ERR_UNSUPPORTED, "embed: segment %d holds reference audio, which has no input here", k);
     if (segs[k].tag == 1 && t_seg < 0) t_seg = k;
     if (segs[k].tag == 2) a_seg = k;
     if (segs[k].tag == 0) v_last = k;

@@ -6,6 +6,7 @@
 // flow-schedule remap (time_shift_sigma), the packed layout
 // (axis_from_sqrt_area, push_audio_grid, Layout::build_full) and the
 // timestep / row assembly at the top of MiniMaxH3::forward.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -57,6 +58,12 @@ uint64_t wait_limit_ns() {
 }
 
 // ------------------------------------------------------------------- plan
+// Where condition rows sit on the schedule ("cortiq_engine/mmh3.rs",
+// VISUAL_COND_TIMESTEP and AUDIO_COND_TIMESTEP, the model's cond_aug and
+// cond_aug_audio): a keyframe or reference row is all but arrived.
+constexpr double kVisualCondTimestep = 0.999;
+constexpr double kAudioCondTimestep = 1.0;
+
 void curve_coords(double t, int grid, int* i0, float* f) {
   const double tc = t < 0.0 ? 0.0 : (t > 1.0 ? 1.0 : t);
   const double p = tc * (double)(grid - 1);
@@ -73,32 +80,34 @@ mmh3_status make_plan(const mmh3_segment* segs, int n_seg, int n, double sigma_v
   if (n_seg < 1 || n_seg > kMaxSeg) return fail(MMH3_ERR_SHAPE, "n_seg=%d not in [1, %d]", n_seg, kMaxSeg);
   if (n < 1) return fail(MMH3_ERR_SHAPE, "n=%d < 1", n);
   uint32_t expect = 0;
-  bool used[2] = {false, false};
+  bool used[kClocks] = {false, false, false, false};
   for (int k = 0; k < n_seg; ++k) {
     const mmh3_segment& s = segs[k];
     if (s.start != expect || s.stop <= s.start)
       return fail(MMH3_ERR_SHAPE, "segment %d [%u, %u) is not contiguous from %u", k, s.start, s.stop, expect);
     if (s.tag > 2) return fail(MMH3_ERR_ARG, "segment %d: tag %d not in {0,1,2}", k, (int)s.tag);
-    if (s.clock > 1) return fail(MMH3_ERR_ARG, "segment %d: clock %d not in {0,1}", k, (int)s.clock);
+    if (s.clock >= kClocks) return fail(MMH3_ERR_ARG, "segment %d: clock %d not in [0, 3]", k, (int)s.clock);
     used[s.clock] = true;
     expect = s.stop;
   }
   if ((int)expect != n) return fail(MMH3_ERR_SHAPE, "segments cover [0, %u), n = %d", expect, n);
   // forward(): sigma_v clamped at 1e-6; t_v = 1 - sigma_v, t_a = 1 - sigma_a;
-  // the distinct timesteps sorted ascending; a clock's slot is its index.
+  // condition rows sit at t_cond = max(t_v, 0.999) (visual) and
+  // t_cond_a = max(t_a, 1) (audio), the model's VISUAL_COND_TIMESTEP and
+  // AUDIO_COND_TIMESTEP; the distinct timesteps of the clocks the segments
+  // use, sorted ascending; a clock's slot is its index in that list.
   const double sv = sigma_v > 1e-6 ? sigma_v : 1e-6;
-  const double t_of[2] = {1.0 - sv, 1.0 - sigma_a};
+  const double t_v = 1.0 - sv, t_a = 1.0 - sigma_a;
+  const double t_of[kClocks] = {t_v, t_a, std::max(t_v, kVisualCondTimestep), std::max(t_a, kAudioCondTimestep)};
   std::vector<double> ts;
-  for (int c = 0; c < 2; ++c)
+  for (int c = 0; c < kClocks; ++c)
     if (used[c]) ts.push_back(t_of[c]);
-  if (ts.size() == 2) {
-    if (ts[1] < ts[0]) std::swap(ts[0], ts[1]);
-    if (ts[0] == ts[1]) ts.pop_back();
-  }
+  std::sort(ts.begin(), ts.end());
+  ts.erase(std::unique(ts.begin(), ts.end()), ts.end());
   *p = Plan{};
   p->n_ts = (int)ts.size();
   for (size_t i = 0; i < ts.size(); ++i) p->ts[i] = ts[i];
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < kClocks; ++c) {
     p->slot[c] = -1;
     if (!used[c]) continue;
     for (int i = 0; i < p->n_ts; ++i)
@@ -165,11 +174,15 @@ struct LayoutBuilder {
     s.clock = (uint8_t)clock;
     segs.push_back(s);
   }
-  mmh3_status emit(mmh3_segment* out_segs, int* n_seg, float* out_pos, int cap, int* n_out) {
+  mmh3_status emit(mmh3_segment* out_segs, int seg_cap, int* n_seg, float* out_pos, int cap, int* n_out) {
     if (n_seg == nullptr || n_out == nullptr || out_segs == nullptr)
       return fail(MMH3_ERR_ARG, "layout: null output pointer");
     *n_out = rows();
     *n_seg = (int)segs.size();
+    if ((int)segs.size() > kMaxSeg)
+      return fail(MMH3_ERR_SHAPE, "layout: %d segments, above the %d a block takes", (int)segs.size(), kMaxSeg);
+    if ((int)segs.size() > seg_cap)
+      return fail(MMH3_ERR_SHAPE, "layout: segment capacity %d < %d segments", seg_cap, (int)segs.size());
     for (size_t k = 0; k < segs.size(); ++k) out_segs[k] = segs[k];
     if (out_pos == nullptr) return MMH3_OK;
     if (cap < rows()) return fail(MMH3_ERR_SHAPE, "layout: pos capacity %d < %d rows", cap, rows());
@@ -178,31 +191,120 @@ struct LayoutBuilder {
   }
 };
 
-}  // namespace
 
-extern "C" mmh3_status mmh3_layout_t2va(int text_len, int latent_t, int lat_h, int lat_w,
-                                        int audio_t, mmh3_segment* segs, int* n_seg, float* pos,
-                                        int pos_capacity, int* n_out) {
-  clear_error();
-  if (text_len < 1 || latent_t < 1 || lat_h < 2 || lat_w < 2 || audio_t < 1 || (lat_h & 1) ||
-      (lat_w & 1))
-    return fail(MMH3_ERR_SHAPE, "t2va: bad sizes text=%d t=%d h=%d w=%d audio=%d", text_len,
-                latent_t, lat_h, lat_w, audio_t);
+// The packed layout of "cortiq_engine/mmh3.rs" Layout::build_full: the
+// text rows (i, 0, 0) in runs of equal modality tag (text_tags, or all
+// text); the reference blocks in order, each advancing the cursor (a still:
+// its own h/w grid at the cursor, +1; standalone audio: t stereo frames,
+// +t; a clip: its soundtrack first, then its frames stepping t by the
+// 5/3 x [1,4,4,4,4] spans, + max(audio frames, spans)); the keyframes on the
+// target grid, pinned to the frame they stand for without moving the
+// cursor (the first frame at the cursor, the last one at cursor + spans -
+// 5/3); then the target audio and the target video from the cursor.
+// Segment clocks: text, audio and video on the flow clocks 0 / 1 / 0,
+// keyframes and reference frames tag video on clock 2, reference audio tag
+// audio on clock 3 (MiniMaxH3::forward's row assignment).
+mmh3_status build_layout(LayoutBuilder& L, int text_len, int latent_t, int lat_h, int lat_w, int audio_t,
+                         const mmh3_keyframe* frames, int n_frames, const mmh3_ref* refs, int n_refs,
+                         const uint8_t* text_tags) {
+  if (text_len < 1 || latent_t < 1 || lat_h < 2 || lat_w < 2 || audio_t < 1 || (lat_h & 1) || (lat_w & 1))
+    return fail(MMH3_ERR_SHAPE, "layout: bad sizes text=%d t=%d h=%d w=%d audio=%d", text_len, latent_t, lat_h,
+                lat_w, audio_t);
+  if (n_frames < 0 || (n_frames > 0 && frames == nullptr) || n_refs < 0 || (n_refs > 0 && refs == nullptr))
+    return fail(MMH3_ERR_ARG, "layout: keyframe / reference list null or negative");
   static const double kFramePerToken[5] = {1.0, 4.0, 4.0, 4.0, 4.0};
   const double kRescale = 5.0 / 3.0;
   const double area = std::sqrt((double)lat_h * (double)lat_w);
   const std::vector<double> hs = axis_from_sqrt_area(lat_h, 2, area);
   const std::vector<double> ws = axis_from_sqrt_area(lat_w, 2, area);
-  LayoutBuilder L;
-  for (int i = 0; i < text_len; ++i) L.row((double)i, 0.0, 0.0);
-  L.seg(0, /*tag text*/ 1, /*clock*/ 0);
-  const double cursor = (double)text_len;
-  // stereo audio, channel-major, w pinned to the frame grid's extremes
-  int a0 = L.rows();
-  for (int ch = 0; ch < 2; ++ch)
-    for (int i = 0; i < audio_t; ++i) L.row(cursor + (double)i, 0.0, ch == 0 ? ws.front() : ws.back());
+  auto audio_grid = [&](double cursor, int t, double w_low, double w_high) {
+    for (int ch = 0; ch < 2; ++ch)
+      for (int i = 0; i < t; ++i) L.row(cursor + (double)i, 0.0, ch == 0 ? w_low : w_high);
+  };
+  // text, in runs of one tag
+  int run0 = 0, prev = -1;
+  for (int i = 0; i < text_len; ++i) {
+    const int tag = text_tags ? text_tags[i] : 1;
+    if (tag > 2) return fail(MMH3_ERR_ARG, "layout: text tag %d of token %d not in {0,1,2}", tag, i);
+    if (i > 0 && tag != prev) {
+      L.seg(run0, prev, 0);
+      run0 = L.rows();
+    }
+    L.row((double)i, 0.0, 0.0);
+    prev = tag;
+  }
+  L.seg(run0, prev, 0);
+  double cursor = (double)text_len;
+  for (int r = 0; r < n_refs; ++r) {
+    const mmh3_ref& ref = refs[r];
+    if (ref.kind == MMH3_REF_IMAGE) {
+      if (ref.lat_h < 2 || ref.lat_w < 2 || (ref.lat_h & 1) || (ref.lat_w & 1))
+        return fail(MMH3_ERR_SHAPE, "layout: reference image %d grid %d x %d", r, ref.lat_h, ref.lat_w);
+      const double a = std::sqrt((double)ref.lat_h * (double)ref.lat_w);
+      const std::vector<double> rh = axis_from_sqrt_area(ref.lat_h, 2, a), rw = axis_from_sqrt_area(ref.lat_w, 2, a);
+      const int s0 = L.rows();
+      for (double h : rh)
+        for (double w : rw) L.row(cursor, h, w);
+      L.seg(s0, 0, 2);
+      cursor += 1.0;
+    } else if (ref.kind == MMH3_REF_AUDIO) {
+      if (ref.audio_t < 0) return fail(MMH3_ERR_SHAPE, "layout: reference audio %d frames %d", r, ref.audio_t);
+      if (ref.audio_t > 0) {
+        const int s0 = L.rows();
+        audio_grid(cursor, ref.audio_t, ws.front(), ws.back());
+        L.seg(s0, 2, 3);
+      }
+      cursor += (double)ref.audio_t;
+    } else if (ref.kind == MMH3_REF_VIDEO) {
+      if (ref.latent_t < 1 || ref.audio_t < 0 || ref.lat_h < 2 || ref.lat_w < 2 || (ref.lat_h & 1) ||
+          (ref.lat_w & 1))
+        return fail(MMH3_ERR_SHAPE, "layout: reference clip %d sizes", r);
+      const double a = std::sqrt((double)ref.lat_h * (double)ref.lat_w);
+      const std::vector<double> rh = axis_from_sqrt_area(ref.lat_h, 2, a), rw = axis_from_sqrt_area(ref.lat_w, 2, a);
+      if (ref.audio_t > 0) {
+        const int s0 = L.rows();
+        audio_grid(cursor, ref.audio_t, rw.front(), rw.back());
+        L.seg(s0, 2, 3);
+      }
+      const int s0 = L.rows();
+      double t = cursor;
+      for (int k = 0; k < ref.latent_t; ++k) {
+        for (double h : rh)
+          for (double w : rw) L.row(t, h, w);
+        t += kRescale * kFramePerToken[k % 5];
+      }
+      L.seg(s0, 0, 2);
+      double spans = 0.0;
+      for (int k = 0; k < ref.latent_t; ++k) spans += kRescale * kFramePerToken[k % 5];
+      cursor += std::max((double)ref.audio_t, spans);
+    } else {
+      return fail(MMH3_ERR_ARG, "layout: reference %d kind %d not in {0,1,2}", r, ref.kind);
+    }
+  }
+  // keyframes: on the target grid, never moving the cursor
+  double spans = 0.0;
+  for (int k = 0; k < latent_t; ++k) spans += kRescale * kFramePerToken[k % 5];
+  for (int f = 0; f < n_frames; ++f) {
+    const mmh3_keyframe& kf = frames[f];
+    double cond_t;
+    if (kf.pixel_index == 0)
+      cond_t = cursor;
+    else if (kf.frame_count > 0 && kf.pixel_index == kf.frame_count - 1)
+      cond_t = cursor + spans - kRescale;
+    else
+      return fail(MMH3_ERR_ARG, "layout: keyframe %d at pixel %d of %d: only the first and last frame anchor one", f,
+                  kf.pixel_index, kf.frame_count);
+    const int s0 = L.rows();
+    for (double h : hs)
+      for (double w : ws) L.row(cond_t, h, w);
+    L.seg(s0, 0, 2);
+  }
+  // stereo audio, channel-major, w pinned to the target grid's extremes
+  const int a0 = L.rows();
+  audio_grid(cursor, audio_t, ws.front(), ws.back());
   L.seg(a0, /*tag audio*/ 2, /*clock*/ 1);
-  int v0 = L.rows();
+  // video: t advances by the per-token frame spans
+  const int v0 = L.rows();
   double t = cursor;
   for (int k = 0; k < latent_t; ++k) {
     for (double h : hs)
@@ -210,7 +312,42 @@ extern "C" mmh3_status mmh3_layout_t2va(int text_len, int latent_t, int lat_h, i
     t += kRescale * kFramePerToken[k % 5];
   }
   L.seg(v0, /*tag video*/ 0, /*clock*/ 0);
-  return L.emit(segs, n_seg, pos, pos_capacity, n_out);
+  return MMH3_OK;
+}
+
+}  // namespace
+
+extern "C" mmh3_status mmh3_layout_t2va(int text_len, int latent_t, int lat_h, int lat_w,
+                                        int audio_t, mmh3_segment* segs, int* n_seg, float* pos,
+                                        int pos_capacity, int* n_out) {
+  clear_error();
+  LayoutBuilder L;
+  mmh3_status st = build_layout(L, text_len, latent_t, lat_h, lat_w, audio_t, nullptr, 0, nullptr, 0, nullptr);
+  if (st != MMH3_OK) return st;
+  return L.emit(segs, 3, n_seg, pos, pos_capacity, n_out);
+}
+
+extern "C" mmh3_status mmh3_layout_fl2va(int text_len, int latent_t, int lat_h, int lat_w, int audio_t,
+                                         const mmh3_keyframe* frames, int n_frames, const uint8_t* text_tags,
+                                         mmh3_segment* segs, int seg_capacity, int* n_seg, float* pos,
+                                         int pos_capacity, int* n_out) {
+  clear_error();
+  LayoutBuilder L;
+  mmh3_status st =
+      build_layout(L, text_len, latent_t, lat_h, lat_w, audio_t, frames, n_frames, nullptr, 0, text_tags);
+  if (st != MMH3_OK) return st;
+  return L.emit(segs, seg_capacity, n_seg, pos, pos_capacity, n_out);
+}
+
+extern "C" mmh3_status mmh3_layout_ref2va(int text_len, int latent_t, int lat_h, int lat_w, int audio_t,
+                                          const mmh3_ref* refs, int n_refs, const uint8_t* text_tags,
+                                          mmh3_segment* segs, int seg_capacity, int* n_seg, float* pos,
+                                          int pos_capacity, int* n_out) {
+  clear_error();
+  LayoutBuilder L;
+  mmh3_status st = build_layout(L, text_len, latent_t, lat_h, lat_w, audio_t, nullptr, 0, refs, n_refs, text_tags);
+  if (st != MMH3_OK) return st;
+  return L.emit(segs, seg_capacity, n_seg, pos, pos_capacity, n_out);
 }
 
 extern "C" mmh3_status mmh3_layout_image(int text_len, int ref_lat_h, int ref_lat_w, int lat_h,
@@ -235,7 +372,7 @@ extern "C" mmh3_status mmh3_layout_image(int text_len, int ref_lat_h, int ref_la
     L.seg(s0, 0, 0);
     cursor += 1.0;
   }
-  return L.emit(segs, n_seg, pos, pos_capacity, n_out);
+  return L.emit(segs, 3, n_seg, pos, pos_capacity, n_out);
 }
 
 extern "C" mmh3_status mmh3_plan_timesteps(const mmh3_segment* segs, int n_seg, int n,

@@ -26,10 +26,14 @@ DevStatus* device_status_ptr();
 int num_sms();
 
 // ------------------------------------------------------------------ plan
+// Clocks of a segment: 0 the video flow clock, 1 the audio flow clock,
+// 2 the visual condition clock (keyframe and reference-image rows), 3 the
+// audio condition clock (reference audio rows).
+constexpr int kClocks = 4;
 struct Plan {
   int n_ts = 0;
-  double ts[2] = {0, 0};
-  int slot[2] = {-1, -1};   // slot of clock 0 / 1 (-1: unused)
+  double ts[kClocks] = {0, 0, 0, 0};
+  int slot[kClocks] = {-1, -1, -1, -1};  // slot of each clock (-1: unused)
   SegRows block_rows{};      // per segment: slot*3 + tag
   SegRows final_rows{};      // per segment: slot
   int seg_tag[kMaxSeg]{};

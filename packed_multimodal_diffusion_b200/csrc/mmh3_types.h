@@ -27,7 +27,7 @@ struct DevStatus {
 
 // Segment table as a kernel parameter: token i reads modulation row
 // row[k] where start[k] <= i < stop[k].
-constexpr int kMaxSeg = 8;
+constexpr int kMaxSeg = 16;
 struct SegRows {
   int n;
   int start[kMaxSeg];

@@ -202,3 +202,79 @@ def test_host_slot_count_matches_header():
     text = open(os.path.join(ROOT, "include", "mmh3.h")).read()
     m = re.search(r"#define MMH3_HOST_SLOTS (\d+)", text)
     assert m and int(m.group(1)) == api.HOST_SLOTS
+
+
+# ---------------------------------------------- keyframe / reference layouts
+FL2VA_CASES = [
+    ((8, 3, 8, 12, 5), [(0, 39), (38, 39)], None),
+    ((20, 3, 16, 20, 20), [(38, 39)], [1] * 5 + [0] * 10 + [1] * 5),
+    ((16, 2, 8, 8, 8), [], None),
+]
+REF2VA_CASES = [
+    ((4, 2, 4, 4, 3), [("image", 4, 6)], None),
+    ((4, 2, 4, 4, 3), [("audio", 3)], None),
+    ((4, 2, 4, 4, 3), [("video", 2, 4, 8, 5)], None),
+    ((10, 3, 16, 20, 6), [("image", 8, 8), ("audio", 4), ("video", 3, 8, 12, 0), ("video", 1, 4, 4, 7)],
+     [1, 1, 1, 0, 0, 0, 0, 1, 1, 1]),
+]
+
+
+@pytest.mark.parametrize("case", range(len(FL2VA_CASES)))
+def test_fl2va_layout_bit_exact_against_oracle(case):
+    sizes, frames, tags = FL2VA_CASES[case]
+    segs, pos = api.layout_fl2va(*sizes, frames, tags)
+    L = O.layout_fl2va(*sizes, frames, text_tags=tags)
+    assert [tuple(s) for s in segs] == [tuple(s) for s in L["segments"]]
+    np.testing.assert_array_equal(pos, L["pos"].astype(np.float32))
+
+
+@pytest.mark.parametrize("case", range(len(REF2VA_CASES)))
+def test_ref2va_layout_bit_exact_against_oracle(case):
+    sizes, refs, tags = REF2VA_CASES[case]
+    segs, pos = api.layout_ref2va(*sizes, refs, tags)
+    L = O.layout_ref2va(*sizes, refs, text_tags=tags)
+    assert [tuple(s) for s in segs] == [tuple(s) for s in L["segments"]]
+    np.testing.assert_array_equal(pos, L["pos"].astype(np.float32))
+
+
+@pytest.mark.parametrize("sigma_v", [1e-9, 1e-4, 0.3, 0.9, 1.0])
+def test_condition_clock_plan_matches_oracle(sigma_v):
+    sa = O.time_shift_sigma(max(sigma_v, 1e-6), 12, 3)
+    for L in (O.layout_fl2va(*FL2VA_CASES[0][0], FL2VA_CASES[0][1]),
+              O.layout_ref2va(*REF2VA_CASES[3][0], REF2VA_CASES[3][1], text_tags=REF2VA_CASES[3][2])):
+        ts_o, slot = O.plan_timesteps(sigma_v, sa, L["segments"])
+        ts, rows = api.plan_timesteps(L["segments"], L["seq_len"], sigma_v, sa)
+        assert ts == ts_o
+        rows_o = O.token_rows(L["segments"], slot, L["seq_len"])
+        assert [int(rows_o[a]) for a, _, _, _ in L["segments"]] == rows
+
+
+def test_layout_errors_and_more_than_two_timesteps_without_modulation():
+    lib = _lib.load()
+    kf = (_lib.Keyframe * 1)(_lib.Keyframe(5, 39))
+    segs = (_lib.Segment * 16)()
+    ns, n = C.c_int(), C.c_int()
+    # a keyframe that is neither the first nor the last frame
+    assert lib.mmh3_layout_fl2va(8, 3, 8, 12, 5, kf, 1, None, segs, 16, C.byref(ns), None, 0, C.byref(n)) == 1
+    assert b"first and the last" in lib.mmh3_last_error() or b"first and last" in lib.mmh3_last_error()
+    # segment capacity below the layout's count
+    kf2 = (_lib.Keyframe * 2)(_lib.Keyframe(0, 39), _lib.Keyframe(38, 39))
+    assert lib.mmh3_layout_fl2va(8, 3, 8, 12, 5, kf2, 2, None, segs, 4, C.byref(ns), None, 0, C.byref(n)) == 2
+    # four distinct timesteps: the block's own adaLN curve is refused before
+    # any launch (nothing below is dereferenced)
+    sizes, refs, tags = REF2VA_CASES[3]
+    L = O.layout_ref2va(*sizes, refs, text_tags=tags)
+    nn = L["seq_len"]
+    d = api.make_dims(256, 2, 128, 512)
+    v = C.c_size_t()
+    assert lib.mmh3_workspace_size(C.byref(d), nn, C.byref(v)) == 0
+    w = _lib.BlockWeights(*([256] * 11))
+    sa = O.time_shift_sigma(0.3, 12, 3)
+    rc = lib.mmh3_block_forward(C.byref(d), C.byref(w), C.c_void_p(256), nn, api.segments(L["segments"]),
+                                len(L["segments"]), None, 0.3, sa, 1, None, C.c_void_p(256), v.value, None)
+    assert rc == 5 and b"two slots" in lib.mmh3_last_error()
+    out = C.c_int()
+    rc = lib.mmh3_adaln_modulation(C.byref(d), C.c_void_p(256), C.c_void_p(256), C.c_void_p(256), 18 * 256,
+                                   api.segments(L["segments"]), len(L["segments"]), nn, 0.3, sa,
+                                   C.c_void_p(256), C.byref(out), None)
+    assert rc == 5 and out.value == 4

@@ -747,3 +747,97 @@ def test_denoise_forward_each_stream_reads_its_own_clocks_final_row():
                              heads, 0.5, 0.2, dims)
     np.testing.assert_allclose(v, -2.0 * video, rtol=0, atol=1e-14)
     np.testing.assert_allclose(a, -4.0 * audio, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------- keyframe / reference layouts
+
+def test_keyframes_sit_between_the_text_and_the_audio_page_test():
+    # "cortiq_engine/mmh3.rs" test keyframes_sit_between_the_text_and_the_audio:
+    # t2va(8, 3, 8, 12, 5) against fl2va with the first and last frame of a
+    # 39-frame clip
+    tl, lt, lh, lw, at = 8, 3, 8, 12, 5
+    base = O.layout_t2va(tl, lt, lh, lw, at)
+    L = O.layout_fl2va(tl, lt, lh, lw, at, [(0, 39), (38, 39)])
+    cond = [s for s, k in zip(L["segments"], L["kinds"]) if k == "Cond"]
+    assert sum(b - a for a, b, _, _ in cond) == 2 * L["frame_rows"] == 48
+    assert L["seq_len"] == base["seq_len"] + 2 * L["frame_rows"] == 138
+    assert L["kinds"] == ["Text", "Cond", "Cond", "Audio", "Video"]
+    seg = {k: s for s, k in zip(L["segments"], L["kinds"])}
+    bseg = dict(zip(base["kinds"], base["segments"]))
+    # a keyframe never advances the cursor
+    assert L["pos"][seg["Audio"][0], 0] == base["pos"][bseg["Audio"][0], 0]
+    assert L["pos"][seg["Video"][0], 0] == base["pos"][bseg["Video"][0], 0]
+    # first frame at the text's end, the last a whole clip further, minus one span
+    assert L["pos"][cond[0][0], 0] == tl
+    spans = sum(O.FRAME_RESCALE * O.FRAME_PER_TOKEN[k % 5] for k in range(lt))
+    assert abs(L["pos"][cond[1][0], 0] - (tl + spans - O.FRAME_RESCALE)) < 1e-12
+    assert abs(L["pos"][cond[1][0], 0] - (8 + 15 - 5 / 3)) < 1e-12           # spans = 5/3 (1+4+4)
+    # both keyframes share the target grid
+    np.testing.assert_array_equal(L["pos"][cond[0][0]:cond[0][1], 1:], L["pos"][seg["Video"][0]:seg["Video"][0] + 24, 1:])
+    # keyframe rows: tag video on the visual condition clock
+    assert all(s[2] == O.TAG_VIDEO and s[3] == O.CLOCK_COND for s in cond)
+    with pytest.raises(ValueError):
+        O.layout_fl2va(tl, lt, lh, lw, at, [(5, 39)])
+
+
+def test_reference_blocks_advance_the_cursor_by_hand():
+    # a still: its own grid at the cursor, cursor + 1
+    L = O.layout_ref2va(4, 2, 4, 4, 3, [("image", 4, 6)])
+    assert L["kinds"] == ["Text", "RefImg", "Audio", "Video"]
+    img = L["segments"][1]
+    assert img[1] - img[0] == 2 * 3 and (img[2], img[3]) == (O.TAG_VIDEO, O.CLOCK_COND)
+    assert (L["pos"][img[0]:img[1], 0] == 4.0).all()
+    a = math.sqrt(24)
+    assert L["pos"][img[0] + 1, 2] == O.axis_from_sqrt_area(6, 2, a)[1]
+    assert L["pos"][L["segments"][2][0], 0] == 5.0 and L["pos"][L["segments"][3][0], 0] == 5.0
+    # standalone audio: t stereo frames from the cursor (target grid's w extremes), cursor + t
+    L = O.layout_ref2va(4, 2, 4, 4, 3, [("audio", 3)])
+    ra = L["segments"][1]
+    assert L["kinds"][1] == "RefAudio" and (ra[2], ra[3]) == (O.TAG_AUDIO, O.CLOCK_COND_AUDIO)
+    np.testing.assert_array_equal(L["pos"][ra[0]:ra[1], 0], [4, 5, 6, 4, 5, 6])
+    w_t = O.axis_from_sqrt_area(4, 2, 4.0)
+    assert L["pos"][ra[0], 2] == w_t[0] and L["pos"][ra[1] - 1, 2] == w_t[-1]
+    assert L["pos"][L["segments"][2][0], 0] == 7.0
+    # a clip: soundtrack first (its own w extremes), frames stepping by the
+    # spans, cursor + max(audio frames, spans)
+    L = O.layout_ref2va(4, 2, 4, 4, 3, [("video", 2, 4, 8, 5)])
+    assert L["kinds"] == ["Text", "RefAudio", "RefImg", "Audio", "Video"]
+    ra, rv = L["segments"][1], L["segments"][2]
+    w_r = O.axis_from_sqrt_area(8, 2, math.sqrt(32))
+    assert L["pos"][ra[0], 2] == w_r[0] and L["pos"][ra[1] - 1, 2] == w_r[-1]
+    assert L["pos"][rv[0], 0] == 4.0 and abs(L["pos"][rv[0] + 8, 0] - (4 + 5 / 3)) < 1e-12
+    assert abs(L["pos"][L["segments"][3][0], 0] - (4 + 25 / 3)) < 1e-12   # max(5, 5/3 + 20/3)
+    # a clip whose soundtrack is longer than its frames
+    L = O.layout_ref2va(4, 2, 4, 4, 3, [("video", 1, 4, 4, 5)])
+    assert L["pos"][L["segments"][3][0], 0] == 9.0                          # max(5, 5/3)
+
+
+def test_condition_rows_hand_enumerated():
+    # fl2va at sigma_v 0.3: t_v 0.7, t_a 28/31, t_cond max(0.7, 0.999)
+    L = O.layout_fl2va(8, 3, 8, 12, 5, [(0, 39)])
+    sa = O.time_shift_sigma(0.3, 12, 3)
+    ts, slot = O.plan_timesteps(0.3, sa, L["segments"])
+    np.testing.assert_allclose(ts, [0.7, 28 / 31, 0.999], rtol=0, atol=1e-15)
+    rows = O.token_rows(L["segments"], slot, L["seq_len"])
+    assert [int(rows[s[0]]) for s in L["segments"]] == [1, 6, 5, 0]
+    # late in sampling t_v passes 0.999: the keyframes share the video slot
+    sv = 1e-4
+    sa = O.time_shift_sigma(sv, 12, 3)
+    ts, slot = O.plan_timesteps(sv, sa, L["segments"])
+    assert len(ts) == 2 and slot[O.CLOCK_COND] == slot[O.CLOCK_VIDEO] == 0
+    rows = O.token_rows(L["segments"], slot, L["seq_len"])
+    assert [int(rows[s[0]]) for s in L["segments"]] == [1, 0, 5, 0]
+    # ref2va with a still and standalone audio: four clocks, four timesteps
+    L = O.layout_ref2va(4, 2, 4, 4, 3, [("image", 4, 4), ("audio", 2)])
+    ts, slot = O.plan_timesteps(0.3, O.time_shift_sigma(0.3, 12, 3), L["segments"])
+    assert len(ts) == 4 and ts[-2:] == [0.999, 1.0]
+    rows = O.token_rows(L["segments"], slot, L["seq_len"])
+    assert [int(rows[s[0]]) for s in L["segments"]] == [1, 6, 11, 5, 0]
+
+
+def test_text_tags_split_the_prompt_into_runs():
+    L = O.layout_fl2va(8, 1, 4, 4, 2, [], text_tags=[1, 1, 0, 0, 1, 1, 1, 1])
+    assert L["segments"][:3] == [(0, 2, 1, 0), (2, 4, 0, 0), (4, 8, 1, 0)]
+    ts, slot = O.plan_timesteps(0.5, 0.2, L["segments"])
+    rows = O.token_rows(L["segments"], slot, L["seq_len"])
+    assert list(rows[:8]) == [1, 1, 0, 0, 1, 1, 1, 1]
