@@ -44,7 +44,8 @@ typedef enum {
   MMH3_ERR_WORKSPACE = 4,    /* workspace missing or too small */
   MMH3_ERR_UNSUPPORTED = 5,  /* more than two distinct timesteps, etc. */
   MMH3_ERR_CUDA = 6,         /* a CUDA runtime / driver call failed */
-  MMH3_ERR_TIMEOUT = 7       /* a kernel gave up waiting (device status) */
+  MMH3_ERR_TIMEOUT = 7,      /* a kernel gave up waiting (device status) */
+  MMH3_ERR_CHECK = 8         /* a device check of the MMH3_CHECK mode failed (device status) */
 } mmh3_status;
 
 typedef enum { MMH3_F32 = 0, MMH3_BF16 = 1 } mmh3_dtype;
@@ -603,6 +604,29 @@ mmh3_status mmh3_device_status(void* stream, int* code, int* site);
  * if a kernel gave up waiting, MMH3_ERR_CUDA if the synchronisation failed.
  * The one entry point besides mmh3_device_status that waits for the GPU. */
 mmh3_status mmh3_status_sync(void* stream, int* device_status);
+
+/* The check mode (no counterpart in the pages; the memory-safety evidence
+ * where no sanitizer runs).  On: MMH3_CHECK=1 in the environment, or
+ * mmh3_set_check(1); mmh3_set_check(-1) returns to the environment's
+ * choice.  While it is on:
+ *  - every token's modulation row is checked against the modulation
+ *    buffer's rows (T_s * 3 for a block, T_s for the heads), every TMA
+ *    operand copy of the GEMMs and of attention against the copy rules
+ *    (x offset a multiple of 16 bytes, no negative coordinate); a failure
+ *    is recorded in the device status word, the access skipped (the
+ *    kernel aborts through its bounded-wait path), never trapped;
+ *  - each workspace region is followed by a 256-byte canary, written at the
+ *    start of a call and verified after every kernel of the block, the
+ *    stack and the heads (mmh3_workspace_size reports the larger size,
+ *    so query it with the mode already set);
+ *  - mmh3_device_status / mmh3_status_sync return MMH3_ERR_CHECK with the
+ *    record (code 6 row, 7 TMA coordinate, 8 canary; the canary's site is
+ *    kernel * 16 + region, kernel as MMH3_PROF_K_*, 8 for the heads).
+ * The flag lives in each device's status word and is written (a
+ * synchronous copy) on the first call that touches a device after the mode
+ * changes: set the mode outside stream capture. */
+void mmh3_set_check(int on);
+int mmh3_check_enabled(void);
 
 /* Bound on every in-kernel wait, in nanoseconds (0 restores the default). */
 void mmh3_set_wait_limit_ns(uint64_t ns);

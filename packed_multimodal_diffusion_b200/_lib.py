@@ -14,7 +14,7 @@ MMH3_F32, MMH3_BF16 = 0, 1
 
 STATUS_NAMES = {0: "MMH3_OK", 1: "MMH3_ERR_ARG", 2: "MMH3_ERR_SHAPE", 3: "MMH3_ERR_ALIGN",
                 4: "MMH3_ERR_WORKSPACE", 5: "MMH3_ERR_UNSUPPORTED", 6: "MMH3_ERR_CUDA",
-                7: "MMH3_ERR_TIMEOUT"}
+                7: "MMH3_ERR_TIMEOUT", 8: "MMH3_ERR_CHECK"}
 
 
 class Mmh3Error(RuntimeError):
@@ -144,6 +144,8 @@ SIGNATURES = {
     "mmh3_device_status": (_I, [_P, C.POINTER(_I), C.POINTER(_I)]),
     "mmh3_status_sync": (_I, [_P, C.POINTER(_I)]),
     "mmh3_set_wait_limit_ns": (None, [C.c_uint64]),
+    "mmh3_set_check": (None, [_I]),
+    "mmh3_check_enabled": (_I, []),
     "mmh3_selftest_wait_timeout": (_I, [C.c_uint64, _P]),
     "mmh3_prof_enable": (None, [_I]),
     "mmh3_prof_collect": (_I, [C.POINTER(C.c_double), _I, C.POINTER(C.c_long)]),

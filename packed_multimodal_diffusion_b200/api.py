@@ -519,6 +519,11 @@ def launch_count() -> int:
     return int(load().mmh3_launch_count())
 
 
+def set_check(on: int) -> None:
+    """The check mode: 1 on, 0 off, -1 the environment's MMH3_CHECK."""
+    load().mmh3_set_check(on)
+
+
 def set_wait_limit_ns(ns: int) -> None:
     load().mmh3_set_wait_limit_ns(ns)
 

@@ -95,6 +95,7 @@ struct Workspace {
   void* head;
   float* fmods;
   size_t bytes;
+  CanaryList canaries;  // MMH3_CHECK mode: one after each region
 };
 
 Workspace carve(const mmh3_dims& d, int n, void* base) {
@@ -103,9 +104,15 @@ Workspace carve(const mmh3_dims& d, int n, void* base) {
   const size_t N = (size_t)n;
   Workspace w{};
   size_t off = 0;
+  const bool canary = check_mode();
   auto take = [&](size_t bytes) {
     uint8_t* p = static_cast<uint8_t*>(base) + off;
     off += align256(bytes);
+    if (canary) {
+      if (base && w.canaries.n < kMaxCanaries)
+        w.canaries.p[w.canaries.n++] = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(base) + off);
+      off += kCanaryBytes;
+    }
     return base ? static_cast<void*>(p) : nullptr;
   };
   w.mods = static_cast<float*>(take(2 * 3 * 6 * H * 4));
@@ -159,6 +166,14 @@ mmh3_status check_block(const mmh3_dims& d, const mmh3_block_weights* w, bool mo
   return MMH3_OK;
 }
 
+// MMH3_CHECK mode: fill the workspace canaries (verify = false) or check
+// them after the kernel kid (verify = true); nothing without canaries.
+mmh3_status canaries(const Workspace& ws, bool verify, int kid, cudaStream_t s) {
+  if (ws.canaries.n == 0) return MMH3_OK;
+  cudaError_t e = launch_canary(ws.canaries, verify, kid, s);
+  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "canary launch");
+}
+
 // norm1-modulate -> qkv+qknorm+rope (the part before attention)
 mmh3_status block_pre(const mmh3_dims& d, const mmh3_block_weights& w, const float* x, int n, const Plan& plan,
                       const float* mods, const float2* cs, const Workspace& ws, cudaStream_t s, PhaseMark& pm) {
@@ -169,11 +184,12 @@ mmh3_status block_pre(const mmh3_dims& d, const mmh3_block_weights& w, const flo
                                   ws.xn1, s);
   if (e != cudaSuccess) return cuda_fail(e, "norm1/modulate launch");
   pm.mark(0, MMH3_PROF_K_NORM1);
-  mmh3_status st = gemm_qkv(dt, ws.xn1, w.wqkv, n, 3 * I, H, d.head_dim, I, w.q_norm, w.k_norm, cs, d.qk_eps,
-                            ws.qkv, s);
+  mmh3_status st = canaries(ws, true, MMH3_PROF_K_NORM1, s);
+  if (st != MMH3_OK) return st;
+  st = gemm_qkv(dt, ws.xn1, w.wqkv, n, 3 * I, H, d.head_dim, I, w.q_norm, w.k_norm, cs, d.qk_eps, ws.qkv, s);
   if (st != MMH3_OK) return st;
   pm.mark(1, MMH3_PROF_K_QKV);
-  return MMH3_OK;
+  return canaries(ws, true, MMH3_PROF_K_QKV, s);
 }
 
 // attention -> out+gated residual -> norm2-modulate -> fc1+SwiGLU -> fc2+gated
@@ -195,21 +211,29 @@ mmh3_status block_post(const mmh3_dims& d, const mmh3_block_weights& w, float* x
                                       act_bytes);
   if (st != MMH3_OK) return st;
   pm.mark(3, MMH3_PROF_K_ATTN);
+  st = canaries(ws, true, MMH3_PROF_K_ATTN, s);
+  if (st != MMH3_OK) return st;
   st = gemm_gated_residual(dt, ws.attn, w.wout, n, H, I, x, mods, stride, 2 * H, plan.block_rows, s);
   if (st != MMH3_OK) return st;
   pm.mark(4, MMH3_PROF_K_OUT);
+  st = canaries(ws, true, MMH3_PROF_K_OUT, s);
+  if (st != MMH3_OK) return st;
   cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm2, d.eps, mods, stride, 3 * H, 4 * H, plan.block_rows, 0,
                                   ws.xn2, s);
   if (e != cudaSuccess) return cuda_fail(e, "norm2/modulate launch");
   pm.mark(0, MMH3_PROF_K_NORM2);
+  st = canaries(ws, true, MMH3_PROF_K_NORM2, s);
+  if (st != MMH3_OK) return st;
   st = gemm_swiglu(dt, ws.xn2, w.wfc1, n, F, H, ws.act, s);
   if (st != MMH3_OK) return st;
   pm.mark(5, MMH3_PROF_K_FC1);
+  st = canaries(ws, true, MMH3_PROF_K_FC1, s);
+  if (st != MMH3_OK) return st;
   st = gemm_gated_residual(dt, ws.act, w.wfc2, n, H, F, x, mods, stride, 5 * H, plan.block_rows, s);
   if (st != MMH3_OK) return st;
   pm.mark(7, MMH3_PROF_K_FC2);
   if (pm.on) ++g_prof_blocks;
-  return MMH3_OK;
+  return canaries(ws, true, MMH3_PROF_K_FC2, s);
 }
 
 // The whole block on one GPU.
@@ -246,7 +270,8 @@ mmh3_status prologue(const mmh3_dims& d, const mmh3_block_weights* w, bool own_m
   }
   cudaError_t e = launch_prologue(ab, own_mods ? 1 : 0, d.rank, d.grid, 18 * d.hidden, plan, ws.mods, 0, pos, n,
                                   d.rope_k, d.rope_theta, ws.cs, s);
-  return e == cudaSuccess ? MMH3_OK : cuda_fail(e, "prologue launch");
+  if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+  return canaries(ws, true, MMH3_PROF_K_PROLOGUE, s);
 }
 
 mmh3_status common_checks(const mmh3_dims* dims, float* x, int n, const float* pos, void* ws,
@@ -298,6 +323,8 @@ mmh3_status mmh3::block_forward_impl(const mmh3_dims* dims, const mmh3_block_wei
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden;
   PhaseMark pm(s, profile);
+  st = canaries(ws, false, 0, s);
+  if (st != MMH3_OK) return st;
   st = prologue(*dims, w, own_mods, plan, ws, pos_dev, n, s);
   if (st != MMH3_OK) return st;
   if (own_mods || pos_dev) pm.mark(0, MMH3_PROF_K_PROLOGUE);
@@ -421,6 +448,8 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
   // first launch also writes the rotation table.  When that region cannot
   // hold one block's rows, each block's modulation goes to ws.mods just
   // before the block.
+  st = canaries(ws, false, 0, s);
+  if (st != MMH3_OK) return st;
   const long long mods_floats = (long long)plan.n_ts * 18 * H;
   const size_t head_bytes = (size_t)n * H * esize_of(dims->act_dtype);
   long long fit = (long long)(head_bytes / ((size_t)mods_floats * 4));
@@ -431,6 +460,8 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                                     pos_dev, n, dims->rope_k, dims->rope_theta, ws.cs, s);
     if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
     pm.mark(0, MMH3_PROF_K_PROLOGUE);
+    st = canaries(ws, true, MMH3_PROF_K_PROLOGUE, s);
+    if (st != MMH3_OK) return st;
   }
   for (int i = 0; i < n_blocks; ++i) {
     if (i % per_launch == 0) {
@@ -445,6 +476,8 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
                                       i == 0 ? pos_dev : nullptr, n, dims->rope_k, dims->rope_theta, ws.cs, s);
       if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
       pm.mark(0, MMH3_PROF_K_PROLOGUE);
+      st = canaries(ws, true, MMH3_PROF_K_PROLOGUE, s);
+      if (st != MMH3_OK) return st;
     }
     const float* mods = mbase + (i % per_launch) * mods_floats;
     st = block_core(*dims, blocks[i], x, n, plan, mods, pos_dev ? ws.cs : nullptr, ws, s, pm);
@@ -465,6 +498,8 @@ mmh3_status mmh3_stack_forward(const mmh3_dims* dims, const mmh3_block_weights* 
     st = gemm_bias_act(dims->act_dtype, ws.head, k == 0 ? heads->w_video : heads->w_audio, rows,
                        k == 0 ? heads->out_video : heads->out_audio, H, k == 0 ? heads->b_video : heads->b_audio, 2,
                        k == 0 ? (void*)out_video : (void*)out_audio, s);
+    if (st != MMH3_OK) return st;
+    st = canaries(ws, true, 8, s);
     if (st != MMH3_OK) return st;
   }
   return MMH3_OK;
@@ -572,6 +607,8 @@ mmh3_status mmh3_block_cp_begin(const mmh3_dims* dims, const mmh3_block_weights*
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   PhaseMark pm(s, false);
+  st = canaries(ws, false, 0, s);
+  if (st != MMH3_OK) return st;
   st = prologue(*dims, w, modulated != 0, plan, ws, pos_dev, n, s);
   if (st != MMH3_OK) return st;
   st = block_pre(*dims, *w, x, n, plan, modulated ? ws.mods : nullptr, pos_dev ? ws.cs : nullptr, ws, s, pm);
@@ -647,6 +684,8 @@ mmh3_status mmh3_refine_text(const mmh3_dims* dims, const void* states, int n, i
   float* h = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + refine_stream_offset(*dims, n));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden;
+  st = canaries(ws, false, 0, s);
+  if (st != MMH3_OK) return st;
   st = gemm_bias_act(dims->act_dtype, states, cond_w, n, H, text_dim, cond_b, 3, h, s);
   if (st != MMH3_OK) return st;
   PhaseMark pm(s, false);

@@ -184,11 +184,25 @@ __global__ void __launch_bounds__(320, 1)
       const int xq = head * HD, xk = k_off + head * HD, xv = v_off + head * HD;
       int in_k = 0, in_v = 0;
       bool ok = true;
-      mbar_expect_tx(bar(B_Q), 2 * Sh::kTileBytes);
-      for (int i = 0; i < 2; ++i)
-        for (int c = 0; c < Sh::kHdBoxes; ++c)
-          tma_load_2d(sbase + Sh::kQOff + i * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_Q),
-                      xq + c * 64, q_row0 + 128 * i);
+      // MMH3_CHECK mode: the x coordinates of every copy this CTA issues and
+      // the first rows of Q and of its keys, before the first copy (the key
+      // rows only grow from there); a failure issues nothing
+      bool q_issued = false;
+      if (status != nullptr && status->check != 0) {
+        for (int c = 0; c < Sh::kHdBoxes && ok; ++c)
+          ok = tma_coords_ok(status, true, xq + c * 64, q_row0, 2) &&
+               tma_coords_ok(status, true, xk + c * 64, kv_row0 + j0 * 128, 2) &&
+               tma_coords_ok(status, true, xv + c * 64, kv_row0 + j0 * 128, 2);
+        if (!ok) *abort_flag = 1;
+      }
+      if (ok) {
+        mbar_expect_tx(bar(B_Q), 2 * Sh::kTileBytes);
+        for (int i = 0; i < 2; ++i)
+          for (int c = 0; c < Sh::kHdBoxes; ++c)
+            tma_load_2d(sbase + Sh::kQOff + i * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_Q),
+                        xq + c * 64, q_row0 + 128 * i);
+        q_issued = true;
+      }
       int j = 0;
       for (; j < n_kv && ok; ++j) {
         const int s = j % KV;
@@ -210,7 +224,7 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) {
         if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, j);
         *abort_flag = 1;
-        mbar_wait(bar(B_Q), 0, limit_ns);
+        if (q_issued) mbar_wait(bar(B_Q), 0, limit_ns);
         for (int i = (in_k > KV ? in_k - KV : 0); i < in_k; ++i)
           mbar_wait(bar(B_KF + i % KV), (uint32_t)((i / KV) & 1), limit_ns);
         for (int i = (in_v > KV ? in_v - KV : 0); i < in_v; ++i)

@@ -504,7 +504,7 @@ struct EpiResidual : NoSetup {
                                              Wait&& wait, const float*) const {
     const float* g = nullptr;
     if (BIAS) g = bias;
-    else if (mods != nullptr) g = mods + (size_t)seg_row(seg, row) * mods_stride + chunk_off;
+    else if (mods != nullptr) g = mods + (size_t)seg_row_checked(seg, row) * mods_stride + chunk_off;
     int c0, c1;
     part_chunks<BN>(part, c0, c1);
     float4 xa[8];
@@ -587,7 +587,7 @@ struct EpiResidualTma : NoSetup {
     if (!st.rows_in) return true;
     const float* g = nullptr;
     if (BIAS) g = bias;
-    else if (mods != nullptr) g = mods + (size_t)seg_row(seg, row) * mods_stride + chunk_off;
+    else if (mods != nullptr) g = mods + (size_t)seg_row_checked(seg, row) * mods_stride + chunk_off;
 #pragma unroll 1
     for (int u = 0; u < units; ++u) {
       const int b = u & 1;
@@ -819,6 +819,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
+      const bool chk = status != nullptr && status->check != 0;
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;  // stages whose copies may still be in flight
@@ -829,6 +830,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (*abort_flag || !mbar_wait(empty_bar(stage), phase ^ 1u, limit_ns)) {
             if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          if (!tma_coords_ok(status, chk, kb * kBK, mt * Sh::BM, ElemTraits<T>::kBytes) ||
+              !tma_coords_ok(status, chk, kb * kBK, nt * BN, ElemTraits<T>::kBytes)) {
             *abort_flag = 1;
             ok = false;
             break;
@@ -1069,6 +1076,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs)
+      const bool chk = status != nullptr && status->check != 0;
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -1081,6 +1089,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (*abort_flag || !mbar_wait(empty_bar(stage), phase ^ 1u, limit_ns)) {
             if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, tile);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          if (!tma_coords_ok(status, chk, kb * kBK, a_row, 2) || !tma_coords_ok(status, chk, kb * kBK, b_row, 2)) {
             *abort_flag = 1;
             ok = false;
             break;

@@ -44,6 +44,17 @@ mmh3_status cuda_fail(cudaError_t e, const char* what) {
   return fail(MMH3_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+static int g_check_override = -1;  // mmh3_set_check; -1: the environment decides
+
+bool check_mode() {
+  if (g_check_override >= 0) return g_check_override != 0;
+  static const bool env_on = [] {
+    const char* v = std::getenv("MMH3_CHECK");
+    return v != nullptr && std::atoi(v) != 0;
+  }();
+  return env_on;
+}
+
 static uint64_t g_limit_override = 0;
 
 uint64_t wait_limit_ns() {
@@ -114,6 +125,11 @@ mmh3_status make_plan(const mmh3_segment* segs, int n_seg, int n, double sigma_v
       if (p->ts[i] == t_of[c]) p->slot[c] = i;
   }
   p->block_rows.n = p->final_rows.n = n_seg;
+  if (check_mode()) {  // rows outside the modulation buffer are recorded on the device
+    p->block_rows.limit = 3 * p->n_ts;
+    p->final_rows.limit = p->n_ts;
+    p->block_rows.status = p->final_rows.status = device_status_ptr();
+  }
   for (int k = 0; k < n_seg; ++k) {
     const int slot = p->slot[segs[k].clock];
     p->block_rows.start[k] = p->final_rows.start[k] = (int)segs[k].start;
@@ -142,6 +158,13 @@ const char* mmh3_last_error(void) { return g_msg; }
 const char* mmh3_version(void) { return "mmh3-b200 0.1 (sm_100a)"; }
 
 void mmh3_set_wait_limit_ns(uint64_t ns) { g_limit_override = ns; }
+
+void mmh3_set_check(int on) {
+  g_check_override = on < 0 ? -1 : (on != 0 ? 1 : 0);
+  device_status_ptr();  // writes the flag on the current device (if there is one)
+}
+
+int mmh3_check_enabled(void) { return check_mode() ? 1 : 0; }
 
 }  // extern "C"
 

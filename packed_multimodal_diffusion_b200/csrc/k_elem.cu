@@ -18,16 +18,47 @@ namespace mmh3 {
 // ------------------------------------------------------------ status word
 __device__ DevStatus g_dev_status;
 
+// The status word of the current device; the first lookup on a device also
+// writes the check-mode flag into it (MMH3_CHECK=1 or mmh3_set_check).
 DevStatus* device_status_ptr() {
   static DevStatus* ptrs[64] = {nullptr};
+  static int flag_written[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   if (ptrs[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dev_status) != cudaSuccess) return nullptr;
     ptrs[dev] = static_cast<DevStatus*>(p);
+    flag_written[dev] = -1;
+  }
+  const int want = check_mode() ? 1 : 0;
+  if (flag_written[dev] != want) {
+    if (cudaMemcpy(&ptrs[dev]->check, &want, sizeof(int), cudaMemcpyHostToDevice) == cudaSuccess)
+      flag_written[dev] = want;
   }
   return ptrs[dev];
+}
+
+// ------------------------------------------------ workspace canaries
+// MMH3_CHECK mode: a 256-byte canary follows each workspace region; fill
+// writes a position-dependent pattern, verify records DEV_CHECK_CANARY
+// (site: kernel * 16 + region) for the first word found changed.
+__global__ void canary_kernel(CanaryList l, int verify, int kernel_id, DevStatus* st) {
+  for (int i = threadIdx.x; i < l.n * (kCanaryBytes / 4); i += blockDim.x) {
+    uint32_t* p = l.p[i / (kCanaryBytes / 4)] + (i % (kCanaryBytes / 4));
+    const uint32_t want = 0xC0FFEE5Au ^ (uint32_t)i;
+    if (!verify)
+      *p = want;
+    else if (*p != want)
+      record_error(st, DEV_CHECK_CANARY, kernel_id * 16 + i / (kCanaryBytes / 4));
+  }
+}
+
+cudaError_t launch_canary(const CanaryList& l, bool verify, int kernel_id, cudaStream_t s) {
+  if (l.n == 0) return cudaSuccess;
+  canary_kernel<<<1, 256, 0, s>>>(l, verify ? 1 : 0, kernel_id, device_status_ptr());
+  count_launch();
+  return cudaGetLastError();
 }
 
 int num_sms() {
@@ -287,7 +318,7 @@ __global__ void __launch_bounds__(256) norm_mod_kernel(const float* __restrict__
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float inv = rsqrtf(ss / (float)H + eps);
   const float4* g4 = reinterpret_cast<const float4*>(g);
-  const float* m = mods ? mods + (size_t)seg_row(seg, row + row_base) * mods_stride : nullptr;
+  const float* m = mods ? mods + (size_t)seg_row_checked(seg, row + row_base) * mods_stride : nullptr;
   TO* o = out + (size_t)row * H;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
@@ -585,11 +616,13 @@ extern "C" mmh3_status mmh3_device_status(void* stream, int* code, int* site) {
   DevStatus h{};
   e = cudaMemcpy(&h, p, sizeof(h), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "device_status: read");
-  const DevStatus zero{};
-  e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+  const int zero[3] = {0, 0, 0};  // code, site, count; the check flag stays
+  e = cudaMemcpy(p, zero, sizeof(zero), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "device_status: clear");
   if (code) *code = h.code;
   if (site) *site = h.site;
+  if (h.code >= DEV_CHECK_ROW)
+    return fail(MMH3_ERR_CHECK, "a device check failed (code %d, site %d, %d records)", h.code, h.site, h.count);
   if (h.code != 0)
     return fail(MMH3_ERR_TIMEOUT, "a kernel gave up waiting (code %d, site %d, %d CTAs)", h.code, h.site,
                 h.count);

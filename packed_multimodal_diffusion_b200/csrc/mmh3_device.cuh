@@ -21,6 +21,16 @@ __device__ __forceinline__ void record_error(DevStatus* st, int code, int site) 
   atomicAdd(&st->count, 1);
 }
 
+// MMH3_CHECK mode: a TMA copy must start at an x coordinate whose byte
+// offset is a multiple of 16 and at non-negative coordinates (a load may
+// run past the far end: it reads zeros).  Returns false, recording the
+// coordinate, when a copy would break that.
+__device__ __forceinline__ bool tma_coords_ok(DevStatus* st, bool chk, int x, int y, int esize) {
+  if (!chk || (x >= 0 && y >= 0 && ((x * esize) & 15) == 0)) return true;
+  record_error(st, DEV_CHECK_TMA, y < 0 ? y : x);
+  return false;
+}
+
 // ------------------------------------------------------------------- helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

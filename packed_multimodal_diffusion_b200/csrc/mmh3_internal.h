@@ -21,6 +21,20 @@ void clear_error();
 bool fault_injected(const char* site);
 mmh3_status cuda_fail(cudaError_t e, const char* what);
 uint64_t wait_limit_ns();
+// MMH3_CHECK mode (MMH3_CHECK=1 in the environment, or mmh3_set_check):
+// device bounds checks and workspace canaries.
+bool check_mode();
+
+// Workspace canaries of the check mode: kCanaryBytes after each region.
+constexpr int kCanaryBytes = 256;
+constexpr int kMaxCanaries = 16;
+struct CanaryList {
+  uint32_t* p[kMaxCanaries];
+  int n;
+};
+// fill (verify = false) or verify the canaries; kernel_id names the kernel
+// that ran just before a verify (MMH3_PROF_K_*, 8 for the output heads)
+cudaError_t launch_canary(const CanaryList& l, bool verify, int kernel_id, cudaStream_t s);
 // Address of the device status word on the current device.
 DevStatus* device_status_ptr();
 int num_sms();

@@ -22,7 +22,7 @@ def declared_symbols():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        for m in re.finditer(r"^\s*(?:mmh3_status|double|void|long long|const char\s*\*)\s*(mmh3_\w+)\s*\(",
+        for m in re.finditer(r"^\s*(?:mmh3_status|double|void|int|long long|const char\s*\*)\s*(mmh3_\w+)\s*\(",
                              text, flags=re.M):
             names.add(m.group(1))
     return names
@@ -278,3 +278,33 @@ def test_layout_errors_and_more_than_two_timesteps_without_modulation():
                                    api.segments(L["segments"]), len(L["segments"]), nn, 0.3, sa,
                                    C.c_void_p(256), C.byref(out), None)
     assert rc == 5 and out.value == 4
+
+
+def test_check_mode_canaries_enlarge_the_workspace_and_clock_validation():
+    d = api.make_dims(256, 2, 128, 512)
+    base = api.workspace_size(d, 300)
+    try:
+        api.set_check(1)
+        assert _lib.load().mmh3_check_enabled() == 1
+        # nine regions, a 256-byte canary after each
+        assert api.workspace_size(d, 300) == base + 9 * 256
+    finally:
+        api.set_check(-1)
+    assert api.workspace_size(d, 300) == base
+    # a forged clock outside the four is refused by the host before any launch
+    with pytest.raises(_lib.Mmh3Error) as e:
+        api.plan_timesteps([(0, 4, 1, 0), (4, 9, 0, 7)], 9, 0.5, 0.2)
+    assert e.value.code == 1 and "clock 7" in str(e.value)
+
+
+def test_workspace_fault_injection_before_any_launch(monkeypatch):
+    lib = _lib.load()
+    d = api.make_dims(256, 2, 128, 512)
+    v = C.c_size_t()
+    assert lib.mmh3_workspace_size(C.byref(d), 300, C.byref(v)) == 0
+    w = _lib.BlockWeights(*([256] * 11))
+    segs = api.segments([(0, 300, 1, 0)])
+    monkeypatch.setenv("MMH3_FAULT", "workspace")
+    rc = lib.mmh3_block_forward(C.byref(d), C.byref(w), C.c_void_p(256), 300, segs, 1, None, 0.5, 0.2, 1, None,
+                                C.c_void_p(256), v.value, None)
+    assert rc == 4 and b"injected fault at workspace" in lib.mmh3_last_error()
