@@ -356,7 +356,9 @@ def run_gpu(args):
     xd = [torch.empty_like(W["x0"]) for _ in range(api.HOST_SLOTS)]
     pd = [torch.empty_like(W["pos_d"]) for _ in range(api.HOST_SLOTS)]
     copy_in, copy_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
-    e2e_steps = max(10, args.steps // 4)
+    # at least 30 steps: the first copy-in and the last copy-out (about
+    # 2.6 ms each at the block workload) are the pipeline's fill and drain
+    e2e_steps = max(30, args.steps)
     e2e_count = [0]
 
     def e2e_step():
