@@ -9,7 +9,7 @@ Bars (floating point):
     |gpu - ref| <= 2e-2 + 2^-7 |ref| -- rounding a value to bf16 alone moves
     it by up to 2^-8 |ref|, which exceeds 2e-2 for |ref| > 5.
   * fp32 modulation vectors: |gpu - oracle| <= 1e-4 |oracle| + 1e-6.
-  * fp32-storage path (tcgen05 kind::tf32 GEMMs, exact-fp32 attention):
+  * fp32-storage path (tcgen05 kind::tf32 GEMMs and attention):
     max-abs <= 5e-3 and cosine >= 0.99995, intermediates + 2^-10 |ref| --
     tf32 rounding (2^-11 relative per operand) is 16x finer than bf16's 2^-7,
     so the bf16 bar tightened by about that factor.

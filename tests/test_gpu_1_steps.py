@@ -142,15 +142,37 @@ def test_attention_multi_sequence(cuda_ok):
         assert_close(out[b * seq:(b + 1) * seq], ref, what=f"sequence {b}")
 
 
-def test_attention_fp32_tf32(cuda_ok):
-    n, heads, hd = 200, 2, 64
+@pytest.mark.parametrize("n_seq,seq,heads", [(1, 1, 1), (1, 64, 4), (1, 128, 1), (1, 129, 2), (1, 200, 2),
+                                             (1, 300, 1), (3, 100, 2)])
+def test_attention_fp32_tf32(cuda_ok, n_seq, seq, heads):
+    # the fp32-storage path on the tensor cores (kind::tf32): one key tile,
+    # ragged tiles, several tiles (online rescale) and several sequences
+    hd = 64
+    n = n_seq * seq
     qkv = _qkv(n, heads, hd, 21, dtype=torch.float32)
+    out = torch.full((n, heads * hd), float("nan"), dtype=torch.float32, device="cuda")
+    api.attention(qkv.cuda(), n_seq, seq, heads, hd, 1 / 8, out)
+    assert api.status_sync() == 0
+    for b in range(n_seq):
+        part = qkv[b * seq:(b + 1) * seq]
+        q, k, v = (f64(t).reshape(seq, heads, hd) for t in part.split(heads * hd, dim=1))
+        ref = O.attention(q, k, v, 1 / 8).reshape(seq, -1)
+        assert_close(out[b * seq:(b + 1) * seq], ref, TF32_MAXABS, TF32_COS, what=f"attention tf32 sequence {b}")
+
+
+def test_attention_fp32_tf32_growing_scores(cuda_ok):
+    # scores that grow along the keys: every key tile raises the row maximum,
+    # so O is rescaled on every tile
+    n, heads, hd = 384, 1, 64
+    qkv = _qkv(n, heads, hd, 23, dtype=torch.float32)
+    qkv[:, 0] = 1.0
+    qkv[:, heads * hd] = 0.01 * math.sqrt(hd) * torch.arange(n, dtype=torch.float32)
     out = torch.empty((n, heads * hd), dtype=torch.float32, device="cuda")
     api.attention(qkv.cuda(), 1, n, heads, hd, 1 / 8, out)
-    api.device_status()
+    assert api.status_sync() == 0
     q, k, v = (f64(t).reshape(n, heads, hd) for t in qkv.split(heads * hd, dim=1))
     ref = O.attention(q, k, v, 1 / 8).reshape(n, -1)
-    assert_close(out, ref, TF32_MAXABS, TF32_COS, what="attention tf32")
+    assert_close(out, ref, TF32_MAXABS, TF32_COS, what="attention tf32, growing scores")
 
 
 def test_bounded_wait_returns_timeout_and_context_survives(cuda_ok):
