@@ -1,12 +1,13 @@
 """The stack against the oracle, with real gates ("cortiq_engine/mmh3.rs",
 forward "blocks" and "heads").
 
-* Teacher-forced at the full stack workload (26 496 tokens, 50 blocks): the
-  GPU stack runs to block i - 1, and the oracle computes block i on the GPU's
-  own x_i for i in {0, 24, 49}, on sampled rows that span text, audio, video
-  and the ragged last tile (k and v for every token).  Block i's output and
-  its delta meet the block bars.  After block 49 both output heads are
-  compared on sampled rows of their streams.
+* Teacher-forced at the full stack workload (26 496 tokens, 50 blocks) and
+  the image workload (8 448 tokens, 50 blocks, one clock): the GPU stack runs
+  to block i - 1, and the oracle computes block i on the GPU's own x_i for
+  i in {0, 24, 49}, on sampled rows that span every segment and the ragged
+  last tile (k and v for every token).  Block i's output and its delta meet
+  the block bars.  After block 49 the output heads (video and audio; the
+  image head on the target image) are compared on sampled rows.
 * A whole 50-block chain at the tiny workload's shape (64 tokens), untruncated,
   in fp32 storage (tf32 GEMMs) and in bf16 storage, against the oracle's
   50-block chain.
@@ -39,15 +40,23 @@ def _host_weights(c, i, bp: api.BlockParams) -> dict:
     return p
 
 
-def test_stack_full_size_teacher_forced_blocks_and_heads(cuda_ok):
-    c = configs.STACK
-    segs, pos = api.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+@pytest.mark.parametrize("workload", ["stack", "image"])
+def test_stack_full_size_teacher_forced_blocks_and_heads(cuda_ok, workload):
+    c = configs.CONFIGS[workload]
+    if c.image_mode:
+        # one clock, two tags; the head reads the target image's rows
+        segs, pos = api.layout_image(c.text_len, c.ref_lat_h, c.ref_lat_w, c.lat_h, c.lat_w)
+        hc = configs.DitConfig(c.name, c.cfg_seed, hidden=c.hidden, heads=c.heads, head_dim=c.head_dim,
+                               ffn=c.ffn, text_len=c.text_len, heads_out=128)
+    else:
+        segs, pos = api.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+        hc = c
     n = pos.shape[0]
-    assert n == 26496
+    assert n == {"stack": 26496, "image": 8448}[workload]
     dims = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn)
     blocks = [api.BlockParams.from_host(dims, configs.block_weights(c, b, device="cuda"), device="cuda")
               for b in range(c.n_blocks)]
-    hw = configs.head_weights(c, device="cuda")
+    hw = configs.head_weights(hc, device="cuda")
     heads = api.HeadParams.from_host(hw, device="cuda")
     x = configs.hidden_states(c, device="cuda")
     pd = torch.as_tensor(pos.astype(np.float32)).cuda()
@@ -84,13 +93,14 @@ def test_stack_full_size_teacher_forced_blocks_and_heads(cuda_ok):
     assert done == c.n_blocks
     # the heads on the GPU's final hidden states
     vs = [s for s in segs if s[2] == 0][-1]
-    as_ = [s for s in segs if s[2] == 2][-1]
+    a_segs = [s for s in segs if s[2] == 2]
     ov = torch.full((vs[1] - vs[0], 128), float("nan"), device="cuda")
-    oa = torch.full((as_[1] - as_[0], 128), float("nan"), device="cuda")
+    oa = torch.full((a_segs[-1][1] - a_segs[-1][0], 128), float("nan"), device="cuda") if a_segs else None
     api.stack_forward(dims, [], heads, xi, segs, pd, sv, sa, ov, oa, ws)
     api.device_status()
     fm = O.final_mods(f64(hw["adaln_w"]), f64(hw["adaln_b"]), f64(hw["adaln_table"]), ts, c.hidden)
-    for (seg, key, out) in ((vs, "video", ov), (as_, "audio", oa)):
+    streams = [(vs, "video", ov)] + ([(a_segs[-1], "audio", oa)] if a_segs else [])
+    for (seg, key, out) in streams:
         r = np.unique(np.concatenate([np.linspace(seg[0], seg[1] - 1, 9).astype(int),
                                       [seg[1] - 1, seg[1] - 2]]))
         ref = O.heads_forward(f64(xi[r]), f64(hw["final_norm"]), fm[slot[seg[3]]],
