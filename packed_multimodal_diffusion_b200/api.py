@@ -22,8 +22,10 @@ __all__ = ["Dims", "Segment", "make_dims", "segments", "layout_t2va", "layout_im
            "block_forward", "stack_forward", "block_forward_host", "block_cp_begin", "block_cp_end", "refine_workspace_size", "refine_text",
            "patch_embed_workspace_size", "patch_embed", "embed_workspace_size", "embed",
            "unpatchify_video", "unpack_audio", "forward_workspace_size", "forward", "VitParams", "vit_fold_qkv", "vit_workspace_size",
-           "vit_layer_forward", "device_status", "selftest_wait_timeout", "set_wait_limit_ns",
-           "MMH3_BF16", "MMH3_F32"]
+           "vit_layer_forward", "vit_dims", "layout_fl2va", "layout_ref2va", "block_forward_noalloc",
+           "workspace_regions", "device_status", "status_sync", "set_check", "selftest_wait_timeout",
+           "set_wait_limit_ns", "launch_count", "prof_enable", "prof_reset", "prof_collect",
+           "prof_collect_kernels", "MMH3_BF16", "MMH3_F32"]
 
 
 def _stream() -> int:
