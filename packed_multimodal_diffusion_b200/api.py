@@ -538,7 +538,7 @@ def workspace_regions(dims: Dims, n: int, ws: torch.Tensor) -> dict:
     es = 2 if dims.act_dtype == MMH3_BF16 else 4
     a256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
     sizes = [("mods", 2 * 3 * 6 * H * 4, torch.float32, (6, 6 * H)),
-             ("cs", n * 3 * dims.rope_k * 8, torch.float32, (n, 3 * dims.rope_k, 2)),
+             ("cs", n * 3 * dims.rope_k * 8, torch.float32, (3 * dims.rope_k, n, 2)),
              ("xn1", n * H * es, act, (n, H)), ("qkv", n * 3 * I * es, act, (n, 3 * I)),
              ("attn", n * I * es, act, (n, I)), ("xn2", n * H * es, act, (n, H)),
              ("act", n * F * es, act, (n, F)), ("head", n * H * es, act, (n, H)),

@@ -266,7 +266,8 @@ struct EpiQkvNormRope {
   int inner;         // heads * HD
   const float* q_norm;
   const float* k_norm;
-  const float2* cs;  // [M, kPairs] (cos, sin), or null: no rotation
+  const float2* cs;  // frequency-major [kPairs, cs_ld] (cos, sin), or null: no rotation
+  int cs_ld;         // rows of the table (the GEMM's M)
   float eps;
   static constexpr int kPairs = 3 * (HD / 8);
   static constexpr int kG = HD / 8;
@@ -317,10 +318,10 @@ struct EpiQkvNormRope {
           ld_acc<kG>(th + j0, lo);
           ld_acc<kG>(th + j0 + kPairs, hi);
           if (row_ok) {
-            const float2* c2 = cs + (size_t)row * kPairs + j0;
+            const float2* c2 = cs + (size_t)j0 * cs_ld + row;
 #pragma unroll
             for (int i = 0; i < kG; ++i) {
-              const float2 e = __ldg(c2 + i);
+              const float2 e = __ldg(c2 + (size_t)i * cs_ld);
               const float yl = lo[i] * inv * w[j0 + i];
               const float yh = hi[i] * inv * w[j0 + kPairs + i];
               lo[i] = yl * e.x - yh * e.y;
@@ -365,7 +366,8 @@ struct EpiQkvNormRopeTma {
   int inner;
   const float* q_norm;
   const float* k_norm;
-  const float2* cs;
+  const float2* cs;  // frequency-major [kPairs, cs_ld] (cos, sin)
+  int cs_ld;         // rows of the table (the GEMM's M)
   float eps;
   static constexpr int HD = 128;
   static constexpr int kPairs = 3 * (HD / 8);  // 48
@@ -415,10 +417,10 @@ struct EpiQkvNormRopeTma {
         float lo[kG], hi[kG];
         ld_acc<kG>(th + j0, lo);
         ld_acc<kG>(th + j0 + kPairs, hi);
-        const float2* c2 = cs + (size_t)(row_ok ? row : 0) * kPairs + j0;
+        const float2* c2 = cs + (size_t)j0 * cs_ld + (row_ok ? row : 0);
 #pragma unroll
         for (int i = 0; i < kG; ++i) {
-          const float2 e = cs ? __ldg(c2 + i) : make_float2(1.f, 0.f);
+          const float2 e = cs ? __ldg(c2 + (size_t)i * cs_ld) : make_float2(1.f, 0.f);
           const float yl = lo[i] * inv * w[j0 + i];
           const float yh = hi[i] * inv * w[j0 + kPairs + i];
           lo[i] = yl * e.x - yh * e.y;

@@ -201,14 +201,17 @@ __global__ void __launch_bounds__(256, 4)
     __syncwarp();
   }
   if constexpr (K > 0) {
-    // rotation table: 256 entries per warp item, grid-stride
+    // rotation table, frequency-major: entry e = j * n + i holds pair j of
+    // row i, so a warp writes (and the qkv epilogue, one row per lane, later
+    // reads) 32 consecutive rows of one pair as one contiguous run.  256
+    // entries per warp item, grid-stride.
     const unsigned cs_total = (unsigned)n * 3u * K;  // < 2^31 (checked by the host)
     for (unsigned e0 = (unsigned)gw * 256u; e0 < cs_total; e0 += (unsigned)n_warps * 256u) {
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const unsigned e = e0 + u * 32 + lane;
         if (e < cs_total) {
-          const unsigned i = e / (3u * K), j = e % (3u * K);
+          const unsigned j = e / (unsigned)n, i = e - j * (unsigned)n;
           const float a = (float)((double)pos[i * 3 + j / K] * (double)sinv[j % K]);
           float sv, cv;
           sincosf(a, &sv, &cv);
@@ -282,9 +285,21 @@ cudaError_t launch_adaln(const float* w, const float* b, const float* table, int
 }
 
 // ------------------------------------------- K2 RMSNorm + modulate gather
-// One warp per token row; VPL float4 per lane (H = 128 * VPL).  Row i reads
-// modulation row seg_row(i + row_base): y = (x * rsqrt(mean x^2 + eps) * g)
-// * (1 + scale) + shift, stored as the GEMM operand dtype.
+// y = (x * rsqrt(mean x^2 + eps) * g) * (1 + scale) + shift for each token
+// row i, with shift / scale from modulation row seg_row(i + row_base),
+// stored as the GEMM operand dtype.  H = 128 * VPL (VPL float4 per lane).
+//
+// Persistent and streaming: warp w of the grid takes rows w, w + W, ...
+// (W warps in all).  Each warp owns kNormStages row buffers in shared memory;
+// its lane 0 fetches rows into them with 1-D bulk copies (evict-first in L2,
+// so the normalised output, which the next GEMM reads, stays there longer).
+// A warp copies the current row from shared memory into registers, hands
+// the buffer to the copy kNormStages rows ahead and normalises from
+// registers, so two rows per warp are in flight while it computes.
+constexpr int kNormStages = 2;
+constexpr size_t kNormSmemBudget = 220 * 1024;
+constexpr int kNormMaxWarps = 8;
+
 __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
   uint2 u;
   u.x = pack_bf16x2(v.x, v.y);
@@ -294,66 +309,152 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 __device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
 template <typename TO, int VPL>
-__global__ void __launch_bounds__(256) norm_mod_kernel(const float* __restrict__ x, int n, int H,
-                                                       const float* __restrict__ g, float eps,
-                                                       const float* __restrict__ mods,
-                                                       int mods_stride, int shift_off,
-                                                       int scale_off, SegRows seg, int row_base,
-                                                       TO* __restrict__ out) {
+__global__ void __launch_bounds__(kNormMaxWarps * 32, 1)
+    norm_mod_kernel(const float* __restrict__ x, int n, int H, const float* __restrict__ g, float eps,
+                    const float* __restrict__ mods, int mods_stride, int shift_off, int scale_off, SegRows seg,
+                    int row_base, TO* __restrict__ out, DevStatus* status, uint64_t limit_ns) {
+  constexpr uint32_t kRowBytes = VPL * 512;
+  extern __shared__ __align__(128) uint8_t norm_smem[];
+  const int warps = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (row >= n) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * H);
-  float4 v[VPL];
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    v[i] = __ldcs(xr + i * 32 + lane);
-    ss = fmaf(v[i].x, v[i].x, ss);
-    ss = fmaf(v[i].y, v[i].y, ss);
-    ss = fmaf(v[i].z, v[i].z, ss);
-    ss = fmaf(v[i].w, v[i].w, ss);
+  const float4* buf = reinterpret_cast<const float4*>(norm_smem + (size_t)warp * kNormStages * kRowBytes);
+  const uint32_t buf_s = smem_u32(buf);
+  const uint32_t bar0 = smem_u32(norm_smem + (size_t)warps * kNormStages * kRowBytes) + 8u * kNormStages * warp;
+  const long long W = (long long)gridDim.x * warps;
+  const long long gw = (long long)blockIdx.x * warps + warp;
+  const int cnt = gw < n ? (int)((n - 1 - gw) / W) + 1 : 0;  // rows of this warp
+  if (cnt == 0) return;  // warp-uniform; the kernel has no CTA-wide barrier
+  uint64_t policy = 0;
+  if (lane == 0) {
+    for (int st = 0; st < kNormStages; ++st) mbar_init(bar0 + 8u * st, 1);
+    fence_mbar_init();
+    policy = policy_evict_first();
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float inv = rsqrtf(ss / (float)H + eps);
+  __syncwarp();
+  auto issue = [&](int i) {  // lane 0: row i of this warp into buffer i % kNormStages
+    const uint32_t st = (uint32_t)(i % kNormStages);
+    mbar_expect_tx(bar0 + 8u * st, kRowBytes);
+    bulk_load_1d(buf_s + st * kRowBytes, x + (size_t)(gw + (long long)i * W) * H, kRowBytes, bar0 + 8u * st,
+                 policy);
+  };
+  if (lane == 0)
+    for (int i = 0; i < kNormStages && i < cnt; ++i) issue(i);
   const float4* g4 = reinterpret_cast<const float4*>(g);
-  const float* m = mods ? mods + (size_t)seg_row_checked(seg, row + row_base) * mods_stride : nullptr;
-  TO* o = out + (size_t)row * H;
+  int i = 0;
+  for (; i < cnt; ++i) {
+    const int st = i % kNormStages;
+    const bool fail = !mbar_wait(bar0 + 8u * st, (uint32_t)((i / kNormStages) & 1), limit_ns);
+    if (__any_sync(0xffffffffu, fail)) break;
+    float4 v[VPL];
+    float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int c4 = i * 32 + lane;
-    const float4 gg = __ldg(g4 + c4);
-    float4 y = make_float4(v[i].x * inv * gg.x, v[i].y * inv * gg.y, v[i].z * inv * gg.z,
-                           v[i].w * inv * gg.w);
-    if (m) {
-      const float4 sh = __ldg(reinterpret_cast<const float4*>(m + shift_off) + c4);
-      const float4 sc = __ldg(reinterpret_cast<const float4*>(m + scale_off) + c4);
-      y.x = fmaf(y.x, 1.0f + sc.x, sh.x);
-      y.y = fmaf(y.y, 1.0f + sc.y, sh.y);
-      y.z = fmaf(y.z, 1.0f + sc.z, sh.z);
-      y.w = fmaf(y.w, 1.0f + sc.w, sh.w);
+    for (int k = 0; k < VPL; ++k) v[k] = buf[st * (VPL * 32) + k * 32 + lane];
+    // every lane holds its part of the row: the buffer takes the next copy
+    // (the proxy fence orders these reads before the copy's writes)
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && i + kNormStages < cnt) issue(i + kNormStages);
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      ss = fmaf(v[k].x, v[k].x, ss);
+      ss = fmaf(v[k].y, v[k].y, ss);
+      ss = fmaf(v[k].z, v[k].z, ss);
+      ss = fmaf(v[k].w, v[k].w, ss);
     }
-    store4(o + 4 * c4, y);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = rsqrtf(ss / (float)H + eps);
+    const int row = (int)(gw + (long long)i * W);
+    const float* m = mods ? mods + (size_t)seg_row_checked(seg, row + row_base) * mods_stride : nullptr;
+    TO* o = out + (size_t)row * H;
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) {
+      const int c4 = k * 32 + lane;
+      const float4 gg = __ldg(g4 + c4);
+      float4 y = make_float4(v[k].x * inv * gg.x, v[k].y * inv * gg.y, v[k].z * inv * gg.z,
+                             v[k].w * inv * gg.w);
+      if (m) {
+        const float4 sh = __ldg(reinterpret_cast<const float4*>(m + shift_off) + c4);
+        const float4 sc = __ldg(reinterpret_cast<const float4*>(m + scale_off) + c4);
+        y.x = fmaf(y.x, 1.0f + sc.x, sh.x);
+        y.y = fmaf(y.y, 1.0f + sc.y, sh.y);
+        y.z = fmaf(y.z, 1.0f + sc.z, sh.z);
+        y.w = fmaf(y.w, 1.0f + sc.w, sh.w);
+      }
+      store4(o + 4 * c4, y);
+    }
   }
+  if (i < cnt && lane == 0) {
+    // gave up on row i: record it, then let the copies still in flight land
+    // (bounded) before the CTA's shared memory is released
+    record_error(status, DEV_TIMEOUT_COPY, (int)(gw + (long long)i * W));
+    for (int k = i; k < cnt && k < i + kNormStages; ++k)
+      mbar_wait(bar0 + 8u * (uint32_t)(k % kNormStages), (uint32_t)((k / kNormStages) & 1), limit_ns);
+  }
+}
+
+// Warps per CTA: as many as the row buffers' shared memory allows (at most
+// kNormMaxWarps; more warps would cap a thread's registers at 168 and
+// spill), fewer only where that leaves a fuller last round of rows (e.g.
+// 13 248 rows on 148 SMs: seven warps a CTA give 13 rounds, 98% full,
+// against 12 rounds, 93% full, with eight).
+template <typename TO, int VPL>
+static cudaError_t norm_mod_launch(const float* x, int n, int H, const float* g, float eps, const float* mods,
+                                   int ms, int so, int co, const SegRows& seg, int rb, TO* out, cudaStream_t s) {
+  constexpr size_t kWarpBytes = (size_t)kNormStages * (VPL * 512 + 8);
+  constexpr int kWarps = kNormSmemBudget / kWarpBytes >= kNormMaxWarps ? kNormMaxWarps
+                                                                         : (int)(kNormSmemBudget / kWarpBytes);
+  static_assert(kWarps >= 1, "RMSNorm row buffers above the shared-memory budget");
+  auto kern = norm_mod_kernel<TO, VPL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kWarps * kWarpBytes));
+  if (e != cudaSuccess) return e;
+  static int per_sm[64][kNormMaxWarps + 1];  // CTAs per SM by warps per CTA (0: not yet asked)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  const long long sms = num_sms();
+  int warps = kWarps, ctas_per_sm = 1;
+  double best = -1.0;
+  for (int w = kWarps; w >= 1 && w >= kWarps - 4; --w) {
+    if (per_sm[dev][w] == 0) {
+      int v = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, w * 32, w * kWarpBytes);
+      if (e != cudaSuccess) return e;
+      per_sm[dev][w] = v > 0 ? v : 1;
+    }
+    const long long lanes = sms * per_sm[dev][w] * w;  // warps resident at once
+    const long long rounds = ((long long)n + lanes - 1) / lanes;
+    const double full = (double)n / (double)(rounds * lanes);
+    if (full > best + 0.02) {
+      best = full;
+      warps = w;
+      ctas_per_sm = per_sm[dev][w];
+    }
+    if (rounds == 1) break;  // one round: fewer warps a CTA only spread the same rows thinner
+  }
+  const long long want = ((long long)n + warps - 1) / warps;
+  const long long cap = sms * ctas_per_sm;
+  const int blocks = (int)(want < cap ? want : cap);
+  kern<<<blocks, warps * 32, warps * kWarpBytes, s>>>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out,
+                                                      device_status_ptr(), wait_limit_ns());
+  count_launch();
+  return cudaGetLastError();
 }
 
 template <typename TO>
 static cudaError_t norm_mod_dispatch(const float* x, int n, int H, const float* g, float eps,
                                      const float* mods, int ms, int so, int co, const SegRows& seg,
                                      int rb, TO* out, cudaStream_t s) {
-  const int blocks = (n + 7) / 8;
   switch (H / 128) {
 #define MMH3_NM(V) \
   case V:          \
-    norm_mod_kernel<TO, V><<<blocks, 256, 0, s>>>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out); count_launch(); break;
+    return norm_mod_launch<TO, V>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out, s);
     MMH3_NM(1) MMH3_NM(2) MMH3_NM(4) MMH3_NM(6) MMH3_NM(8) MMH3_NM(16) MMH3_NM(21) MMH3_NM(24)
     MMH3_NM(32)
 #undef MMH3_NM
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_norm_mod(int dtype, const float* x, int n, int H, const float* g, float eps,
@@ -621,7 +722,7 @@ extern "C" mmh3_status mmh3_device_status(void* stream, int* code, int* site) {
   if (e != cudaSuccess) return cuda_fail(e, "device_status: clear");
   if (code) *code = h.code;
   if (site) *site = h.site;
-  if (h.code >= DEV_CHECK_ROW)
+  if (dev_err_is_check(h.code))
     return fail(MMH3_ERR_CHECK, "a device check failed (code %d, site %d, %d records)", h.code, h.site, h.count);
   if (h.code != 0)
     return fail(MMH3_ERR_TIMEOUT, "a kernel gave up waiting (code %d, site %d, %d CTAs)", h.code, h.site,

@@ -207,22 +207,22 @@ mmh3_status gemm_qkv(int dtype, const void* A, const void* B, int M, int N, int 
                      float eps, void* out, cudaStream_t s) {
   if (dtype == MMH3_BF16 && head_dim == 128) {
     if (use_pairs(M, N, 256)) {
-      EpiQkvNormRopeTma<256> e{N, inner, q_norm, k_norm, cs, eps};
+      EpiQkvNormRopeTma<256> e{N, inner, q_norm, k_norm, cs, M, eps};
       return run_gemm2<256>(A, B, M, N, K, e, s, out, N);
     }
-    EpiQkvNormRope<__nv_bfloat16, 128, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, eps};
+    EpiQkvNormRope<__nv_bfloat16, 128, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, M, eps};
     return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
   }
   if (dtype == MMH3_BF16 && head_dim == 64) {
-    EpiQkvNormRope<__nv_bfloat16, 64, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, eps};
+    EpiQkvNormRope<__nv_bfloat16, 64, 256> e{static_cast<__nv_bfloat16*>(out), N, inner, q_norm, k_norm, cs, M, eps};
     return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
   }
   if (dtype == MMH3_F32 && head_dim == 64) {
-    EpiQkvNormRope<float, 64, 256> e{static_cast<float*>(out), N, inner, q_norm, k_norm, cs, eps};
+    EpiQkvNormRope<float, 64, 256> e{static_cast<float*>(out), N, inner, q_norm, k_norm, cs, M, eps};
     return run_gemm<float, 256>(A, B, M, N, K, e, s);
   }
   if (dtype == MMH3_F32 && head_dim == 128) {
-    EpiQkvNormRope<float, 128, 256> e{static_cast<float*>(out), N, inner, q_norm, k_norm, cs, eps};
+    EpiQkvNormRope<float, 128, 256> e{static_cast<float*>(out), N, inner, q_norm, k_norm, cs, M, eps};
     return run_gemm<float, 256>(A, B, M, N, K, e, s);
   }
   return fail(MMH3_ERR_SHAPE, "qkv: head_dim %d unsupported", head_dim);

@@ -118,6 +118,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// L2 policy that marks the lines a load brings in as first to evict (data
+// read once, e.g. a row normalised and never read again by this kernel).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 1-D bulk copy (no tensor map) of `bytes` from global to shared memory,
+// completing on `bar`.  Both addresses 16-byte aligned, bytes a multiple of
+// 16 and below 2^20 (one mbarrier phase's transaction count).
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                             uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy (the
 // tensor core reads operands through it).
 __device__ __forceinline__ void fence_proxy_async_smem() {

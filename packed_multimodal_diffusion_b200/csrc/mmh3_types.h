@@ -20,7 +20,12 @@ enum DevErr : int {
   DEV_CHECK_ROW = 6,     // a token's modulation row outside [0, rows)
   DEV_CHECK_TMA = 7,     // a TMA copy at an unaligned or negative coordinate
   DEV_CHECK_CANARY = 8,  // a workspace canary overwritten (site: kernel * 16 + region)
+  DEV_TIMEOUT_COPY = 9,  // a bulk row copy that never landed (site: the row)
 };
+
+__host__ __device__ __forceinline__ bool dev_err_is_check(int code) {
+  return code >= DEV_CHECK_ROW && code <= DEV_CHECK_CANARY;
+}
 
 struct DevStatus {
   int code;   // first DevErr recorded (0 = none)
