@@ -418,8 +418,9 @@ def run_gpu(args):
                      "frac_burst": achieved / peaks["bf16_tflops"],
                      "frac_sustained": achieved / peaks["bf16_tflops_sustained"],
                      "traffic": traffic,
-                     "traffic_unit": ("bytes per attention step (whole-unit launch, split-tail launch and "
-                                      "merge when the last wave is split)" if dom == "attention"
+                     "traffic_unit": ("bytes per attention step (the attention launch, whole units and "
+                                      "split tail in one grid, and the merge when the tail is split)"
+                                      if dom == "attention"
                                       else "bytes/launch"),
                      "algorithmic_bytes": 2 * n * 3 * 2688 + 2 * n * 2688},
         "phases_ms_per_block": {k: round(v / max(1, nblocks), 4) for k, v in phases.items()},

@@ -267,7 +267,8 @@ mmh3_status mmh3_attention(const void* qkv, int n_seq, int seq, int heads, int h
  * when that shortens the wave enough: f in 2..8 minimises
  * ceil(tail * f / SMs) / f, each piece keeps at least 32 key tiles of 128,
  * and the split is made only if the tail's time drops to 0.6 of a unit or
- * less.  The CTAs' partial results (unnormalised O,
+ * less.  The pieces run in the same launch as the whole units, after them,
+ * so the SMs that finish first take them.  The CTAs' partial results (unnormalised O,
  * running maximum, row sum: 256 x (head_dim + 4) fp32 per CTA) go to scratch
  * and are then merged.  Without room in scratch (or with scratch NULL)
  * nothing is split.  The result equals mmh3_attention's up to the order of

@@ -107,7 +107,7 @@ template <int HD>
 __global__ void __launch_bounds__(320, 1)
     attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tmkv,
                     __nv_bfloat16* __restrict__ out, int ldo, int seq, int seq_kv, int k_off, int v_off,
-                    float scale_log2, int heads, int unit0, int split, float* __restrict__ part,
+                    float scale_log2, int heads, int whole, int split, float* __restrict__ part,
                     DevStatus* status, uint64_t limit_ns) {
   using Sh = Attn2Shape<HD>;
   constexpr int KV = Sh::kKV;
@@ -133,13 +133,18 @@ __global__ void __launch_bounds__(320, 1)
   // Keys / values: rows [z*seq_kv, (z+1)*seq_kv) of `tmkv`, k at column
   // k_off, v at v_off (the same panel for a whole sequence on one GPU; the
   // gathered K|V rows of all ranks for a sequence split over ranks).
-  // Work unit u = unit0 + blockIdx.x / split: 256 query rows (q pair) of one
-  // head of one sequence.  With split > 1 the unit's key tiles are divided
-  // into `split` contiguous ranges, one per CTA, and each CTA writes its
-  // unnormalised partial result to `part` for attn_merge_kernel.
+  // Work unit: 256 query rows (q pair) of one head of one sequence.  CTAs
+  // [0, whole) compute whole units u = blockIdx.x.  The rest are the tail:
+  // CTA whole + b, b = t * split + piece, computes key range `piece` of the
+  // `split` contiguous ranges of unit whole + t and writes its unnormalised
+  // partial result to part slot b for attn_merge_kernel.  One grid holds
+  // both, so the hardware hands tail pieces to the SMs that finish their
+  // whole units first.
   const int nq = (seq + 255) / 256;
-  const int u = unit0 + (int)blockIdx.x / split;
-  const int piece = (int)blockIdx.x % split;
+  const int tb = (int)blockIdx.x - whole;  // tail CTA index; < 0: a whole unit
+  const int sp = tb < 0 ? 1 : split;
+  const int u = tb < 0 ? (int)blockIdx.x : whole + tb / split;
+  const int piece = tb < 0 ? 0 : tb % split;
   const int qpair = u % nq;
   const int head = (u / nq) % heads;
   const int zseq = u / (nq * heads);
@@ -147,8 +152,8 @@ __global__ void __launch_bounds__(320, 1)
   const int kv_row0 = zseq * seq_kv;
   const int q_row0 = seq_row0 + qpair * 256;
   const int kv_tiles = (seq_kv + 127) / 128;
-  const int j0 = piece * kv_tiles / split;              // first key tile of this CTA
-  const int n_kv = (piece + 1) * kv_tiles / split - j0;  // key tiles of this CTA (>= 1)
+  const int j0 = piece * kv_tiles / sp;              // first key tile of this CTA
+  const int n_kv = (piece + 1) * kv_tiles / sp - j0;  // key tiles of this CTA (>= 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q), 1);
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const int qr = qpair * 256 + wg * 128 + r;
       const bool row_ok = qr < seq;
-      if (split == 1) {
+      if (sp == 1) {
         const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
         __nv_bfloat16* dst = out + (size_t)(seq_row0 + qr) * ldo + head * HD;
 #pragma unroll 1
@@ -431,7 +436,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       } else {
         // partial: O unnormalised (relative to m_ref), then m_ref and l_sum
-        float* dst = part + ((size_t)blockIdx.x * 256 + wg * 128 + r) * Attn2Shape<HD>::kPartStride;
+        float* dst = part + ((size_t)tb * 256 + wg * 128 + r) * Attn2Shape<HD>::kPartStride;
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           float v[32];

@@ -174,8 +174,8 @@ def test_block_forward_host_pipelined_matches_device_calls(cuda_ok):
 
 def test_launch_count_of_one_block(cuda_ok):
     # prologue (adaLN curve + rotation table), 2 x norm/modulate, 4 GEMMs,
-    # attention: 8 kernels (attention adds a split launch and a merge when
-    # its last wave is split)
+    # attention: 8 kernels (attention adds a merge launch when its last wave
+    # is split)
     dims_o, dims_c = small_dims()
     segs, pos = t2va(20, 3, 16, 20, 20)
     n = int(pos.shape[0])
