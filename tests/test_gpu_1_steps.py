@@ -199,7 +199,10 @@ def test_attention_split_tail(cuda_ok, n_seq, seq, heads, hd):
     scale = 1 / math.sqrt(hd)
     out = torch.full((n, heads * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
     scratch = torch.empty(160 * 256 * (hd + 4) * 4, dtype=torch.uint8, device="cuda")
+    c0 = api.launch_count()
     api.attention_ws(qkv, n_seq, seq, heads, hd, scale, out, scratch)
+    # the whole units and the split tail are one grid; a split adds only the merge
+    assert api.launch_count() - c0 == (1 if seq == 700 else 2)
     plain = torch.empty_like(out)
     api.attention(qkv, n_seq, seq, heads, hd, scale, plain)
     api.device_status()
