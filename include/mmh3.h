@@ -656,8 +656,8 @@ void mmh3_prof_reset(void);
  * holds the prologue and both RMSNorm + modulate launches).  The prologue
  * is one launch that evaluates the adaLN curve of one block (of up to 64
  * blocks at once in mmh3_stack_forward) and writes the rotation table.
- * Attention counts its whole step (the main launch and, when its last wave
- * is split, the tail launch and the merge). */
+ * Attention counts its whole step (its launch, whole units and any split
+ * tail in one grid, and the merge when the tail is split). */
 #define MMH3_PROF_K_PROLOGUE 0 /* adaLN curve -> modulation, rotation table */
 #define MMH3_PROF_K_NORM1 1    /* segment gather + RMSNorm(norm1) + modulate */
 #define MMH3_PROF_K_QKV 2      /* qkv GEMM + qk-norm + rotation */
