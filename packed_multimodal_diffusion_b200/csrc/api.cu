@@ -321,7 +321,6 @@ mmh3_status mmh3::block_forward_impl(const mmh3_dims* dims, const mmh3_block_wei
     }
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int H = dims->hidden;
   PhaseMark pm(s, profile);
   st = canaries(ws, false, 0, s);
   if (st != MMH3_OK) return st;

@@ -179,6 +179,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
   // S_i at columns 128 i, O_i at 256 + HD i
   auto t_s = [&](int i) { return tmem + 128u * i; };
   auto t_o = [&](int i) { return tmem + 256u + (uint32_t)HD * i; };
@@ -467,6 +469,8 @@ template <int HD>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ part, int split,
                                                          __nv_bfloat16* __restrict__ out, int ldo, int seq,
                                                          int heads, int unit0) {
+  pdl_launch_dependents();
+  pdl_wait();
   static_assert(HD == 128 || HD == 64, "head_dim");
   constexpr int kLaneCols = HD / 32;  // 4 or 2
   const int nq = (seq + 255) / 256;

@@ -812,6 +812,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
 
   const int m_tiles = (M + Sh::BM - 1) / Sh::BM;
   const int n_tiles = (N + BN - 1) / BN;
@@ -1067,6 +1069,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
 
   const int m_tiles = (M + 2 * Sh::BM - 1) / (2 * Sh::BM);
   const int n_tiles = (N + BN - 1) / BN;

@@ -330,14 +330,16 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
   // one grid: the whole units first, then the tail pieces (dispatched in
   // block order, so SMs that finish early take the pieces)
   float* part = split ? static_cast<float*>(scratch) : nullptr;
-  kern<<<whole + (split ? tail * f : 0), Sh::kThreads, Sh::kSmem, s>>>(
-      tm, tkv, o, inner, seq, seq_kv, k_off, v_off, sl2, heads, whole, f, part, device_status_ptr(), wait_limit_ns());
+  e = launch_pdl(kern, dim3(whole + (split ? tail * f : 0)), dim3(Sh::kThreads), Sh::kSmem, s, tm, tkv, o, inner, seq,
+                 seq_kv, k_off, v_off, sl2, heads, whole, f, part, device_status_ptr(), wait_limit_ns());
   count_launch();
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (split) {
-    attn_merge_kernel<HD><<<tail * 32, 256, 0, s>>>(part, f, o, inner, seq, heads, units - tail); count_launch();
-    e = cudaGetLastError();
+    e = launch_pdl(attn_merge_kernel<HD>, dim3(tail * 32), dim3(256), 0, s, part, f, o, inner, seq, heads,
+                   units - tail);
+    count_launch();
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "attention merge launch");
   }
   return MMH3_OK;

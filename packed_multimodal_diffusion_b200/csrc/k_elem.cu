@@ -141,6 +141,8 @@ __global__ void __launch_bounds__(256, 4)
     prologue_kernel(AdalnBatch ab, int n_ab, int rank, int rows_per_slot, int n_ts, CurveArgs ca,
                     float* __restrict__ mods, long long mods_stride, const float* __restrict__ pos, int n,
                     InvFreq inv, float2* __restrict__ cs) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ __align__(16) float part[8][32 * 8];
   __shared__ __align__(16) float coord[8][32];
   __shared__ float sinv[K > 0 ? K : 1];
@@ -260,19 +262,20 @@ cudaError_t launch_prologue(const AdalnBatch& ab, int n_ab, int rank, int grid, 
   long long blocks = (items + 7) / 8;
   if (blocks > (long long)num_sms() * 4) blocks = (long long)num_sms() * 4;  // 32 warps per SM
   const int g = (int)blocks;
+  cudaError_t e;
   if (kk == 16)
-    prologue_kernel<16><<<g, 256, 0, s>>>(ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods, mods_stride, pos, n,
-                                          inv, cs);
+    e = launch_pdl(prologue_kernel<16>, dim3(g), dim3(256), 0, s, ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods,
+                   mods_stride, pos, n, inv, cs);
   else if (kk == 8)
-    prologue_kernel<8><<<g, 256, 0, s>>>(ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods, mods_stride, pos, n,
-                                         inv, cs);
+    e = launch_pdl(prologue_kernel<8>, dim3(g), dim3(256), 0, s, ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods,
+                   mods_stride, pos, n, inv, cs);
   else if (kk == 0)
-    prologue_kernel<0><<<g, 256, 0, s>>>(ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods, mods_stride, pos, n,
-                                         inv, cs);
+    e = launch_pdl(prologue_kernel<0>, dim3(g), dim3(256), 0, s, ab, n_ab, rank, rows_per_slot, plan.n_ts, ca, mods,
+                   mods_stride, pos, n, inv, cs);
   else
     return cudaErrorInvalidValue;
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_adaln(const float* w, const float* b, const float* table, int rank, int grid,
@@ -313,6 +316,8 @@ __global__ void __launch_bounds__(kNormMaxWarps * 32, 1)
     norm_mod_kernel(const float* __restrict__ x, int n, int H, const float* __restrict__ g, float eps,
                     const float* __restrict__ mods, int mods_stride, int shift_off, int scale_off, SegRows seg,
                     int row_base, TO* __restrict__ out, DevStatus* status, uint64_t limit_ns) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr uint32_t kRowBytes = VPL * 512;
   extern __shared__ __align__(128) uint8_t norm_smem[];
   const int warps = blockDim.x >> 5;
@@ -435,9 +440,10 @@ static cudaError_t norm_mod_launch(const float* x, int n, int H, const float* g,
   const long long want = ((long long)n + warps - 1) / warps;
   const long long cap = sms * ctas_per_sm;
   const int blocks = (int)(want < cap ? want : cap);
-  kern<<<blocks, warps * 32, warps * kWarpBytes, s>>>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out,
-                                                      device_status_ptr(), wait_limit_ns());
+  e = launch_pdl(kern, dim3(blocks), dim3(warps * 32), warps * kWarpBytes, s, x, n, H, g, eps, mods, ms, so, co, seg,
+                 rb, out, device_status_ptr(), wait_limit_ns());
   count_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -118,9 +118,10 @@ static mmh3_status run_gemm(const void* A, const void* B, int M, int N, int K, c
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
   const int gm = group_m_for(K, (N + BN - 1) / BN, m_tiles, 128);
-  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, gm, epi, device_status_ptr(), wait_limit_ns());
+  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kGemmThreads), smem, s, ta, tb, tc, M, N, K, gm, epi,
+                             device_status_ptr(), wait_limit_ns());
   count_launch();
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return MMH3_OK;
 }
@@ -189,9 +190,10 @@ static mmh3_status run_gemm2(const void* A, const void* B, int M, int N, int K, 
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   if (fault_injected("launch")) return fail(MMH3_ERR_CUDA, "injected fault at launch");
   const int gm = group_m_for(K, (N + BN - 1) / BN, m_tiles, 256);
-  kern<<<2 * pairs, kGemmThreads, smem, s>>>(ta, tb, tc, M, N, K, gm, epi, device_status_ptr(), wait_limit_ns());
+  cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(kGemmThreads), smem, s, ta, tb, tc, M, N, K, gm, epi,
+                             device_status_ptr(), wait_limit_ns());
   count_launch();
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
   return MMH3_OK;
 }

@@ -37,6 +37,24 @@ struct CanaryList {
 cudaError_t launch_canary(const CanaryList& l, bool verify, int kernel_id, cudaStream_t s);
 // Address of the device status word on the current device.
 DevStatus* device_status_ptr();
+
+// Launch with programmatic stream serialization (see pdl_wait): the kernel
+// must call pdl_wait() before its first global memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 int num_sms();
 
 // ------------------------------------------------------------------ plan
