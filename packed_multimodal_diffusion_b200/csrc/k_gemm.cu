@@ -234,19 +234,22 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
                                 float* x, const float* mods, int mods_stride, int chunk_off,
                                 const SegRows& seg, cudaStream_t s) {
   if (dtype == MMH3_BF16) {
-    // CTA pairs with 192-wide tiles for the out projection and for fc2
-    // (K = 4H): with the warp-wide MMA issue, fc2 on pairs measured 0.545 ms
-    // against 0.642 on single CTAs with 224-wide tiles, and 256-wide pair
-    // tiles 0.560.  x is moved by TMA (staged read-modify-write) when N is a
-    // multiple of 32.
+    // CTA pairs with 256-wide tiles for the out projection and for fc2
+    // (K = 4H), even where N leaves the last column tile half empty (N =
+    // 2688: 10.5 tiles).  Per SM and 64-deep k-block a 256 x 192 pair tile
+    // moves 28 KB through shared memory twice (TMA in, MMA out) in 384 MMA
+    // cycles, about 146 B/clk against the 128 B/clk shared memory gives; a
+    // 256 x 256 tile needs 125.  Measured in the same calls: fc2 0.540-0.545
+    // against 0.550-0.553 ms with 192-wide tiles, out unchanged.  x is moved
+    // by TMA (staged read-modify-write) when N is a multiple of 32.
     const bool staged = N % 32 == 0;
-    if (staged && N % 192 == 0 && use_pairs(M, N, 192)) {
-      EpiResidualTma<192, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
-      return run_gemm2<192>(A, B, M, N, K, e, s, x, N, 4);
-    }
     if (staged && use_pairs(M, N, 256)) {
       EpiResidualTma<256, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
       return run_gemm2<256>(A, B, M, N, K, e, s, x, N, 4);
+    }
+    if (staged && N % 192 == 0 && use_pairs(M, N, 192)) {
+      EpiResidualTma<192, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
+      return run_gemm2<192>(A, B, M, N, K, e, s, x, N, 4);
     }
     if (staged && N % 224 == 0) {
       EpiResidualTma<224, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
