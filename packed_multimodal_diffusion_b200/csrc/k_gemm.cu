@@ -240,8 +240,8 @@ mmh3_status gemm_gated_residual(int dtype, const void* A, const void* B, int M, 
     // moves 28 KB through shared memory twice (TMA in, MMA out) in 384 MMA
     // cycles, about 146 B/clk against the 128 B/clk shared memory gives; a
     // 256 x 256 tile needs 125.  Measured in the same calls: fc2 0.540-0.545
-    // against 0.550-0.553 ms with 192-wide tiles, out unchanged.  x is moved
-    // by TMA (staged read-modify-write) when N is a multiple of 32.
+    // against 0.550-0.553 ms with 192-wide tiles, out unchanged.  When N is a
+    // multiple of 32 the update is added into x by tensor reduce-adds.
     const bool staged = N % 32 == 0;
     if (staged && use_pairs(M, N, 256)) {
       EpiResidualTma<256, false> e{{}, N, mods, mods_stride, chunk_off, seg, nullptr};
