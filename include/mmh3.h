@@ -25,6 +25,12 @@
  *  - Kernel waits are bounded (default 2 s, MMH3_WAIT_LIMIT_MS or
  *    mmh3_set_wait_limit_ns); a kernel that gives up records a device status
  *    that mmh3_device_status() returns as MMH3_ERR_TIMEOUT.
+ *  - The block's kernels use programmatic dependent launch: each is launched
+ *    with programmatic stream serialization, lets the next kernel of the
+ *    stream launch early, and waits (griddepcontrol.wait) for its
+ *    predecessor before touching global memory.  A caller's own kernel
+ *    launched after them without that attribute runs in plain stream order;
+ *    one launched with it must itself wait before reading their outputs.
  */
 #ifndef MMH3_H_
 #define MMH3_H_
