@@ -362,6 +362,15 @@ def run_gpu(args):
     kernels = api.prof_collect_kernels()
     api.device_status()
 
+    # ---- the same step replayed from a CUDA graph (one stream capture of
+    # the block's launches), from the power state the timed pass started from
+    time.sleep(PROFILE_PAUSE_S)
+    for _ in range(max(3, args.warmup)):
+        step()
+    g_per, g_ms, g_kernels, g_clocks = time_graph(step, args.steps, max(3, args.warmup))
+    api.device_status()
+    g_ms_max = max_over_ranks(g_ms, device, world)
+
     # ---- end to end through the C ABI with host buffers (pinned), copies
     # inside the timed region: each step copies its input in and its result
     # out (mmh3_block_forward_host); three device slots let a step's
@@ -448,6 +457,8 @@ def run_gpu(args):
                 "d2h_bytes_per_step": int(W["x0"].numel() * 4)},
         "gpu_launches": launches,
         "clocks": clocks,
+        "graph": {"value": job_throughput(world, n, args.steps, g_ms_max), "unit": UNIT,
+                  **graph_entry(g_per, g_ms_max, g_kernels, g_clocks, args.steps)},
     }
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline()
@@ -563,6 +574,45 @@ def _time(fn, steps, warmup):
     return e0.elapsed_time(e1) / steps
 
 
+def time_graph(fn, steps, warmup):
+    """`fn` captured once into a CUDA graph (stream capture; the library's
+    launches, programmatic edges included, become the graph's nodes), then
+    `warmup` untimed replays and `steps` timed ones, with a CUDA event on the
+    current stream before every replay and after the last.  Returns the
+    per-replay ms, the total ms, the library kernels one replay launches and
+    the clocks sampled while timing."""
+    import torch
+
+    from packed_multimodal_diffusion_b200 import api
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    k0 = api.launch_count()
+    with torch.cuda.graph(g):
+        fn()
+    kernels = api.launch_count() - k0
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev[0].record()
+        for i in range(steps):
+            g.replay()
+            ev[i + 1].record()
+        torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total = ev[0].elapsed_time(ev[-1])
+    g.reset()
+    return per, total, kernels, clk.summary()
+
+
+def graph_entry(per, total, kernels, clocks, steps) -> dict:
+    return {"ms_per_step": total / steps,
+            "step_ms": {"median": statistics.median(per), "p10": percentile(per, 10),
+                        "p90": percentile(per, 90), "mean": total / steps},
+            "kernels_per_step": kernels, "clocks": clocks}
+
+
 def run_workload(args):
     """One JSON line for the stack, image, SigLIP or tiny workload (device-timed
     with CUDA events, weights generated on the device from the seeded streams,
@@ -583,6 +633,10 @@ def run_workload(args):
         x = configs.vit_inputs(c, device=dev)
         ws = torch.empty(api.vit_workspace_size(d, c.batch, c.seq), dtype=torch.uint8, device=dev)
         ms = _time(lambda: api.vit_layer_forward(d, params, x, c.batch, c.seq, ws), steps, warmup)
+        clocks = _time.clocks
+        api.device_status()
+        graph = graph_entry(*time_graph(lambda: api.vit_layer_forward(d, params, x, c.batch, c.seq, ws),
+                                        steps, warmup), steps)
         api.device_status()
         rows = c.batch * c.seq
         flop = 2.0 * rows * c.hidden * (3 * c.hidden + c.hidden + 2 * c.mlp) + 4.0 * c.batch * c.seq ** 2 * c.hidden
@@ -592,7 +646,7 @@ def run_workload(args):
                     config={"workload": "SigLIP layer: 32 images x 1024 tokens, hidden 768, 12x64 heads, "
                                         "MLP 3072 tanh-GELU, LayerNorm pre-norm"},
                     context="the pages quote 61.9 ms/layer for batch 1 on an unnamed CPU",
-                    clocks=_time.clocks)
+                    clocks=clocks, graph={"value": graph["ms_per_step"], "unit": "ms/layer", **graph})
         print(json.dumps(line), flush=True)
         return
     c = {"stack": configs.STACK, "image": configs.IMAGE, "tiny": configs.TINY}[args.workload]
@@ -639,6 +693,8 @@ def run_workload(args):
     phases, nblocks = api.prof_collect()
     kernels = api.prof_collect_kernels()
     api.device_status()
+    graph = graph_entry(*time_graph(step, steps, warmup), steps)
+    api.device_status()
     flops = block_flops(n, c.hidden, c.heads * c.head_dim, c.ffn)
     per_block = {k: v / max(1, nblocks) for k, v in phases.items() if v > 0}
     peak, peak_kind, _ = choose_peak(peaks, clocks, ms * steps / 1e3)
@@ -657,7 +713,8 @@ def run_workload(args):
                                  blocks_per_prologue=min(c.n_blocks, 64),
                                  act_bytes=4 if c.act_dtype == torch.float32 else 2), peaks["hbm_gbs"])},
                 config={"workload": f"{c.name}: n {n}, hidden {c.hidden}, {c.heads}x{c.head_dim} heads, "
-                                    f"SwiGLU {c.ffn}, {c.n_blocks} blocks" + (", output heads" if heads else "")})
+                                    f"SwiGLU {c.ffn}, {c.n_blocks} blocks" + (", output heads" if heads else "")},
+                graph={"value": graph["ms_per_step"], "unit": "ms/forward", **graph})
     print(json.dumps(line), flush=True)
 
 

@@ -31,6 +31,14 @@
  *    predecessor before touching global memory.  A caller's own kernel
  *    launched after them without that attribute runs in plain stream order;
  *    one launched with it must itself wait before reading their outputs.
+ *  - Stream capture: the forward entry points (block, stack, encoder layer,
+ *    attention) put only kernel launches and asynchronous copies on
+ *    `stream`, so they can be captured into a CUDA graph (the programmatic
+ *    launches become programmatic edges).  Make one uncaptured call on the
+ *    device first: the first call writes the check-mode flag into the status
+ *    word with a synchronous copy.  mmh3_device_status, mmh3_status_sync,
+ *    mmh3_prof_collect and the host-buffer pipeline's first call synchronise
+ *    and are not capturable.
  */
 #ifndef MMH3_H_
 #define MMH3_H_

@@ -218,3 +218,52 @@ def test_block_caller_modulation_replaces_the_adaln_curve(cuda_ok):
     own, _, _ = oracle_block(w, x, segs, pos, sv, sa, dims_o)
     from gpu_common import cosine
     assert cosine(own - f64(x), ref - f64(x)) < BF16_COS
+
+
+def _graph_vs_eager(dims_c, w, segs, pos, sv, sa, xs, launches):
+    """One block forward captured in a CUDA graph, then replayed on each input
+    of `xs` (copied into the captured x): every replay equals the eager call on
+    the same input, bit for bit, and the capture holds `launches` kernels."""
+    n, H = xs[0].shape
+    params = api.BlockParams.from_host(dims_c, w, device="cuda")
+    pd = torch.as_tensor(np.asarray(pos, np.float32)).cuda()
+    ws = torch.empty(api.workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
+    xg = xs[0].cuda().clone()
+    api.block_forward(dims_c, params, xg, segs, pd, sv, sa, ws)  # first-use set-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    c0 = api.launch_count()
+    with torch.cuda.graph(g):
+        api.block_forward(dims_c, params, xg, segs, pd, sv, sa, ws)
+    assert api.launch_count() - c0 == launches
+    for k, x in enumerate(xs):
+        xg.copy_(x.cuda())
+        g.replay()
+        ref = x.cuda().clone()
+        api.block_forward(dims_c, params, ref, segs, pd, sv, sa, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(xg, ref), f"replay {k}"
+    g.reset()
+    assert api.status_sync() == 0
+
+
+def test_block_graph_replay_matches_eager(cuda_ok):
+    dims_o, dims_c = small_dims()
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    n = int(pos.shape[0])
+    w = small_block_weights(38, 256, 2, 128, 512)
+    xs = [configs.synth.normal((n, 256), 110 + k, 1.0) for k in range(3)]
+    _graph_vs_eager(dims_c, w, segs, pos, *sigma_pair(0.5), xs, 8)
+
+
+def test_block_workload_graph_replay_matches_eager(cuda_ok):
+    # the bench's launch configuration: the attention's last wave is split,
+    # so the capture holds the merge launch as well
+    c = configs.BLOCK
+    segs, pos = t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+    n = int(pos.shape[0])
+    w = configs.block_weights(c, 0, device="cuda")
+    x0 = configs.hidden_states(c, device="cuda")
+    xs = [x0, x0 * 0.5]
+    dims_c = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn)
+    _graph_vs_eager(dims_c, w, segs, pos, *sigma_pair(c.sigma_v), xs, 9)

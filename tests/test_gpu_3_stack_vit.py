@@ -128,3 +128,66 @@ def test_vit_layer_full_size_sampled_images(cuda_ok):
         rows = slice(img * cfg.seq, (img + 1) * cfg.seq)
         assert_close(xg[rows], ref, what=f"image {img}")
         assert_close(xg[rows].cpu().double() - x[rows].double(), ref - f64(x[rows]), what=f"image {img} delta")
+
+
+def _capture(fn):
+    """fn() run once eagerly (first-use set-up), then captured in a CUDA graph."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+@pytest.mark.parametrize("act,heads,head_dim,ffn", [(torch.bfloat16, 2, 128, 512), (torch.float32, 4, 64, 1024)])
+def test_stack_graph_replay_matches_eager(cuda_ok, act, heads, head_dim, ffn):
+    # three blocks and the output heads in one captured graph (bf16 operands,
+    # and fp32 storage with tf32 tensor-core GEMMs): a replay on a new input
+    # equals the eager stack on it, bit for bit, heads included
+    dims_o, dims_c = small_dims(heads=heads, head_dim=head_dim, ffn=ffn, act=act)
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    n = int(pos.shape[0])
+    bp = [api.BlockParams.from_host(dims_c, small_block_weights(70 + i, 256, heads, head_dim, ffn, wdtype=act))
+          for i in range(3)]
+    hp = api.HeadParams.from_host(_small_heads(71, 256))
+    pd = torch.as_tensor(np.asarray(pos, np.float32)).cuda()
+    vseg = [s for s in segs if s[2] == 0][-1]
+    aseg = [s for s in segs if s[2] == 2][-1]
+    ws = torch.empty(api.workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
+    sv, sa = sigma_pair(0.5)
+
+    def run(xd, ov, oa):
+        api.stack_forward(dims_c, bp, hp, xd, segs, pd, sv, sa, ov, oa, ws)
+
+    xg = configs.synth.normal((n, 256), 83, 1.0).cuda()
+    ovg = torch.empty((vseg[1] - vseg[0], 128), device="cuda")
+    oag = torch.empty((aseg[1] - aseg[0], 128), device="cuda")
+    g = _capture(lambda: run(xg, ovg, oag))
+    x_new = configs.synth.normal((n, 256), 84, 1.0).cuda()
+    xg.copy_(x_new)
+    g.replay()
+    xe, ove, oae = x_new.clone(), torch.empty_like(ovg), torch.empty_like(oag)
+    run(xe, ove, oae)
+    torch.cuda.synchronize()
+    g.reset()
+    assert api.status_sync() == 0
+    assert torch.equal(xg, xe) and torch.equal(ovg, ove) and torch.equal(oag, oae)
+
+
+def test_vit_layer_graph_replay_matches_eager(cuda_ok):
+    cfg = _vit_small()
+    d = api.vit_dims(cfg.hidden, cfg.heads, cfg.head_dim, cfg.mlp, cfg.ln_eps)
+    params = api.VitParams.from_host(d, configs.vit_weights(cfg))
+    x = configs.vit_inputs(cfg).cuda()
+    ws = torch.empty(api.vit_workspace_size(d, cfg.batch, cfg.seq), dtype=torch.uint8, device="cuda")
+    xg = x.clone()
+    g = _capture(lambda: api.vit_layer_forward(d, params, xg, cfg.batch, cfg.seq, ws))
+    xg.copy_(x)
+    g.replay()
+    xe = x.clone()
+    api.vit_layer_forward(d, params, xe, cfg.batch, cfg.seq, ws)
+    torch.cuda.synchronize()
+    g.reset()
+    assert api.status_sync() == 0
+    assert torch.equal(xg, xe)
