@@ -638,14 +638,38 @@ def run_workload(args):
         graph = graph_entry(*time_graph(lambda: api.vit_layer_forward(d, params, x, c.batch, c.seq, ws),
                                         steps, warmup), steps)
         api.device_status()
+        # the phase profiler's pass over the same number of layers
+        api.prof_reset()
+        api.prof_enable(True)
+        for _ in range(steps):
+            api.vit_layer_forward(d, params, x, c.batch, c.seq, ws)
+        torch.cuda.synchronize()
+        api.prof_enable(False)
+        phases, nlayers = api.prof_collect()
+        kernels = api.prof_collect_kernels()
+        api.device_status()
         rows = c.batch * c.seq
-        flop = 2.0 * rows * c.hidden * (3 * c.hidden + c.hidden + 2 * c.mlp) + 4.0 * c.batch * c.seq ** 2 * c.hidden
+        # LayerNorm reads x (fp32) and writes its bf16 output once
+        ln_bytes = rows * c.hidden * 4 + rows * c.hidden * 2
+        hbm_ln = hbm_fractions(kernels, {"norm1": ln_bytes, "norm2": ln_bytes}, peaks["hbm_gbs"])
+        H, Fm = c.hidden, c.mlp
+        vflops = {"qkv gemm": 2.0 * rows * H * 3 * H, "attention": 4.0 * c.batch * c.seq ** 2 * H,
+                  "out gemm": 2.0 * rows * H * H, "fc1 gemm": 2.0 * rows * H * Fm, "fc2 gemm": 2.0 * rows * Fm * H}
+        per_layer = {k: v / max(1, nlayers) for k, v in phases.items() if v > 0}
+        peak, _, _ = choose_peak(peaks, clocks, ms * steps / 1e3)
+        flop = sum(vflops.values())
         line.update(metric="SigLIP encoder layer time (bf16, 1 B200)", value=ms, unit="ms/layer",
                     higher_is_better=False, dtype="bf16", tokens_per_s=rows / (ms / 1e3),
                     tflops_per_s=flop / (ms / 1e3) / 1e12,
                     config={"workload": "SigLIP layer: 32 images x 1024 tokens, hidden 768, 12x64 heads, "
                                         "MLP 3072 tanh-GELU, LayerNorm pre-norm"},
                     context="the pages quote 61.9 ms/layer for batch 1 on an unnamed CPU",
+                    phases_ms_per_layer={k: round(v, 4) for k, v in per_layer.items()},
+                    phase_frac_of_peak={k: round(vflops[k] / (per_layer[k] / 1e3) / 1e12 / peak, 4)
+                                        for k in vflops if k in per_layer},
+                    peak_tflops=peak,
+                    hbm_kernels={"peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                                 **{("ln1" if k == "norm1" else "ln2"): v for k, v in hbm_ln.items()}},
                     clocks=clocks, graph={"value": graph["ms_per_step"], "unit": "ms/layer", **graph})
         print(json.dumps(line), flush=True)
         return

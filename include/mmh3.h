@@ -261,12 +261,14 @@ mmh3_status mmh3_prepare_fc1(const mmh3_dims* dims, const void* fc1_gate_up, voi
  * n tokens.  Layout (each region 256-byte aligned, in this order): mods fp32
  * [2*3, 6H]; rope (cos, sin) fp32x2 [n, 3*rope_k]; xn1 [n, H]; qkv [n, 3*inner]
  * (q and k after qk-norm + rotation); attn [n, inner]; xn2 [n, H]; act [n, F];
- * head scratch [n, H] and final mods fp32 [2, 2H] -- all act dtype unless
- * stated.  After a block call the regions hold that block's intermediates. */
+ * head scratch [n, H]; final mods fp32 [2, 2H]; attention's work counter
+ * (16 bytes, zeroed by the block's first RMSNorm launch) -- all act dtype
+ * unless stated.  After a block call the regions hold that block's
+ * intermediates. */
 mmh3_status mmh3_workspace_size(const mmh3_dims* dims, int n, size_t* bytes);
 
-/* Full bidirectional attention over packed sequences (one 128-row query
- * tile per CTA, tcgen05): for each sequence b < n_seq of `seq` tokens
+/* Full bidirectional attention over packed sequences (work units of two
+ * 128-row query tiles of one head, tcgen05): for each sequence b < n_seq of `seq` tokens
  * starting at row b*seq of the qkv panel [n_seq*seq, 3*heads*head_dim]
  * (rows [q | k | v], heads contiguous, act dtype, device), per head:
  * out = softmax(q k^T * scale) v, written to out [n_seq*seq, heads*head_dim]
@@ -275,16 +277,19 @@ mmh3_status mmh3_workspace_size(const mmh3_dims* dims, int n, size_t* bytes);
 mmh3_status mmh3_attention(const void* qkv, int n_seq, int seq, int heads, int head_dim,
                            int act_dtype, float scale, void* out, void* stream);
 
-/* mmh3_attention with a scratch region for the last wave (bf16 only).
- * Work units of 256 query rows of one head fill the SMs in waves.  The
- * units of the last, partial wave are split along the keys over f CTAs
- * when that shortens the wave enough: f in 2..8 minimises
+/* mmh3_attention with a scratch region (bf16 only).  Its first 256 bytes
+ * hold a work counter (zeroed on the stream by a memset), and the launch is
+ * persistent: one CTA per SM takes work items from the counter until none
+ * is left.  Work units of 256 query rows of one head fill the SMs in
+ * waves.  The units of the last, partial wave are split along the keys
+ * into f items when that shortens the wave enough: f in 2..8 minimises
  * ceil(tail * f / SMs) / f, each piece keeps at least 32 key tiles of 128,
  * and the split is made only if the tail's time drops to 0.6 of a unit or
- * less.  The pieces run in the same launch as the whole units, after them,
- * so the SMs that finish first take them.  The CTAs' partial results (unnormalised O,
- * running maximum, row sum: 256 x (head_dim + 4) fp32 per CTA) go to scratch
- * and are then merged.  Without room in scratch (or with scratch NULL)
+ * less.  The pieces come after the whole units, so the SMs that finish
+ * first take them.  Their partial results (unnormalised O, running
+ * maximum, row sum: 256 x (head_dim + 4) fp32 per piece) go to scratch
+ * after the counter and are then merged.  With scratch NULL (or under 256
+ * bytes) every item is its own CTA; without room for the partial results
  * nothing is split.  The result equals mmh3_attention's up to the order of
  * the softmax sums.  The block entry points give attention this region from
  * their workspace (the SwiGLU activation region, free until fc1; the
@@ -594,7 +599,8 @@ mmh3_status mmh3_vit_fold_qkv(const mmh3_vit_dims* dims, const void* wq, const v
                               void* wqkv, float* bqkv, void* stream);
 
 /* Workspace: h [B*S, H] bf16, qkv [B*S, 3H] bf16, attn [B*S, H] bf16,
- * act [B*S, mlp] bf16 (256-byte aligned regions, in this order). */
+ * act [B*S, mlp] bf16, attention's work counter (16 bytes, zeroed by LN1)
+ * (256-byte aligned regions, in this order). */
 mmh3_status mmh3_vit_workspace_size(const mmh3_vit_dims* dims, int batch, int seq, size_t* bytes);
 
 /* One pre-norm encoder layer, in place on x [batch*seq, H] fp32
@@ -660,8 +666,12 @@ mmh3_status mmh3_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  * mmh3_prof_enable(1) makes the block entry points record CUDA events on
  * their stream between launches; mmh3_prof_collect waits for the recorded
  * events and adds their times into ms[0..min(n_slots,9)) (cumulative since
- * the last reset), with *n_blocks the number of blocks profiled.  Not thread
- * safe; the events are created lazily and reused. */
+ * the last reset), with *n_blocks the number of blocks profiled.  The
+ * encoder layer (mmh3_vit_layer_forward) records into the same slots and
+ * counts as one block: its two LayerNorms in slot 0 (kernels NORM1, NORM2),
+ * qkv + bias in 1, attention in 3, out + bias + residual in 4, fc1 + bias +
+ * GELU in 5, fc2 + bias + residual in 7.  Not thread safe; the events are
+ * created lazily and reused. */
 void mmh3_prof_enable(int on);
 mmh3_status mmh3_prof_collect(double* ms, int n_slots, long* n_blocks);
 void mmh3_prof_reset(void);

@@ -542,7 +542,7 @@ def workspace_regions(dims: Dims, n: int, ws: torch.Tensor) -> dict:
              ("xn1", n * H * es, act, (n, H)), ("qkv", n * 3 * I * es, act, (n, 3 * I)),
              ("attn", n * I * es, act, (n, I)), ("xn2", n * H * es, act, (n, H)),
              ("act", n * F * es, act, (n, F)), ("head", n * H * es, act, (n, H)),
-             ("fmods", 2 * 2 * H * 4, torch.float32, (2, 2 * H))]
+             ("fmods", 2 * 2 * H * 4, torch.float32, (2, 2 * H)), ("sched", 16, torch.int32, (4,))]
     out, off = {}, 0
     raw = ws.view(torch.uint8)
     for name, nbytes, dt, shape in sizes:

@@ -94,6 +94,7 @@ struct Workspace {
   void* act;
   void* head;
   float* fmods;
+  unsigned* sched;  // attention's work counter (zeroed by the block's first RMSNorm)
   size_t bytes;
   CanaryList canaries;  // MMH3_CHECK mode: one after each region
 };
@@ -124,6 +125,7 @@ Workspace carve(const mmh3_dims& d, int n, void* base) {
   w.act = take(N * F * es);
   w.head = take(N * H * es);
   w.fmods = static_cast<float*>(take(2 * 2 * H * 4));
+  w.sched = static_cast<unsigned*>(take(16));
   w.bytes = off;
   return w;
 }
@@ -181,7 +183,7 @@ mmh3_status block_pre(const mmh3_dims& d, const mmh3_block_weights& w, const flo
   const int dt = d.act_dtype;
   const int stride = 6 * H;
   cudaError_t e = launch_norm_mod(dt, x, n, H, w.norm1, d.eps, mods, stride, 0 * H, 1 * H, plan.block_rows, 0,
-                                  ws.xn1, s);
+                                  ws.xn1, s, ws.sched);
   if (e != cudaSuccess) return cuda_fail(e, "norm1/modulate launch");
   pm.mark(0, MMH3_PROF_K_NORM1);
   mmh3_status st = canaries(ws, true, MMH3_PROF_K_NORM1, s);
@@ -206,9 +208,10 @@ mmh3_status block_post(const mmh3_dims& d, const mmh3_block_weights& w, float* x
   // results of split attention units
   const size_t act_bytes = (size_t)n * F * esize_of(dt);
   mmh3_status st = kv_all == nullptr
-                       ? attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, scale, ws.attn, s, ws.act, act_bytes)
+                       ? attention(dt, ws.qkv, 1, n, d.heads, d.head_dim, scale, ws.attn, s, ws.act, act_bytes,
+                                   ws.sched)
                        : attention_kv(dt, ws.qkv, n, kv_all, n_kv, d.heads, d.head_dim, scale, ws.attn, s, ws.act,
-                                      act_bytes);
+                                      act_bytes, ws.sched);
   if (st != MMH3_OK) return st;
   pm.mark(3, MMH3_PROF_K_ATTN);
   st = canaries(ws, true, MMH3_PROF_K_ATTN, s);
@@ -948,7 +951,7 @@ static mmh3_status check_vit(const mmh3_vit_dims* d) {
 }
 
 static size_t vit_carve(const mmh3_vit_dims& d, size_t rows, void* base, void** h, void** qkv, void** attn,
-                        void** act) {
+                        void** act, void** sched) {
   size_t off = 0;
   auto take = [&](size_t bytes) {
     void* p = base ? static_cast<void*>(static_cast<uint8_t*>(base) + off) : nullptr;
@@ -959,6 +962,7 @@ static size_t vit_carve(const mmh3_vit_dims& d, size_t rows, void* base, void** 
   *qkv = take(rows * 3 * d.hidden * 2);
   *attn = take(rows * d.hidden * 2);
   *act = take(rows * d.mlp * 2);
+  *sched = take(16);
   return off;
 }
 
@@ -967,8 +971,8 @@ mmh3_status mmh3_vit_workspace_size(const mmh3_vit_dims* dims, int batch, int se
   mmh3_status st = check_vit(dims);
   if (st != MMH3_OK) return st;
   if (bytes == nullptr || batch < 0 || seq < 0) return fail(MMH3_ERR_ARG, "vit workspace args");
-  void *a, *b, *c, *e;
-  *bytes = vit_carve(*dims, (size_t)batch * seq, nullptr, &a, &b, &c, &e);
+  void *a, *b, *c, *e, *f;
+  *bytes = vit_carve(*dims, (size_t)batch * seq, nullptr, &a, &b, &c, &e, &f);
   return MMH3_OK;
 }
 
@@ -998,29 +1002,44 @@ mmh3_status mmh3_vit_layer_forward(const mmh3_vit_dims* dims, const mmh3_vit_wei
   }
   if (batch < 1 || seq < 1) return fail(MMH3_ERR_SHAPE, "vit: batch %d seq %d", batch, seq);
   if (misaligned(x) || misaligned(workspace)) return fail(MMH3_ERR_ALIGN, "vit: x / workspace alignment");
-  void *h, *qkv, *attn, *act;
+  void *h, *qkv, *attn, *act, *sched;
   const size_t rows = (size_t)batch * seq;
-  const size_t need = vit_carve(*dims, rows, nullptr, &h, &qkv, &attn, &act);
+  const size_t need = vit_carve(*dims, rows, nullptr, &h, &qkv, &attn, &act, &sched);
   if (workspace == nullptr || ws_bytes < need)
     return fail(MMH3_ERR_WORKSPACE, "vit workspace %zu < %zu", ws_bytes, need);
-  vit_carve(*dims, rows, workspace, &h, &qkv, &attn, &act);
+  vit_carve(*dims, rows, workspace, &h, &qkv, &attn, &act, &sched);
+  unsigned* ticket = static_cast<unsigned*>(sched);  // attention's work counter, zeroed by LN1
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = dims->hidden, M = (int)rows;
-  cudaError_t e = launch_layernorm(x, M, H, w->ln1_g, w->ln1_b, dims->ln_eps, static_cast<__nv_bfloat16*>(h), s);
+  // profiler slots as the block's: LayerNorm in the norm slot, the four
+  // projections in the GEMM slots, attention in its own
+  PhaseMark pm(s, true);
+  cudaError_t e =
+      launch_layernorm(x, M, H, w->ln1_g, w->ln1_b, dims->ln_eps, static_cast<__nv_bfloat16*>(h), s, ticket);
   if (e != cudaSuccess) return cuda_fail(e, "ln1 launch");
+  pm.mark(0, MMH3_PROF_K_NORM1);
   st = gemm_bias_act(MMH3_BF16, h, w->wqkv, M, 3 * H, H, w->bqkv, 0, qkv, s);
   if (st != MMH3_OK) return st;
+  pm.mark(1, MMH3_PROF_K_QKV);
   // h is free between the qkv projection and LN2: it holds the partial
   // results of split attention units
-  st = attention(MMH3_BF16, qkv, batch, seq, dims->heads, dims->head_dim, 1.0f, attn, s, h, rows * H * 2);
+  st = attention(MMH3_BF16, qkv, batch, seq, dims->heads, dims->head_dim, 1.0f, attn, s, h, rows * H * 2, ticket);
   if (st != MMH3_OK) return st;
+  pm.mark(3, MMH3_PROF_K_ATTN);
   st = gemm_bias_residual(MMH3_BF16, attn, w->wo, M, H, H, w->bo, x, s);
   if (st != MMH3_OK) return st;
+  pm.mark(4, MMH3_PROF_K_OUT);
   e = launch_layernorm(x, M, H, w->ln2_g, w->ln2_b, dims->ln_eps, static_cast<__nv_bfloat16*>(h), s);
   if (e != cudaSuccess) return cuda_fail(e, "ln2 launch");
+  pm.mark(0, MMH3_PROF_K_NORM2);
   st = gemm_bias_act(MMH3_BF16, h, w->w1, M, dims->mlp, H, w->b1, 1, act, s);
   if (st != MMH3_OK) return st;
-  return gemm_bias_residual(MMH3_BF16, act, w->w2, M, H, dims->mlp, w->b2, x, s);
+  pm.mark(5, MMH3_PROF_K_FC1);
+  st = gemm_bias_residual(MMH3_BF16, act, w->w2, M, H, dims->mlp, w->b2, x, s);
+  if (st != MMH3_OK) return st;
+  pm.mark(7, MMH3_PROF_K_FC2);
+  if (pm.on) ++g_prof_blocks;
+  return MMH3_OK;
 }
 
 // ---------------------------------------------------------------- profiler

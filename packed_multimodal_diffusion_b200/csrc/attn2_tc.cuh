@@ -30,6 +30,17 @@
 // While softmax 1 works on S1(j) the tensor core computes O0 += P0 V_j and
 // S0(j+1); while softmax 0 works on S0(j+1) it computes O1 += P1 V_j and
 // S1(j+1).
+//
+// With a ticket counter the kernel is persistent: one CTA per SM takes work
+// items (a whole unit, or one key range of a split unit) from the counter
+// until none is left, the producer one item ahead, and hands each to the
+// MMA and softmax warps through a two-slot ring in shared memory (a full
+// and an empty mbarrier per slot).  Between items the K/V ring and the
+// per-tile barriers run on; the producer reloads Q once the previous item's
+// last S MMAs are done (B_QE), so the copy and the next item's first S MMAs
+// overlap that item's last softmax and epilogue, and the item's first P.V
+// waits until the softmax warps have read the previous O out (B_OE).
+// Without a counter each CTA computes the one item blockIdx.x.
 #pragma once
 
 #include <type_traits>
@@ -107,8 +118,8 @@ template <int HD>
 __global__ void __launch_bounds__(320, 1)
     attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tmkv,
                     __nv_bfloat16* __restrict__ out, int ldo, int seq, int seq_kv, int k_off, int v_off,
-                    float scale_log2, int heads, int whole, int split, float* __restrict__ part,
-                    DevStatus* status, uint64_t limit_ns) {
+                    float scale_log2, int heads, int whole, int split, int total, unsigned* __restrict__ ticket,
+                    float* __restrict__ part, DevStatus* status, uint64_t limit_ns) {
   using Sh = Attn2Shape<HD>;
   constexpr int KV = Sh::kKV;
   constexpr uint32_t kIdescS = make_idesc(false, 128, 128, false, false);
@@ -120,9 +131,11 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int B_Q = 0;
   constexpr int B_KF = 1, B_KE = B_KF + KV, B_VF = B_KE + KV, B_VE = B_VF + KV;
   constexpr int B_SF = B_VE + KV, B_PF = B_SF + 2, B_PH = B_PF + 2, B_OF = B_PH + 2, B_DRAIN = B_OF + 1;
-  constexpr int kNumBars = B_DRAIN + 1;
+  constexpr int B_QE = B_DRAIN + 1, B_OE = B_QE + 1, B_IF = B_OE + 1, B_IE = B_IF + 2;
+  constexpr int kNumBars = B_IE + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* items = reinterpret_cast<volatile int*>(tmem_slot + 2);  // the two-slot work ring
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = smem_u32(smem);
@@ -133,27 +146,40 @@ __global__ void __launch_bounds__(320, 1)
   // Keys / values: rows [z*seq_kv, (z+1)*seq_kv) of `tmkv`, k at column
   // k_off, v at v_off (the same panel for a whole sequence on one GPU; the
   // gathered K|V rows of all ranks for a sequence split over ranks).
-  // Work unit: 256 query rows (q pair) of one head of one sequence.  CTAs
-  // [0, whole) compute whole units u = blockIdx.x.  The rest are the tail:
-  // CTA whole + b, b = t * split + piece, computes key range `piece` of the
-  // `split` contiguous ranges of unit whole + t and writes its unnormalised
-  // partial result to part slot b for attn_merge_kernel.  One grid holds
-  // both, so the hardware hands tail pieces to the SMs that finish their
-  // whole units first.
+  // Work item w < total.  Items [0, whole) are whole units u = w (256
+  // query rows of one head of one sequence, u = (zseq*heads + head)*nq +
+  // qpair, all key tiles).  The rest are the tail: item whole + b, b = t *
+  // split + piece, computes key range `piece` of the `split` contiguous
+  // ranges of unit whole + t and writes its unnormalised partial result to
+  // part slot b for attn_merge_kernel.
   const int nq = (seq + 255) / 256;
-  const int tb = (int)blockIdx.x - whole;  // tail CTA index; < 0: a whole unit
-  const int sp = tb < 0 ? 1 : split;
-  const int u = tb < 0 ? (int)blockIdx.x : whole + tb / split;
-  const int piece = tb < 0 ? 0 : tb % split;
-  const int qpair = u % nq;
-  const int head = (u / nq) % heads;
-  const int zseq = u / (nq * heads);
-  const int seq_row0 = zseq * seq;
-  const int kv_row0 = zseq * seq_kv;
-  const int q_row0 = seq_row0 + qpair * 256;
   const int kv_tiles = (seq_kv + 127) / 128;
-  const int j0 = piece * kv_tiles / sp;              // first key tile of this CTA
-  const int n_kv = (piece + 1) * kv_tiles / sp - j0;  // key tiles of this CTA (>= 1)
+  struct Item {
+    int u, j0, n, tb;  // unit, first key tile, key tiles, tail index (< 0: whole)
+  };
+  auto item_of = [&](int w) {
+    Item it;
+    it.tb = w - whole;
+    const int sp = it.tb < 0 ? 1 : split;
+    it.u = it.tb < 0 ? w : whole + it.tb / split;
+    const int piece = it.tb < 0 ? 0 : it.tb % split;
+    it.j0 = piece * kv_tiles / sp;
+    it.n = (piece + 1) * kv_tiles / sp - it.j0;
+    return it;
+  };
+  struct Unit {
+    int head, qpair, seq_row0, kv_row0, q_row0;
+  };
+  auto unit_of = [&](int u) {
+    Unit r;
+    r.qpair = u % nq;
+    r.head = (u / nq) % heads;
+    const int zseq = u / (nq * heads);
+    r.seq_row0 = zseq * seq;
+    r.kv_row0 = zseq * seq_kv;
+    r.q_row0 = r.seq_row0 + r.qpair * 256;
+    return r;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q), 1);
@@ -167,9 +193,13 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(B_SF + i), 1);
       mbar_init(bar(B_PF + i), 128);
       mbar_init(bar(B_PH + i), 128);
+      mbar_init(bar(B_IF + i), 1);
+      mbar_init(bar(B_IE + i), 9);  // the MMA warp and the eight softmax warps
     }
     mbar_init(bar(B_OF), 1);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_QE), 1);
+    mbar_init(bar(B_OE), 256);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch(&tm);
@@ -188,50 +218,87 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      const int xq = head * HD, xk = k_off + head * HD, xv = v_off + head * HD;
-      int in_k = 0, in_v = 0;
+      // Takes the CTA's items from the ticket counter (one ahead, so the
+      // atomic's latency hides behind the current item) and hands each to
+      // the other roles through the work ring.  Per item: Q0 and Q1 (once
+      // the previous item's S MMAs have read the old ones), then its K / V
+      // tiles through the two-stage ring, whose counter c runs on across
+      // items.  Without a counter the CTA's one item is blockIdx.x.
+      const bool chk = status != nullptr && status->check != 0;
+      int c = 0, in_k = 0, in_v = 0, q_last = -1;
+      bool q_pending = false;  // a Q copy no role has waited for yet (the last one)
       bool ok = true;
-      // MMH3_CHECK mode: the x coordinates of every copy this CTA issues and
-      // the first rows of Q and of its keys, before the first copy (the key
-      // rows only grow from there); a failure issues nothing
-      bool q_issued = false;
-      if (status != nullptr && status->check != 0) {
-        for (int c = 0; c < Sh::kHdBoxes && ok; ++c)
-          ok = tma_coords_ok(status, true, xq + c * 64, q_row0, 2) &&
-               tma_coords_ok(status, true, xk + c * 64, kv_row0 + j0 * 128, 2) &&
-               tma_coords_ok(status, true, xv + c * 64, kv_row0 + j0 * 128, 2);
-        if (!ok) *abort_flag = 1;
-      }
-      if (ok) {
+      unsigned next = ticket != nullptr ? atomicAdd(ticket, 1u) : blockIdx.x;
+      for (int k = 0; ok; ++k) {
+        const int w = next < (unsigned)total ? (int)next : total;
+        // slot k & 1 is free once every role has read item k - 2
+        if (!mbar_wait_ab(bar(B_IE + (k & 1)), (uint32_t)(((k >> 1) & 1) ^ 1), limit_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        items[k & 1] = w;
+        mbar_arrive(bar(B_IF + (k & 1)));
+        if (w >= total) break;
+        next = ticket != nullptr ? atomicAdd(ticket, 1u) : (unsigned)total;
+        const Item it = item_of(w);
+        const Unit un = unit_of(it.u);
+        const int xq = un.head * HD, xk = k_off + un.head * HD, xv = v_off + un.head * HD;
+        // MMH3_CHECK mode: the x coordinates of every copy of the item and
+        // the first rows of Q and of its keys (the key rows only grow from
+        // there); a failure issues nothing
+        if (chk) {
+          bool fine = true;
+          for (int cc = 0; cc < Sh::kHdBoxes && fine; ++cc)
+            fine = tma_coords_ok(status, true, xq + cc * 64, un.q_row0, 2) &&
+                   tma_coords_ok(status, true, xk + cc * 64, un.kv_row0 + it.j0 * 128, 2) &&
+                   tma_coords_ok(status, true, xv + cc * 64, un.kv_row0 + it.j0 * 128, 2);
+          if (!fine) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+        }
+        if (k > 0 && !mbar_wait_ab(bar(B_QE), (uint32_t)((k - 1) & 1), limit_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
         mbar_expect_tx(bar(B_Q), 2 * Sh::kTileBytes);
         for (int i = 0; i < 2; ++i)
-          for (int c = 0; c < Sh::kHdBoxes; ++c)
-            tma_load_2d(sbase + Sh::kQOff + i * Sh::kTileBytes + c * Sh::kBoxBytes, &tm, bar(B_Q),
-                        xq + c * 64, q_row0 + 128 * i);
-        q_issued = true;
-      }
-      int j = 0;
-      for (; j < n_kv && ok; ++j) {
-        const int s = j % KV;
-        const uint32_t ph = (uint32_t)((j / KV) & 1);
-        const int y = kv_row0 + (j0 + j) * 128;
-        if (!mbar_wait_ab(bar(B_KE + s), ph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(bar(B_KF + s), Sh::kTileBytes);
-        for (int c = 0; c < Sh::kHdBoxes; ++c)
-          tma_load_2d(sbase + Sh::kKOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tmkv, bar(B_KF + s),
-                      xk + c * 64, y);
-        in_k = j + 1;
-        if (!mbar_wait_ab(bar(B_VE + s), ph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(bar(B_VF + s), Sh::kTileBytes);
-        for (int c = 0; c < Sh::kHdBoxes; ++c)
-          tma_load_2d(sbase + Sh::kVOff + s * Sh::kTileBytes + c * Sh::kBoxBytes, &tmkv, bar(B_VF + s),
-                      xv + c * 64, y);
-        in_v = j + 1;
+          for (int cc = 0; cc < Sh::kHdBoxes; ++cc)
+            tma_load_2d(sbase + Sh::kQOff + i * Sh::kTileBytes + cc * Sh::kBoxBytes, &tm, bar(B_Q),
+                        xq + cc * 64, un.q_row0 + 128 * i);
+        q_last = k;
+        q_pending = true;
+        for (int j = it.j0; j < it.j0 + it.n && ok; ++j, ++c) {
+          const int s = c % KV;
+          const uint32_t ph = (uint32_t)((c / KV) & 1);
+          const int y = un.kv_row0 + j * 128;
+          if (!mbar_wait_ab(bar(B_KE + s), ph ^ 1u, limit_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(bar(B_KF + s), Sh::kTileBytes);
+          for (int cc = 0; cc < Sh::kHdBoxes; ++cc)
+            tma_load_2d(sbase + Sh::kKOff + s * Sh::kTileBytes + cc * Sh::kBoxBytes, &tmkv, bar(B_KF + s),
+                        xk + cc * 64, y);
+          in_k = c + 1;
+          if (!mbar_wait_ab(bar(B_VE + s), ph ^ 1u, limit_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(bar(B_VF + s), Sh::kTileBytes);
+          for (int cc = 0; cc < Sh::kHdBoxes; ++cc)
+            tma_load_2d(sbase + Sh::kVOff + s * Sh::kTileBytes + cc * Sh::kBoxBytes, &tmkv, bar(B_VF + s),
+                        xv + cc * 64, y);
+          in_v = c + 1;
+        }
       }
       if (!ok) {
-        if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, j);
+        if (!*abort_flag) record_error(status, DEV_TIMEOUT_PRODUCER, c);
         *abort_flag = 1;
-        if (q_issued) mbar_wait(bar(B_Q), 0, limit_ns);
+        // let the copies still in flight land (bounded) before the CTA's
+        // shared memory is released
+        if (q_pending) mbar_wait(bar(B_Q), (uint32_t)(q_last & 1), limit_ns);
         for (int i = (in_k > KV ? in_k - KV : 0); i < in_k; ++i)
           mbar_wait(bar(B_KF + i % KV), (uint32_t)((i / KV) & 1), limit_ns);
         for (int i = (in_v > KV ? in_v - KV : 0); i < in_v; ++i)
@@ -245,10 +312,13 @@ __global__ void __launch_bounds__(320, 1)
     // same) issues every MMA and commit.  Stage indices are compile-time
     // (the loop body is instantiated per K/V stage), so each descriptor is a
     // base plus a constant.
-    // Order: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
-    // S_i(j+1) goes right after PV_i(j), so the tensor core computes
-    // S0(j+1) while softmax 1 still works on S1(j).  Each PV_i(j) is issued
-    // in two halves of 64 keys, the first once P_i's first half is released.
+    // Order within an item: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) |
+    // PV0(1) S0(2) ...  S_i(j+1) goes right after PV_i(j), so the tensor
+    // core computes S0(j+1) while softmax 1 still works on S1(j).  Each
+    // PV_i(j) is issued in two halves of 64 keys, the first once P_i's first
+    // half is released.  The key-tile counter c (stages and barrier phases)
+    // runs on across items; an item's first S MMAs follow the previous
+    // item's last P.V, so they overlap that item's epilogue.
     static_assert(KV == 2, "the issue loop is written for two K/V stages");
     const uint64_t dk_major = sdesc_sw128(sbase, 16, 1024);           // Q, K: K-major
     const uint64_t dv_major = sdesc_sw128(sbase, Sh::kBoxBytes, 1024);  // V: MN-major
@@ -274,13 +344,16 @@ __global__ void __launch_bounds__(320, 1)
                       kIdescO, (!first || ks > 0) ? 1u : 0u);
       }
     };
-    // One key tile j in stage st: PV0(j) [S0(j+1)] PV1(j) [S1(j+1)].
-    auto step = [&](int j, auto stage) -> bool {
+    // Key tile j of an item of n tiles (item k), counter c, in stage st:
+    // PV0(j) [S0(j+1)] PV1(j) [S1(j+1)].  The item's first P.V overwrites O,
+    // so it waits until the softmax warps have read the previous item's O.
+    auto step = [&](int k, int j, int n, int c, auto stage) -> bool {
       constexpr int st = decltype(stage)::value;
       const std::integral_constant<int, 1 - st> next{};
-      const uint32_t pj = (uint32_t)(j & 1);
-      const uint32_t pv = (uint32_t)((j / KV) & 1);
-      const bool more = j + 1 < n_kv;
+      const uint32_t pj = (uint32_t)(c & 1);
+      const uint32_t pv = (uint32_t)((c / KV) & 1);
+      const bool more = j + 1 < n;
+      if (j == 0 && k > 0 && !wait(B_OE, (uint32_t)((k - 1) & 1))) return false;
       if (!wait(B_VF + st, pv) || !wait(B_PH + 0, pj)) return false;
       tc_fence_after();
       issue_pv(0, 0, j == 0, stage);
@@ -288,7 +361,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       issue_pv(0, 1, j == 0, stage);
       if (more) {
-        if (!wait(B_KF + 1 - st, (uint32_t)(((j + 1) / KV) & 1))) return false;
+        if (!wait(B_KF + 1 - st, (uint32_t)(((c + 1) / KV) & 1))) return false;
         tc_fence_after();
         issue_s(0, next);
       }
@@ -302,20 +375,44 @@ __global__ void __launch_bounds__(320, 1)
       if (more) {
         issue_s(1, next);
         umma_commit_elect(bar(B_KE + 1 - st));
+        // the item's last S MMAs: once they are done, the producer may load
+        // the next item's Q while this tile's softmax and P.V run
+        if (j + 2 == n) umma_commit_elect(bar(B_QE));
       }
       return true;
     };
     const std::integral_constant<int, 0> stage0{};
     const std::integral_constant<int, 1> stage1{};
-    bool ok = wait(B_Q, 0) && wait(B_KF + 0, 0);
-    if (ok) {
+    int c = 0;
+    auto body = [&](int k, int n) -> bool {
+      if (!wait(B_Q, (uint32_t)(k & 1)) || !wait(B_KF + (c & 1), (uint32_t)((c / KV) & 1))) return false;
       tc_fence_after();
-      issue_s(0, stage0);
-      issue_s(1, stage0);
-      umma_commit_elect(bar(B_KE + 0));
+      if (c & 1) {
+        issue_s(0, stage1);
+        issue_s(1, stage1);
+      } else {
+        issue_s(0, stage0);
+        issue_s(1, stage0);
+      }
+      umma_commit_elect(bar(B_KE + (c & 1)));
+      if (n == 1) umma_commit_elect(bar(B_QE));  // no further S MMA reads this Q
+      for (int j = 0; j < n; ++j, ++c)
+        if (!((c & 1) ? step(k, j, n, c, stage1) : step(k, j, n, c, stage0))) return false;
+      umma_commit_elect(bar(B_OF));  // O of this item complete
+      return true;
+    };
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      if (!wait(B_IF + (k & 1), (uint32_t)((k >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      const int w = items[k & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_IE + (k & 1)));
+      if (w >= total) break;
+      ok = body(k, item_of(w).n);
     }
-    for (int j = 0; j < n_kv && ok; ++j) ok = (j & 1) ? step(j, stage1) : step(j, stage0);
-    if (ok) umma_commit_elect(bar(B_OF));
     if (!ok) {
       if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_MMA, blockIdx.x);
       __syncwarp();
@@ -331,125 +428,148 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = (uint32_t)(lgrp * 32) << 16;
     const uint32_t ts = t_s(wg) + lane_off;
     const uint32_t to = t_o(wg) + lane_off;
-    float m_ref = 0.f, l_sum = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      {
-        const bool fail = !mbar_wait_ab(bar(B_SF + wg), (uint32_t)(j & 1), limit_ns, abort_flag);
-        if (__any_sync(0xffffffffu, fail)) { ok = false; break; }
-      }
-      tc_fence_after();
-      float s[128];
-      {
-        uint32_t u0[32], u1[32], u2[32], u3[32];
-        tmem_ld32(ts + 0, u0);
-        tmem_ld32(ts + 32, u1);
-        tmem_ld32(ts + 64, u2);
-        tmem_ld32(ts + 96, u3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(u0[i]);
-          s[32 + i] = __uint_as_float(u1[i]);
-          s[64 + i] = __uint_as_float(u2[i]);
-          s[96 + i] = __uint_as_float(u3[i]);
+    int c = 0;
+    // item k = w: its key tiles are c .. c_end - 1 of the CTA's count;
+    // valid = keys of its first tile that exist
+    auto body = [&](int k, int w, int valid, int c_end) -> bool {
+      float m_ref = 0.f, l_sum = 0.f;
+      for (bool first = true; c < c_end; ++c, valid -= 128, first = false) {
+        {
+          const bool fail = !mbar_wait_ab(bar(B_SF + wg), (uint32_t)(c & 1), limit_ns, abort_flag);
+          if (__any_sync(0xffffffffu, fail)) return false;
         }
-      }
-      const int valid = seq_kv - (j0 + j) * 128;
-      if (valid < 128) {
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          tmem_ld32(ts + 0, u0);
+          tmem_ld32(ts + 32, u1);
+          tmem_ld32(ts + 64, u2);
+          tmem_ld32(ts + 96, u3);
+          tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 128; ++k)
-          if (k >= valid) s[k] = -INFINITY;
-      }
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-      float pm[8];
-      if (j == 0) {
-        // first key tile: the row maximum before any exponential
-        attn_row_max(s, pm);
-        m_ref = attn_max8(pm) * scale_log2;
-        attn_exp_slices<0, 2, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
-      } else {
-        // keys 0..63 against the current reference, with the maximum of
-        // keys 64..127 folded in.  The lower half needs no maximum of its
-        // own: its exponentials are non-negative, so a lower-half sum of at
-        // most 2^8 bounds each of them by 2^8, i.e. no lower score exceeds
-        // the reference by more than 8 (log2 domain).  A row whose lower
-        // sum or upper maximum fails that bound rescales to its full row
-        // maximum and redoes the lower half.
-#pragma unroll
-        for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
-        attn_exp_slices<0, 2, true>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
-        const float m_hi = attn_max8(pm) * scale_log2;
-        const float lo_sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-        const bool need = lo_sum > 256.0f || m_hi > m_ref + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          // O_i holds every earlier product (see the kernel comment).
-          attn_row_max(s, pm);
-          const float m_new = need ? fmaxf(attn_max8(pm) * scale_log2, m_ref) : m_ref;
-          const float f = ex2_approx(m_ref - m_new);
-          l_sum *= f;
-          m_ref = m_new;
-#pragma unroll 1
-          for (int c = 0; c < HD / 16; ++c) {
-            uint32_t u[16];
-            tmem_ld16(to + c * 16, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i2 = 0; i2 < 16; ++i2) u[i2] = __float_as_uint(__uint_as_float(u[i2]) * f);
-            tmem_st16(to + c * 16, u);
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(u0[i]);
+            s[32 + i] = __uint_as_float(u1[i]);
+            s[64 + i] = __uint_as_float(u2[i]);
+            s[96 + i] = __uint_as_float(u3[i]);
           }
-          tmem_wait_st();
-          acc0 = make_float2(0.f, 0.f);
-          acc1 = make_float2(0.f, 0.f);
-          attn_exp_slices<0, 2, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
         }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_PH + wg));
-      attn_exp_slices<2, 4, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
-      l_sum += (acc0.x + acc0.y) + (acc1.x + acc1.y);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_PF + wg));
-    }
-    if (ok) {
-      const bool fail = !mbar_wait_ab(bar(B_OF), 0, limit_ns, abort_flag);
-      if (__any_sync(0xffffffffu, fail)) ok = false;
-    }
-    if (!ok) {
-      if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_SOFTMAX, blockIdx.x);
-      *abort_flag = 1;
-    }
-    if (__all_sync(0xffffffffu, ok)) {
-      tc_fence_after();
-      const int qr = qpair * 256 + wg * 128 + r;
-      const bool row_ok = qr < seq;
-      if (sp == 1) {
-        const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
-        __nv_bfloat16* dst = out + (size_t)(seq_row0 + qr) * ldo + head * HD;
+        if (valid < 128) {
+#pragma unroll
+          for (int kk = 0; kk < 128; ++kk)
+            if (kk >= valid) s[kk] = -INFINITY;
+        }
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        float pm[8];
+        if (first) {
+          // first key tile: the row maximum before any exponential
+          attn_row_max(s, pm);
+          m_ref = attn_max8(pm) * scale_log2;
+          attn_exp_slices<0, 2, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
+        } else {
+          // keys 0..63 against the current reference, with the maximum of
+          // keys 64..127 folded in.  The lower half needs no maximum of its
+          // own: its exponentials are non-negative, so a lower-half sum of at
+          // most 2^8 bounds each of them by 2^8, i.e. no lower score exceeds
+          // the reference by more than 8 (log2 domain).  A row whose lower
+          // sum or upper maximum fails that bound rescales to its full row
+          // maximum and redoes the lower half.
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
+          attn_exp_slices<0, 2, true>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
+          const float m_hi = attn_max8(pm) * scale_log2;
+          const float lo_sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+          const bool need = lo_sum > 256.0f || m_hi > m_ref + 8.0f;
+          if (__any_sync(0xffffffffu, need)) {
+            // O_i holds every earlier product of the item (see the kernel comment).
+            attn_row_max(s, pm);
+            const float m_new = need ? fmaxf(attn_max8(pm) * scale_log2, m_ref) : m_ref;
+            const float f = ex2_approx(m_ref - m_new);
+            l_sum *= f;
+            m_ref = m_new;
 #pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
+            for (int cc = 0; cc < HD / 16; ++cc) {
+              uint32_t uu[16];
+              tmem_ld16(to + cc * 16, uu);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i2 = 0; i2 < 16; ++i2) uu[i2] = __float_as_uint(__uint_as_float(uu[i2]) * f);
+              tmem_st16(to + cc * 16, uu);
+            }
+            tmem_wait_st();
+            acc0 = make_float2(0.f, 0.f);
+            acc1 = make_float2(0.f, 0.f);
+            attn_exp_slices<0, 2, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PH + wg));
+        attn_exp_slices<2, 4, false>(s, ts, scale_log2, m_ref, acc0, acc1, pm);
+        l_sum += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PF + wg));
+      }
+      {
+        const bool fail = !mbar_wait_ab(bar(B_OF), (uint32_t)(k & 1), limit_ns, abort_flag);
+        if (__any_sync(0xffffffffu, fail)) return false;
+      }
+      tc_fence_after();
+      const Item it = item_of(w);
+      const Unit un = unit_of(it.u);
+      const int qr = un.qpair * 256 + wg * 128 + r;
+      const bool row_ok = qr < seq;
+      if (it.tb < 0) {
+        const float inv = l_sum > 0.f ? 1.0f / l_sum : 0.f;
+        __nv_bfloat16* dst = out + (size_t)(un.seq_row0 + qr) * ldo + un.head * HD;
+#pragma unroll 1
+        for (int cc = 0; cc < HD / 32; ++cc) {
           float v[32];
-          ld_acc32(to + c * 32, v);
+          ld_acc32(to + cc * 32, v);
 #pragma unroll
           for (int i2 = 0; i2 < 32; ++i2) v[i2] *= inv;
-          if (row_ok) store32(dst + c * 32, v);
+          if (row_ok) store32(dst + cc * 32, v);
         }
       } else {
         // partial: O unnormalised (relative to m_ref), then m_ref and l_sum
-        float* dst = part + ((size_t)tb * 256 + wg * 128 + r) * Attn2Shape<HD>::kPartStride;
+        float* dst = part + ((size_t)it.tb * 256 + wg * 128 + r) * Sh::kPartStride;
 #pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
+        for (int cc = 0; cc < HD / 32; ++cc) {
           float v[32];
-          ld_acc32(to + c * 32, v);
-          if (row_ok) store32(dst + c * 32, v);
+          ld_acc32(to + cc * 32, v);
+          if (row_ok) store32(dst + cc * 32, v);
         }
         if (row_ok) {
           dst[HD] = m_ref;
           dst[HD + 1] = l_sum;
         }
       }
+      // this thread's O is read: the next item's first P.V may overwrite it
+      tc_fence_before();
+      mbar_arrive(bar(B_OE));
+      return true;
+    };
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      {
+        const bool fail = !mbar_wait_ab(bar(B_IF + (k & 1)), (uint32_t)((k >> 1) & 1), limit_ns, abort_flag);
+        if (__any_sync(0xffffffffu, fail)) {
+          ok = false;
+          break;
+        }
+      }
+      const int w = items[k & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_IE + (k & 1)));
+      if (w >= total) break;
+      const Item it = item_of(w);
+      ok = body(k, w, seq_kv - it.j0 * 128, c + it.n);
+    }
+    if (!ok) {
+      if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_SOFTMAX, blockIdx.x);
+      *abort_flag = 1;
     }
   }
   __syncthreads();

@@ -67,9 +67,15 @@ __device__ __forceinline__ void ld_acc32(uint32_t taddr, float (&v)[32]) {
 // 1 + e^-g = inf it gives 0, the limit); the result is rounded to bf16.
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// The tanh form of GELU, 0.5 x (1 + tanh(u)) with u = sqrt(2/pi) (x +
+// 0.044715 x^3), evaluated through the identity 0.5 (1 + tanh(u)) =
+// 1 / (1 + e^(-2u)): x / (1 + e^(-2u)), one exponential and one fast
+// reciprocal division, as silu above (for x far below zero the divisor
+// overflows to inf and the result is 0, the limit).
 __device__ __forceinline__ float gelu_tanh_f(float x) {
-  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-  return 0.5f * x * (1.0f + tanhf(k0 * (x + 0.044715f * x * x * x)));
+  const float k2 = -1.5957691216057308f;  // -2 sqrt(2/pi)
+  const float u2 = k2 * x * fmaf(0.044715f * x, x, 1.0f);
+  return __fdividef(x, 1.0f + __expf(u2));
 }
 
 // ------------------------------------------------------------- epilogues

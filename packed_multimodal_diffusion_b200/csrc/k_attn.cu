@@ -1,6 +1,7 @@
 // Host launcher of the tcgen05 attention kernel ("cortiq_engine/mmh3.rs",
 // attention: full bidirectional softmax attention per head over the packed
 // sequence; "ffai-argus 0.7.0 src/siglip.rs": attention inside each image).
+#include <algorithm>
 #include <cmath>
 
 #include "attn2_tc.cuh"
@@ -267,16 +268,24 @@ static mmh3_status run_attn_f32(const void* qkv, int n_seq, int seq, int heads, 
 // column 0, v at inner); the map covers exactly n_seq*seq_kv rows, so rows
 // a caller padded beyond them are never read.
 //
-// Work units (256 query rows of one head) fill the SMs in waves, one CTA per
-// SM.  When splitting the units of the last, partial wave along the keys
-// shortens it (and `scratch` has room for the partial results), each tail
-// unit runs as f CTAs over contiguous key ranges and attn_merge_kernel
-// combines their results.  The tail's CTAs follow the whole units in the
-// same grid, so the SMs that finish their whole units first (they differ by
-// 5-8% in speed) take them, with no launch boundary in between.
+// Work units (256 query rows of one head) fill the SMs in waves, one unit
+// per SM at a time.  When splitting the units of the last, partial wave
+// along the keys shortens it (and `scratch` has room for the partial
+// results), each tail unit runs as f items over contiguous key ranges and
+// attn_merge_kernel combines their results.  The tail's items follow the
+// whole units, so the SMs that finish their whole units first (they differ
+// by 5-8% in speed) take them, with no launch boundary in between.
+// The launch is persistent when it has a ticket counter: one CTA per SM
+// takes the items in order from the counter (`ticket`, zeroed by an earlier
+// kernel of the same call, or else the first kTicketBytes of scratch, zeroed
+// here by a memset).  Without either, it is one CTA per item, dispatched in
+// order by the hardware.
+constexpr size_t kTicketBytes = 256;
+
 template <int HD>
 static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv, int seq_kv, int heads,
-                             float scale, void* out, void* scratch, size_t scratch_bytes, cudaStream_t s) {
+                             float scale, void* out, void* scratch, size_t scratch_bytes, unsigned* ticket,
+                             cudaStream_t s) {
   using Sh = Attn2Shape<HD>;
   static_assert(Sh::kSmem <= 232448, "attention shared memory above the per-CTA limit");
   const int inner = heads * HD;
@@ -311,8 +320,16 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
   // Measured at 13248 keys, f = 2: -3%; at 8448 keys f = 4 (16 tiles a
   // piece): +6%; at 26496 keys f = 5 (0.8 of a unit): +1%; 32 x 1024 keys
   // f = 2 (4 tiles a piece): +7%.
+  if ((reinterpret_cast<uintptr_t>(scratch) & 15) != 0) scratch = nullptr;
+  bool reset_ticket = false;
+  if (ticket == nullptr && scratch != nullptr && scratch_bytes >= kTicketBytes) {
+    ticket = static_cast<unsigned*>(scratch);
+    scratch = static_cast<uint8_t*>(scratch) + kTicketBytes;
+    scratch_bytes -= kTicketBytes;
+    reset_ticket = true;
+  }
   int f = 1;
-  if (tail > 0 && scratch != nullptr && (reinterpret_cast<uintptr_t>(scratch) & 15) == 0) {
+  if (tail > 0 && scratch != nullptr) {
     double best = 1.0;
     for (int c = 2; c <= 8 && kv_tiles / c >= 32; ++c) {
       if ((size_t)tail * c * Sh::kPartBytesPerCta > scratch_bytes) break;
@@ -329,9 +346,15 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
   const int whole = split ? units - tail : units;
   // one grid: the whole units first, then the tail pieces (dispatched in
   // block order, so SMs that finish early take the pieces)
+  const int total = whole + (split ? tail * f : 0);
   float* part = split ? static_cast<float*>(scratch) : nullptr;
-  e = launch_pdl(kern, dim3(whole + (split ? tail * f : 0)), dim3(Sh::kThreads), Sh::kSmem, s, tm, tkv, o, inner, seq,
-                 seq_kv, k_off, v_off, sl2, heads, whole, f, part, device_status_ptr(), wait_limit_ns());
+  if (reset_ticket) {
+    e = cudaMemsetAsync(ticket, 0, sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_fail(e, "attention: ticket reset");
+  }
+  e = launch_pdl(kern, dim3(ticket != nullptr ? std::min(total, sms) : total), dim3(Sh::kThreads), Sh::kSmem, s, tm,
+                 tkv, o, inner, seq, seq_kv, k_off, v_off, sl2, heads, whole, f, total, ticket, part,
+                 device_status_ptr(), wait_limit_ns());
   count_launch();
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
@@ -346,28 +369,29 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
 }
 
 mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads, int head_dim,
-                      float scale, void* out, cudaStream_t s, void* scratch, size_t scratch_bytes) {
+                      float scale, void* out, cudaStream_t s, void* scratch, size_t scratch_bytes, unsigned* ticket) {
   if (n_seq <= 0 || seq <= 0) return MMH3_OK;
   if ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "attention: pointer not 16-byte aligned");
   if (dtype == MMH3_BF16 && head_dim == 128)
-    return run_attn2<128>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, scratch, scratch_bytes, s);
+    return run_attn2<128>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, scratch, scratch_bytes, ticket, s);
   if (dtype == MMH3_BF16 && head_dim == 64)
-    return run_attn2<64>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, scratch, scratch_bytes, s);
+    return run_attn2<64>(qkv, n_seq, seq, nullptr, 0, heads, scale, out, scratch, scratch_bytes, ticket, s);
   if (dtype == MMH3_F32 && head_dim == 64) return run_attn_f32<64>(qkv, n_seq, seq, heads, scale, out, s);
   return fail(MMH3_ERR_SHAPE, "attention: dtype %d head_dim %d unsupported", dtype, head_dim);
 }
 
 mmh3_status attention_kv(int dtype, const void* q_panel, int n_q, const void* kv, int n_kv, int heads,
-                         int head_dim, float scale, void* out, cudaStream_t s, void* scratch, size_t scratch_bytes) {
+                         int head_dim, float scale, void* out, cudaStream_t s, void* scratch, size_t scratch_bytes,
+                         unsigned* ticket) {
   if (n_q <= 0) return MMH3_OK;
   if (n_kv <= 0) return fail(MMH3_ERR_SHAPE, "attention: %d keys", n_kv);
   if ((reinterpret_cast<uintptr_t>(q_panel) | reinterpret_cast<uintptr_t>(kv) | reinterpret_cast<uintptr_t>(out)) & 15)
     return fail(MMH3_ERR_ALIGN, "attention: pointer not 16-byte aligned");
   if (dtype == MMH3_BF16 && head_dim == 128)
-    return run_attn2<128>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, scratch, scratch_bytes, s);
+    return run_attn2<128>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, scratch, scratch_bytes, ticket, s);
   if (dtype == MMH3_BF16 && head_dim == 64)
-    return run_attn2<64>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, scratch, scratch_bytes, s);
+    return run_attn2<64>(q_panel, 1, n_q, kv, n_kv, heads, scale, out, scratch, scratch_bytes, ticket, s);
   return fail(MMH3_ERR_UNSUPPORTED, "attention over gathered K|V: bf16 only (dtype %d, head_dim %d)", dtype,
               head_dim);
 }

@@ -315,9 +315,11 @@ template <typename TO, int VPL>
 __global__ void __launch_bounds__(kNormMaxWarps * 32, 1)
     norm_mod_kernel(const float* __restrict__ x, int n, int H, const float* __restrict__ g, float eps,
                     const float* __restrict__ mods, int mods_stride, int shift_off, int scale_off, SegRows seg,
-                    int row_base, TO* __restrict__ out, DevStatus* status, uint64_t limit_ns) {
+                    int row_base, TO* __restrict__ out, unsigned* zero_word, DevStatus* status,
+                    uint64_t limit_ns) {
   pdl_launch_dependents();
   pdl_wait();
+  if (zero_word != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
   constexpr uint32_t kRowBytes = VPL * 512;
   extern __shared__ __align__(128) uint8_t norm_smem[];
   const int warps = blockDim.x >> 5;
@@ -405,7 +407,8 @@ __global__ void __launch_bounds__(kNormMaxWarps * 32, 1)
 // against 12 rounds, 93% full, with eight).
 template <typename TO, int VPL>
 static cudaError_t norm_mod_launch(const float* x, int n, int H, const float* g, float eps, const float* mods,
-                                   int ms, int so, int co, const SegRows& seg, int rb, TO* out, cudaStream_t s) {
+                                   int ms, int so, int co, const SegRows& seg, int rb, TO* out, cudaStream_t s,
+                                   unsigned* zw) {
   constexpr size_t kWarpBytes = (size_t)kNormStages * (VPL * 512 + 8);
   constexpr int kWarps = kNormSmemBudget / kWarpBytes >= kNormMaxWarps ? kNormMaxWarps
                                                                          : (int)(kNormSmemBudget / kWarpBytes);
@@ -441,7 +444,7 @@ static cudaError_t norm_mod_launch(const float* x, int n, int H, const float* g,
   const long long cap = sms * ctas_per_sm;
   const int blocks = (int)(want < cap ? want : cap);
   e = launch_pdl(kern, dim3(blocks), dim3(warps * 32), warps * kWarpBytes, s, x, n, H, g, eps, mods, ms, so, co, seg,
-                 rb, out, device_status_ptr(), wait_limit_ns());
+                 rb, out, zw, device_status_ptr(), wait_limit_ns());
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -450,11 +453,11 @@ static cudaError_t norm_mod_launch(const float* x, int n, int H, const float* g,
 template <typename TO>
 static cudaError_t norm_mod_dispatch(const float* x, int n, int H, const float* g, float eps,
                                      const float* mods, int ms, int so, int co, const SegRows& seg,
-                                     int rb, TO* out, cudaStream_t s) {
+                                     int rb, TO* out, cudaStream_t s, unsigned* zw) {
   switch (H / 128) {
 #define MMH3_NM(V) \
   case V:          \
-    return norm_mod_launch<TO, V>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out, s);
+    return norm_mod_launch<TO, V>(x, n, H, g, eps, mods, ms, so, co, seg, rb, out, s, zw);
     MMH3_NM(1) MMH3_NM(2) MMH3_NM(4) MMH3_NM(6) MMH3_NM(8) MMH3_NM(16) MMH3_NM(21) MMH3_NM(24)
     MMH3_NM(32)
 #undef MMH3_NM
@@ -465,13 +468,13 @@ static cudaError_t norm_mod_dispatch(const float* x, int n, int H, const float* 
 
 cudaError_t launch_norm_mod(int dtype, const float* x, int n, int H, const float* g, float eps,
                             const float* mods, int mods_stride, int shift_off, int scale_off,
-                            const SegRows& seg, int row_base, void* out, cudaStream_t s) {
+                            const SegRows& seg, int row_base, void* out, cudaStream_t s, unsigned* zero_word) {
   if (n <= 0) return cudaSuccess;
   if (dtype == MMH3_BF16)
     return norm_mod_dispatch(x, n, H, g, eps, mods, mods_stride, shift_off, scale_off, seg, row_base,
-                             static_cast<__nv_bfloat16*>(out), s);
+                             static_cast<__nv_bfloat16*>(out), s, zero_word);
   return norm_mod_dispatch(x, n, H, g, eps, mods, mods_stride, shift_off, scale_off, seg, row_base,
-                           static_cast<float*>(out), s);
+                           static_cast<float*>(out), s, zero_word);
 }
 
 // ------------------------------------------------------------ LayerNorm
@@ -480,7 +483,8 @@ template <int VPL>
 __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict__ x, int n, int H,
                                                         const float* __restrict__ g,
                                                         const float* __restrict__ b, float eps,
-                                                        __nv_bfloat16* __restrict__ out) {
+                                                        __nv_bfloat16* __restrict__ out, unsigned* zero_word) {
+  if (zero_word != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= n) return;
@@ -519,12 +523,12 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float* __restrict_
 }
 
 cudaError_t launch_layernorm(const float* x, int n, int H, const float* g, const float* b,
-                             float eps, __nv_bfloat16* out, cudaStream_t s) {
+                             float eps, __nv_bfloat16* out, cudaStream_t s, unsigned* zero_word) {
   if (n <= 0) return cudaSuccess;
   const int blocks = (n + 7) / 8;
   switch (H / 128) {
 #define MMH3_LN(V) \
-  case V: layernorm_kernel<V><<<blocks, 256, 0, s>>>(x, n, H, g, b, eps, out); count_launch(); break;
+  case V: layernorm_kernel<V><<<blocks, 256, 0, s>>>(x, n, H, g, b, eps, out, zero_word); count_launch(); break;
     MMH3_LN(2) MMH3_LN(4) MMH3_LN(6) MMH3_LN(8) MMH3_LN(16) MMH3_LN(21)
 #undef MMH3_LN
     default:

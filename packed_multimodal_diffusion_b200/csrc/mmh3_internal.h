@@ -91,11 +91,15 @@ struct AdalnBatch {
 cudaError_t launch_prologue(const AdalnBatch& ab, int n_ab, int rank, int grid, int rows_per_slot,
                             const Plan& plan, float* mods, long long mods_stride, const float* pos, int n,
                             int k, float theta, float2* cs, cudaStream_t s);
+// zero_word (optional): a 4-byte word the launch sets to 0 (the attention
+// ticket counter of the same call, ready before the attention launch reads
+// it, since every launch in between waits for its predecessor)
 cudaError_t launch_norm_mod(int dtype, const float* x, int n, int H, const float* g, float eps,
                             const float* mods, int mods_stride, int shift_off, int scale_off,
-                            const SegRows& seg, int row_base, void* out, cudaStream_t s);
+                            const SegRows& seg, int row_base, void* out, cudaStream_t s,
+                            unsigned* zero_word = nullptr);
 cudaError_t launch_layernorm(const float* x, int n, int H, const float* g, const float* b,
-                             float eps, __nv_bfloat16* out, cudaStream_t s);
+                             float eps, __nv_bfloat16* out, cudaStream_t s, unsigned* zero_word = nullptr);
 cudaError_t launch_rows(const SegRows& seg, int n, int32_t* rows, cudaStream_t s);
 cudaError_t launch_fc1_tile(int esize, const void* in, void* out, int F, int H, cudaStream_t s);
 cudaError_t launch_vit_fold(const void* wq, const void* wk, const void* wv, const float* bq,
@@ -125,12 +129,16 @@ mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N,
                           const float* bias, int mode, void* out, cudaStream_t s);
 mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,
                                const float* bias, float* x, cudaStream_t s);
+// scratch: room for the split tail's partial results; ticket: the work
+// counter of a persistent launch, already zeroed on the stream (null: the
+// first 256 bytes of scratch serve, zeroed by a memset; without scratch the
+// launch is one CTA per work item).
 mmh3_status attention(int dtype, const void* qkv, int n_seq, int seq, int heads, int head_dim,
                       float scale, void* out, cudaStream_t s, void* scratch = nullptr,
-                      size_t scratch_bytes = 0);
+                      size_t scratch_bytes = 0, unsigned* ticket = nullptr);
 mmh3_status attention_kv(int dtype, const void* q_panel, int n_q, const void* kv, int n_kv, int heads,
                          int head_dim, float scale, void* out, cudaStream_t s, void* scratch = nullptr,
-                         size_t scratch_bytes = 0);
+                         size_t scratch_bytes = 0, unsigned* ticket = nullptr);
 
 // The block on a caller-provided scratch region (see mmh3_workspace_size);
 // mods_or_null: the caller's modulation [T_s*3, 6H] fp32 (device) in place

@@ -286,8 +286,9 @@ def test_check_mode_canaries_enlarge_the_workspace_and_clock_validation():
     try:
         api.set_check(1)
         assert _lib.load().mmh3_check_enabled() == 1
-        # nine regions, a 256-byte canary after each
-        assert api.workspace_size(d, 300) == base + 9 * 256
+        # ten regions (the last one attention's work counter), a 256-byte
+        # canary after each
+        assert api.workspace_size(d, 300) == base + 10 * 256
     finally:
         api.set_check(-1)
     assert api.workspace_size(d, 300) == base
