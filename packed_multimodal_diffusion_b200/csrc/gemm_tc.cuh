@@ -78,6 +78,21 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   return __fdividef(x, 1.0f + __expf(u2));
 }
 
+// The same for a pair, with the multiplications and additions as packed
+// f32x2 operations: x / (1 + 2^(x (c1 + c3 x^2))) with c1 = -2 sqrt(2/pi)
+// log2(e) and c3 = 0.044715 c1, one ex2 and one reciprocal (both MUFU) per
+// element.  The divisor is at least 1; it overflows to inf for x far below
+// zero, where the reciprocal gives 0, the limit.
+__device__ __forceinline__ float2 gelu_tanh_f2(float2 x) {
+  const float c1 = -2.3022082f;               // -2 sqrt(2/pi) log2(e)
+  const float c3 = -0.10294324f;              // 0.044715 * c1
+  const float2 x2 = __fmul2_rn(x, x);
+  const float2 a = __ffma2_rn(x2, make_float2(c3, c3), make_float2(c1, c1));
+  const float2 u = __fmul2_rn(x, a);
+  const float2 d = __fadd2_rn(make_float2(ex2_approx(u.x), ex2_approx(u.y)), make_float2(1.0f, 1.0f));
+  return __fmul2_rn(x, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
 // ------------------------------------------------------------- epilogues
 constexpr int kEpiParts = 1;         // epilogue warp sets (4 warps each)
 
@@ -428,10 +443,12 @@ struct EpiBiasActTma : NoSetup {
         float v[32];
         ld_acc<32>(tacc + u * 64 + h * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float t = v[i] + __ldg(bias + col + h * 32 + i);
-          if (MODE == 1) t = gelu_tanh_f(t);
-          v[i] = t;
+        for (int i = 0; i < 32; i += 2) {
+          float2 t = __fadd2_rn(make_float2(v[i], v[i + 1]),
+                                make_float2(__ldg(bias + col + h * 32 + i), __ldg(bias + col + h * 32 + i + 1)));
+          if (MODE == 1) t = gelu_tanh_f2(t);
+          v[i] = t.x;
+          v[i + 1] = t.y;
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) ch[h * 4 + q] = pack8_bf16(v + 8 * q);

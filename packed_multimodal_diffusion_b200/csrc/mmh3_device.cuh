@@ -303,6 +303,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------- CTA pairs (2-SM)
 // A cluster of two CTAs on one TPC shares one tcgen05 MMA of M = 256: each
 // CTA holds its 128 rows of A and half of B's rows in its own shared
