@@ -423,6 +423,7 @@ struct EpiQkvNormRopeTma {
 };
 
 // out = act(acc + bias), bf16, with tensor-store output (pair kernel).
+// bias must be 16-byte aligned (it is read as float4).
 template <int BN, int MODE>
 struct EpiBiasActTma : NoSetup {
   static constexpr int kStageOut = 32768;
@@ -437,18 +438,31 @@ struct EpiBiasActTma : NoSetup {
     for (int u = 0; u < BN / 64; ++u) {
       const int col = n0 + u * 64;
       if (col >= N) break;
+      // both 32-column halves of the unit in flight before one wait
+      uint32_t r[2][32];
+      tmem_ld32(tacc + u * 64, r[0]);
+      tmem_ld32(tacc + u * 64 + 32, r[1]);
+      tmem_wait_ld();
       uint4 ch[8];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float v[32];
-        ld_acc<32>(tacc + u * 64 + h * 32, v);
+        const float4* b4 = reinterpret_cast<const float4*>(bias + col + h * 32);  // 16-byte aligned
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float2 t = __fadd2_rn(make_float2(v[i], v[i + 1]),
-                                make_float2(__ldg(bias + col + h * 32 + i), __ldg(bias + col + h * 32 + i + 1)));
-          if (MODE == 1) t = gelu_tanh_f2(t);
-          v[i] = t.x;
-          v[i + 1] = t.y;
+        for (int i = 0; i < 32; i += 4) {
+          const float4 b = __ldg(b4 + i / 4);
+          float2 t0 = __fadd2_rn(make_float2(__uint_as_float(r[h][i]), __uint_as_float(r[h][i + 1])),
+                                 make_float2(b.x, b.y));
+          float2 t1 = __fadd2_rn(make_float2(__uint_as_float(r[h][i + 2]), __uint_as_float(r[h][i + 3])),
+                                 make_float2(b.z, b.w));
+          if (MODE == 1) {
+            t0 = gelu_tanh_f2(t0);
+            t1 = gelu_tanh_f2(t1);
+          }
+          v[i] = t0.x;
+          v[i + 1] = t0.y;
+          v[i + 2] = t1.x;
+          v[i + 3] = t1.y;
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) ch[h * 4 + q] = pack8_bf16(v + 8 * q);

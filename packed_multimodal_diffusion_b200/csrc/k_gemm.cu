@@ -307,15 +307,17 @@ mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N,
     return run_gemm<float, 128>(A, B, M, N, K, e, s);
   }
   if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias/gelu epilogue: bf16 only");
+  // the pair kernel's epilogue reads the bias as float4
+  const bool bias16 = (reinterpret_cast<uintptr_t>(bias) & 15) == 0;
   if (mode == 1) {
-    if (use_pairs(M, N, 256) && N % 64 == 0) {
+    if (use_pairs(M, N, 256) && N % 64 == 0 && bias16) {
       EpiBiasActTma<256, 1> et{{}, N, bias};
       return run_gemm2<256>(A, B, M, N, K, et, s, out, N);
     }
     EpiBiasAct<__nv_bfloat16, 256, 1> e{{}, static_cast<__nv_bfloat16*>(out), N, bias};
     return run_gemm<__nv_bfloat16, 256>(A, B, M, N, K, e, s);
   }
-  if (use_pairs(M, N, 256) && N % 64 == 0) {
+  if (use_pairs(M, N, 256) && N % 64 == 0 && bias16) {
     EpiBiasActTma<256, 0> et{{}, N, bias};
     return run_gemm2<256>(A, B, M, N, K, et, s, out, N);
   }
@@ -326,6 +328,8 @@ mmh3_status gemm_bias_act(int dtype, const void* A, const void* B, int M, int N,
 mmh3_status gemm_bias_residual(int dtype, const void* A, const void* B, int M, int N, int K,
                                const float* bias, float* x, cudaStream_t s) {
   if (dtype != MMH3_BF16) return fail(MMH3_ERR_UNSUPPORTED, "bias residual epilogue: bf16 only");
+  if ((reinterpret_cast<uintptr_t>(bias) & 15) != 0)  // both epilogues read it as float4
+    return fail(MMH3_ERR_ALIGN, "bias residual epilogue: bias not 16-byte aligned");
   if (use_pairs(M, N, 256) && N % 32 == 0) {
     EpiResidualTma<256, true> et{{}, N, nullptr, 0, 0, SegRows{}, bias};
     return run_gemm2<256>(A, B, M, N, K, et, s, x, N, 4);
