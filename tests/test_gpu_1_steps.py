@@ -216,6 +216,35 @@ def test_attention_split_tail(cuda_ok, n_seq, seq, heads, hd):
         assert_close(out[b * seq:(b + 1) * seq][sel], ref, what=f"split tail sequence {b}")
 
 
+@pytest.mark.parametrize("n_seq,seq,heads,hd", [(4, 2048, 21, 128), (32, 1024, 12, 64), (200, 100, 2, 64),
+                                                (3, 700, 8, 128)])
+def test_attention_persistent_matches_one_cta_per_item(cuda_ok, n_seq, seq, heads, hd):
+    # a 256-byte scratch holds only the work counter: the launch is
+    # persistent (148 CTAs, each walking several items through the work
+    # ring; 100-key sequences give one-tile items) and nothing is split, so
+    # every item computes exactly what the launch without scratch (one CTA
+    # per item) computes: equal bit for bit, and sampled rows against the
+    # oracle
+    n = n_seq * seq
+    qkv = _qkv(n, heads, hd, 500 + seq).cuda()
+    scale = 1 / math.sqrt(hd)
+    out = torch.full((n, heads * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    counter_only = torch.empty(256, dtype=torch.uint8, device="cuda")
+    c0 = api.launch_count()
+    api.attention_ws(qkv, n_seq, seq, heads, hd, scale, out, counter_only)
+    assert api.launch_count() - c0 == 1
+    plain = torch.empty_like(out)
+    api.attention(qkv, n_seq, seq, heads, hd, scale, plain)
+    assert api.status_sync() == 0
+    assert torch.equal(out, plain)
+    for b in (0, n_seq - 1):
+        part = qkv[b * seq:(b + 1) * seq].cpu()
+        q, k, v = (f64(t).reshape(seq, heads, hd) for t in part.split(heads * hd, dim=1))
+        sel = np.arange(0, seq, 37)
+        ref = O.attention(q, k, v, scale, q_rows=sel).reshape(len(sel), -1)
+        assert_close(out[b * seq:(b + 1) * seq][sel.tolist()], ref, what=f"persistent, sequence {b}")
+
+
 def test_attention_split_tail_with_rescales(cuda_ok):
     # 12288 keys x 1 head split in three with scores of std ~5: rows rescale
     # inside each piece, the pieces end with different reference maxima, and
