@@ -141,6 +141,40 @@ def test_block_pair_tile_boundaries(cuda_ok, layout):
     _check_block(dims_o, dims_c, w, x, segs, pos, sv, sa, (BF16_MAXABS, BF16_COS, BF16_STORE_REL))
 
 
+def test_block_hidden_128_half_empty_tiles(cuda_ok):
+    # hidden 128: the out and fc2 projections (N = 128) have one 256-wide
+    # column tile per pair tile, whose upper CTA's half of B lies wholly
+    # beyond N (zero-filled, its columns skipped by the epilogue)
+    dims_o, dims_c = small_dims(hidden=128, heads=1, head_dim=128, ffn=256)
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    n = int(pos.shape[0])
+    w = small_block_weights(39, 128, 1, 128, 256)
+    x = configs.synth.normal((n, 128), 86, 1.0)
+    _check_block(dims_o, dims_c, w, x, segs, pos, *sigma_pair(0.5), (BF16_MAXABS, BF16_COS, BF16_STORE_REL))
+
+
+def test_block_full_hidden_short_sequence(cuda_ok):
+    # the block's own sizes (hidden 2688, 21 x 128 heads, SwiGLU 10752) at
+    # 300 tokens: two pair-tile rows (the second one partly beyond n), 10.5
+    # column tiles for out and fc2, 84 for fc1, 31.5 for qkv, attention in
+    # three key tiles; sampled rows against the oracle
+    c = configs.BLOCK
+    segs, pos = t2va(20, 3, 16, 20, 20)
+    n = int(pos.shape[0])
+    assert 257 <= n <= 512
+    w = configs.block_weights(c, 0)
+    x = configs.hidden_states(c, n)
+    sv, sa = sigma_pair(c.sigma_v)
+    dims_c = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn)
+    xg, reg = run_block(dims_c, w, x, segs, pos, sv, sa)
+    sample = [0, 1, 100, 255, 256, n - 1]
+    keep = {}
+    ref, _, _ = oracle_block(w, x, segs, pos, sv, sa, c.dims(), sample_rows=sample, keep=keep)
+    assert_close(reg["attn"][sample], keep["attn"], what="attn rows", rel=BF16_STORE_REL)
+    assert_close(xg[sample], ref, what="x_out rows")
+    assert_close(xg[sample].cpu().double() - x[sample].double(), ref - f64(x[sample]), what="delta rows")
+
+
 def test_block_forward_host_pipelined_matches_device_calls(cuda_ok):
     # seven calls rotating over the slots with different inputs: each result
     # is the device block's on the same input, bit for bit
