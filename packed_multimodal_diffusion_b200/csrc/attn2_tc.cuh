@@ -1,9 +1,10 @@
-// Bidirectional flash attention on tcgen05, two query tiles per CTA.
+// Bidirectional flash attention on tcgen05, two query tiles per work item.
 //
-// One CTA computes two 128-row query tiles (256 rows) of one head, so each
-// K/V tile fetched by TMA serves 256 query rows.  Tensor memory (512
-// columns) holds S0 | S1 | O0 | O1.
-//   warp 0      TMA producer: Q0 and Q1 once, then K_j / V_j (two stages)
+// A work item is two 128-row query tiles (256 rows) of one head, over all
+// its keys or one key range of them, so each K/V tile fetched by TMA serves
+// 256 query rows.  Tensor memory (512 columns) holds S0 | S1 | O0 | O1.
+//   warp 0      TMA producer: Q0 and Q1 of the item, then its K_j / V_j
+//               (two stages)
 //   warp 1      MMA issuer (the whole warp runs the loop, one elected lane
 //               issues): S0 = Q0 K_0^T, S1 = Q1 K_0^T, then per key tile
 //               j: O0 += P0 V_j (once P0 is written), S0 = Q0 K_{j+1}^T,
