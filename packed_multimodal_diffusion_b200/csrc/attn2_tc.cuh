@@ -38,9 +38,13 @@
 // MMA and softmax warps through a two-slot ring in shared memory (a full
 // and an empty mbarrier per slot).  Between items the K/V ring and the
 // per-tile barriers run on; the producer reloads Q once the previous item's
-// last S MMAs are done (B_QE), so the copy and the next item's first S MMAs
-// overlap that item's last softmax and epilogue, and the item's first P.V
-// waits until the softmax warps have read the previous O out (B_OE).
+// last S MMAs are done (B_QE).  The MMA warp reads the next item from the
+// ring during the current item's last key tile and issues the next item's
+// first S0 right after that tile's PV0 and its first S1 after PV1, as
+// inside an item, so the two query tiles keep their alternation across
+// items.  Each query tile's O is signalled complete on its own barrier
+// (B_OF + i), and the next item's first P.V waits until both softmax
+// warpgroups have read their O out (B_OE + i).
 // Without a counter each CTA computes the one item blockIdx.x.
 #pragma once
 
@@ -131,8 +135,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::kBarOff);
   constexpr int B_Q = 0;
   constexpr int B_KF = 1, B_KE = B_KF + KV, B_VF = B_KE + KV, B_VE = B_VF + KV;
-  constexpr int B_SF = B_VE + KV, B_PF = B_SF + 2, B_PH = B_PF + 2, B_OF = B_PH + 2, B_DRAIN = B_OF + 1;
-  constexpr int B_QE = B_DRAIN + 1, B_OE = B_QE + 1, B_IF = B_OE + 1, B_IE = B_IF + 2;
+  constexpr int B_SF = B_VE + KV, B_PF = B_SF + 2, B_PH = B_PF + 2, B_OF = B_PH + 2, B_DRAIN = B_OF + 2;
+  constexpr int B_QE = B_DRAIN + 1, B_OE = B_QE + 1, B_IF = B_OE + 2, B_IE = B_IF + 2;
   constexpr int kNumBars = B_IE + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -196,11 +200,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(B_PH + i), 128);
       mbar_init(bar(B_IF + i), 1);
       mbar_init(bar(B_IE + i), 9);  // the MMA warp and the eight softmax warps
+      mbar_init(bar(B_OF + i), 1);
+      mbar_init(bar(B_OE + i), 128);
     }
-    mbar_init(bar(B_OF), 1);
     mbar_init(bar(B_DRAIN), 1);
     mbar_init(bar(B_QE), 1);
-    mbar_init(bar(B_OE), 256);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch(&tm);
@@ -354,7 +358,8 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t pj = (uint32_t)(c & 1);
       const uint32_t pv = (uint32_t)((c / KV) & 1);
       const bool more = j + 1 < n;
-      if (j == 0 && k > 0 && !wait(B_OE, (uint32_t)((k - 1) & 1))) return false;
+      if (j == 0 && k > 0 && (!wait(B_OE + 0, (uint32_t)((k - 1) & 1)) || !wait(B_OE + 1, (uint32_t)((k - 1) & 1))))
+        return false;
       if (!wait(B_VF + st, pv) || !wait(B_PH + 0, pj)) return false;
       tc_fence_after();
       issue_pv(0, 0, j == 0, stage);
@@ -382,37 +387,90 @@ __global__ void __launch_bounds__(320, 1)
       }
       return true;
     };
-    const std::integral_constant<int, 0> stage0{};
-    const std::integral_constant<int, 1> stage1{};
-    int c = 0;
-    auto body = [&](int k, int n) -> bool {
-      if (!wait(B_Q, (uint32_t)(k & 1)) || !wait(B_KF + (c & 1), (uint32_t)((c / KV) & 1))) return false;
+    // The item's last key tile (j = n - 1): PV0 and PV1 as in step, each
+    // query tile's O signalled complete on its own barrier (B_OF + i) right
+    // after its last P.V, and, when a next item follows (n_next > 0 key
+    // tiles), that item's first S0 issued right after PV0 and its first S1
+    // after PV1, as inside an item, so the two query tiles keep their
+    // alternation across items.
+    auto last_step = [&](int k, int j, int c, int n_next, auto stage) -> bool {
+      constexpr int st = decltype(stage)::value;
+      const std::integral_constant<int, 1 - st> next{};
+      const uint32_t pj = (uint32_t)(c & 1);
+      const uint32_t pv = (uint32_t)((c / KV) & 1);
+      if (j == 0 && k > 0 && (!wait(B_OE + 0, (uint32_t)((k - 1) & 1)) || !wait(B_OE + 1, (uint32_t)((k - 1) & 1))))
+        return false;
+      if (!wait(B_VF + st, pv) || !wait(B_PH + 0, pj)) return false;
       tc_fence_after();
-      if (c & 1) {
-        issue_s(0, stage1);
-        issue_s(1, stage1);
-      } else {
-        issue_s(0, stage0);
-        issue_s(1, stage0);
+      issue_pv(0, 0, j == 0, stage);
+      if (!wait(B_PF + 0, pj)) return false;
+      tc_fence_after();
+      issue_pv(0, 1, j == 0, stage);
+      umma_commit_elect(bar(B_OF + 0));
+      if (n_next > 0) {
+        if (!wait(B_Q, (uint32_t)((k + 1) & 1)) || !wait(B_KF + 1 - st, (uint32_t)(((c + 1) / KV) & 1))) return false;
+        tc_fence_after();
+        issue_s(0, next);
       }
-      umma_commit_elect(bar(B_KE + (c & 1)));
-      if (n == 1) umma_commit_elect(bar(B_QE));  // no further S MMA reads this Q
-      for (int j = 0; j < n; ++j, ++c)
-        if (!((c & 1) ? step(k, j, n, c, stage1) : step(k, j, n, c, stage0))) return false;
-      umma_commit_elect(bar(B_OF));  // O of this item complete
+      if (!wait(B_PH + 1, pj)) return false;
+      tc_fence_after();
+      issue_pv(1, 0, j == 0, stage);
+      if (!wait(B_PF + 1, pj)) return false;
+      tc_fence_after();
+      issue_pv(1, 1, j == 0, stage);
+      umma_commit_elect(bar(B_VE + st));
+      umma_commit_elect(bar(B_OF + 1));
+      if (n_next > 0) {
+        issue_s(1, next);
+        umma_commit_elect(bar(B_KE + 1 - st));
+        if (n_next == 1) umma_commit_elect(bar(B_QE));  // the next item's only S MMAs
+      }
       return true;
     };
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      if (!wait(B_IF + (k & 1), (uint32_t)((k >> 1) & 1))) {
+    const std::integral_constant<int, 0> stage0{};
+    const std::integral_constant<int, 1> stage1{};
+    // item kk from the work ring (warp-uniform); false on timeout
+    auto fetch = [&](int kk, int& w_out) -> bool {
+      if (!wait(B_IF + (kk & 1), (uint32_t)((kk >> 1) & 1))) return false;
+      w_out = items[kk & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_IE + (kk & 1)));
+      return true;
+    };
+    int c = 0;
+    int w = total;
+    bool ok = fetch(0, w);
+    bool s_issued = false;  // the item's first S MMAs went out with the previous item's last tile
+    for (int k = 0; ok && w < total; ++k) {
+      const int n = item_of(w).n;
+      if (!s_issued) {
+        if (!wait(B_Q, (uint32_t)(k & 1)) || !wait(B_KF + (c & 1), (uint32_t)((c / KV) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (c & 1) {
+          issue_s(0, stage1);
+          issue_s(1, stage1);
+        } else {
+          issue_s(0, stage0);
+          issue_s(1, stage0);
+        }
+        umma_commit_elect(bar(B_KE + (c & 1)));
+        if (n == 1) umma_commit_elect(bar(B_QE));  // no further S MMA reads this Q
+      }
+      for (int j = 0; j + 1 < n && ok; ++j, ++c) ok = (c & 1) ? step(k, j, n, c, stage1) : step(k, j, n, c, stage0);
+      if (!ok) break;
+      int w_next = total;
+      if (!fetch(k + 1, w_next)) {
         ok = false;
         break;
       }
-      const int w = items[k & 1];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_IE + (k & 1)));
-      if (w >= total) break;
-      ok = body(k, item_of(w).n);
+      const int n_next = w_next < total ? item_of(w_next).n : 0;
+      ok = (c & 1) ? last_step(k, n - 1, c, n_next, stage1) : last_step(k, n - 1, c, n_next, stage0);
+      ++c;
+      s_issued = n_next > 0;
+      w = w_next;
     }
     if (!ok) {
       if (lane == 0 && !*abort_flag) record_error(status, DEV_TIMEOUT_MMA, blockIdx.x);
@@ -514,7 +572,7 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(bar(B_PF + wg));
       }
       {
-        const bool fail = !mbar_wait_ab(bar(B_OF), (uint32_t)(k & 1), limit_ns, abort_flag);
+        const bool fail = !mbar_wait_ab(bar(B_OF + wg), (uint32_t)(k & 1), limit_ns, abort_flag);
         if (__any_sync(0xffffffffu, fail)) return false;
       }
       tc_fence_after();
@@ -549,7 +607,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       // this thread's O is read: the next item's first P.V may overwrite it
       tc_fence_before();
-      mbar_arrive(bar(B_OE));
+      mbar_arrive(bar(B_OE + wg));
       return true;
     };
     bool ok = true;
