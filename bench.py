@@ -48,10 +48,14 @@ def parse():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="b200", choices=["b200", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--workload", default="block", choices=["block", "stack", "image", "siglip", "tiny"],
+    p.add_argument("--workload", default="block",
+                   choices=["block", "stack", "image", "siglip", "tiny", "cp", "refine", "denoise"],
                    help="block (default) prints the benchmark line; the others print one JSON line "
                         "each for the remaining workloads (stack: 50 blocks + heads, image: 50 "
-                        "blocks, siglip: one encoder layer x 32 images, tiny: fp32 block)")
+                        "blocks, siglip: one encoder layer x 32 images, tiny: fp32 block, cp: the "
+                        "block over 2 and 4 sequence shards run one after another on one GPU, "
+                        "refine: the token refiner, denoise: one whole denoise call at the stack "
+                        "shape with embed and unpacking)")
     return p.parse_args()
 
 
@@ -742,10 +746,141 @@ def run_workload(args):
     print(json.dumps(line), flush=True)
 
 
+def run_next(args):
+    """JSON lines for the rows around the block: the block over sequence
+    shards (context parallel; the shards run one after another on one GPU,
+    so the time is the compute of all shards, without any exchange), the
+    token refiner, and one whole denoise call (embed, 50 blocks, heads,
+    unpacking) at the stack shape."""
+    import numpy as np
+    import torch
+
+    from packed_multimodal_diffusion_b200 import api, configs, shard
+    torch.cuda.set_device(0)
+    dev = "cuda"
+    steps, warmup = max(1, args.steps), max(1, args.warmup)
+    line = {"workload": args.workload, "data": "synthetic", "steps": steps, "warmup": warmup,
+            "higher_is_better": False, "dtype": "bf16"}
+    if args.workload == "cp":
+        c = configs.BLOCK
+        segs, pos = api.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+        n = pos.shape[0]
+        dims = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn)
+        params = api.BlockParams.from_host(dims, configs.block_weights(c, 0, device=dev), device=dev)
+        x0 = configs.hidden_states(c, device=dev)
+        pd = torch.as_tensor(pos.astype(np.float32), device=dev)
+        sv = c.sigma_v
+        sa = api.time_shift_sigma(max(sv, 1e-6), 12.0, 3.0)
+        inner = c.heads * c.head_dim
+        ws1 = torch.empty(api.workspace_size(dims, n), dtype=torch.uint8, device=dev)
+        x1 = x0.clone()
+        one = _time(lambda: api.block_forward(dims, params, x1, segs, pd, sv, sa, ws1), steps, warmup)
+        del ws1
+        worlds = {}
+        for world in (2, 4):
+            m, parts = shard.shard_rows(n, world)
+            kv_all = torch.empty((world * m, 2 * inner), dtype=torch.bfloat16, device=dev)
+            xs = [x0[r0:r0 + rows].clone() for r0, rows in parts]
+            wss = [torch.empty(api.workspace_size(dims, max(rows, 1)), dtype=torch.uint8, device=dev)
+                   for _, rows in parts]
+            ssegs = [shard.shard_segments(segs, r0, rows) for r0, rows in parts]
+            pss = [pd[r0:r0 + rows].clone() for r0, rows in parts]
+
+            def run():
+                for r, (r0, rows) in enumerate(parts):
+                    api.block_cp_begin(dims, params, xs[r], ssegs[r], pss[r], sv, sa, kv_all[r * m:r * m + rows],
+                                       wss[r])
+                for r, (r0, rows) in enumerate(parts):
+                    api.block_cp_end(dims, params, xs[r], ssegs[r], sv, sa, kv_all, n, wss[r])
+
+            ms = _time(run, steps, warmup)
+            api.device_status()
+            worlds[f"shards_{world}"] = {"ms_all_shards": ms, "ms_per_shard": ms / world,
+                                         "rows_per_shard": m, "kv_exchange_bytes_per_rank": 2 * n * 2 * inner}
+            del wss, kv_all
+        line.update(metric="block over sequence shards, compute only (bf16, 1 B200)", value=one,
+                    unit="ms/block (one GPU, whole sequence)", shards=worlds,
+                    config={"workload": f"block: n {n}, hidden 2688, 21x128 heads, SwiGLU 10752; shards "
+                                        "emulated one after another on one GPU, K|V gathered in place"},
+                    clocks=_time.clocks)
+    elif args.workload == "refine":
+        c = configs.BLOCK
+        text_dim, n_blocks, n = 4096, 2, c.text_len
+        dims = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn)
+        sd = lambda j: configs.synth.tensor_seed(7, 800 + j)  # noqa: E731
+        states = configs.synth.normal((n, text_dim), sd(0), 1.0, dtype=torch.bfloat16, device=dev)
+        cond_w = configs.synth.normal((c.hidden, text_dim), sd(1), text_dim ** -0.5, dtype=torch.bfloat16,
+                                      device=dev)
+        cond_b = configs.synth.normal((c.hidden,), sd(2), 0.1, device=dev)
+        norm = configs.synth.normal((c.hidden,), sd(3), 0.1, 1.0, device=dev)
+        blocks = [api.BlockParams.from_host(dims, configs.block_weights(c, 10 + b, device=dev), device=dev)
+                  for b in range(n_blocks)]
+        out = torch.empty((n, c.hidden), dtype=torch.float32, device=dev)
+        ws = torch.empty(api.refine_workspace_size(dims, n), dtype=torch.uint8, device=dev)
+        ms = _time(lambda: api.refine_text(dims, states, cond_w, cond_b, blocks, norm, 1e-6, out, ws), steps,
+                   warmup)
+        api.device_status()
+        line.update(metric="token refiner time (bf16, 1 B200)", value=ms, unit="ms/call",
+                    config={"workload": f"token refiner: {n} text tokens of width {text_dim} (assumed), "
+                                        f"projection to hidden 2688, {n_blocks} unmodulated unrotated blocks "
+                                        "(21x128 heads, SwiGLU 10752), final RMSNorm"},
+                    clocks=_time.clocks)
+    else:  # denoise
+        c = configs.STACK
+        segs, pos = api.layout_t2va(c.text_len, c.latent_t, c.lat_h, c.lat_w, c.audio_t)
+        n = pos.shape[0]
+        H, Cv, Ca = c.hidden, c.heads_out // 4, c.heads_out
+        dims = api.make_dims(c.hidden, c.heads, c.head_dim, c.ffn)
+        sd = lambda j: configs.synth.tensor_seed(8, 900 + j)  # noqa: E731
+        text = configs.synth.normal((c.text_len, H), sd(0), 1.0, device=dev)
+        video = configs.synth.normal((Cv, c.latent_t, c.lat_h, c.lat_w), sd(1), 1.0, device=dev)
+        audio = configs.synth.normal((Ca, 2, c.audio_t), sd(2), 1.0, device=dev)
+        ew = (configs.synth.normal((H, 4 * Cv), sd(3), (4 * Cv) ** -0.5, dtype=torch.bfloat16, device=dev),
+              configs.synth.normal((H,), sd(4), 0.1, device=dev),
+              configs.synth.normal((H, Ca), sd(5), Ca ** -0.5, dtype=torch.bfloat16, device=dev),
+              configs.synth.normal((H,), sd(6), 0.1, device=dev))
+        blocks = [api.BlockParams.from_host(dims, configs.block_weights(c, b, device=dev), device=dev)
+                  for b in range(c.n_blocks)]
+        heads = api.HeadParams.from_host(configs.head_weights(c, device=dev), device=dev)
+        pd = torch.as_tensor(pos.astype(np.float32), device=dev)
+        x = torch.empty((n, H), device=dev)
+        vo = torch.empty_like(video)
+        ao = torch.empty_like(audio)
+        ws = torch.empty(api.forward_workspace_size(dims, n, text, video, audio), dtype=torch.uint8, device=dev)
+        sv = c.sigma_v
+        sa = api.time_shift_sigma(max(sv, 1e-6), 12.0, 3.0)
+        ms = _time(lambda: api.forward(dims, segs, n, pd, sv, sa, text, video, audio, ew, blocks, heads, x, vo,
+                                       ao, ws), steps, warmup)
+        clocks = _time.clocks
+        ews = torch.empty(api.embed_workspace_size(dims, text, video, audio), dtype=torch.uint8, device=dev)
+        ms_embed = _time(lambda: api.embed(dims, segs, n, text, video, audio, *ew, x, ews), steps, warmup)
+        vseg = [sg for sg in segs if sg[2] == 0][-1]
+        aseg = [sg for sg in segs if sg[2] == 2]
+        vrows = torch.empty((vseg[1] - vseg[0], 4 * Cv), device=dev)
+        arows = torch.empty((aseg[-1][1] - aseg[0][0], Ca), device=dev)
+
+        def unpack():
+            api.unpatchify_video(vrows, Cv, c.latent_t, c.lat_h, c.lat_w, vo)
+            api.unpack_audio(arows, Ca, c.audio_t, ao)
+
+        ms_unpack = _time(unpack, steps, warmup)
+        api.device_status()
+        line.update(metric="denoise call time (bf16, 1 B200)", value=ms, unit="ms/call",
+                    embed_ms=ms_embed, unpack_ms=ms_unpack,
+                    config={"workload": f"one denoise evaluation at the stack shape: embed (text {c.text_len} x "
+                                        f"{H}, video latents {Cv}x{c.latent_t}x{c.lat_h}x{c.lat_w} patchified "
+                                        f"2x2, audio {Ca}x2x{c.audio_t}), 50 blocks (n {n}), both heads "
+                                        "(128 each), unpatchify and audio unpacking"},
+                    clocks=clocks)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload in ("cp", "refine", "denoise"):
+        run_next(args)
     elif args.workload != "block":
         run_workload(args)
     else:
