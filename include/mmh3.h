@@ -32,9 +32,10 @@
  *    launched after them without that attribute runs in plain stream order;
  *    one launched with it must itself wait before reading their outputs.
  *  - Stream capture: the forward entry points (block, stack, encoder layer,
- *    attention) put only kernel launches and asynchronous copies on
- *    `stream`, so they can be captured into a CUDA graph (the programmatic
- *    launches become programmatic edges).  Make one uncaptured call on the
+ *    attention, token refiner, the whole denoise call) put only kernel
+ *    launches, asynchronous copies and memsets on `stream`, so they can be
+ *    captured into a CUDA graph (the programmatic launches become
+ *    programmatic edges).  Make one uncaptured call on the
  *    device first: the first call writes the check-mode flag into the status
  *    word with a synchronous copy.  mmh3_device_status, mmh3_status_sync,
  *    mmh3_prof_collect and the host-buffer pipeline's first call synchronise

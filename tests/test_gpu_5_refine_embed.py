@@ -190,3 +190,62 @@ def test_denoise_forward_end_to_end(cuda_ok):
     api.device_status()
     assert_close(vo, rv, BF16_MAXABS, BF16_COS, "video velocity")
     assert_close(ao, ra, BF16_MAXABS, BF16_COS, "audio velocity")
+
+
+def _graph_equals_eager(fn, outs):
+    """fn() once eagerly, then captured in a CUDA graph and replayed; the
+    replay's outputs equal the eager call's bit for bit."""
+    fn()
+    torch.cuda.synchronize()
+    eager = [t.clone() for t in outs]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for t in outs:
+        t.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    g.reset()
+    assert api.status_sync() == 0
+    for a, b in zip(outs, eager):
+        assert torch.equal(a, b)
+
+
+def test_denoise_forward_graph_replay(cuda_ok):
+    # mmh3_forward (embed, two blocks, heads, unpatchify / unpack) captured
+    # in a CUDA graph
+    dims_o, dims_c = small_dims()
+    H, Cv, Ca = 256, 8, 32
+    L = O.layout_t2va(8, 2, 8, 12, 6)
+    segs, n = L["segments"], L["seq_len"]
+    d = [configs.synth.normal((8, H), 681, 1.0).cuda(), _bf16_exact((Cv, 2, 8, 12), 682).cuda(),
+         _bf16_exact((Ca, 2, 6), 683).cuda()]
+    ew = tuple(t.cuda() for t in _embed_weights(H, Cv, Ca))
+    bp = [api.BlockParams.from_host(dims_c, small_block_weights(690 + i, H, 2, 128, 512)) for i in range(2)]
+    cfg = configs.DitConfig("fwdg", 69, hidden=H, heads=2, head_dim=128, ffn=512, text_len=1, heads_out=32)
+    heads = configs.head_weights(cfg)
+    heads["w_audio"] = configs.synth.normal((Ca, H), 684, 0.02).to(torch.bfloat16)
+    heads["b_audio"] = configs.synth.normal((Ca,), 685, 0.02)
+    hp = api.HeadParams.from_host(heads)
+    pos = torch.as_tensor(np.asarray(L["pos"], np.float32)).cuda()
+    x = torch.empty((n, H), device="cuda")
+    vo = torch.empty(d[1].shape, device="cuda")
+    ao = torch.empty(d[2].shape, device="cuda")
+    ws = torch.empty(api.forward_workspace_size(dims_c, n, *d), dtype=torch.uint8, device="cuda")
+    sv, sa = 0.5, O.time_shift_sigma(0.5, 12.0, 3.0)
+    _graph_equals_eager(lambda: api.forward(dims_c, segs, n, pos, sv, sa, *d, ew, bp, hp, x, vo, ao, ws),
+                        [x, vo, ao])
+
+
+def test_refine_graph_replay(cuda_ok):
+    dims_o, dims_c = small_dims()
+    n, text_dim = 77, 384
+    states = configs.synth.normal((n, text_dim), 701, 1.0).to(torch.bfloat16).cuda()
+    cond_w = configs.synth.normal((256, text_dim), 702, text_dim ** -0.5).to(torch.bfloat16).cuda()
+    cond_b = configs.synth.normal((256,), 703, 0.1).cuda()
+    norm = (1.0 + configs.synth.normal((256,), 704, 0.1)).cuda()
+    blocks = [api.BlockParams.from_host(dims_c, small_block_weights(710 + i, 256, 2, 128, 512)) for i in range(2)]
+    out = torch.empty((n, 256), dtype=torch.float32, device="cuda")
+    ws = torch.empty(api.refine_workspace_size(dims_c, n), dtype=torch.uint8, device="cuda")
+    _graph_equals_eager(lambda: api.refine_text(dims_c, states, cond_w, cond_b, blocks, norm, 1e-6, out, ws),
+                        [out])
