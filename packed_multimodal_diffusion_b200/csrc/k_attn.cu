@@ -344,8 +344,9 @@ static mmh3_status run_attn2(const void* qkv, int n_seq, int seq, const void* kv
   const bool split = f >= 2;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   const int whole = split ? units - tail : units;
-  // one grid: the whole units first, then the tail pieces (dispatched in
-  // block order, so SMs that finish early take the pieces)
+  // one launch: the whole units first, then the tail pieces (taken in order
+  // from the ticket counter, or dispatched in block order without one, so
+  // the SMs that finish early take the pieces)
   const int total = whole + (split ? tail * f : 0);
   float* part = split ? static_cast<float*>(scratch) : nullptr;
   if (reset_ticket) {
